@@ -1,0 +1,378 @@
+"""Pins for the CPU oracle (no GPU).
+
+Each test ties an oracle function to something other than the oracle itself:
+brute force on tiny inputs, the pages' own sort-by-expert example, closed
+forms, invariants, and special cases that reduce to textbook routines computed
+with torch / scipy on the CPU.  A plausible slip in the oracle (a dropped
+term, a wrong sign or index, a transposed operand, an unstable order, a wrong
+rounding) fails at least one of them.
+
+Pages cited (titles):
+  "MoE 推理中的 Expert Parallel、KV Cache 与大规模专家并行架构解析" (§1, §2, §7, §8)
+  "MoE 推理架构深度实战：从 Expert Parallelism 到 DeepSeek-V3 的工程落地" (§2.1 router code, §3.1)
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+RNG = np.random.default_rng(1234)
+
+
+# --------------------------------------------------------------------------- helpers (test side)
+
+def bf16_bits(a: np.ndarray) -> np.ndarray:
+    """float -> bf16 bit patterns via torch (round to nearest even)."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_to_f64(a: np.ndarray) -> np.ndarray:
+    return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def rand_bf16(shape, std=1.0):
+    return bf16_bits((RNG.standard_normal(shape) * std).astype(np.float32))
+
+
+def ulp_diff_bf16(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Distance in bf16 ulps between two bf16 bit arrays (same-sign finite values)."""
+    def key(x):
+        x = x.astype(np.int32)
+        return np.where(x & 0x8000, -(x & 0x7FFF), x & 0x7FFF)
+    return np.abs(key(a) - key(b))
+
+
+def torch_bf16_round_f64(v: torch.Tensor) -> torch.Tensor:
+    return v.to(torch.float32).to(torch.bfloat16)
+
+
+# --------------------------------------------------------------------------- bf16 rounding
+
+def test_bf16_round_closed_forms():
+    # exact ties round to the even mantissa
+    assert oracle.bf16_round(1.0 + 2.0 ** -8) == 0x3F80          # tie between 1 and 1+2^-7 -> 1
+    assert oracle.bf16_round(1.0 + 3 * 2.0 ** -8) == 0x3F82      # tie -> 1+2^-6 (even)
+    assert oracle.bf16_round(-(1.0 + 2.0 ** -8)) == 0xBF80
+    # one rounding from double: just above a tie rounds up (an fp32 detour would round to even)
+    assert oracle.bf16_round(1.0 + 2.0 ** -8 + 2.0 ** -40) == 0x3F81
+    assert oracle.bf16_round(0.0) == 0x0000
+    assert oracle.bf16_round(-2.5) == 0xC020
+    assert oracle.bf16_round(3.0e38) == 0x7F62
+
+
+def test_bf16_round_matches_torch_on_fp32_values():
+    v = (RNG.standard_normal(4000) * np.exp(RNG.uniform(-20, 20, 4000))).astype(np.float32)
+    ours = np.array([oracle.bf16_round(float(x)) for x in v], dtype=np.uint16)
+    assert np.array_equal(ours, bf16_bits(v))
+
+
+# --------------------------------------------------------------------------- router logits
+
+def test_router_logits_vs_torch_matmul():
+    T, d, E = 37, 192, 13
+    x, wg = rand_bf16((T, d)), rand_bf16((E, d), 1 / math.sqrt(d))
+    ours = oracle.router_logits(x, wg)
+    ref = (torch.from_numpy(bf16_to_f64(x)) @ torch.from_numpy(bf16_to_f64(wg)).T).to(torch.float32).numpy()
+    # both sum exact bf16 products in double; only the order differs -> at most 1 fp32 ulp
+    assert np.all(np.abs(ours - ref) <= np.spacing(np.abs(ref)))
+    assert np.mean(ours == ref) > 0.99
+
+
+# --------------------------------------------------------------------------- routing
+
+def brute_topk(keys: np.ndarray, k: int) -> np.ndarray:
+    """k rounds of argmax, removing the winner; np.argmax breaks ties to the lowest index."""
+    T = keys.shape[0]
+    out = np.empty((T, k), np.int32)
+    for t in range(T):
+        kk = keys[t].astype(np.float64).copy()
+        for j in range(k):
+            e = int(np.argmax(kk))
+            out[t, j] = e
+            kk[e] = -np.inf
+    return out
+
+
+@pytest.mark.parametrize("E,k", [(8, 1), (8, 2), (13, 4), (64, 2), (256, 8), (5, 5)])
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_route_vs_bruteforce(E, k, with_bias):
+    T = 150
+    logits = RNG.standard_normal((T, E)).astype(np.float32)
+    bias = RNG.uniform(-0.1, 0.1, E).astype(np.float32) if with_bias else None
+    idx, w = oracle.route(logits, k, bias)
+    keys = logits + (bias if bias is not None else np.float32(0))      # fp32 add
+    assert np.array_equal(idx, brute_topk(keys, k))
+    # weights: softmax over the chosen subset of the UNBIASED logits (equal to the
+    # renormalised full softmax by shift/scale invariance)
+    for t in range(T):
+        ref = scipy.special.softmax(logits[t, idx[t]].astype(np.float64))
+        np.testing.assert_allclose(w[t], ref, rtol=2e-7, atol=1e-9)
+    np.testing.assert_allclose(w.astype(np.float64).sum(1), 1.0, atol=1e-6)
+
+
+def test_route_ties_break_to_lower_expert():
+    T, E, k = 300, 16, 4
+    logits = RNG.integers(-3, 3, (T, E)).astype(np.float32)     # many exact ties
+    logits[0, :] = 0.0                                          # all tied
+    logits[1, :] = -0.0
+    logits[1, 5] = 0.0                                          # -0 == +0
+    idx, w = oracle.route(logits, k)
+    assert np.array_equal(idx, brute_topk(logits, k))
+    assert list(idx[0]) == [0, 1, 2, 3]
+    assert list(idx[1]) == [0, 1, 2, 3]
+    np.testing.assert_allclose(w[0], 0.25, rtol=1e-7)
+
+
+def test_route_k1_is_argmax_with_unit_weight():
+    logits = RNG.standard_normal((500, 32)).astype(np.float32)
+    idx, w = oracle.route(logits, 1)
+    assert np.array_equal(idx[:, 0], np.argmax(logits, axis=1))
+    assert np.all(w == 1.0)
+
+
+def test_route_k_equals_E_gives_full_softmax():
+    logits = (RNG.standard_normal((64, 12)) * 3).astype(np.float32)
+    idx, w = oracle.route(logits, 12)
+    p = scipy.special.softmax(logits.astype(np.float64), axis=1)
+    for t in range(64):
+        assert np.all(np.diff(logits[t, idx[t]]) <= 0)         # descending
+        np.testing.assert_allclose(w[t], p[t, idx[t]], rtol=2e-7)
+
+
+def test_route_bias_selects_but_does_not_weight():
+    T, E, k = 50, 32, 3
+    logits = RNG.standard_normal((T, E)).astype(np.float32)
+    forced = [4, 9, 30]
+    bias = np.zeros(E, np.float32)
+    bias[forced] = 100.0
+    idx, w = oracle.route(logits, k, bias)
+    for t in range(T):
+        assert sorted(idx[t]) == forced
+        ref = scipy.special.softmax(logits[t, idx[t]].astype(np.float64))
+        np.testing.assert_allclose(w[t], ref, rtol=2e-7)
+
+
+def test_route_shift_invariance():
+    logits = RNG.standard_normal((80, 24)).astype(np.float32)
+    i1, w1 = oracle.route(logits, 3)
+    i2, w2 = oracle.route(logits + np.float32(8.0), 3)
+    assert np.array_equal(i1, i2)
+    np.testing.assert_allclose(w1, w2, rtol=3e-6)
+
+
+def test_route_rejects_nonfinite():
+    logits = np.zeros((4, 8), np.float32)
+    logits[2, 3] = np.inf
+    with pytest.raises(ValueError):
+        oracle.route(logits, 2)
+
+
+# --------------------------------------------------------------------------- capacity
+
+def test_capacity_values():
+    # router formula int(num_tokens / num_experts * factor), Python int() truncation
+    for T, E, k, cf in [(4096, 8, 2, 1.25), (4096, 8, 2, 2.0), (1000, 7, 3, 1.1), (1, 64, 2, 1.25),
+                        (16384, 128, 8, 1.0), (999, 10, 1, 0.3)]:
+        assert oracle.capacity(T, E, k, cf, oracle.CAP_PER_TOKEN) == int(T / E * cf)
+        assert oracle.capacity(T, E, k, cf, oracle.CAP_PER_ASSIGNMENT) == int(T * k / E * cf)
+    assert oracle.capacity(32768, 64, 2, 1.25, oracle.CAP_PER_ASSIGNMENT) == 1280
+    assert oracle.capacity(32768, 64, 2, 1.25, oracle.CAP_PER_TOKEN) == 640
+    assert oracle.capacity(4096, 8, 2, 2.0, oracle.CAP_PER_TOKEN) == 1024      # eval factor 2.0
+    assert oracle.capacity(10, 3, 1, 0.9, oracle.CAP_PER_TOKEN) == 3            # 3.0000000000000004 -> 3
+    assert oracle.capacity(10, 3, 1, 1.0, oracle.CAP_NONE) == -1
+
+
+# --------------------------------------------------------------------------- dispatch
+
+def random_idx(T, E, k):
+    return np.stack([RNG.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+
+
+def brute_dispatch(idx, E, C):
+    """Per expert: the ascending list of tokens routed to it; keep its first C."""
+    T, k = idx.shape
+    lists = [[t for t in range(T) if e in idx[t]] for e in range(E)]
+    kept = [l if C < 0 else l[:C] for l in lists]
+    offsets = np.concatenate([[0], np.cumsum([len(l) for l in kept])]).astype(np.int32)
+    dest = np.full((T, k), -1, np.int32)
+    src = np.empty(offsets[-1], np.int32)
+    for e in range(E):
+        for pos, t in enumerate(kept[e]):
+            j = int(np.where(idx[t] == e)[0][0])
+            dest[t, j] = offsets[e] + pos
+            src[offsets[e] + pos] = t
+    return [len(l) for l in lists], [len(l) for l in kept], offsets, dest, src
+
+
+@pytest.mark.parametrize("T,E,k,C", [(200, 8, 2, -1), (200, 8, 2, 30), (333, 16, 4, 50), (64, 8, 8, 5),
+                                     (100, 4, 1, 0), (257, 32, 3, 1000), (1, 8, 2, -1)])
+def test_dispatch_vs_bruteforce(T, E, k, C):
+    idx = random_idx(T, E, k)
+    r = oracle.dispatch(idx, E, C)
+    craw, cnt, off, dest, src = brute_dispatch(idx, E, C)
+    assert np.array_equal(r["counts_raw"], craw)
+    assert np.array_equal(r["counts"], cnt)
+    assert np.array_equal(r["offsets"], off)
+    assert np.array_equal(r["dest"], dest)
+    assert np.array_equal(r["src_token"], src)
+    # invariants
+    assert r["counts_raw"].sum() == T * k
+    assert np.array_equal(r["counts_raw"], np.bincount(idx.ravel(), minlength=E))
+    drops = int((r["dest"] < 0).sum())
+    assert r["counts"].sum() == T * k - drops == r["N"]
+    if C >= 0:
+        assert np.array_equal(r["counts"], np.minimum(r["counts_raw"], C))
+    else:
+        assert drops == 0
+    assert np.all(np.diff(r["offsets"]) >= 0)
+    kept = r["dest"] >= 0
+    tt = np.repeat(np.arange(T)[:, None], k, 1)
+    assert np.array_equal(r["src_token"][r["dest"][kept]], tt[kept])
+
+
+def test_dispatch_zero_capacity_drops_everything():
+    idx = random_idx(40, 8, 2)
+    r = oracle.dispatch(idx, 8, 0)
+    assert r["N"] == 0 and np.all(r["dest"] == -1) and np.all(r["offsets"] == 0)
+
+
+def test_permutation_matches_pages_example():
+    rows = [l.split() for l in open(os.path.join(HERE, "golden", "permutation_example.txt"))
+            if l.strip() and not l.startswith("#")]
+    experts, sorted_ids, src_expected = ([int(v) for v in r] for r in rows)
+    idx = np.array(experts, np.int32)[:, None]
+    r = oracle.dispatch(idx, 8, -1)
+    assert list(r["src_token"]) == src_expected
+    assert [experts[t] for t in r["src_token"]] == sorted_ids
+
+
+# --------------------------------------------------------------------------- permute / combine
+
+def test_unpermute_identity_k1():
+    T, d, E = 90, 64, 8
+    x = rand_bf16((T, d))
+    idx = random_idx(T, E, 1)
+    r = oracle.dispatch(idx, E, -1)
+    xp = oracle.gather(x, r["dest"], r["N"])
+    out = oracle.combine(xp, r["dest"], np.ones((T, 1), np.float32))
+    assert np.array_equal(out, x)
+
+
+def test_unpermute_identity_k4_weights_sum_to_one():
+    T, d, E, k = 70, 32, 16, 4
+    x = rand_bf16((T, d))
+    logits = RNG.standard_normal((T, E)).astype(np.float32)
+    idx, w = oracle.route(logits, k)
+    r = oracle.dispatch(idx, E, -1)
+    xp = oracle.gather(x, r["dest"], r["N"])
+    out = oracle.combine(xp, r["dest"], w)
+    assert np.array_equal(out, x)
+
+
+def test_combine_dropped_slots_contribute_zero_and_shared_added():
+    T, d, k = 3, 8, 2
+    y = bf16_bits(np.arange(4 * d, dtype=np.float32).reshape(4, d) / 8)
+    dest = np.array([[0, -1], [-1, -1], [2, 3]], np.int32)
+    w = np.array([[0.75, 0.25], [0.5, 0.5], [0.5, 0.5]], np.float32)
+    ysh = bf16_bits(np.full((T, d), 0.5, np.float32))
+    out = bf16_to_f64(oracle.combine(y, dest, w, ysh))
+    yf = bf16_to_f64(y)
+    np.testing.assert_array_equal(out[0], 0.75 * yf[0] + 0.5)
+    np.testing.assert_array_equal(out[1], 0.5)
+    np.testing.assert_allclose(out[2], bf16_to_f64(bf16_bits((0.5 * yf[2] + 0.5 * yf[3] + 0.5).astype(np.float32))))
+
+
+# --------------------------------------------------------------------------- experts
+
+def textbook_swiglu(x, W1, W3, W2):
+    """torch float64 dense SwiGLU FFN, W2 (silu(W1 x) * (W3 x)), with bf16 stores of h and y."""
+    X = torch.from_numpy(bf16_to_f64(x))
+    g = X @ torch.from_numpy(bf16_to_f64(W1)).T
+    u = X @ torch.from_numpy(bf16_to_f64(W3)).T
+    h = torch_bf16_round_f64(torch.nn.functional.silu(g) * u)
+    y = torch_bf16_round_f64(h.to(torch.float64) @ torch.from_numpy(bf16_to_f64(W2)).T)
+    to_bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)
+    return to_bits(h), to_bits(y)
+
+
+def test_expert_ffn_vs_textbook():
+    rows, d, f = 24, 96, 160
+    x = rand_bf16((rows, d))
+    W1, W3 = rand_bf16((f, d), d ** -0.5), rand_bf16((f, d), d ** -0.5)
+    W2 = rand_bf16((d, f), f ** -0.5)
+    h, y = oracle.expert_ffn(x, W1, W3, W2)
+    h_ref, y_ref = textbook_swiglu(x, W1, W3, W2)
+    # only summation order (and torch's fp32 detour when rounding) differ: <= 1 bf16 ulp, nearly all exact
+    assert ulp_diff_bf16(h, h_ref).max() <= 1 and np.mean(h == h_ref) > 0.99
+    assert ulp_diff_bf16(y, y_ref).max() <= 1 and np.mean(y == y_ref) > 0.97
+
+
+def test_layer_single_expert_is_dense_swiglu():
+    T, d, f = 40, 64, 128
+    x = rand_bf16((T, d))
+    wg = rand_bf16((1, d), d ** -0.5)
+    W1, W3 = rand_bf16((1, f, d), d ** -0.5), rand_bf16((1, f, d), d ** -0.5)
+    W2 = rand_bf16((1, d, f), f ** -0.5)
+    r = oracle.layer_forward(x, wg, W1, W3, W2, k=1)
+    _, y_ref = textbook_swiglu(x, W1[0], W3[0], W2[0])
+    assert np.all(r["w"] == 1.0) and np.all(r["idx"] == 0)
+    assert ulp_diff_bf16(r["out"], y_ref).max() <= 1 and np.mean(r["out"] == y_ref) > 0.97
+
+
+def test_layer_equals_dense_weighted_sum_over_all_experts():
+    T, d, E, k, f = 48, 64, 8, 2, 96
+    x = rand_bf16((T, d))
+    wg = rand_bf16((E, d), d ** -0.5)
+    W1, W3 = rand_bf16((E, f, d), d ** -0.5), rand_bf16((E, f, d), d ** -0.5)
+    W2 = rand_bf16((E, d, f), f ** -0.5)
+    r = oracle.layer_forward(x, wg, W1, W3, W2, k=k)
+    # every expert on every token (textbook), gates zero off the selected set
+    G = np.zeros((T, E))
+    for t in range(T):
+        G[t, r["idx"][t]] = r["w"][t]
+    acc = np.zeros((T, d))
+    for e in range(E):
+        _, ye = textbook_swiglu(x, W1[e], W3[e], W2[e])
+        acc += G[:, e:e + 1] * bf16_to_f64(ye)
+    ref = bf16_bits(acc.astype(np.float32))
+    assert ulp_diff_bf16(r["out"], ref).max() <= 2 and np.mean(r["out"] == ref) > 0.95
+
+
+def test_shared_expert_alone_when_routed_outputs_vanish():
+    T, d, E, k, f, fs = 32, 64, 4, 2, 64, 128
+    x = rand_bf16((T, d))
+    wg = rand_bf16((E, d), d ** -0.5)
+    W1, W3 = rand_bf16((E, f, d), d ** -0.5), rand_bf16((E, f, d), d ** -0.5)
+    W2 = np.zeros((E, d, f), np.uint16)                                    # routed experts output 0
+    W1s, W3s, W2s = rand_bf16((fs, d), d ** -0.5), rand_bf16((fs, d), d ** -0.5), rand_bf16((d, fs), fs ** -0.5)
+    r = oracle.layer_forward(x, wg, W1, W3, W2, k=k, W1s=W1s, W3s=W3s, W2s=W2s)
+    _, ysh = textbook_swiglu(x, W1s, W3s, W2s)
+    assert ulp_diff_bf16(r["out"], ysh).max() <= 1
+    assert np.array_equal(r["out"], r["y_shared"])
+
+
+def test_layer_zero_capacity_outputs_zero():
+    T, d, E, k, f = 16, 32, 4, 2, 64
+    x = rand_bf16((T, d))
+    wg = rand_bf16((E, d), d ** -0.5)
+    W1, W3, W2 = rand_bf16((E, f, d)), rand_bf16((E, f, d)), rand_bf16((E, d, f))
+    r = oracle.layer_forward(x, wg, W1, W3, W2, k=k, C=0)
+    assert r["N"] == 0 and np.all(bf16_to_f64(r["out"]) == 0)
+
+
+def test_layer_routes_supplied_logits():
+    T, d, E, k, f = 20, 32, 8, 2, 64
+    x = rand_bf16((T, d))
+    wg = rand_bf16((E, d), d ** -0.5)
+    W1, W3, W2 = rand_bf16((E, f, d)), rand_bf16((E, f, d)), rand_bf16((E, d, f))
+    logits = RNG.standard_normal((T, E)).astype(np.float32)
+    r = oracle.layer_forward(x, wg, W1, W3, W2, k=k, logits_in=logits)
+    i2, _ = oracle.route(logits, k)
+    assert np.array_equal(r["idx"], i2) and np.array_equal(r["logits"], logits)
