@@ -1,0 +1,384 @@
+#!/usr/bin/env python
+"""Benchmark: MoE-layer tokens/s on B200 (Router -> Permutation -> Expert GEMM -> Combine).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral] [--impl ours|reference]
+
+One step = one moe_layer_forward over one batch of T tokens whose inputs already sit in
+HBM (router GEMM, top-k, histogram/scan/permute, grouped GEMM1 + SwiGLU, grouped GEMM2,
+combine).  Under torchrun each rank runs its own token batch against replicated weights
+(no collective on the data path: weak scaling) and the time is the max over ranks.
+
+Rank 0 prints one JSON line: value (tokens/s over all ranks), the dominant kernel's
+roofline (its CUDA-event duration inside the timed region vs MEASURED_PEAKS.json),
+an end-to-end number through the public API with host buffers, the SM clocks seen,
+and (at N=1) the CPU oracle timed on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s on 1 B200; % of BF16 tensor or HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 9   # router GEMM, top-k, count, scan, scatter, gather, GEMM1, GEMM2, combine
+
+DESCR = {
+    "tiny": "tiny MoE layer T=128 d=256 E=8 top-2 f=512",
+    "mixtral": "Mixtral-like prefill T=4096 d=4096 E=8 top-2 SwiGLU f=14336",
+    "qwen3": "Qwen3-235B-A22B-like prefill T=16384 d=4096 E=128 top-8 f=1536",
+    "dsv3": "DeepSeek-V3-like decode T=256 d=7168 E=256 top-8 f=2048 + shared f=2048, selection bias",
+    "skew": "skewed routing T=32768 d=4096 E=64 top-2 f=2048 Zipf(1.2), capacity int(T*k/E*1.25)",
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mixtral", choices=list(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for n in ("grouped_gemm.cuh", "ptx.cuh"):
+        h.update(open(os.path.join(ROOT, "moe_layer_router_b200", "csrc", n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on this kernel source."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    src = kernel_source_hash()
+    for line in open(p):
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload \
+                and parts[2] == src:
+            return float(parts[3])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.dev = device_index
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.dev)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            p = [s.strip() for s in line.split(",")]
+            if len(p) < 8:
+                continue
+            try:
+                rows.append((float(p[0]), float(p[1]), p[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm = np.array([r[0] for r in rows])
+        mx = max(r[1] for r in rows)
+        loaded = sm[sm >= 0.5 * np.max(sm)]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[2][i].lower() == "active"})
+        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------ oracle (CPU) legs
+
+def host_weights(wl):
+    inp = synth.Inputs(wl)
+    w = dict(wg=inp.wg(), w1=inp.w1(), w3=inp.w3(), w2=inp.w2(), bias=inp.bias(),
+             w1s=inp.shared("w1s"), w3s=inp.shared("w3s"), w2s=inp.shared("w2s"))
+    return inp, w
+
+
+def oracle_step(oracle, wl, inp, w, t0, S):
+    x = inp.x_rows(t0, S).reshape(S, wl.d)
+    C = oracle.capacity(wl.T, wl.E, wl.k, wl.capacity_factor, wl.cap_mode)
+    if C >= 0:   # the capacity of the full batch, scaled to the sample
+        C = max(0, int(C * S / wl.T))
+    t = time.perf_counter()
+    oracle.layer_forward(x, w["wg"], w["w1"], w["w3"], w["w2"], k=wl.k, C=C, bias=w["bias"],
+                         W1s=w["w1s"], W3s=w["w3s"], W2s=w["w2s"])
+    return time.perf_counter() - t
+
+
+def cpu_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def sample_size(oracle, wl, inp, w, seconds):
+    """Tokens in one oracle sample so that it takes about `seconds` (calibrated on a small run)."""
+    s0 = min(wl.T, 16)
+    dt = oracle_step(oracle, wl, inp, w, 0, s0)
+    S = int(s0 * seconds / max(dt, 1e-3))
+    return max(1, min(wl.T, S)), dt, s0
+
+
+def cpu_baseline(wl, seconds):
+    import oracle
+    inp, w = host_weights(wl)
+    S, _, _ = sample_size(oracle, wl, inp, w, seconds)
+    dt = oracle_step(oracle, wl, inp, w, 0, S)
+    return {"value": S / dt, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"oracle layer forward on the first {S} of {wl.T} tokens ({dt:.1f} s, capacity scaled to "
+                      f"the sample), double-precision sums, OpenMP over rows"}
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    inp, w = host_weights(wl)
+    per_step = min(8.0, 150.0 / max(1, args.steps + args.warmup))
+    S, _, _ = sample_size(oracle, wl, inp, w, per_step)
+    for i in range(args.warmup):
+        oracle_step(oracle, wl, inp, w, 0, S)
+    tot = 0.0
+    for i in range(args.steps):
+        tot += oracle_step(oracle, wl, inp, w, (i * S) % max(1, wl.T - S + 1), S)
+    value = S * args.steps / tot
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": DESCR[wl.name], "global_batch": S, "sample_tokens_per_step": S},
+            "cpu_baseline": {"kind": "oracle", "cores": cpu_threads(), "value": value, "unit": "tokens/s",
+                             "sample": f"{S} of {wl.T} tokens per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------ GPU leg
+
+def gemm1_work(wl, N):
+    """Algorithmic FLOPs and bytes of one launch of the first grouped GEMM (W1/W3 + SwiGLU)."""
+    flops = 4.0 * N * wl.d * wl.f + 4.0 * wl.T * wl.d * wl.f_shared
+    return flops
+
+
+def gemm1_bytes(wl, N, touched):
+    b = touched * 2.0 * wl.f * wl.d * 2            # W1, W3 of touched experts
+    b += N * wl.d * 2 + N * wl.f * 2                # x_perm read, h write
+    if wl.f_shared:
+        b += 2.0 * wl.f_shared * wl.d * 2 + wl.T * wl.d * 2 + wl.T * wl.f_shared * 2
+    return b
+
+
+def layer_work(wl, N, touched):
+    flops = 6.0 * N * wl.d * wl.f + 2.0 * wl.T * wl.d * wl.E + 6.0 * wl.T * wl.d * wl.f_shared
+    b = touched * 3.0 * wl.f * wl.d * 2 + wl.E * wl.d * 2 + 3.0 * wl.f_shared * wl.d * 2
+    b += wl.T * wl.d * 2 + 2 * N * wl.d * 2 + 2 * N * wl.f * 2 + 2 * N * wl.d * 2 + wl.T * wl.d * 2
+    if wl.f_shared:
+        b += 2 * wl.T * wl.f_shared * 2 + 2 * wl.T * wl.d * 2
+    return flops, b
+
+
+def main():
+    args = parse()
+    wl = synth.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, wl, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    import moe_layer_router_b200 as moe
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    # inputs: replicated weights, a distinct token batch per rank
+    tensors = synth.device_tensors(wl, dev, names=["wg", "w1", "w3", "w2", "w1s", "w3s", "w2s", "bias"])
+    inp = synth.Inputs(wl)
+    x_host = torch.from_numpy(inp.x_rows(rank * wl.T, wl.T).view(np.int16)).view(torch.bfloat16).reshape(wl.T, wl.d)
+    x = x_host.to(dev)
+    T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
+    ws = torch.empty(moe.moe_workspace_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device=dev)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    W = tensors
+
+    def fwd(xin, o, events=None):
+        moe.moe_layer_forward_ex(xin, W["wg"], W["bias"], W["w1"], W["w3"], W["w2"], W.get("w1s"), W.get("w3s"),
+                                 W.get("w2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, o, ws, events)
+
+    for _ in range(max(3, args.warmup)):
+        fwd(x, out)
+    torch.cuda.synchronize()
+    rc = moe.moe_get_error()
+    if rc != 0:
+        raise RuntimeError(f"device error after warm-up: {moe.strerror(rc)}")
+
+    K = args.steps
+    evs = [{n: torch.cuda.Event(enable_timing=True) for n in moe.STAGES} for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            fwd(x, out, evs[i])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = evs[0]["route"].elapsed_time(evs[K - 1]["end"])
+    stage_ms = {}
+    for a, b in zip(moe.STAGES[:-1], moe.STAGES[1:]):
+        stage_ms[a] = float(np.mean([e[a].elapsed_time(e[b]) for e in evs]))
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    value = world * T * K / (total_ms / 1000.0)
+
+    # kept rows and touched experts of the (deterministic) routing
+    L = moe.moe_workspace_layout(T, d, E, k, f, fs)
+    counts = moe.workspace_view(ws, L, "counts", (E,), torch.int32).cpu().numpy()
+    craw = moe.workspace_view(ws, L, "counts_raw", (E,), torch.int32).cpu().numpy()
+    N = int(counts.sum())
+    touched = int((counts > 0).sum())
+
+    # end to end through the public API: pinned host input -> layer -> host output, every step
+    x_pin = x_host.pin_memory()
+    out_pin = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
+    x_e2e = torch.empty_like(x)
+    for _ in range(2):
+        x_e2e.copy_(x_pin, non_blocking=True)
+        moe.moe_layer_forward(x_e2e, W["wg"], W["bias"], W["w1"], W["w3"], W["w2"], W.get("w1s"), W.get("w3s"),
+                              W.get("w2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, out, ws)
+        out_pin.copy_(out, non_blocking=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(K):
+        x_e2e.copy_(x_pin, non_blocking=True)
+        moe.moe_layer_forward(x_e2e, W["wg"], W["bias"], W["w1"], W["w3"], W["w2"], W.get("w1s"), W.get("w3s"),
+                              W.get("w2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, out, ws)
+        out_pin.copy_(out, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_value = world * T * K / (float(te.item()) / 1000.0)
+    rc = moe.moe_get_error()
+    if rc != 0:
+        raise RuntimeError(f"device error: {moe.strerror(rc)}")
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    peaks, peak_src = load_peaks()
+    g1_ms = stage_ms["gate_up"]
+    decode = wl.name == "dsv3"
+    if decode:
+        alg = gemm1_bytes(wl, N, touched)
+        achieved = alg / (g1_ms / 1000.0) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    else:
+        alg = gemm1_work(wl, N)
+        achieved = alg / (g1_ms / 1000.0) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"]}
+    roof["traffic"] = recorded_traffic("gate_up", wl.name)
+    roof["kernel"] = "grouped_gemm_kernel<EPI_SWIGLU> (gate_up: W1/W3 + SwiGLU)"
+    roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if decode else 'bf16_tflops'}, burst)"
+    roof["algorithmic_per_launch"] = alg
+    lf, lb = layer_work(wl, N, touched)
+    step_s = total_ms / K / 1000.0
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded Philox4x32-10 + Box-Muller; random-init weights)",
+        "config": {"workload": DESCR[wl.name], "global_batch": world * T, "seq_len": T, "parallelism": f"dp{world}",
+                   "l2": "working set larger than L2 (expert weights %.2f GB per step)" % (
+                       touched * 3.0 * f * d * 2 / 1e9)},
+        "roofline": roof,
+        "layer": {"tflops": lf / step_s / 1e12, "gbs": lb / step_s / 1e9,
+                  "tensor_frac": lf / step_s / 1e12 / peaks["bf16_tflops"],
+                  "hbm_frac": lb / step_s / 1e9 / peaks["hbm_gbs"], "kept_rows": N, "touched_experts": touched,
+                  "drop_rate": 1.0 - N / float(T * k), "load_var_raw": float(np.var(craw)),
+                  "load_var_kept": float(np.var(counts)), "max_rows": int(counts.max()),
+                  "min_rows": int(counts.min())},
+        "stages_ms": stage_ms,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
+                "d2h_bytes_per_step": T * d * 2},
+        "gpu_launches": KERNELS_PER_STEP * K,
+        "clocks": clk.summary(),
+    }
+    if wl.zipf_s > 0:
+        p = craw / craw.sum()
+        line["layer"]["zipf_l1_error"] = float(np.abs(p - inp.zipf_target()).sum())
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,202 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) MoE layer forward.
+ *
+ * The layer (Router -> Permutation -> Expert GEMM -> Combine) as the pages define it:
+ *   [EP-KV]  "MoE 推理中的 Expert Parallel、KV Cache 与大规模专家并行架构解析"
+ *            §1 (FFN with a SwiGLU gate), §2 (router + top-k experts + weighted combine,
+ *            y = g5 E5(x) + g18 E18(x)), §7 (restore token order and aggregate),
+ *            §8 (count, sort and pack tokens by expert, grouped GEMM), §10 (data path).
+ *   [EP-DS3] "MoE 推理架构深度实战：从 Expert Parallelism 到 DeepSeek-V3 的工程落地"
+ *            §2.1 router code (gate Linear without bias, softmax, top-k, renormalise,
+ *            per-expert bias, bincount, capacity int(tokens/experts*factor)),
+ *            §3.1 (sort the routing by expert id).
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers to row-major, contiguous buffers that the
+ *     caller owns (allocates and frees).  Pointers must be 16-byte aligned.
+ *   - bf16 tensors are passed as moe_bf16 (the 16-bit pattern of a bfloat16).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream)
+ *     and runs asynchronously.  The library never allocates device memory, never
+ *     frees it and never synchronises, except moe_get_error().
+ *   - The return value is a HOST-side status: argument validation and launch errors.
+ *     Faults detected on the device (a non-finite router score, a bounded wait that
+ *     ran out) are recorded in a per-device error word read by moe_get_error().
+ *   - Shapes: 1 <= T, d % 64 == 0, f % 64 == 0, 1 <= k <= 32, k <= E <= 1024,
+ *     T*k < 2^31.  A violation returns MOE_ERR_SHAPE and launches nothing.
+ *   - Counts, offsets and the permutation stay on the device; no call reads them back,
+ *     so a sequence of calls can be captured into a CUDA graph.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16;   /* bit pattern of one bfloat16 */
+typedef void* moe_stream_t;  /* cudaStream_t */
+
+enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1, /* null pointer where one is required, bad enum value */
+    MOE_ERR_SHAPE = -2,       /* shape outside the supported range */
+    MOE_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned */
+    MOE_ERR_WORKSPACE = -4,   /* ws_bytes smaller than moe_workspace_bytes() */
+    MOE_ERR_CUDA = -5,        /* a CUDA runtime / driver call failed */
+    MOE_ERR_TIMEOUT = -6,     /* device: a bounded wait inside a kernel ran out */
+    MOE_ERR_CHECK = -7,       /* device: non-finite router score or inconsistent offsets */
+    MOE_ERR_DEVICE = -8       /* the current device is not sm_100 */
+};
+
+enum moe_cap_mode {
+    MOE_CAP_NONE = 0,           /* no capacity limit */
+    MOE_CAP_PER_TOKEN = 1,      /* C = int(T / E * factor): the router's get_expert_capacity, [EP-DS3] §2.1 */
+    MOE_CAP_PER_ASSIGNMENT = 2  /* C = int(T * k / E * factor): one slot per routed assignment */
+};
+
+/*
+ * Capacity per expert, computed in double and truncated toward zero like Python's int()
+ * ([EP-DS3] §2.1, capacity = int(num_tokens / num_experts * factor)).
+ * Returns -1 (unlimited) for MOE_CAP_NONE or an unknown mode.
+ */
+int64_t moe_capacity(int T, int E, int k, double capacity_factor, int cap_mode);
+
+/*
+ * Bytes of device workspace that moe_layer_forward() needs for these shapes
+ * (f_shared = 0: no shared expert).  The same size also covers moe_route(),
+ * moe_permute() and moe_expert_ffn() for the same T, d, E, k, f.
+ * Writes *bytes; returns MOE_OK or MOE_ERR_SHAPE / MOE_ERR_INVALID_ARG.
+ */
+int moe_workspace_bytes(int T, int d, int E, int k, int f, int f_shared, size_t* bytes);
+
+/*
+ * Router ([EP-DS3] §2.1 steps 1-4): logits = x Wg^T (fp32 accumulate on tensor cores),
+ * then per token the k largest keys logit_e + bias_e (ties -> lower e, slots in
+ * descending key order), and weights w_j = softmax(logits)_idx_j / sum over the k
+ * selected, from the UNBIASED logits (the bias steers selection only).
+ *   x         [T, d] bf16           hidden states (ignored if logits_in != NULL)
+ *   Wg        [E, d] bf16           router weight (ignored if logits_in != NULL)
+ *   bias      [E] fp32 or NULL      per-expert selection bias
+ *   logits_in [T, E] fp32 or NULL   route these scores instead of computing x Wg^T
+ *   logits_out[T, E] fp32 or NULL   receives the computed logits
+ *   idx       [T, k] int32          selected experts
+ *   w         [T, k] fp32           routing weights
+ *   ws / ws_bytes                   workspace (moe_workspace_bytes)
+ * Non-finite keys set MOE_ERR_CHECK in the device error word.
+ */
+int moe_route(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const float* logits_in,
+              int T, int d, int E, int k, float* logits_out, int32_t* idx, float* w,
+              void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Dispatch ([EP-KV] §8 count / sort / pack; [EP-DS3] §2.1 bincount + capacity, §3.1 sort by
+ * expert id): per-expert histogram, capacity in token order (per expert the first
+ * `capacity` assignments by ascending token index are kept; capacity < 0 = unlimited),
+ * exclusive scan, and a stable permutation of the kept assignments into contiguous
+ * per-expert row blocks.
+ *   x          [T, d] bf16           hidden states
+ *   idx        [T, k] int32          experts per token (distinct within a token, in [0, E))
+ *   counts_raw [E] int32             assignments per expert before the capacity limit
+ *   counts     [E] int32             kept assignments per expert
+ *   offsets    [E+1] int32           exclusive scan of counts; offsets[E] = N kept rows
+ *   dest       [T, k] int32          row of (t, j) in x_perm, or -1 if dropped
+ *   src_token  [T*k] int32           src_token[r] = token of row r, for r < N
+ *   x_perm     [T*k, d] bf16         x_perm[dest[t,j]] = x[t]; rows >= N untouched
+ */
+int moe_permute(const moe_bf16* x, const int32_t* idx, int T, int d, int E, int k, int64_t capacity,
+                int32_t* counts_raw, int32_t* counts, int32_t* offsets, int32_t* dest, int32_t* src_token,
+                moe_bf16* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Experts ([EP-KV] §1 and §8): for every expert e, on rows [offsets[e], offsets[e+1]) of x_perm,
+ *   h = bf16( silu(x_perm W1_e^T) * (x_perm W3_e^T) ),  y_perm = bf16( h W2_e^T ),
+ * two grouped GEMMs on the tcgen05 tensor cores (fp32 accumulate in tensor memory),
+ * SwiGLU fused into the first one's epilogue.  silu(a) = a / (1 + e^-a).
+ *   x_perm   [max_rows, d] bf16      permuted hidden states (max_rows >= offsets[E], usually T*k)
+ *   offsets  [E+1] int32 (device)    per-expert row ranges
+ *   W1, W3   [E, f, d] bf16          gate / up projections
+ *   W2       [E, d, f] bf16          down projection
+ *   h        [max_rows, f] bf16      intermediate (written for rows < offsets[E])
+ *   y_perm   [max_rows, d] bf16      expert outputs
+ */
+int moe_expert_ffn(const moe_bf16* x_perm, const int32_t* offsets, int max_rows, int E, int d, int f,
+                   const moe_bf16* W1, const moe_bf16* W3, const moe_bf16* W2,
+                   moe_bf16* h, moe_bf16* y_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Combine ([EP-KV] §2 weighted sum, §7 restore order and aggregate):
+ *   out[t] = bf16( sum_{j = 0..k-1, dest[t,j] >= 0} w[t,j] * y_perm[dest[t,j]]  (+ y_shared[t]) )
+ * accumulated in fp32 in slot order j = 0..k-1, the shared expert added last with
+ * weight 1; no atomics, so the result is deterministic.
+ *   y_shared [T, d] bf16 or NULL
+ */
+int moe_combine(const moe_bf16* y_perm, const int32_t* dest, const float* w, const moe_bf16* y_shared,
+                int T, int d, int k, moe_bf16* out, moe_stream_t stream);
+
+/*
+ * The whole layer: moe_route -> moe_permute -> moe_expert_ffn (+ the shared expert, run
+ * in the same grouped-GEMM launches on all T tokens) -> moe_combine.
+ *   W1s, W3s [f_shared, d], W2s [d, f_shared] bf16, all NULL and f_shared = 0 for none
+ *   ([EP-KV] §3: routed and shared experts side by side).
+ *   capacity = moe_capacity(T, E, k, capacity_factor, cap_mode).
+ *   out [T, d] bf16.
+ * Intermediates live in the workspace (layout: moe_workspace_layout()).
+ */
+int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias,
+                      const moe_bf16* W1, const moe_bf16* W3, const moe_bf16* W2,
+                      const moe_bf16* W1s, const moe_bf16* W3s, const moe_bf16* W2s, int f_shared,
+                      int T, int d, int E, int k, int f, double capacity_factor, int cap_mode,
+                      moe_bf16* out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Optional stage markers for measurement.  Each non-NULL member is a cudaEvent_t that
+ * moe_layer_forward_ex() records on `stream` at the boundary it names; NULL members are
+ * skipped.  Recording adds no work to the layer.
+ */
+typedef struct moe_stage_events {
+    void* route;     /* before the router GEMM */
+    void* topk;      /* before the top-k / softmax kernel */
+    void* permute;   /* before the histogram / scan / scatter / gather kernels */
+    void* gate_up;   /* before the first grouped GEMM (W1/W3 + SwiGLU) */
+    void* down;      /* before the second grouped GEMM (W2) */
+    void* combine;   /* before the combine kernel */
+    void* end;       /* after the combine kernel */
+} moe_stage_events;
+
+/* moe_layer_forward() with optional stage markers (events may be NULL). */
+int moe_layer_forward_ex(const moe_bf16* x, const moe_bf16* Wg, const float* bias,
+                         const moe_bf16* W1, const moe_bf16* W3, const moe_bf16* W2,
+                         const moe_bf16* W1s, const moe_bf16* W3s, const moe_bf16* W2s, int f_shared,
+                         int T, int d, int E, int k, int f, double capacity_factor, int cap_mode,
+                         moe_bf16* out, void* ws, size_t ws_bytes, moe_stream_t stream,
+                         const moe_stage_events* events);
+
+/*
+ * Byte offsets of the intermediates that moe_layer_forward() leaves in its workspace,
+ * so that a caller (a test) can read them after the call:
+ *   off[0] logits [T,E] fp32   off[1] idx [T,k] int32   off[2] w [T,k] fp32
+ *   off[3] counts_raw [E]      off[4] counts [E]        off[5] offsets [E+1]
+ *   off[6] dest [T,k]          off[7] src_token [T*k]   off[8] x_perm [T*k,d] bf16
+ *   off[9] h [T*k,f] bf16      off[10] y_perm [T*k,d]   off[11] y_shared [T,d] bf16
+ * Returns MOE_OK or a shape error.
+ */
+int moe_workspace_layout(int T, int d, int E, int k, int f, int f_shared, size_t off[12]);
+
+/*
+ * Synchronises `stream`, returns the first device-side error recorded on the current
+ * device since the last call (MOE_OK if none) and clears it.  The error word is shared
+ * by all streams of the device.
+ */
+int moe_get_error(moe_stream_t stream);
+
+/* Static text for a status code. */
+const char* moe_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

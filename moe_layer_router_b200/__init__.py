@@ -1,0 +1,186 @@
+"""B200 (sm_100a) MoE layer forward: Python binding of the C ABI in include/moe.h.
+
+Argument marshalling only.  Every step of the layer runs in the CUDA kernels of
+``libmoe_b200.so``; this module passes device pointers, sizes and the current
+torch stream, and turns a non-zero status into ``MoeError``.  There is no CPU
+fallback: if the library is missing, importing the binding raises.
+
+Names follow the C ABI: ``moe_route``, ``moe_permute``, ``moe_expert_ffn``,
+``moe_combine``, ``moe_layer_forward``, plus the helpers ``moe_capacity``,
+``moe_workspace_bytes``, ``moe_workspace_layout``, ``moe_get_error``,
+``moe_strerror``.  Tensors are torch tensors (bf16 / fp32 / int32, contiguous);
+``None`` passes NULL.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_SHAPE = -2
+MOE_ERR_ALIGN = -3
+MOE_ERR_WORKSPACE = -4
+MOE_ERR_CUDA = -5
+MOE_ERR_TIMEOUT = -6
+MOE_ERR_CHECK = -7
+MOE_ERR_DEVICE = -8
+
+MOE_CAP_NONE, MOE_CAP_PER_TOKEN, MOE_CAP_PER_ASSIGNMENT = 0, 1, 2
+
+# Names of the intermediates moe_layer_forward leaves in its workspace (moe_workspace_layout order).
+WS_NAMES = ["logits", "idx", "w", "counts_raw", "counts", "offsets", "dest", "src_token",
+            "x_perm", "h", "y_perm", "y_shared"]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {strerror(code)} ({code})")
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with __graft_entry__.build() "
+                      "(python -m moe_layer_router_b200.build)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp, _i32, _i64, _dbl, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double, ctypes.c_size_t
+
+_lib.moe_capacity.argtypes = [_i32, _i32, _i32, _dbl, _i32]
+_lib.moe_capacity.restype = _i64
+_lib.moe_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(_sz)]
+_lib.moe_workspace_layout.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(_sz)]
+_lib.moe_route.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.moe_permute.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.moe_expert_ffn.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.moe_combine.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp]
+_lib.moe_layer_forward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
+                                   _i32, _i32, _i32, _i32, _i32, _dbl, _i32, _vp, _vp, _sz, _vp]
+_lib.moe_layer_forward_ex.argtypes = _lib.moe_layer_forward.argtypes + [_vp]
+_lib.moe_get_error.argtypes = [_vp]
+_lib.moe_strerror.argtypes = [_i32]
+_lib.moe_strerror.restype = ctypes.c_char_p
+for _n in ("moe_workspace_bytes", "moe_workspace_layout", "moe_route", "moe_permute", "moe_expert_ffn",
+           "moe_combine", "moe_layer_forward", "moe_layer_forward_ex", "moe_get_error"):
+    getattr(_lib, _n).restype = _i32
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return _lib.moe_strerror(int(code)).decode()
+
+
+moe_strerror = strerror
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != MOE_OK:
+        raise MoeError(rc, where)
+
+
+def _nbytes(t) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def moe_capacity(T: int, E: int, k: int, capacity_factor: float, cap_mode: int) -> int:
+    return int(_lib.moe_capacity(T, E, k, float(capacity_factor), cap_mode))
+
+
+def moe_workspace_bytes(T: int, d: int, E: int, k: int, f: int, f_shared: int = 0) -> int:
+    out = _sz(0)
+    _check(_lib.moe_workspace_bytes(T, d, E, k, f, f_shared, ctypes.byref(out)), "moe_workspace_bytes")
+    return int(out.value)
+
+
+def moe_workspace_layout(T: int, d: int, E: int, k: int, f: int, f_shared: int = 0) -> dict:
+    arr = (_sz * 12)()
+    _check(_lib.moe_workspace_layout(T, d, E, k, f, f_shared, arr), "moe_workspace_layout")
+    return {n: int(arr[i]) for i, n in enumerate(WS_NAMES)}
+
+
+def moe_route(x, Wg, bias, logits_in, T, d, E, k, logits_out, idx, w, ws, stream=None) -> None:
+    _check(_lib.moe_route(_ptr(x), _ptr(Wg), _ptr(bias), _ptr(logits_in), T, d, E, k, _ptr(logits_out),
+                          _ptr(idx), _ptr(w), _ptr(ws), _nbytes(ws), _stream(stream)), "moe_route")
+
+
+def moe_permute(x, idx, T, d, E, k, capacity, counts_raw, counts, offsets, dest, src_token, x_perm, ws,
+                stream=None) -> None:
+    _check(_lib.moe_permute(_ptr(x), _ptr(idx), T, d, E, k, int(capacity), _ptr(counts_raw), _ptr(counts),
+                            _ptr(offsets), _ptr(dest), _ptr(src_token), _ptr(x_perm), _ptr(ws), _nbytes(ws),
+                            _stream(stream)), "moe_permute")
+
+
+def moe_expert_ffn(x_perm, offsets, max_rows, E, d, f, W1, W3, W2, h, y_perm, ws, stream=None) -> None:
+    _check(_lib.moe_expert_ffn(_ptr(x_perm), _ptr(offsets), max_rows, E, d, f, _ptr(W1), _ptr(W3), _ptr(W2),
+                               _ptr(h), _ptr(y_perm), _ptr(ws), _nbytes(ws), _stream(stream)), "moe_expert_ffn")
+
+
+def moe_combine(y_perm, dest, w, y_shared, T, d, k, out, stream=None) -> None:
+    _check(_lib.moe_combine(_ptr(y_perm), _ptr(dest), _ptr(w), _ptr(y_shared), T, d, k, _ptr(out),
+                            _stream(stream)), "moe_combine")
+
+
+def moe_layer_forward(x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, f_shared, T, d, E, k, f, capacity_factor, cap_mode,
+                      out, ws, stream=None) -> None:
+    _check(_lib.moe_layer_forward(_ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(W1s),
+                                  _ptr(W3s), _ptr(W2s), f_shared, T, d, E, k, f, float(capacity_factor), cap_mode,
+                                  _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream)), "moe_layer_forward")
+
+
+STAGES = ["route", "topk", "permute", "gate_up", "down", "combine", "end"]
+
+
+class moe_stage_events(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in STAGES]
+
+
+def moe_layer_forward_ex(x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, f_shared, T, d, E, k, f, capacity_factor,
+                         cap_mode, out, ws, events: Optional[dict] = None, stream=None) -> None:
+    """moe_layer_forward with optional stage markers: events = {stage name: torch.cuda.Event}."""
+    ev = None
+    if events:
+        ev = moe_stage_events(*[events[n].cuda_event if n in events and events[n] is not None else None
+                                for n in STAGES])
+    _check(_lib.moe_layer_forward_ex(_ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(W1s),
+                                     _ptr(W3s), _ptr(W2s), f_shared, T, d, E, k, f, float(capacity_factor),
+                                     cap_mode, _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream),
+                                     ctypes.byref(ev) if ev is not None else None), "moe_layer_forward_ex")
+
+
+def moe_get_error(stream=None) -> int:
+    return int(_lib.moe_get_error(_stream(stream)))
+
+
+def workspace_view(ws, layout: dict, name: str, shape, dtype):
+    """A typed view of one intermediate inside a moe_layer_forward workspace (uint8 tensor)."""
+    import torch
+    n = 1
+    for s in shape:
+        n *= s
+    nb = n * torch.empty((), dtype=dtype).element_size()
+    o = layout[name]
+    return ws[o:o + nb].view(dtype).view(*shape)

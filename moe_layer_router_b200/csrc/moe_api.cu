@@ -1,0 +1,546 @@
+// moe_api.cu - the C ABI (include/moe.h): argument validation, TMA descriptors, launches.
+//
+// The host side never allocates device memory and never synchronises (except
+// moe_get_error).  Every launch goes to the caller's stream.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "grouped_gemm.cuh"
+#include "route_permute_combine.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool init = false;
+    bool ok = false;
+    int sms = 0;
+    bool gemm_attr = false;
+    bool permute_attr = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mutex;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int device_info(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo& di = g_dev[dev];
+    if (!di.init) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        di.ok = (major == 10 && minor == 0);
+        di.init = true;
+    }
+    if (!di.ok) return MOE_ERR_DEVICE;
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return MOE_ERR_CUDA;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    *out = &di;
+    return MOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+int check_shape(int T, int d, int E, int k, int f) {
+    if (T < 1 || d < 64 || d % 64 || f < 64 || f % 64 || k < 1 || k > MAX_TOPK || E < k || E > 1024)
+        return MOE_ERR_SHAPE;
+    if ((long long)T * k >= (1ll << 31)) return MOE_ERR_SHAPE;
+    return MOE_OK;
+}
+
+// 2-D bf16 tensor map [rows, inner], box [box_rows, 64], 128-byte swizzle, zero fill outside.
+int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {(cuuint32_t)GEMM_BK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+template <int EPI>
+int launch_gemm(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& b0b,
+                const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& b1b, const GemmParams& p,
+                long long tiles_upper, cudaStream_t s) {
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        static bool attr_set[kMaxDevices][3] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (!attr_set[dev][EPI]) {
+            if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     GEMM_SMEM_BYTES) != cudaSuccess)
+                return MOE_ERR_CUDA;
+            attr_set[dev][EPI] = true;
+        }
+    }
+    if (tiles_upper <= 0) return MOE_OK;
+    const int grid = (int)(tiles_upper < di->sms ? tiles_upper : di->sms);
+    grouped_gemm_kernel<EPI><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, s>>>(a0, b0, b0b, a1, b1, b1b, p);
+    return launch_status();
+}
+
+// ------------------------------------------------------------------ workspace layouts
+
+struct LayerLayout {
+    size_t off[12];
+    size_t blk_cnt, rank_local, mprefix, h_shared;
+    size_t total;
+};
+
+int permute_blocks(int T) { return (T + PERMUTE_TOKENS - 1) / PERMUTE_TOKENS; }
+
+LayerLayout layer_layout(int T, int d, int E, int k, int f, int f_shared) {
+    LayerLayout L;
+    const size_t Tk = (size_t)T * k;
+    size_t cur = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = cur;
+        cur = align256(cur + bytes);
+        return o;
+    };
+    L.off[0] = take((size_t)T * E * 4);
+    L.off[1] = take(Tk * 4);
+    L.off[2] = take(Tk * 4);
+    L.off[3] = take((size_t)E * 4);
+    L.off[4] = take((size_t)E * 4);
+    L.off[5] = take((size_t)(E + 1) * 4);
+    L.off[6] = take(Tk * 4);
+    L.off[7] = take(Tk * 4);
+    L.off[8] = take(Tk * d * 2);
+    L.off[9] = take(Tk * f * 2);
+    L.off[10] = take(Tk * d * 2);
+    L.off[11] = take(f_shared > 0 ? (size_t)T * d * 2 : 0);
+    L.h_shared = take(f_shared > 0 ? (size_t)T * f_shared * 2 : 0);
+    L.blk_cnt = take((size_t)permute_blocks(T) * E * 4);
+    L.rank_local = take(Tk * 4);
+    L.mprefix = take((size_t)(E + 1) * 4);
+    L.total = cur;
+    return L;
+}
+
+// scratch used by moe_permute: blk_cnt + rank_local + mprefix
+size_t permute_scratch_bytes(int T, int E, int k, size_t* o_blk, size_t* o_rank, size_t* o_mp) {
+    size_t cur = 0;
+    *o_blk = cur;
+    cur = align256(cur + (size_t)permute_blocks(T) * E * 4);
+    *o_rank = cur;
+    cur = align256(cur + (size_t)T * k * 4);
+    *o_mp = cur;
+    cur = align256(cur + (size_t)(E + 1) * 4);
+    return cur;
+}
+
+// ------------------------------------------------------------------ stage launchers
+
+int run_router_gemm(DeviceInfo* di, const moe_bf16* x, const moe_bf16* Wg, int T, int d, int E, float* logits,
+                    cudaStream_t s) {
+    const int npad = E <= 256 ? ((E + 15) / 16) * 16 : 256;
+    CUtensorMap a, b;
+    int rc;
+    if ((rc = make_map(&a, x, d, T, GEMM_BM)) != MOE_OK) return rc;
+    if ((rc = make_map(&b, Wg, d, E, npad)) != MOE_OK) return rc;
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    GemmClass& c = p.cls[1];
+    c.K = d;
+    c.n_out = E;
+    c.ntiles = (E + npad - 1) / npad;
+    c.b_group_rows = 0;
+    c.b_tile_rows = npad;
+    c.mma_n = npad;
+    c.out = logits;
+    c.ldo = E;
+    c.out_row0 = 0;
+    c.out_rows = T;
+    p.cls[0] = c;
+    p.offsets = nullptr;
+    p.mprefix = nullptr;
+    p.E = E;
+    p.dense_rows = T;
+    const long long tiles = (long long)((T + GEMM_BM - 1) / GEMM_BM) * c.ntiles;
+    return launch_gemm<EPI_LOGITS>(di, a, b, b, a, b, b, p, tiles, s);
+}
+
+int run_topk(const float* logits, const float* bias, int T, int E, int k, int32_t* idx, float* w, cudaStream_t s) {
+    const int blocks = (T + 7) / 8;
+    const int epl = (E + 31) / 32;
+    if (epl <= 1) topk_softmax_kernel<1><<<blocks, 256, 0, s>>>(logits, bias, T, E, k, idx, w);
+    else if (epl <= 2) topk_softmax_kernel<2><<<blocks, 256, 0, s>>>(logits, bias, T, E, k, idx, w);
+    else if (epl <= 4) topk_softmax_kernel<4><<<blocks, 256, 0, s>>>(logits, bias, T, E, k, idx, w);
+    else if (epl <= 8) topk_softmax_kernel<8><<<blocks, 256, 0, s>>>(logits, bias, T, E, k, idx, w);
+    else if (epl <= 16) topk_softmax_kernel<16><<<blocks, 256, 0, s>>>(logits, bias, T, E, k, idx, w);
+    else topk_softmax_kernel<32><<<blocks, 256, 0, s>>>(logits, bias, T, E, k, idx, w);
+    return launch_status();
+}
+
+int run_permute(DeviceInfo* di, const moe_bf16* x, const int32_t* idx, int T, int d, int E, int k, long long C,
+                int32_t* counts_raw, int32_t* counts, int32_t* offsets, int32_t* dest, int32_t* src_token,
+                moe_bf16* x_perm, int32_t* blk_cnt, int32_t* rank_local, int32_t* mprefix, cudaStream_t s) {
+    const int nb = permute_blocks(T);
+    const size_t smem = (size_t)(PERMUTE_WARPS * E + PERMUTE_TOKENS * k) * sizeof(int);
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!di->permute_attr) {
+            if (cudaFuncSetAttribute(permute_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (PERMUTE_WARPS * 1024 + PERMUTE_TOKENS * MAX_TOPK) * (int)sizeof(int)) !=
+                cudaSuccess)
+                return MOE_ERR_CUDA;
+            di->permute_attr = true;
+        }
+    }
+    permute_count_kernel<<<nb, PERMUTE_TOKENS, smem, s>>>(idx, T, E, k, blk_cnt, rank_local);
+    permute_scan_kernel<<<1, 1024, 0, s>>>(blk_cnt, nb, E, C, counts_raw, counts, offsets, mprefix);
+    permute_scatter_kernel<<<nb, PERMUTE_TOKENS, 0, s>>>(idx, rank_local, blk_cnt, offsets, T, E, k, C, dest,
+                                                          src_token);
+    gather_rows_kernel<<<(T + 7) / 8, 256, 0, s>>>(reinterpret_cast<const uint4*>(x), dest, T, d, k,
+                                                    reinterpret_cast<uint4*>(x_perm));
+    return launch_status();
+}
+
+// Both grouped GEMMs of the expert FFN.  Class 0: routed experts on x_perm rows given by
+// offsets/mprefix.  Class 1 (optional): the shared expert on all T rows of x.
+struct FfnArgs {
+    const moe_bf16* x_perm;
+    const int32_t* offsets;
+    const int32_t* mprefix;
+    int max_rows, E, d, f;
+    const moe_bf16 *W1, *W3, *W2;
+    moe_bf16 *h, *y_perm;
+    // shared expert (f_shared = 0: none)
+    const moe_bf16* x;
+    int T, f_shared;
+    const moe_bf16 *W1s, *W3s, *W2s;
+    moe_bf16 *h_shared, *y_shared;
+};
+
+int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_down = nullptr) {
+    const bool shared = a.f_shared > 0;
+    const bool routed = a.max_rows > 0;
+    int rc;
+    // ---- GEMM1: h = silu(x W1^T) * (x W3^T)
+    {
+        CUtensorMap A0, B0, B0b, A1, B1, B1b;
+        if (routed) {
+            if ((rc = make_map(&A0, a.x_perm, a.d, a.max_rows, GEMM_BM)) != MOE_OK) return rc;
+            if ((rc = make_map(&B0, a.W1, a.d, (uint64_t)a.E * a.f, 128)) != MOE_OK) return rc;
+            if ((rc = make_map(&B0b, a.W3, a.d, (uint64_t)a.E * a.f, 128)) != MOE_OK) return rc;
+        }
+        if (shared) {
+            if ((rc = make_map(&A1, a.x, a.d, a.T, GEMM_BM)) != MOE_OK) return rc;
+            if ((rc = make_map(&B1, a.W1s, a.d, a.f_shared, 128)) != MOE_OK) return rc;
+            if ((rc = make_map(&B1b, a.W3s, a.d, a.f_shared, 128)) != MOE_OK) return rc;
+        }
+        if (!routed) { A0 = A1; B0 = B1; B0b = B1b; }
+        if (!shared) { A1 = A0; B1 = B0; B1b = B0b; }
+        GemmParams p;
+        memset(&p, 0, sizeof(p));
+        GemmClass& c0 = p.cls[0];
+        c0.K = a.d; c0.n_out = a.f; c0.ntiles = (a.f + 127) / 128; c0.b_group_rows = a.f; c0.b_tile_rows = 128;
+        c0.mma_n = 256; c0.out = a.h; c0.ldo = a.f; c0.out_row0 = 0; c0.out_rows = a.max_rows;
+        GemmClass& c1 = p.cls[1];
+        c1.K = a.d; c1.n_out = a.f_shared; c1.ntiles = (a.f_shared + 127) / 128; c1.b_group_rows = 0;
+        c1.b_tile_rows = 128; c1.mma_n = 256; c1.out = a.h_shared; c1.ldo = a.f_shared; c1.out_row0 = 0;
+        c1.out_rows = a.T;
+        p.offsets = routed ? a.offsets : nullptr;
+        p.mprefix = a.mprefix;
+        p.E = a.E;
+        p.dense_rows = shared ? a.T : 0;
+        long long tiles = 0;
+        if (routed) tiles += ((long long)(a.max_rows + GEMM_BM - 1) / GEMM_BM + a.E) * c0.ntiles;
+        if (shared) tiles += (long long)((a.T + GEMM_BM - 1) / GEMM_BM) * c1.ntiles;
+        if ((rc = launch_gemm<EPI_SWIGLU>(di, A0, B0, B0b, A1, B1, B1b, p, tiles, s)) != MOE_OK) return rc;
+    }
+    if (ev_down && cudaEventRecord(ev_down, s) != cudaSuccess) return MOE_ERR_CUDA;
+    // ---- GEMM2: y = h W2^T
+    {
+        CUtensorMap A0, B0, A1, B1;
+        if (routed) {
+            if ((rc = make_map(&A0, a.h, a.f, a.max_rows, GEMM_BM)) != MOE_OK) return rc;
+            if ((rc = make_map(&B0, a.W2, a.f, (uint64_t)a.E * a.d, 256)) != MOE_OK) return rc;
+        }
+        if (shared) {
+            if ((rc = make_map(&A1, a.h_shared, a.f_shared, a.T, GEMM_BM)) != MOE_OK) return rc;
+            if ((rc = make_map(&B1, a.W2s, a.f_shared, a.d, 256)) != MOE_OK) return rc;
+        }
+        if (!routed) { A0 = A1; B0 = B1; }
+        if (!shared) { A1 = A0; B1 = B0; }
+        GemmParams p;
+        memset(&p, 0, sizeof(p));
+        GemmClass& c0 = p.cls[0];
+        c0.K = a.f; c0.n_out = a.d; c0.ntiles = (a.d + 255) / 256; c0.b_group_rows = a.d; c0.b_tile_rows = 256;
+        c0.mma_n = 256; c0.out = a.y_perm; c0.ldo = a.d; c0.out_row0 = 0; c0.out_rows = a.max_rows;
+        GemmClass& c1 = p.cls[1];
+        c1.K = a.f_shared; c1.n_out = a.d; c1.ntiles = (a.d + 255) / 256; c1.b_group_rows = 0; c1.b_tile_rows = 256;
+        c1.mma_n = 256; c1.out = a.y_shared; c1.ldo = a.d; c1.out_row0 = 0; c1.out_rows = a.T;
+        p.offsets = routed ? a.offsets : nullptr;
+        p.mprefix = a.mprefix;
+        p.E = a.E;
+        p.dense_rows = shared ? a.T : 0;
+        long long tiles = 0;
+        if (routed) tiles += ((long long)(a.max_rows + GEMM_BM - 1) / GEMM_BM + a.E) * c0.ntiles;
+        if (shared) tiles += (long long)((a.T + GEMM_BM - 1) / GEMM_BM) * c1.ntiles;
+        if ((rc = launch_gemm<EPI_STORE>(di, A0, B0, B0, A1, B1, B1, p, tiles, s)) != MOE_OK) return rc;
+    }
+    return MOE_OK;
+}
+
+int run_combine(const moe_bf16* y_perm, const int32_t* dest, const float* w, const moe_bf16* y_shared, int T, int d,
+                int k, moe_bf16* out, cudaStream_t s) {
+    combine_kernel<<<(T + 7) / 8, 256, 0, s>>>(reinterpret_cast<const uint4*>(y_perm), dest, w,
+                                                reinterpret_cast<const uint4*>(y_shared), T, d, k,
+                                                reinterpret_cast<uint4*>(out));
+    return launch_status();
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+#define MOE_REQUIRE(cond, code) \
+    do {                        \
+        if (!(cond)) return (code); \
+    } while (0)
+
+extern "C" {
+
+int64_t moe_capacity(int T, int E, int k, double capacity_factor, int cap_mode) {
+    if (E <= 0) return -1;
+    if (cap_mode == MOE_CAP_PER_TOKEN) return (int64_t)((double)T / (double)E * capacity_factor);
+    if (cap_mode == MOE_CAP_PER_ASSIGNMENT) return (int64_t)((double)T * (double)k / (double)E * capacity_factor);
+    return -1;
+}
+
+int moe_workspace_bytes(int T, int d, int E, int k, int f, int f_shared, size_t* bytes) {
+    MOE_REQUIRE(bytes != nullptr, MOE_ERR_INVALID_ARG);
+    int rc = check_shape(T, d, E, k, f);
+    if (rc != MOE_OK) return rc;
+    MOE_REQUIRE(f_shared >= 0 && f_shared % 64 == 0, MOE_ERR_SHAPE);
+    *bytes = layer_layout(T, d, E, k, f, f_shared).total;
+    return MOE_OK;
+}
+
+int moe_workspace_layout(int T, int d, int E, int k, int f, int f_shared, size_t off[12]) {
+    MOE_REQUIRE(off != nullptr, MOE_ERR_INVALID_ARG);
+    int rc = check_shape(T, d, E, k, f);
+    if (rc != MOE_OK) return rc;
+    MOE_REQUIRE(f_shared >= 0 && f_shared % 64 == 0, MOE_ERR_SHAPE);
+    LayerLayout L = layer_layout(T, d, E, k, f, f_shared);
+    for (int i = 0; i < 12; ++i) off[i] = L.off[i];
+    return MOE_OK;
+}
+
+int moe_route(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const float* logits_in, int T, int d, int E,
+              int k, float* logits_out, int32_t* idx, float* w, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    MOE_REQUIRE(T >= 1 && k >= 1 && k <= MAX_TOPK && E >= k && E <= 1024 && (long long)T * k < (1ll << 31),
+                MOE_ERR_SHAPE);
+    MOE_REQUIRE(idx && w, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(idx) && aligned16(w) && aligned16(bias) && aligned16(logits_in) && aligned16(logits_out),
+                MOE_ERR_ALIGN);
+    DeviceInfo* di;
+    int rc = device_info(&di);
+    if (rc != MOE_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const float* logits = logits_in;
+    if (!logits_in) {
+        MOE_REQUIRE(x && Wg, MOE_ERR_INVALID_ARG);
+        MOE_REQUIRE(d >= 64 && d % 64 == 0, MOE_ERR_SHAPE);
+        MOE_REQUIRE(aligned16(x) && aligned16(Wg), MOE_ERR_ALIGN);
+        float* dst = logits_out;
+        if (!dst) {
+            MOE_REQUIRE(ws && ws_bytes >= (size_t)T * E * 4, MOE_ERR_WORKSPACE);
+            MOE_REQUIRE(aligned16(ws), MOE_ERR_ALIGN);
+            dst = static_cast<float*>(ws);
+        }
+        if ((rc = run_router_gemm(di, x, Wg, T, d, E, dst, s)) != MOE_OK) return rc;
+        logits = dst;
+    } else if (logits_out && logits_out != logits_in) {
+        if (cudaMemcpyAsync(logits_out, logits_in, (size_t)T * E * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    return run_topk(logits, bias, T, E, k, idx, w, s);
+}
+
+int moe_permute(const moe_bf16* x, const int32_t* idx, int T, int d, int E, int k, int64_t capacity,
+                int32_t* counts_raw, int32_t* counts, int32_t* offsets, int32_t* dest, int32_t* src_token,
+                moe_bf16* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    int rc = check_shape(T, d, E, k, 64);
+    if (rc != MOE_OK) return rc;
+    MOE_REQUIRE(x && idx && counts_raw && counts && offsets && dest && src_token && x_perm && ws, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(x) && aligned16(x_perm) && aligned16(idx) && aligned16(dest) && aligned16(ws),
+                MOE_ERR_ALIGN);
+    size_t o_blk, o_rank, o_mp;
+    const size_t need = permute_scratch_bytes(T, E, k, &o_blk, &o_rank, &o_mp);
+    MOE_REQUIRE(ws_bytes >= need, MOE_ERR_WORKSPACE);
+    DeviceInfo* di;
+    if ((rc = device_info(&di)) != MOE_OK) return rc;
+    char* base = static_cast<char*>(ws);
+    return run_permute(di, x, idx, T, d, E, k, capacity < 0 ? -1 : (long long)capacity, counts_raw, counts, offsets,
+                       dest, src_token, x_perm, reinterpret_cast<int32_t*>(base + o_blk),
+                       reinterpret_cast<int32_t*>(base + o_rank), reinterpret_cast<int32_t*>(base + o_mp),
+                       static_cast<cudaStream_t>(stream));
+}
+
+int moe_expert_ffn(const moe_bf16* x_perm, const int32_t* offsets, int max_rows, int E, int d, int f,
+                   const moe_bf16* W1, const moe_bf16* W3, const moe_bf16* W2, moe_bf16* h, moe_bf16* y_perm,
+                   void* ws, size_t ws_bytes, moe_stream_t stream) {
+    MOE_REQUIRE(max_rows >= 0 && E >= 1 && E <= 1024 && d >= 64 && d % 64 == 0 && f >= 64 && f % 64 == 0,
+                MOE_ERR_SHAPE);
+    MOE_REQUIRE(x_perm && offsets && W1 && W3 && W2 && h && y_perm && ws, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(x_perm) && aligned16(W1) && aligned16(W3) && aligned16(W2) && aligned16(h) &&
+                    aligned16(y_perm) && aligned16(ws),
+                MOE_ERR_ALIGN);
+    MOE_REQUIRE(ws_bytes >= (size_t)(E + 1) * 4, MOE_ERR_WORKSPACE);
+    DeviceInfo* di;
+    int rc = device_info(&di);
+    if (rc != MOE_OK) return rc;
+    if (max_rows == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t* mprefix = static_cast<int32_t*>(ws);
+    tile_prefix_kernel<<<1, 1024, 0, s>>>(offsets, E, max_rows, mprefix);
+    if ((rc = launch_status()) != MOE_OK) return rc;
+    FfnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x_perm = x_perm; a.offsets = offsets; a.mprefix = mprefix; a.max_rows = max_rows; a.E = E; a.d = d; a.f = f;
+    a.W1 = W1; a.W3 = W3; a.W2 = W2; a.h = h; a.y_perm = y_perm;
+    a.f_shared = 0;
+    return run_expert_ffn(di, a, s);
+}
+
+int moe_combine(const moe_bf16* y_perm, const int32_t* dest, const float* w, const moe_bf16* y_shared, int T, int d,
+                int k, moe_bf16* out, moe_stream_t stream) {
+    MOE_REQUIRE(T >= 1 && d >= 64 && d % 64 == 0 && k >= 1 && k <= MAX_TOPK, MOE_ERR_SHAPE);
+    MOE_REQUIRE(y_perm && dest && w && out, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(y_perm) && aligned16(y_shared) && aligned16(out), MOE_ERR_ALIGN);
+    DeviceInfo* di;
+    int rc = device_info(&di);
+    if (rc != MOE_OK) return rc;
+    return run_combine(y_perm, dest, w, y_shared, T, d, k, out, static_cast<cudaStream_t>(stream));
+}
+
+int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const moe_bf16* W1, const moe_bf16* W3,
+                      const moe_bf16* W2, const moe_bf16* W1s, const moe_bf16* W3s, const moe_bf16* W2s, int f_shared,
+                      int T, int d, int E, int k, int f, double capacity_factor, int cap_mode, moe_bf16* out, void* ws,
+                      size_t ws_bytes, moe_stream_t stream) {
+    return moe_layer_forward_ex(x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, f_shared, T, d, E, k, f, capacity_factor,
+                                cap_mode, out, ws, ws_bytes, stream, nullptr);
+}
+
+int moe_layer_forward_ex(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const moe_bf16* W1,
+                         const moe_bf16* W3, const moe_bf16* W2, const moe_bf16* W1s, const moe_bf16* W3s,
+                         const moe_bf16* W2s, int f_shared, int T, int d, int E, int k, int f, double capacity_factor,
+                         int cap_mode, moe_bf16* out, void* ws, size_t ws_bytes, moe_stream_t stream,
+                         const moe_stage_events* events) {
+    int rc = check_shape(T, d, E, k, f);
+    if (rc != MOE_OK) return rc;
+    MOE_REQUIRE(f_shared >= 0 && f_shared % 64 == 0, MOE_ERR_SHAPE);
+    MOE_REQUIRE(cap_mode >= MOE_CAP_NONE && cap_mode <= MOE_CAP_PER_ASSIGNMENT, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(x && Wg && W1 && W3 && W2 && out && ws, MOE_ERR_INVALID_ARG);
+    const bool shared = f_shared > 0;
+    MOE_REQUIRE(!shared || (W1s && W3s && W2s), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(x) && aligned16(Wg) && aligned16(bias) && aligned16(W1) && aligned16(W3) && aligned16(W2) &&
+                    aligned16(W1s) && aligned16(W3s) && aligned16(W2s) && aligned16(out) && aligned16(ws),
+                MOE_ERR_ALIGN);
+    const LayerLayout L = layer_layout(T, d, E, k, f, f_shared);
+    MOE_REQUIRE(ws_bytes >= L.total, MOE_ERR_WORKSPACE);
+    DeviceInfo* di;
+    if ((rc = device_info(&di)) != MOE_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* base = static_cast<char*>(ws);
+    float* logits = reinterpret_cast<float*>(base + L.off[0]);
+    int32_t* idx = reinterpret_cast<int32_t*>(base + L.off[1]);
+    float* w = reinterpret_cast<float*>(base + L.off[2]);
+    int32_t* counts_raw = reinterpret_cast<int32_t*>(base + L.off[3]);
+    int32_t* counts = reinterpret_cast<int32_t*>(base + L.off[4]);
+    int32_t* offsets = reinterpret_cast<int32_t*>(base + L.off[5]);
+    int32_t* dest = reinterpret_cast<int32_t*>(base + L.off[6]);
+    int32_t* src = reinterpret_cast<int32_t*>(base + L.off[7]);
+    moe_bf16* x_perm = reinterpret_cast<moe_bf16*>(base + L.off[8]);
+    moe_bf16* h = reinterpret_cast<moe_bf16*>(base + L.off[9]);
+    moe_bf16* y_perm = reinterpret_cast<moe_bf16*>(base + L.off[10]);
+    moe_bf16* y_shared = shared ? reinterpret_cast<moe_bf16*>(base + L.off[11]) : nullptr;
+    moe_bf16* h_shared = shared ? reinterpret_cast<moe_bf16*>(base + L.h_shared) : nullptr;
+    int32_t* blk_cnt = reinterpret_cast<int32_t*>(base + L.blk_cnt);
+    int32_t* rank_local = reinterpret_cast<int32_t*>(base + L.rank_local);
+    int32_t* mprefix = reinterpret_cast<int32_t*>(base + L.mprefix);
+
+    moe_stage_events ev;
+    memset(&ev, 0, sizeof(ev));
+    if (events) ev = *events;
+    auto mark = [&](void* e) { return e == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(e), s) == cudaSuccess; };
+
+    const long long C = moe_capacity(T, E, k, capacity_factor, cap_mode);
+    if (!mark(ev.route)) return MOE_ERR_CUDA;
+    if ((rc = run_router_gemm(di, x, Wg, T, d, E, logits, s)) != MOE_OK) return rc;
+    if (!mark(ev.topk)) return MOE_ERR_CUDA;
+    if ((rc = run_topk(logits, bias, T, E, k, idx, w, s)) != MOE_OK) return rc;
+    if (!mark(ev.permute)) return MOE_ERR_CUDA;
+    if ((rc = run_permute(di, x, idx, T, d, E, k, C, counts_raw, counts, offsets, dest, src, x_perm, blk_cnt,
+                          rank_local, mprefix, s)) != MOE_OK)
+        return rc;
+    if (!mark(ev.gate_up)) return MOE_ERR_CUDA;
+    FfnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x_perm = x_perm; a.offsets = offsets; a.mprefix = mprefix; a.max_rows = T * k; a.E = E; a.d = d; a.f = f;
+    a.W1 = W1; a.W3 = W3; a.W2 = W2; a.h = h; a.y_perm = y_perm;
+    a.x = x; a.T = T; a.f_shared = f_shared; a.W1s = W1s; a.W3s = W3s; a.W2s = W2s;
+    a.h_shared = h_shared; a.y_shared = y_shared;
+    if ((rc = run_expert_ffn(di, a, s, static_cast<cudaEvent_t>(ev.down))) != MOE_OK) return rc;
+    if (!mark(ev.combine)) return MOE_ERR_CUDA;
+    if ((rc = run_combine(y_perm, dest, w, y_shared, T, d, k, out, s)) != MOE_OK) return rc;
+    return mark(ev.end) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_get_error(moe_stream_t stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int v = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&v, g_moe_error, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_moe_error, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    return v;
+}
+
+const char* moe_strerror(int code) {
+    switch (code) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_SHAPE: return "unsupported shape";
+        case MOE_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case MOE_ERR_WORKSPACE: return "workspace too small";
+        case MOE_ERR_CUDA: return "CUDA runtime error";
+        case MOE_ERR_TIMEOUT: return "device wait timed out";
+        case MOE_ERR_CHECK: return "device check failed (non-finite score or bad offsets)";
+        case MOE_ERR_DEVICE: return "device is not sm_100";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

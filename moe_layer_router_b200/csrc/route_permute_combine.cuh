@@ -1,0 +1,372 @@
+// route_permute_combine.cuh - the HBM-/latency-bound stages of the layer.
+//
+//   topk_softmax_kernel   router top-k + renormalised softmax weights, one warp per token
+//                         ([EP-DS3] §2.1 steps 1-4)
+//   permute_count_kernel  per-block expert histogram + stable rank of every assignment
+//   permute_scan_kernel   grid-wide scan: block bases, counts, capacity, offsets, m-tile prefix
+//   permute_scatter_kernel  dest / src_token from the ranks ([EP-KV] §8, [EP-DS3] §3.1)
+//   gather_rows_kernel    x_perm[dest] = x[t], one warp per token, 16-byte vectors
+//   combine_kernel        out[t] = sum_j w * y_perm[dest] (+ y_shared), one warp per token
+//                         ([EP-KV] §2, §7)
+//   tile_prefix_kernel    m-tile prefix of the grouped GEMM from offsets (with checks)
+#pragma once
+
+#include "ptx.cuh"
+
+namespace moe {
+
+constexpr int PERMUTE_TOKENS = 256;   // tokens per block in the count / scatter kernels
+constexpr int PERMUTE_WARPS = PERMUTE_TOKENS / 32;
+constexpr int MAX_TOPK = 32;
+
+// ---------------------------------------------------------------- block scan (<= 1024 threads)
+
+// Exclusive scan of v over the block; returns the prefix, *total gets the block sum.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* total) {
+    __shared__ int warp_sums[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nwarps = (blockDim.x + 31) >> 5;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += n;
+    }
+    if (lane == 31) warp_sums[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        int s = lane < nwarps ? warp_sums[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += n;
+        }
+        warp_sums[lane] = s;   // inclusive over warps
+    }
+    __syncthreads();
+    const int before = warp ? warp_sums[warp - 1] : 0;
+    *total = warp_sums[nwarps - 1];
+    __syncthreads();
+    return before + inc - v;
+}
+
+// ---------------------------------------------------------------- router top-k
+
+// key order: larger key first, equal keys -> lower expert index
+__device__ __forceinline__ bool key_before(float ka, int ea, float kb, int eb) {
+    return ka > kb || (ka == kb && ea < eb);
+}
+
+// EPL = logits held per lane (E <= 32*EPL).  One warp per token.
+template <int EPL>
+__global__ void __launch_bounds__(256)
+topk_softmax_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k,
+                    int32_t* __restrict__ idx, float* __restrict__ w) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const float* row = logits + (size_t)t * E;
+    float L[EPL], key[EPL];
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) {
+            L[i] = __ldg(row + e);
+            key[i] = __fadd_rn(L[i], bias ? __ldg(bias + e) : 0.0f);   // fp32 add, no contraction
+            bad |= !isfinite(key[i]) || !isfinite(L[i]);
+        } else {
+            L[i] = 0.0f;
+            key[i] = -INFINITY;
+        }
+    }
+    if (__any_sync(0xffffffffu, bad)) {
+        if (lane == 0) record_error(-7 /* MOE_ERR_CHECK */);
+    }
+    uint32_t used = 0;                 // bit i: element i of this lane already selected
+    int my_e = 0;
+    float my_l = -INFINITY;            // lane j < k keeps slot j
+    for (int j = 0; j < k; ++j) {
+        float bk = -INFINITY, bl = 0.0f;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !((used >> i) & 1u) && key_before(key[i], e, bk, be)) {
+                bk = key[i];
+                be = e;
+                bl = L[i];
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            const float ol = __shfl_xor_sync(0xffffffffu, bl, o);
+            if (key_before(ok, oe, bk, be)) {
+                bk = ok;
+                be = oe;
+                bl = ol;
+            }
+        }
+        if (be < E && (be & 31) == lane) used |= 1u << (be >> 5);
+        if (lane == j) {
+            my_e = be < E ? be : 0;
+            my_l = bl;
+        }
+    }
+    // w_j = exp(L_j - m) / sum_sel exp(L_i - m), m = max selected logit: the softmax over
+    // all E renormalised over the selected k (the common factors cancel).
+    float m = lane < k ? my_l : -INFINITY;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float ex = lane < k ? expf(my_l - m) : 0.0f;
+    float s = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane < k) {
+        idx[(size_t)t * k + lane] = my_e;
+        w[(size_t)t * k + lane] = ex / s;
+    }
+}
+
+// ---------------------------------------------------------------- permutation
+
+// Block b owns tokens [256 b, 256 b + 256).  Writes blk_cnt[b, e] (assignments to e in the
+// block) and rank_local[t, j] = #{t' < t in the block : e = idx[t, j] is among idx[t', :]},
+// i.e. the stable (token-order) rank of (t, j) inside its block and expert.
+// Dynamic smem: (PERMUTE_WARPS * E + PERMUTE_TOKENS * k) ints.
+__global__ void __launch_bounds__(PERMUTE_TOKENS)
+permute_count_kernel(const int32_t* __restrict__ idx, int T, int E, int k, int32_t* __restrict__ blk_cnt,
+                     int32_t* __restrict__ rank_local) {
+    extern __shared__ int psm[];
+    int* wcnt = psm;                              // [PERMUTE_WARPS][E]
+    int* sidx = psm + PERMUTE_WARPS * E;          // [PERMUTE_TOKENS][k]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t0 = blockIdx.x * PERMUTE_TOKENS;
+    for (int i = threadIdx.x; i < PERMUTE_WARPS * E; i += blockDim.x) wcnt[i] = 0;
+    for (int i = threadIdx.x; i < PERMUTE_TOKENS * k; i += blockDim.x) {
+        const int t = t0 + i / k;
+        int e = t < T ? __ldg(idx + (size_t)t0 * k + i) : -1;
+        if (e >= E || e < -1) {
+            record_error(-7 /* MOE_ERR_CHECK */);
+            e = -1;
+        }
+        sidx[i] = e;
+    }
+    __syncthreads();
+    const int me = warp * 32 + lane;              // token index inside the block
+    const int t = t0 + me;
+    // rank inside the warp: lower lanes of this warp whose token routes to the same expert
+    for (int j = 0; j < k; ++j) {
+        const int e = sidx[me * k + j];
+        int r = 0;
+        for (int l = 0; l < 32; ++l) {
+            const int* other = sidx + (warp * 32 + l) * k;
+            int hit = 0;
+            for (int j2 = 0; j2 < k; ++j2) hit |= (other[j2] == e);
+            r += (l < lane) & hit;
+        }
+        if (e >= 0) {
+            atomicAdd(&wcnt[warp * E + e], 1);
+            rank_local[(size_t)t * k + j] = r;
+        }
+    }
+    __syncthreads();
+    // per expert: exclusive prefix over warps, block total
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = 0;
+        for (int w2 = 0; w2 < PERMUTE_WARPS; ++w2) {
+            const int c = wcnt[w2 * E + e];
+            wcnt[w2 * E + e] = run;
+            run += c;
+        }
+        blk_cnt[(size_t)blockIdx.x * E + e] = run;
+    }
+    __syncthreads();
+    if (t < T) {
+        for (int j = 0; j < k; ++j) {
+            const int e = sidx[me * k + j];
+            if (e >= 0) rank_local[(size_t)t * k + j] += wcnt[warp * E + e];
+        }
+    }
+}
+
+// One block of 1024 threads.  In place, blk_cnt[b, e] becomes the number of assignments to
+// e in blocks before b.  Then counts_raw, counts = min(raw, C), offsets = exclusive scan
+// of counts, and mprefix = exclusive scan of ceil(counts / 128) (the GEMM m-tiles).
+__global__ void __launch_bounds__(1024)
+permute_scan_kernel(int32_t* __restrict__ blk_cnt, int nb, int E, long long C, int32_t* __restrict__ counts_raw,
+                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ mprefix) {
+    __shared__ int part[1024];
+    __shared__ int tot[1024];
+    const int P = blockDim.x / E;                 // partitions of the block range per expert
+    const int tid = threadIdx.x;
+    const int e = tid % E, pi = tid / E;
+    const bool active = pi < P;
+    const int chunk = (nb + P - 1) / P;
+    const int b0 = pi * chunk, b1 = min(nb, b0 + chunk);
+    int s = 0;
+    if (active)
+        for (int b = b0; b < b1; ++b) s += blk_cnt[(size_t)b * E + e];
+    part[tid] = s;
+    __syncthreads();
+    if (active && pi == 0) {
+        int run = 0;
+        for (int q = 0; q < P; ++q) {
+            const int v = part[q * E + e];
+            part[q * E + e] = run;
+            run += v;
+        }
+        tot[e] = run;
+    }
+    __syncthreads();
+    if (active) {
+        int run = part[tid];
+        for (int b = b0; b < b1; ++b) {
+            const int c = blk_cnt[(size_t)b * E + e];
+            blk_cnt[(size_t)b * E + e] = run;
+            run += c;
+        }
+    }
+    const int raw = tid < E ? tot[tid] : 0;
+    const int kept = tid < E ? (C < 0 ? raw : (int)min((long long)raw, C)) : 0;
+    int total;
+    const int off = block_exclusive_scan(kept, &total);
+    const int mt = (kept + 127) / 128;
+    int mtotal;
+    const int moff = block_exclusive_scan(mt, &mtotal);
+    if (tid < E) {
+        counts_raw[tid] = raw;
+        counts[tid] = kept;
+        offsets[tid] = off;
+        mprefix[tid] = moff;
+    }
+    if (tid == 0) {
+        offsets[E] = total;
+        mprefix[E] = mtotal;
+    }
+}
+
+__global__ void __launch_bounds__(PERMUTE_TOKENS)
+permute_scatter_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ rank_local,
+                       const int32_t* __restrict__ blk_base, const int32_t* __restrict__ offsets, int T, int E,
+                       int k, long long C, int32_t* __restrict__ dest, int32_t* __restrict__ src_token) {
+    const int t = blockIdx.x * PERMUTE_TOKENS + threadIdx.x;
+    if (t >= T) return;
+    for (int j = 0; j < k; ++j) {
+        const int e = __ldg(idx + (size_t)t * k + j);
+        int d = -1;
+        if (e >= 0 && e < E) {
+            const long long r = (long long)__ldg(blk_base + (size_t)blockIdx.x * E + e) + __ldg(rank_local + (size_t)t * k + j);
+            if (C < 0 || r < C) {
+                d = __ldg(offsets + e) + (int)r;
+                src_token[d] = t;
+            }
+        }
+        dest[(size_t)t * k + j] = d;
+    }
+}
+
+// x_perm[dest[t, j]] = x[t]; one warp per token reads the row once and writes it k times.
+__global__ void __launch_bounds__(256)
+gather_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ dest, int T, int d, int k,
+                   uint4* __restrict__ x_perm) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const int nvec = d / 8;
+    const int dj = lane < k ? __ldg(dest + (size_t)t * k + lane) : -1;
+    const uint4* src = x + (size_t)t * nvec;
+    for (int base = 0; base < nvec; base += 32) {
+        const int c = base + lane;
+        const bool ok = c < nvec;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (ok) v = __ldg(src + c);
+        for (int j = 0; j < k; ++j) {
+            const int r = __shfl_sync(0xffffffffu, dj, j);
+            if (ok && r >= 0) x_perm[(size_t)r * nvec + c] = v;
+        }
+    }
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// out[t] = bf16( sum_{j=0..k-1, dest>=0} w[t,j] * y_perm[dest[t,j]] + y_shared[t] ), fp32 FMA in j order.
+__global__ void __launch_bounds__(256)
+combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ dest, const float* __restrict__ w,
+               const uint4* __restrict__ y_shared, int T, int d, int k, uint4* __restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const int nvec = d / 8;
+    const int dj = lane < k ? __ldg(dest + (size_t)t * k + lane) : -1;
+    const float wj = lane < k ? __ldg(w + (size_t)t * k + lane) : 0.0f;
+    for (int base = 0; base < nvec; base += 32) {
+        const int c = base + lane;
+        const bool ok = c < nvec;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const int r = __shfl_sync(0xffffffffu, dj, j);
+            const float wv = __shfl_sync(0xffffffffu, wj, j);
+            if (ok && r >= 0) {
+                float f[8];
+                bf16x8_to_f32(__ldg(y_perm + (size_t)r * nvec + c), f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(wv, f[i], acc[i]);
+            }
+        }
+        if (ok) {
+            if (y_shared) {
+                float f[8];
+                bf16x8_to_f32(__ldg(y_shared + (size_t)t * nvec + c), f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], f[i]);
+            }
+            out[(size_t)t * nvec + c] = make_uint4(f32x2_to_bf16x2(acc[0], acc[1]), f32x2_to_bf16x2(acc[2], acc[3]),
+                                                   f32x2_to_bf16x2(acc[4], acc[5]), f32x2_to_bf16x2(acc[6], acc[7]));
+        }
+    }
+}
+
+// mprefix = exclusive scan of ceil((offsets[e+1]-offsets[e]) / 128).  If offsets are not a
+// monotone sequence starting at 0 and ending <= max_rows, records MOE_ERR_CHECK and
+// writes an all-zero prefix (no GEMM tile runs).
+__global__ void __launch_bounds__(1024)
+tile_prefix_kernel(const int32_t* __restrict__ offsets, int E, int max_rows, int32_t* __restrict__ mprefix) {
+    __shared__ int bad;
+    const int e = threadIdx.x;
+    if (e == 0) bad = 0;
+    __syncthreads();
+    int mt = 0;
+    if (e < E) {
+        const int a = offsets[e], b = offsets[e + 1];
+        if (a < 0 || b < a || b > max_rows || (e == 0 && a != 0)) bad = 1;
+        mt = (b - a + 127) / 128;
+    }
+    __syncthreads();
+    if (bad) mt = 0;
+    int total;
+    const int moff = block_exclusive_scan(mt, &total);
+    if (e < E) mprefix[e] = moff;
+    if (e == 0) {
+        mprefix[E] = total;
+        if (bad) record_error(-7 /* MOE_ERR_CHECK */);
+    }
+}
+
+}  // namespace moe

@@ -232,3 +232,54 @@ class Inputs:
         if wl.bias_range <= 0:
             return None
         return uniform_f32(wl.seed, TID["bias"], 0, wl.E, -wl.bias_range, wl.bias_range)
+
+
+def device_tensors(wl: Workload, device, names=None, chunk_elems: int = 1 << 27) -> dict:
+    """Generate the workload's tensors on the host and copy them to `device` (torch).
+
+    Large expert tensors are produced in chunks of whole experts into pinned staging
+    buffers, so host memory stays bounded.  bf16 tensors come back as torch.bfloat16.
+    Keys: x, wg, w1, w3, w2, [w1s, w3s, w2s], [bias].
+    """
+    import torch
+
+    inp = Inputs(wl)
+    want = names or ["x", "wg", "w1", "w3", "w2", "w1s", "w3s", "w2s", "bias"]
+    out = {}
+
+    def to_dev_bf16(a: np.ndarray, shape):
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).reshape(shape)
+        return t.to(device)
+
+    if "x" in want:
+        out["x"] = to_dev_bf16(inp.x_rows(0, wl.T), (wl.T, wl.d))
+    if "wg" in want:
+        out["wg"] = to_dev_bf16(inp.wg().ravel(), (wl.E, wl.d))
+    per = wl.f * wl.d
+    ne = max(1, min(wl.E, chunk_elems // per))
+    stage = [torch.empty(ne * per, dtype=torch.int16).pin_memory() for _ in range(2)]
+    for name in ("w1", "w3", "w2"):
+        if name not in want:
+            continue
+        shape = (wl.E, wl.d, wl.f) if name == "w2" else (wl.E, wl.f, wl.d)
+        dst = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        flat = dst.view(-1).view(torch.int16)
+        i = 0
+        for e0 in range(0, wl.E, ne):
+            n = min(ne, wl.E - e0)
+            buf = stage[i & 1]
+            torch.cuda.current_stream(device).synchronize()   # buffer free again
+            inp.expert_rows(name, e0, n, out=buf.numpy()[: n * per].view(np.uint16))
+            flat[e0 * per:(e0 + n) * per].copy_(buf[: n * per], non_blocking=True)
+            i += 1
+        torch.cuda.current_stream(device).synchronize()
+        out[name] = dst
+    if wl.has_shared:
+        for name in ("w1s", "w3s", "w2s"):
+            if name in want:
+                a = inp.shared(name)
+                out[name] = to_dev_bf16(a.ravel(), a.shape)
+    if "bias" in want:
+        b = inp.bias()
+        out["bias"] = torch.from_numpy(b).to(device) if b is not None else None
+    return out

@@ -1,0 +1,90 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol the header declares,
+and its host-only logic (capacity, workspace sizes, argument validation) behaves."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+LIB = os.path.join(ROOT, "moe_layer_router_b200", "libmoe_b200.so")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        from moe_layer_router_b200.build import build
+        build()
+    return ctypes.CDLL(LIB)
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s+\**(moe_[a-z_0-9]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_layer_entry_points():
+    names = declared_functions()
+    for n in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward"):
+        assert n in names
+    assert len(names) >= 10
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert set(declared_functions()) <= exported
+
+
+def test_capacity_host(lib):
+    lib.moe_capacity.restype = ctypes.c_int64
+    lib.moe_capacity.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int]
+    assert lib.moe_capacity(32768, 64, 2, 1.25, 2) == 1280
+    assert lib.moe_capacity(32768, 64, 2, 1.25, 1) == 640
+    assert lib.moe_capacity(4096, 8, 2, 2.0, 1) == 1024
+    assert lib.moe_capacity(10, 3, 1, 0.9, 1) == 3
+    assert lib.moe_capacity(10, 3, 1, 0.9, 0) == -1
+    for T, E, k, cf in [(1000, 7, 3, 1.1), (999, 10, 1, 0.3), (16384, 128, 8, 1.0)]:
+        assert lib.moe_capacity(T, E, k, cf, 1) == int(T / E * cf)
+        assert lib.moe_capacity(T, E, k, cf, 2) == int(T * k / E * cf)
+
+
+def test_workspace_sizes_and_layout(lib):
+    sz = ctypes.c_size_t(0)
+    lib.moe_workspace_bytes.argtypes = [ctypes.c_int] * 6 + [ctypes.POINTER(ctypes.c_size_t)]
+    assert lib.moe_workspace_bytes(4096, 4096, 8, 2, 14336, 0, ctypes.byref(sz)) == 0
+    T, d, E, k, f = 4096, 4096, 8, 2, 14336
+    big = T * k * d * 2 * 2 + T * k * f * 2
+    assert big < sz.value < big * 1.05
+    off = (ctypes.c_size_t * 12)()
+    lib.moe_workspace_layout.argtypes = [ctypes.c_int] * 6 + [ctypes.c_size_t * 12]
+    assert lib.moe_workspace_layout(T, d, E, k, f, 0, off) == 0
+    offs = list(off)
+    assert all(o % 256 == 0 for o in offs)
+    assert offs[:11] == sorted(offs[:11]) and offs[10] + T * k * d * 2 <= sz.value
+    # shape checks: d % 64, k <= 32, k <= E, E <= 1024
+    for args in [(128, 100, 8, 2, 512), (128, 256, 8, 33, 512), (128, 256, 4, 8, 512), (128, 256, 2000, 2, 512),
+                 (0, 256, 8, 2, 512), (128, 256, 8, 2, 500)]:
+        assert lib.moe_workspace_bytes(*args, 0, ctypes.byref(sz)) == -2
+
+
+def test_entry_points_validate_before_touching_the_device(lib):
+    vp = ctypes.c_void_p
+    # a bad shape is rejected on the host, without a GPU
+    lib.moe_layer_forward.argtypes = [vp] * 9 + [ctypes.c_int] * 6 + [ctypes.c_double, ctypes.c_int, vp, vp,
+                                                                         ctypes.c_size_t, vp]
+    assert lib.moe_layer_forward(*([None] * 9), 0, 128, 100, 8, 2, 512, 1.0, 0, None, None, 0, None) == -2
+    assert lib.moe_layer_forward(*([None] * 9), 0, 128, 256, 8, 2, 512, 1.0, 0, None, None, 0, None) == -1
+    assert lib.moe_layer_forward(*([None] * 9), 0, 128, 256, 8, 2, 512, 1.0, 7, None, None, 0, None) == -1
+    lib.moe_combine.argtypes = [vp, vp, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp]
+    assert lib.moe_combine(None, None, None, None, 8, 64, 2, None, None) == -1
+    assert lib.moe_combine(16, 16, 16, None, 8, 65, 2, 16, None) == -2
+    assert lib.moe_combine(16, 16, 16, None, 8, 64, 2, 17, None) == -3     # misaligned out
+    lib.moe_strerror.restype = ctypes.c_char_p
+    assert lib.moe_strerror(-4) == b"workspace too small"

@@ -1,0 +1,255 @@
+"""GPU parity of each stage of the CUDA path against the CPU oracle (through the C ABI).
+
+Bars: routing indices, counts, offsets, dest, src_token and x_perm bit-exact given the
+same fp32 logits; routing weights rel 1e-5; logits within the fp32-accumulation bound of
+_util.logits_tol; h within 1e-3 + 8e-3|ref| (one bf16 ulp plus cancellation floor);
+expert outputs and layer outputs within 1e-2 + 2e-2|ref|.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from _util import assert_layer_close, bf16_bits, bits_to_f64, logits_tol, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def moe():
+    import moe_layer_router_b200 as m
+    assert torch.cuda.is_available()
+    return m
+
+
+def _logits(T, E, tid=100, scale=1.0):
+    return (synth.normal_f64(0, tid, 0, T * E) * scale).astype(np.float32).reshape(T, E)
+
+
+def _bf16(n_rows, n_cols, tid, std=1.0):
+    return synth.normal_bf16(0, tid, 0, n_rows * n_cols, std).reshape(n_rows, n_cols)
+
+
+def _ws(moe, T, d, E, k, f=64, f_shared=0):
+    return torch.empty(moe.moe_workspace_bytes(T, d, E, k, f, f_shared), dtype=torch.uint8, device="cuda")
+
+
+# ----------------------------------------------------------------------------- routing
+
+@pytest.mark.parametrize("T,E,k,with_bias", [(128, 8, 2, False), (1000, 8, 2, False), (777, 128, 8, False),
+                                             (256, 256, 8, True), (300, 64, 2, False), (100, 1024, 32, True),
+                                             (50, 5, 5, False), (33, 40, 1, True)])
+def test_route_on_supplied_logits_bit_exact(moe, T, E, k, with_bias):
+    logits = _logits(T, E)
+    bias = synth.uniform_f32(0, 101, 0, E, -0.1, 0.1) if with_bias else None
+    idx_o, w_o = oracle.route(logits, k, bias)
+    lg = torch.from_numpy(logits).cuda()
+    b = torch.from_numpy(bias).cuda() if bias is not None else None
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    moe.moe_route(None, None, b, lg, T, 64, E, k, None, idx, w, None)
+    assert moe.moe_get_error() == 0
+    assert np.array_equal(idx.cpu().numpy(), idx_o)
+    np.testing.assert_allclose(w.cpu().numpy(), w_o, rtol=1e-5, atol=1e-7)
+
+
+def test_route_ties_break_to_lower_expert(moe):
+    T, E, k = 512, 64, 8
+    logits = np.round(_logits(T, E, tid=103) * 1.5).astype(np.float32)   # many exact ties
+    logits[0] = 0.0
+    idx_o, w_o = oracle.route(logits, k)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    moe.moe_route(None, None, None, torch.from_numpy(logits).cuda(), T, 64, E, k, None, idx, w, None)
+    assert moe.moe_get_error() == 0
+    assert np.array_equal(idx.cpu().numpy(), idx_o)
+    assert list(idx_o[0]) == list(range(8))
+    np.testing.assert_allclose(w.cpu().numpy(), w_o, rtol=1e-5, atol=1e-7)
+
+
+def test_route_nonfinite_score_sets_check_error(moe):
+    T, E, k = 16, 8, 2
+    logits = _logits(T, E)
+    logits[3, 5] = np.nan
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    moe.moe_route(None, None, None, torch.from_numpy(logits).cuda(), T, 64, E, k, None, idx, w, None)
+    assert moe.moe_get_error() == moe.MOE_ERR_CHECK
+    assert moe.moe_get_error() == 0          # cleared by the read
+
+
+# ----------------------------------------------------------------------------- permutation
+
+@pytest.mark.parametrize("T,d,E,k,C", [(128, 256, 8, 2, -1), (1000, 128, 8, 2, 100), (777, 64, 128, 8, -1),
+                                       (777, 64, 128, 8, 40), (2000, 192, 64, 2, 0), (513, 64, 16, 4, 70),
+                                       (1, 64, 8, 2, -1), (300, 64, 1024, 32, 5), (4099, 128, 32, 3, 300)])
+def test_permute_bit_exact(moe, T, d, E, k, C):
+    idx, _ = oracle.route(_logits(T, E, tid=104), k)
+    x = _bf16(T, d, 105)
+    r = oracle.dispatch(idx, E, C)
+    xp = oracle.gather(x, r["dest"], r["N"])
+    dev = lambda a: torch.from_numpy(a).cuda()
+    craw = torch.full((E,), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.full((E,), -7, dtype=torch.int32, device="cuda")
+    off = torch.full((E + 1,), -7, dtype=torch.int32, device="cuda")
+    dest = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
+    src = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
+    x_perm = torch.zeros((T * k, d), dtype=torch.bfloat16, device="cuda")
+    ws = _ws(moe, T, d, E, k)
+    moe.moe_permute(to_dev_bf16(x), dev(idx), T, d, E, k, C, craw, cnt, off, dest, src, x_perm, ws)
+    assert moe.moe_get_error() == 0
+    N = r["N"]
+    assert np.array_equal(craw.cpu().numpy(), r["counts_raw"])
+    assert np.array_equal(cnt.cpu().numpy(), r["counts"])
+    assert np.array_equal(off.cpu().numpy(), r["offsets"])
+    assert np.array_equal(dest.cpu().numpy(), r["dest"])
+    assert np.array_equal(src.cpu().numpy()[:N], r["src_token"])
+    assert np.array_equal(bf16_bits(x_perm)[:N], xp)
+
+
+# ----------------------------------------------------------------------------- combine
+
+@pytest.mark.parametrize("with_shared", [False, True])
+def test_combine(moe, with_shared):
+    T, d, E, k, C = 300, 256, 16, 4, 50
+    idx, w = oracle.route(_logits(T, E, tid=106), k)
+    r = oracle.dispatch(idx, E, C)
+    y_perm = _bf16(T * k, d, 107)
+    ysh = _bf16(T, d, 108) if with_shared else None
+    ref = oracle.combine(y_perm[: max(r["N"], 1)], r["dest"], w, ysh)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine(to_dev_bf16(y_perm), torch.from_numpy(r["dest"]).cuda(), torch.from_numpy(w).cuda(),
+                    to_dev_bf16(ysh) if ysh is not None else None, T, d, k, out)
+    assert moe.moe_get_error() == 0
+    got = bf16_bits(out)
+    assert_layer_close(got, ref)
+    assert np.mean(got == ref) > 0.99
+    assert (r["dest"] < 0).any()                  # drops exercised
+
+
+# ----------------------------------------------------------------------------- router GEMM
+
+@pytest.mark.parametrize("T,d,E", [(128, 256, 8), (300, 512, 128), (129, 1024, 256), (200, 256, 300), (64, 7168, 256),
+                                   (1000, 4096, 64), (17, 64, 40), (130, 128, 1024)])
+def test_router_gemm(moe, T, d, E):
+    k = min(2, E)
+    x = _bf16(T, d, 109)
+    wg = _bf16(E, d, 110, std=d ** -0.5)
+    logits = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    moe.moe_route(to_dev_bf16(x), to_dev_bf16(wg), None, None, T, d, E, k, logits, idx, w, _ws(moe, T, d, E, k))
+    assert moe.moe_get_error() == 0
+    g = logits.cpu().numpy()
+    ref = oracle.router_logits(x, wg)
+    tol = logits_tol(x, wg)
+    assert np.all(np.abs(g.astype(np.float64) - ref) <= tol), float(np.max(np.abs(g - ref) / tol))
+    i2, w2 = oracle.route(g, k)
+    assert np.array_equal(idx.cpu().numpy(), i2)
+    np.testing.assert_allclose(w.cpu().numpy(), w2, rtol=1e-5, atol=1e-7)
+
+
+# ----------------------------------------------------------------------------- expert FFN
+
+@pytest.mark.parametrize("counts,d,f", [([0, 1, 127, 128, 129, 300, 5, 0], 256, 512), ([200, 200, 200], 128, 320),
+                                        ([1], 64, 64), ([0, 0, 0], 128, 128), ([17, 260, 3, 64], 448, 192),
+                                        ([513, 1, 700], 1024, 1536)])
+def test_expert_ffn(moe, counts, d, f):
+    E = len(counts)
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    N = int(off[-1])
+    max_rows = N + 37
+    x_perm = _bf16(max_rows, d, 111)
+    W1 = _bf16(E * f, d, 112, d ** -0.5).reshape(E, f, d)
+    W3 = _bf16(E * f, d, 113, d ** -0.5).reshape(E, f, d)
+    W2 = _bf16(E * d, f, 114, f ** -0.5).reshape(E, d, f)
+    h = torch.full((max_rows, f), 7.0, dtype=torch.bfloat16, device="cuda")
+    y = torch.full((max_rows, d), 7.0, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(4096 * 4, dtype=torch.uint8, device="cuda")
+    moe.moe_expert_ffn(to_dev_bf16(x_perm), torch.from_numpy(off).cuda(), max_rows, E, d, f, to_dev_bf16(W1),
+                       to_dev_bf16(W3), to_dev_bf16(W2), h, y, ws)
+    assert moe.moe_get_error() == 0
+    hg, yg = bf16_bits(h), bf16_bits(y)
+    for e in range(E):
+        a, b = off[e], off[e + 1]
+        if a == b:
+            continue
+        ho, yo = oracle.expert_ffn(x_perm[a:b], W1[e], W3[e], W2[e])
+        dh = np.abs(bits_to_f64(hg[a:b]) - bits_to_f64(ho))
+        assert np.all(dh <= 1e-3 + 8e-3 * np.abs(bits_to_f64(ho))), f"h of expert {e}"
+        assert_layer_close(yg[a:b], yo, f"y of expert {e}")
+        assert np.mean(yg[a:b] == yo) > 0.9
+    # rows past the last group are never written (tiles straddling a group edge are masked)
+    assert np.all(bits_to_f64(hg[N:]) == 7.0) and np.all(bits_to_f64(yg[N:]) == 7.0)
+
+
+def test_expert_ffn_rejects_bad_offsets(moe):
+    E, d, f, max_rows = 4, 64, 64, 100
+    off = np.array([0, 10, 5, 20, 30], np.int32)          # not monotone
+    z = lambda *s: torch.zeros(s, dtype=torch.bfloat16, device="cuda")
+    y = torch.full((max_rows, d), 3.0, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(4096, dtype=torch.uint8, device="cuda")
+    moe.moe_expert_ffn(z(max_rows, d), torch.from_numpy(off).cuda(), max_rows, E, d, f, z(E, f, d), z(E, f, d),
+                       z(E, d, f), z(max_rows, f), y, ws)
+    assert moe.moe_get_error() == moe.MOE_ERR_CHECK
+    assert torch.all(y == 3.0)                             # no tile ran
+
+
+# ----------------------------------------------------------------------------- whole layer, small
+
+SMALL = [
+    dict(name="tiny", wl=synth.WORKLOADS["tiny"]),
+    dict(name="all-options", wl=synth.Workload("all", 300, 256, 16, 4, 320, f_shared=192, bias_range=0.1,
+                                               cap_mode=synth.CAP_PER_TOKEN, capacity_factor=1.25)),
+    dict(name="per-assignment-cap", wl=synth.Workload("cap", 513, 128, 8, 2, 128, cap_mode=synth.CAP_PER_ASSIGNMENT,
+                                                      capacity_factor=0.8)),
+    dict(name="single-expert", wl=synth.Workload("one", 200, 128, 1, 1, 256)),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c["name"] for c in SMALL])
+def test_layer_small_all_intermediates(moe, case):
+    wl = case["wl"]
+    inp = synth.Inputs(wl)
+    x, wg, W1, W3, W2 = inp.x(), inp.wg(), inp.w1(), inp.w3(), inp.w2()
+    bias = inp.bias()
+    W1s, W3s, W2s = inp.shared("w1s"), inp.shared("w3s"), inp.shared("w2s")
+    T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
+    C = oracle.capacity(T, E, k, wl.capacity_factor, wl.cap_mode)
+    assert moe.moe_capacity(T, E, k, wl.capacity_factor, wl.cap_mode) == C
+    dv = lambda a: to_dev_bf16(a) if a is not None else None
+    ws = _ws(moe, T, d, E, k, f, fs)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_layer_forward(dv(x), dv(wg), torch.from_numpy(bias).cuda() if bias is not None else None, dv(W1), dv(W3),
+                          dv(W2), dv(W1s), dv(W3s), dv(W2s), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, out, ws)
+    assert moe.moe_get_error() == 0
+    L = moe.moe_workspace_layout(T, d, E, k, f, fs)
+    v = lambda n, s, dt: moe.workspace_view(ws, L, n, s, dt).cpu()
+    g_logits = v("logits", (T, E), torch.float32).numpy()
+    # (i) logits
+    ref_logits = oracle.router_logits(x, wg)
+    assert np.all(np.abs(g_logits.astype(np.float64) - ref_logits) <= logits_tol(x, wg))
+    # (ii) routing from the GPU's logits: bit-exact; everything downstream fed the same logits
+    ref = oracle.layer_forward(x, wg, W1, W3, W2, k=k, C=C, bias=bias, logits_in=g_logits, W1s=W1s, W3s=W3s, W2s=W2s)
+    assert np.array_equal(v("idx", (T, k), torch.int32).numpy(), ref["idx"])
+    np.testing.assert_allclose(v("w", (T, k), torch.float32).numpy(), ref["w"], rtol=1e-5, atol=1e-7)
+    for n in ("counts_raw", "counts"):
+        assert np.array_equal(v(n, (E,), torch.int32).numpy(), ref[n])
+    assert np.array_equal(v("offsets", (E + 1,), torch.int32).numpy(), ref["offsets"])
+    assert np.array_equal(v("dest", (T, k), torch.int32).numpy(), ref["dest"])
+    N = ref["N"]
+    assert np.array_equal(v("src_token", (T * k,), torch.int32).numpy()[:N], ref["src_token"])
+    xp = bf16_bits(v("x_perm", (T * k, d), torch.bfloat16))[:N]
+    assert np.array_equal(xp, oracle.gather(x, ref["dest"], N))
+    # (iii) routing from the oracle's own logits, on tokens without a near tie at the k-th key
+    own_idx, _ = oracle.route(ref_logits.astype(np.float32), k, bias)
+    keys = np.sort(ref_logits + (bias if bias is not None else 0), axis=1)[:, ::-1]
+    clear = (keys[:, k - 1] - keys[:, k]) >= 1e-5 if k < E else np.ones(T, bool)
+    assert np.array_equal(own_idx[clear], ref["idx"][clear])
+    # (iv) outputs
+    got = bf16_bits(out)
+    assert_layer_close(got, ref["out"])
+    assert np.mean(got == ref["out"]) > 0.9
+    if fs:
+        assert_layer_close(bf16_bits(v("y_shared", (T, d), torch.bfloat16)), ref["y_shared"], "y_shared")
