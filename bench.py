@@ -270,6 +270,9 @@ def main():
 
     K = args.steps
     evs = [{n: torch.cuda.Event(enable_timing=True) for n in moe.STAGES} for _ in range(K)]
+    for e in evs:               # torch creates the CUDA event on its first record
+        for ev in e.values():
+            ev.record()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()

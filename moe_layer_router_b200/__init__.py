@@ -45,7 +45,7 @@ class MoeError(RuntimeError):
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with __graft_entry__.build() "
-                      "(python -m moe_layer_router_b200.build)")
+                      "(python moe_layer_router_b200/build.py)")
 
 _lib = ctypes.CDLL(LIB_PATH)
 _vp, _i32, _i64, _dbl, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double, ctypes.c_size_t

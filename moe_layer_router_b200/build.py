@@ -1,6 +1,7 @@
 """Build libmoe_b200.so (sm_100a) in-tree with nvcc.
 
-    python -m moe_layer_router_b200.build        # or: from moe_layer_router_b200.build import build
+    python moe_layer_router_b200/build.py [--force] [--ptxas-v]
+    (run by path: importing the package itself needs the built library)
 
 The library is one translation unit (csrc/moe_api.cu) that includes the kernels.
 """

@@ -15,8 +15,8 @@ LIB = os.path.join(ROOT, "moe_layer_router_b200", "libmoe_b200.so")
 @pytest.fixture(scope="module")
 def lib():
     if not os.path.exists(LIB):
-        from moe_layer_router_b200.build import build
-        build()
+        import __graft_entry__
+        __graft_entry__.build()
     return ctypes.CDLL(LIB)
 
 
