@@ -111,6 +111,26 @@ int moe_permute(const moe_bf16* x, const int32_t* idx, int T, int d, int E, int 
                 moe_bf16* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_permute() for callers that cannot allocate device memory.  No counterpart on the
+ * pages: it exists because some callers have no way to allocate at the point of the call
+ * (a plugin inside a framework that owns all device memory, an engine whose memory plan
+ * is fixed at start-up, a program that must not call cudaMalloc, which can synchronise
+ * the device).  Same arguments and results as moe_permute() minus the workspace: the
+ * scratch lives in a fixed array of MOE_NOALLOC_SCRATCH_BYTES compiled into the library,
+ * which every GPU that loads the library holds until exit.
+ *   - Sizes whose scratch, ceil(T/256)*E*4 + T*k*4 + (E+1)*4 bytes (each part rounded up
+ *     to 256), exceeds MOE_NOALLOC_SCRATCH_BYTES return MOE_ERR_WORKSPACE; nothing runs.
+ *   - The first call on a device, with that device current, looks up the array's device
+ *     address (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Calls on one device share the array: calls whose kernels overlap on the GPU race.
+ *   - Allocates and frees nothing.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES (4u << 20)
+int moe_permute_noalloc(const moe_bf16* x, const int32_t* idx, int T, int d, int E, int k, int64_t capacity,
+                        int32_t* counts_raw, int32_t* counts, int32_t* offsets, int32_t* dest,
+                        int32_t* src_token, moe_bf16* x_perm, moe_stream_t stream);
+
+/*
  * Experts ([EP-KV] §1 and §8): for every expert e, on rows [offsets[e], offsets[e+1]) of x_perm,
  *   h = bf16( silu(x_perm W1_e^T) * (x_perm W3_e^T) ),  y_perm = bf16( h W2_e^T ),
  * two grouped GEMMs on the tcgen05 tensor cores (fp32 accumulate in tensor memory),

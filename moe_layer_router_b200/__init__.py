@@ -56,6 +56,8 @@ _lib.moe_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32, ctypes.
 _lib.moe_workspace_layout.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(_sz)]
 _lib.moe_route.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.moe_permute.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.moe_permute_noalloc.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.moe_permute_noalloc.restype = _i32
 _lib.moe_expert_ffn.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.moe_combine.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp]
 _lib.moe_layer_forward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
@@ -132,6 +134,18 @@ def moe_permute(x, idx, T, d, E, k, capacity, counts_raw, counts, offsets, dest,
     _check(_lib.moe_permute(_ptr(x), _ptr(idx), T, d, E, k, int(capacity), _ptr(counts_raw), _ptr(counts),
                             _ptr(offsets), _ptr(dest), _ptr(src_token), _ptr(x_perm), _ptr(ws), _nbytes(ws),
                             _stream(stream)), "moe_permute")
+
+
+MOE_NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def moe_permute_noalloc(x, idx, T, d, E, k, capacity, counts_raw, counts, offsets, dest, src_token, x_perm,
+                        stream=None) -> None:
+    """moe_permute without a workspace, for callers that cannot allocate device memory: the
+    scratch is a fixed 4 MiB array inside the library (shared by all calls on a device)."""
+    _check(_lib.moe_permute_noalloc(_ptr(x), _ptr(idx), T, d, E, k, int(capacity), _ptr(counts_raw), _ptr(counts),
+                                    _ptr(offsets), _ptr(dest), _ptr(src_token), _ptr(x_perm), _stream(stream)),
+           "moe_permute_noalloc")
 
 
 def moe_expert_ffn(x_perm, offsets, max_rows, E, d, f, W1, W3, W2, h, y_perm, ws, stream=None) -> None:

@@ -544,3 +544,6 @@ const char* moe_strerror(int code) {
 }
 
 }  // extern "C"
+
+// The no-allocation variant of moe_permute shares this translation unit.
+#include "moe_noalloc.cu"
