@@ -41,6 +41,8 @@ DESCR = {
     "qwen3": "Qwen3-235B-A22B-like prefill T=16384 d=4096 E=128 top-8 f=1536",
     "dsv3": "DeepSeek-V3-like decode T=256 d=7168 E=256 top-8 f=2048 + shared f=2048, selection bias",
     "skew": "skewed routing T=32768 d=4096 E=64 top-2 f=2048 Zipf(1.2), capacity int(T*k/E*1.25)",
+    "mixtral2e": "profiling case: Mixtral-like layer cut to T=2048, E=2 (same tile shapes)",
+    "dsv3_32e": "profiling case: DeepSeek-V3-like decode cut to T=32, E=32 (same tile shapes)",
 }
 
 
@@ -336,7 +338,7 @@ def main():
 
     peaks, peak_src = load_peaks()
     g1_ms = stage_ms["gate_up"]
-    decode = wl.name == "dsv3"
+    decode = wl.name.startswith("dsv3")
     if decode:
         alg = gemm1_bytes(wl, N, touched)
         achieved = alg / (g1_ms / 1000.0) / 1e9

@@ -1,0 +1,299 @@
+// grouped_gemm_pair.cuh - the grouped GEMM on CTA pairs (tcgen05 cta_group::2), for the
+// expert FFN when experts hold many rows (prefill).
+//
+// Same products, group classes, tile walk and epilogues as grouped_gemm.cuh, but a tile is
+// 256 rows x 256 columns computed by a cluster of two CTAs on two SMs:
+//   - CTA r (r = 0, 1) loads rows [128 r, 128 r + 128) of the A tile and its half of the B
+//     tile into its own shared memory (no multicast): for GEMM1 CTA 0 loads the W1 rows and
+//     CTA 1 the same rows of W3; for GEMM2 CTA r loads W2 rows [n0 + 128 r, n0 + 128 r + 128).
+//   - both CTAs' copies complete on the leader's (CTA 0) full barrier; one thread of the leader
+//     issues tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16), which reads both CTAs'
+//     halves and accumulates rows [128 r, 128 r + 128) into CTA r's tensor memory.
+//   - the leader's commits arrive on both CTAs' barriers (empty stage, accumulator full);
+//     every epilogue warp of both CTAs arrives on the leader's accumulator-empty barrier.
+// Per SM this halves the B operand traffic of a 1-SM M = 128 tile and leaves room for a
+// 6-stage ring (A 16 KB + B 16 KB per stage per CTA).
+#pragma once
+
+#include "grouped_gemm.cuh"
+
+namespace moe {
+
+constexpr int PAIR_BM = 256;                 // rows per pair tile
+constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_A_BYTES = 128 * GEMM_BK * 2;   // 16 KB per CTA
+constexpr int PAIR_B_BYTES = 128 * GEMM_BK * 2;   // 16 KB per CTA
+constexpr int PAIR_SMEM_BYTES = PAIR_STAGES * (PAIR_A_BYTES + PAIR_B_BYTES) + 1024 + 256;
+
+// Tile walk with 256-row m-tiles (mprefix counts 256-row tiles per group).
+__device__ __forceinline__ int pair_total_tiles(const GemmParams& p, int& routed_tiles) {
+    routed_tiles = p.offsets ? __ldg(p.mprefix + p.E) * p.cls[0].ntiles : 0;
+    const int dense = p.dense_rows ? ((p.dense_rows + PAIR_BM - 1) / PAIR_BM) * p.cls[1].ntiles : 0;
+    return routed_tiles + dense;
+}
+
+struct PairTile {
+    int cls;
+    int a_row;   // first A row of the pair tile
+    int rows;    // valid rows of the pair tile (<= 256)
+    int group;
+    int n_idx;
+};
+
+__device__ __forceinline__ PairTile pair_decode_tile(const GemmParams& p, int t, int routed_tiles) {
+    PairTile ti;
+    if (t < routed_tiles) {
+        const GemmClass& c = p.cls[0];
+        const int q = t / c.ntiles;
+        int lo = 0, hi = p.E;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(p.mprefix + mid) <= q) lo = mid; else hi = mid;
+        }
+        const int g = lo;
+        const int mp = __ldg(p.mprefix + g);
+        const int mt = __ldg(p.mprefix + g + 1) - mp;
+        const int local = t - mp * c.ntiles;
+        const int m = local % mt, n = local / mt;
+        const int r0 = __ldg(p.offsets + g) + m * PAIR_BM;
+        ti.cls = 0;
+        ti.group = g;
+        ti.a_row = r0;
+        ti.rows = min(PAIR_BM, __ldg(p.offsets + g + 1) - r0);
+        ti.n_idx = n;
+    } else {
+        const GemmClass& c = p.cls[1];
+        const int mt = (p.dense_rows + PAIR_BM - 1) / PAIR_BM;
+        const int local = t - routed_tiles;
+        const int m = local % mt, n = local / mt;
+        ti.cls = 1;
+        ti.group = 0;
+        ti.a_row = m * PAIR_BM;
+        ti.rows = min(PAIR_BM, p.dense_rows - ti.a_row);
+        ti.n_idx = n;
+        (void)c;
+    }
+    return ti;
+}
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
+grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                         const __grid_constant__ CUtensorMap tmB0b, const __grid_constant__ CUtensorMap tmA1,
+                         const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB1b,
+                         const __grid_constant__ GemmParams p) {
+    static_assert(EPI == EPI_SWIGLU || EPI == EPI_STORE, "pair tiles serve the expert GEMMs");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + PAIR_STAGES * PAIR_A_BYTES;
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sB + PAIR_STAGES * PAIR_B_BYTES);
+    uint64_t* empty_bar = full_bar + PAIR_STAGES;
+    uint64_t* tfull_bar = empty_bar + PAIR_STAGES;
+    uint64_t* tempty_bar = tfull_bar + 2;
+    uint64_t* drain_bar = tempty_bar + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();          // 0 = leader, 1 = peer
+    const bool leader = rank == 0;
+    const int pair_id = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < PAIR_STAGES; ++s) {
+            mbar_init(full_bar + s, 1);      // leader: its producer's expect_tx; bytes of both CTAs
+            mbar_init(empty_bar + s, 1);     // one multicast commit from the leader's MMA thread
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar + a, 1);     // one multicast commit
+            mbar_init(tempty_bar + a, 256);  // leader: 128 epilogue threads x 2 CTAs
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmA0);
+        prefetch_tensormap(&tmB0);
+        prefetch_tensormap(&tmB0b);
+        prefetch_tensormap(&tmA1);
+        prefetch_tensormap(&tmB1);
+        prefetch_tensormap(&tmB1b);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, GEMM_TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();          // both CTAs' barriers initialised before any remote use
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    int routed_tiles;
+    const int total = pair_total_tiles(p, routed_tiles);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            const uint64_t pol_a = policy_evict_last();
+            const uint64_t pol_b = policy_evict_normal();
+            const uint32_t full_leader0 = map_to_cta(full_bar, 0);
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int t = pair_id; t < total && ok; t += npairs) {
+                const PairTile ti = pair_decode_tile(p, t, routed_tiles);
+                const GemmClass& c = p.cls[ti.cls];
+                const CUtensorMap* mA = ti.cls ? &tmA1 : &tmA0;
+                const CUtensorMap* mB;
+                int b_row;
+                if (EPI == EPI_SWIGLU) {       // CTA 0: W1 rows (gate), CTA 1: the same rows of W3 (up)
+                    mB = ti.cls ? (leader ? &tmB1 : &tmB1b) : (leader ? &tmB0 : &tmB0b);
+                    b_row = ti.group * c.b_group_rows + ti.n_idx * 128;
+                } else {                       // CTA r: rows [n0 + 128 r, n0 + 128 r + 128) of W2
+                    mB = ti.cls ? &tmB1 : &tmB0;
+                    b_row = ti.group * c.b_group_rows + ti.n_idx * 256 + (int)rank * 128;
+                }
+                const int a_row = ti.a_row + (int)rank * 128;
+                const int nk = c.K / GEMM_BK;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(empty_bar + stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+                    const uint32_t fb = full_leader0 + (uint32_t)stage * 8u;
+                    if (leader) mbar_arrive_expect_tx(full_bar + stage, 2u * (PAIR_A_BYTES + PAIR_B_BYTES));
+                    tma_load_2d_pair(sA + stage * PAIR_A_BYTES, mA, fb, kb * GEMM_BK, a_row, pol_a);
+                    tma_load_2d_pair(sB + stage * PAIR_B_BYTES, mB, fb, kb * GEMM_BK, b_row, pol_b);
+                    ++issued;
+                    if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok && leader) {
+                // the leader's full barriers count both CTAs' copies; let those in flight land
+                const int n = issued < PAIR_STAGES ? issued : PAIR_STAGES;
+                for (int i = 1; i <= n; ++i) {
+                    const int q = issued - i;
+                    mbar_wait(full_bar + (q % PAIR_STAGES), (uint32_t)((q / PAIR_STAGES) & 1), nullptr);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer (leader only)
+        if (lane == 0 && leader) {
+            const uint32_t idesc = idesc_bf16_f32(PAIR_BM, 256);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool any = false, ok = true;
+            for (int t = pair_id; t < total && ok; t += npairs) {
+                const PairTile ti = pair_decode_tile(p, t, routed_tiles);
+                const GemmClass& c = p.cls[ti.cls];
+                const int nk = c.K / GEMM_BK;
+                if (!mbar_wait(tempty_bar + acc, acc_phase ^ 1u, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * GEMM_ACC_COLS);
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(full_bar + stage, phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t ad = smem_desc_k_sw128(sA + stage * PAIR_A_BYTES);
+                    const uint64_t bd = smem_desc_k_sw128(sB + stage * PAIR_B_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < GEMM_BK / 16; ++kk)
+                        umma_bf16_pair(d_tmem, ad + 2ull * kk, bd + 2ull * kk, idesc, (kb | kk) != 0);
+                    umma_commit_pair(empty_bar + stage, 0x3);
+                    any = true;
+                    if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                umma_commit_pair(tfull_bar + acc, 0x3);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+            }
+            if (any) {
+                umma_commit_pair(drain_bar, 0x1);
+                mbar_wait(drain_bar, 0, nullptr);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------------ epilogue (both CTAs)
+        const int sub = warp & 3;
+        const int row_in_cta = sub * 32 + lane;
+        const uint32_t tempty_leader0 = map_to_cta(tempty_bar, 0);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = pair_id; t < total; t += npairs) {
+            const PairTile ti = pair_decode_tile(p, t, routed_tiles);
+            const GemmClass& c = p.cls[ti.cls];
+            const bool ready = mbar_wait(tfull_bar + acc, acc_phase, abort_flag);
+            if (!__all_sync(0xffffffffu, ready)) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + (uint32_t)(acc * GEMM_ACC_COLS) + ((uint32_t)(sub * 32) << 16);
+            const int row_in_tile = (int)rank * 128 + row_in_cta;
+            const long long orow = c.out_row0 + ti.a_row + row_in_tile;
+            const bool row_ok = row_in_tile < ti.rows && orow >= 0 && orow < c.out_rows;
+            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(c.out) + orow * c.ldo;
+            if (EPI == EPI_SWIGLU) {
+#pragma unroll 1
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t g[32], u[32];
+                    __syncwarp();
+                    tmem_ld_32cols(tbase + ch * 32, g);
+                    tmem_ld_32cols(tbase + 128 + ch * 32, u);
+                    tmem_ld_wait();
+                    const int col0 = ti.n_idx * 128 + ch * 32;
+                    if (row_ok && col0 < c.n_out) {
+                        uint32_t packed[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+                            const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+                            const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+                            const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+                            packed[i] = pack_bf16x2(h0, h1);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(out + col0);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t v[32];
+                    __syncwarp();
+                    tmem_ld_32cols(tbase + ch * 32, v);
+                    tmem_ld_wait();
+                    const int col0 = ti.n_idx * 256 + ch * 32;
+                    if (row_ok && col0 < c.n_out) {
+                        uint32_t packed[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                        uint4* dst = reinterpret_cast<uint4*>(out + col0);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive_cluster(tempty_leader0 + (uint32_t)acc * 8u);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    __syncthreads();
+    cluster_sync_all();          // the leader's MMAs have drained; no remote arrivals remain
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, GEMM_TMEM_COLS);
+    }
+}
+
+}  // namespace moe

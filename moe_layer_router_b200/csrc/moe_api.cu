@@ -8,6 +8,7 @@
 
 #include "../../include/moe.h"
 #include "grouped_gemm.cuh"
+#include "grouped_gemm_pair.cuh"
 #include "route_permute_combine.cuh"
 
 namespace moe {
@@ -103,6 +104,32 @@ int launch_gemm(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b0, co
     grouped_gemm_kernel<EPI><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, s>>>(a0, b0, b0b, a1, b1, b1b, p);
     return launch_status();
 }
+
+template <int EPI>
+int launch_gemm_pair(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& b0b,
+                     const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& b1b, const GemmParams& p,
+                     long long tiles_upper, cudaStream_t s) {
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        static bool attr_set[kMaxDevices][3] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (!attr_set[dev][EPI]) {
+            if (cudaFuncSetAttribute(grouped_gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     PAIR_SMEM_BYTES) != cudaSuccess)
+                return MOE_ERR_CUDA;
+            attr_set[dev][EPI] = true;
+        }
+    }
+    if (tiles_upper <= 0) return MOE_OK;
+    const long long pairs = di->sms / 2;
+    const int grid = 2 * (int)(tiles_upper < pairs ? tiles_upper : pairs);
+    grouped_gemm_pair_kernel<EPI><<<grid, GEMM_THREADS, PAIR_SMEM_BYTES, s>>>(a0, b0, b0b, a1, b1, b1b, p);
+    return launch_status();
+}
+
+// Pair (2-SM) tiles pay off when experts average at least one full 256-row tile.
+bool use_pair_tiles(long long rows, int E) { return rows >= 256ll * E; }
 
 // ------------------------------------------------------------------ workspace layouts
 
@@ -200,7 +227,8 @@ int run_topk(const float* logits, const float* bias, int T, int E, int k, int32_
 
 int run_permute(DeviceInfo* di, const moe_bf16* x, const int32_t* idx, int T, int d, int E, int k, long long C,
                 int32_t* counts_raw, int32_t* counts, int32_t* offsets, int32_t* dest, int32_t* src_token,
-                moe_bf16* x_perm, int32_t* blk_cnt, int32_t* rank_local, int32_t* mprefix, cudaStream_t s) {
+                moe_bf16* x_perm, int32_t* blk_cnt, int32_t* rank_local, int32_t* mprefix, cudaStream_t s,
+                int tile_rows = GEMM_BM) {
     const int nb = permute_blocks(T);
     const size_t smem = (size_t)(PERMUTE_WARPS * E + PERMUTE_TOKENS * k) * sizeof(int);
     {
@@ -214,7 +242,7 @@ int run_permute(DeviceInfo* di, const moe_bf16* x, const int32_t* idx, int T, in
         }
     }
     permute_count_kernel<<<nb, PERMUTE_TOKENS, smem, s>>>(idx, T, E, k, blk_cnt, rank_local);
-    permute_scan_kernel<<<1, 1024, 0, s>>>(blk_cnt, nb, E, C, counts_raw, counts, offsets, mprefix);
+    permute_scan_kernel<<<1, 1024, 0, s>>>(blk_cnt, nb, E, C, counts_raw, counts, offsets, mprefix, tile_rows);
     permute_scatter_kernel<<<nb, PERMUTE_TOKENS, 0, s>>>(idx, rank_local, blk_cnt, offsets, T, E, k, C, dest,
                                                           src_token);
     gather_rows_kernel<<<(T + 7) / 8, 256, 0, s>>>(reinterpret_cast<const uint4*>(x), dest, T, d, k,
@@ -236,6 +264,7 @@ struct FfnArgs {
     int T, f_shared;
     const moe_bf16 *W1s, *W3s, *W2s;
     moe_bf16 *h_shared, *y_shared;
+    bool pair;   // 2-SM tiles (mprefix counts 256-row tiles) instead of 1-SM tiles (128 rows)
 };
 
 int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_down = nullptr) {
@@ -271,9 +300,12 @@ int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t
         p.E = a.E;
         p.dense_rows = shared ? a.T : 0;
         long long tiles = 0;
-        if (routed) tiles += ((long long)(a.max_rows + GEMM_BM - 1) / GEMM_BM + a.E) * c0.ntiles;
-        if (shared) tiles += (long long)((a.T + GEMM_BM - 1) / GEMM_BM) * c1.ntiles;
-        if ((rc = launch_gemm<EPI_SWIGLU>(di, A0, B0, B0b, A1, B1, B1b, p, tiles, s)) != MOE_OK) return rc;
+        const int bm = a.pair ? PAIR_BM : GEMM_BM;
+        if (routed) tiles += ((long long)(a.max_rows + bm - 1) / bm + a.E) * c0.ntiles;
+        if (shared) tiles += (long long)((a.T + bm - 1) / bm) * c1.ntiles;
+        rc = a.pair ? launch_gemm_pair<EPI_SWIGLU>(di, A0, B0, B0b, A1, B1, B1b, p, tiles, s)
+                    : launch_gemm<EPI_SWIGLU>(di, A0, B0, B0b, A1, B1, B1b, p, tiles, s);
+        if (rc != MOE_OK) return rc;
     }
     if (ev_down && cudaEventRecord(ev_down, s) != cudaSuccess) return MOE_ERR_CUDA;
     // ---- GEMM2: y = h W2^T
@@ -281,11 +313,11 @@ int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t
         CUtensorMap A0, B0, A1, B1;
         if (routed) {
             if ((rc = make_map(&A0, a.h, a.f, a.max_rows, GEMM_BM)) != MOE_OK) return rc;
-            if ((rc = make_map(&B0, a.W2, a.f, (uint64_t)a.E * a.d, 256)) != MOE_OK) return rc;
+            if ((rc = make_map(&B0, a.W2, a.f, (uint64_t)a.E * a.d, a.pair ? 128 : 256)) != MOE_OK) return rc;
         }
         if (shared) {
             if ((rc = make_map(&A1, a.h_shared, a.f_shared, a.T, GEMM_BM)) != MOE_OK) return rc;
-            if ((rc = make_map(&B1, a.W2s, a.f_shared, a.d, 256)) != MOE_OK) return rc;
+            if ((rc = make_map(&B1, a.W2s, a.f_shared, a.d, a.pair ? 128 : 256)) != MOE_OK) return rc;
         }
         if (!routed) { A0 = A1; B0 = B1; }
         if (!shared) { A1 = A0; B1 = B0; }
@@ -302,9 +334,12 @@ int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t
         p.E = a.E;
         p.dense_rows = shared ? a.T : 0;
         long long tiles = 0;
-        if (routed) tiles += ((long long)(a.max_rows + GEMM_BM - 1) / GEMM_BM + a.E) * c0.ntiles;
-        if (shared) tiles += (long long)((a.T + GEMM_BM - 1) / GEMM_BM) * c1.ntiles;
-        if ((rc = launch_gemm<EPI_STORE>(di, A0, B0, B0, A1, B1, B1, p, tiles, s)) != MOE_OK) return rc;
+        const int bm = a.pair ? PAIR_BM : GEMM_BM;
+        if (routed) tiles += ((long long)(a.max_rows + bm - 1) / bm + a.E) * c0.ntiles;
+        if (shared) tiles += (long long)((a.T + bm - 1) / bm) * c1.ntiles;
+        rc = a.pair ? launch_gemm_pair<EPI_STORE>(di, A0, B0, B0, A1, B1, B1, p, tiles, s)
+                    : launch_gemm<EPI_STORE>(di, A0, B0, B0, A1, B1, B1, p, tiles, s);
+        if (rc != MOE_OK) return rc;
     }
     return MOE_OK;
 }
@@ -422,13 +457,15 @@ int moe_expert_ffn(const moe_bf16* x_perm, const int32_t* offsets, int max_rows,
     if (max_rows == 0) return MOE_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int32_t* mprefix = static_cast<int32_t*>(ws);
-    tile_prefix_kernel<<<1, 1024, 0, s>>>(offsets, E, max_rows, mprefix);
+    const bool pair = use_pair_tiles(max_rows, E);
+    tile_prefix_kernel<<<1, 1024, 0, s>>>(offsets, E, max_rows, pair ? PAIR_BM : GEMM_BM, mprefix);
     if ((rc = launch_status()) != MOE_OK) return rc;
     FfnArgs a;
     memset(&a, 0, sizeof(a));
     a.x_perm = x_perm; a.offsets = offsets; a.mprefix = mprefix; a.max_rows = max_rows; a.E = E; a.d = d; a.f = f;
     a.W1 = W1; a.W3 = W3; a.W2 = W2; a.h = h; a.y_perm = y_perm;
     a.f_shared = 0;
+    a.pair = pair;
     return run_expert_ffn(di, a, s);
 }
 
@@ -500,8 +537,9 @@ int moe_layer_forward_ex(const moe_bf16* x, const moe_bf16* Wg, const float* bia
     if (!mark(ev.topk)) return MOE_ERR_CUDA;
     if ((rc = run_topk(logits, bias, T, E, k, idx, w, s)) != MOE_OK) return rc;
     if (!mark(ev.permute)) return MOE_ERR_CUDA;
+    const bool pair = use_pair_tiles((long long)T * k, E);
     if ((rc = run_permute(di, x, idx, T, d, E, k, C, counts_raw, counts, offsets, dest, src, x_perm, blk_cnt,
-                          rank_local, mprefix, s)) != MOE_OK)
+                          rank_local, mprefix, s, pair ? PAIR_BM : GEMM_BM)) != MOE_OK)
         return rc;
     if (!mark(ev.gate_up)) return MOE_ERR_CUDA;
     FfnArgs a;
@@ -510,6 +548,7 @@ int moe_layer_forward_ex(const moe_bf16* x, const moe_bf16* Wg, const float* bia
     a.W1 = W1; a.W3 = W3; a.W2 = W2; a.h = h; a.y_perm = y_perm;
     a.x = x; a.T = T; a.f_shared = f_shared; a.W1s = W1s; a.W3s = W3s; a.W2s = W2s;
     a.h_shared = h_shared; a.y_shared = y_shared;
+    a.pair = pair;
     if ((rc = run_expert_ffn(di, a, s, static_cast<cudaEvent_t>(ev.down))) != MOE_OK) return rc;
     if (!mark(ev.combine)) return MOE_ERR_CUDA;
     if ((rc = run_combine(y_perm, dest, w, y_shared, T, d, k, out, s)) != MOE_OK) return rc;

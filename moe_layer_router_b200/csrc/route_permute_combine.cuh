@@ -194,10 +194,11 @@ permute_count_kernel(const int32_t* __restrict__ idx, int T, int E, int k, int32
 
 // One block of 1024 threads.  In place, blk_cnt[b, e] becomes the number of assignments to
 // e in blocks before b.  Then counts_raw, counts = min(raw, C), offsets = exclusive scan
-// of counts, and mprefix = exclusive scan of ceil(counts / 128) (the GEMM m-tiles).
+// of counts, and mprefix = exclusive scan of ceil(counts / tile_rows) (the GEMM m-tiles).
 __global__ void __launch_bounds__(1024)
 permute_scan_kernel(int32_t* __restrict__ blk_cnt, int nb, int E, long long C, int32_t* __restrict__ counts_raw,
-                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ mprefix) {
+                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ mprefix,
+                    int tile_rows) {
     __shared__ int part[1024];
     __shared__ int tot[1024];
     const int P = blockDim.x / E;                 // partitions of the block range per expert
@@ -233,7 +234,7 @@ permute_scan_kernel(int32_t* __restrict__ blk_cnt, int nb, int E, long long C, i
     const int kept = tid < E ? (C < 0 ? raw : (int)min((long long)raw, C)) : 0;
     int total;
     const int off = block_exclusive_scan(kept, &total);
-    const int mt = (kept + 127) / 128;
+    const int mt = (kept + tile_rows - 1) / tile_rows;
     int mtotal;
     const int moff = block_exclusive_scan(mt, &mtotal);
     if (tid < E) {
@@ -343,11 +344,12 @@ combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ des
     }
 }
 
-// mprefix = exclusive scan of ceil((offsets[e+1]-offsets[e]) / 128).  If offsets are not a
+// mprefix = exclusive scan of ceil((offsets[e+1]-offsets[e]) / tile_rows).  If offsets are not a
 // monotone sequence starting at 0 and ending <= max_rows, records MOE_ERR_CHECK and
 // writes an all-zero prefix (no GEMM tile runs).
 __global__ void __launch_bounds__(1024)
-tile_prefix_kernel(const int32_t* __restrict__ offsets, int E, int max_rows, int32_t* __restrict__ mprefix) {
+tile_prefix_kernel(const int32_t* __restrict__ offsets, int E, int max_rows, int tile_rows,
+                   int32_t* __restrict__ mprefix) {
     __shared__ int bad;
     const int e = threadIdx.x;
     if (e == 0) bad = 0;
@@ -356,7 +358,7 @@ tile_prefix_kernel(const int32_t* __restrict__ offsets, int E, int max_rows, int
     if (e < E) {
         const int a = offsets[e], b = offsets[e + 1];
         if (a < 0 || b < a || b > max_rows || (e == 0 && a != 0)) bad = 1;
-        mt = (b - a + 127) / 128;
+        mt = (b - a + tile_rows - 1) / tile_rows;
     }
     __syncthreads();
     if (bad) mt = 0;

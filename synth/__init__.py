@@ -147,6 +147,12 @@ WORKLOADS = {
     "skew": Workload("skew", 32768, 4096, 64, 2, 2048, cap_mode=CAP_PER_ASSIGNMENT, capacity_factor=1.25, zipf_s=1.2),
 }
 WORKLOAD_ORDER = ["tiny", "mixtral", "qwen3", "dsv3", "skew"]
+# Smaller cases with the same per-tile shapes, for profiler captures that must stay small.
+PROFILE_WORKLOADS = {
+    "mixtral2e": Workload("mixtral2e", 2048, 4096, 2, 2, 14336),
+    "dsv3_32e": Workload("dsv3_32e", 32, 7168, 32, 8, 2048, f_shared=2048, bias_range=0.1),
+}
+WORKLOADS.update(PROFILE_WORKLOADS)
 
 
 class Inputs:

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synth
-from _util import assert_layer_close, bf16_bits, bits_to_f64, logits_tol, to_dev_bf16
+from _util import assert_layer_close, bf16_bits, bits_to_f64, logits_tol, to_dev_bf16, ulp_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -124,7 +124,7 @@ def test_combine(moe, with_shared):
     assert moe.moe_get_error() == 0
     got = bf16_bits(out)
     assert_layer_close(got, ref)
-    assert np.mean(got == ref) > 0.99
+    assert np.mean(ulp_bf16(got, ref) <= 1) > 0.999
     assert (r["dest"] < 0).any()                  # drops exercised
 
 
@@ -152,9 +152,12 @@ def test_router_gemm(moe, T, d, E):
 
 # ----------------------------------------------------------------------------- expert FFN
 
+# groups averaging >= 256 rows run on CTA-pair (2-SM) tiles, the others on 1-SM tiles
 @pytest.mark.parametrize("counts,d,f", [([0, 1, 127, 128, 129, 300, 5, 0], 256, 512), ([200, 200, 200], 128, 320),
                                         ([1], 64, 64), ([0, 0, 0], 128, 128), ([17, 260, 3, 64], 448, 192),
-                                        ([513, 1, 700], 1024, 1536)])
+                                        ([513, 1, 700], 1024, 1536),
+                                        ([0, 1, 255, 256, 257, 700, 5, 1000], 256, 512),
+                                        ([300, 0, 600], 448, 192), ([2000], 128, 128)])
 def test_expert_ffn(moe, counts, d, f):
     E = len(counts)
     off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
@@ -179,7 +182,7 @@ def test_expert_ffn(moe, counts, d, f):
         dh = np.abs(bits_to_f64(hg[a:b]) - bits_to_f64(ho))
         assert np.all(dh <= 1e-3 + 8e-3 * np.abs(bits_to_f64(ho))), f"h of expert {e}"
         assert_layer_close(yg[a:b], yo, f"y of expert {e}")
-        assert np.mean(yg[a:b] == yo) > 0.9
+        assert np.mean(ulp_bf16(yg[a:b], yo) <= 1) > 0.99
     # rows past the last group are never written (tiles straddling a group edge are masked)
     assert np.all(bits_to_f64(hg[N:]) == 7.0) and np.all(bits_to_f64(yg[N:]) == 7.0)
 
@@ -205,6 +208,8 @@ SMALL = [
     dict(name="per-assignment-cap", wl=synth.Workload("cap", 513, 128, 8, 2, 128, cap_mode=synth.CAP_PER_ASSIGNMENT,
                                                       capacity_factor=0.8)),
     dict(name="single-expert", wl=synth.Workload("one", 200, 128, 1, 1, 256)),
+    dict(name="pair-tiles-shared-cap", wl=synth.Workload("pairs", 1500, 256, 4, 2, 384, f_shared=256, bias_range=0.1,
+                                                         cap_mode=synth.CAP_PER_TOKEN, capacity_factor=1.5)),
 ]
 
 
@@ -250,6 +255,6 @@ def test_layer_small_all_intermediates(moe, case):
     # (iv) outputs
     got = bf16_bits(out)
     assert_layer_close(got, ref["out"])
-    assert np.mean(got == ref["out"]) > 0.9
+    assert np.mean(ulp_bf16(got, ref["out"]) <= 1) > 0.99
     if fs:
         assert_layer_close(bf16_bits(v("y_shared", (T, d), torch.bfloat16)), ref["y_shared"], "y_shared")
