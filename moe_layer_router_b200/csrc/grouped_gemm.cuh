@@ -33,18 +33,25 @@ namespace moe {
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 64;                       // one 128-byte swizzle row of bf16
-constexpr int GEMM_STAGES = 4;
+constexpr int GEMM_STAGES = 4;                        // stages when B tiles are 256 rows
+constexpr int GEMM_MAX_STAGES = 12;
 constexpr int GEMM_A_BYTES = GEMM_BM * GEMM_BK * 2;   // 16 KB
 constexpr int GEMM_B_BYTES = 256 * GEMM_BK * 2;       // 32 KB (N <= 256)
 constexpr int GEMM_ACC_COLS = 256;
 constexpr int GEMM_TMEM_COLS = 512;
 constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_SMEM_MAX = 232448;                 // 227 KB opt-in per CTA
 constexpr int GEMM_SMEM_BYTES = GEMM_STAGES * (GEMM_A_BYTES + GEMM_B_BYTES) + 1024 + 256;
+
+// Shared memory of a ring of `stages` slots, each one A tile and one B slot of b_slot bytes.
+__host__ __device__ constexpr int gemm_smem_bytes(int stages, int b_slot) {
+    return stages * (GEMM_A_BYTES + b_slot) + 1024 + 256;
+}
 
 enum { EPI_LOGITS = 0, EPI_SWIGLU = 1, EPI_STORE = 2 };
 
 struct GemmClass {
-    int K;              // reduction length, multiple of 64
+    int K;              // reduction length per tile (per split), multiple of 64
     int n_out;          // valid output columns
     int ntiles;         // tiles along N
     int b_group_rows;   // rows between consecutive groups in the B tensor(s)
@@ -54,6 +61,8 @@ struct GemmClass {
     long long ldo;      // output row stride in elements
     long long out_row0; // added to the tile's A row to get the output row
     long long out_rows; // output rows available (stores at or beyond are dropped)
+    int ksplit;         // dense class: K is cut into ksplit slices of K each (>= 1)
+    long long split_stride;  // output elements between the partial results of two slices
 };
 
 struct GemmParams {
@@ -62,6 +71,8 @@ struct GemmParams {
     const int32_t* mprefix;  // [E+1] prefix of per-group m-tile counts (class 0)
     int E;
     int dense_rows;          // rows of class 1 (0 = no class 1)
+    int stages;              // ring slots (<= GEMM_MAX_STAGES)
+    int b_slot;              // bytes of one B slot (multiple of 1024)
 };
 
 struct TileInfo {
@@ -70,11 +81,13 @@ struct TileInfo {
     int rows;    // valid rows (<= 128)
     int b_row;   // first B row (gate half for SwiGLU)
     int n_idx;   // tile index along N
+    int ks;      // K slice (dense class with ksplit > 1)
 };
 
 __device__ __forceinline__ int gemm_total_tiles(const GemmParams& p, int& routed_tiles) {
     routed_tiles = p.offsets ? __ldg(p.mprefix + p.E) * p.cls[0].ntiles : 0;
-    const int dense = p.dense_rows ? ((p.dense_rows + GEMM_BM - 1) / GEMM_BM) * p.cls[1].ntiles : 0;
+    const int dense =
+        p.dense_rows ? ((p.dense_rows + GEMM_BM - 1) / GEMM_BM) * p.cls[1].ntiles * p.cls[1].ksplit : 0;
     return routed_tiles + dense;
 }
 
@@ -99,16 +112,19 @@ __device__ __forceinline__ TileInfo gemm_decode_tile(const GemmParams& p, int t,
         ti.rows = min(GEMM_BM, __ldg(p.offsets + g + 1) - r0);
         ti.n_idx = n;
         ti.b_row = g * c.b_group_rows + n * c.b_tile_rows;
+        ti.ks = 0;
     } else {
         const GemmClass& c = p.cls[1];
         const int mt = (p.dense_rows + GEMM_BM - 1) / GEMM_BM;
         const int local = t - routed_tiles;
-        const int m = local % mt, n = local / mt;
+        const int m = local % mt, rest = local / mt;
+        const int n = rest % c.ntiles;
         ti.cls = 1;
         ti.a_row = m * GEMM_BM;
         ti.rows = min(GEMM_BM, p.dense_rows - ti.a_row);
         ti.n_idx = n;
         ti.b_row = n * c.b_tile_rows;
+        ti.ks = rest / c.ntiles;
     }
     return ti;
 }
@@ -126,11 +142,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
                     const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int S = p.stages;
     uint8_t* sA = smem;
-    uint8_t* sB = smem + GEMM_STAGES * GEMM_A_BYTES;
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sB + GEMM_STAGES * GEMM_B_BYTES);
-    uint64_t* empty_bar = full_bar + GEMM_STAGES;
-    uint64_t* tfull_bar = empty_bar + GEMM_STAGES;
+    uint8_t* sB = smem + S * GEMM_A_BYTES;
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sB + S * p.b_slot);
+    uint64_t* empty_bar = full_bar + S;
+    uint64_t* tfull_bar = empty_bar + S;
     uint64_t* tempty_bar = tfull_bar + 2;
     uint64_t* drain_bar = tempty_bar + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
@@ -140,7 +157,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < GEMM_STAGES; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(full_bar + s, 1);
             mbar_init(empty_bar + s, 1);
         }
@@ -190,27 +207,28 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
                 const CUtensorMap* mB = ti.cls ? &tmB1 : &tmB0;
                 const CUtensorMap* mBb = ti.cls ? &tmB1b : &tmB0b;
                 const int nk = c.K / GEMM_BK;
+                const int k0 = ti.ks * c.K;
                 const uint32_t bytes =
                     GEMM_A_BYTES + (EPI == EPI_SWIGLU ? 2u : 1u) * (uint32_t)c.b_tile_rows * GEMM_BK * 2u;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(empty_bar + stage, phase ^ 1u, abort_flag)) { ok = false; break; }
                     mbar_arrive_expect_tx(full_bar + stage, bytes);
                     uint8_t* a_dst = sA + stage * GEMM_A_BYTES;
-                    uint8_t* b_dst = sB + stage * GEMM_B_BYTES;
-                    tma_load_2d(a_dst, mA, full_bar + stage, kb * GEMM_BK, ti.a_row, pol_a);
-                    tma_load_2d(b_dst, mB, full_bar + stage, kb * GEMM_BK, ti.b_row, pol_b);
+                    uint8_t* b_dst = sB + stage * p.b_slot;
+                    tma_load_2d(a_dst, mA, full_bar + stage, k0 + kb * GEMM_BK, ti.a_row, pol_a);
+                    tma_load_2d(b_dst, mB, full_bar + stage, k0 + kb * GEMM_BK, ti.b_row, pol_b);
                     if (EPI == EPI_SWIGLU)
-                        tma_load_2d(b_dst + 128 * 128, mBb, full_bar + stage, kb * GEMM_BK, ti.b_row, pol_b);
+                        tma_load_2d(b_dst + 128 * 128, mBb, full_bar + stage, k0 + kb * GEMM_BK, ti.b_row, pol_b);
                     ++issued;
-                    if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1u; }
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
             }
             if (!ok) {
                 // another role gave up: let the copies already in flight land before exit
-                const int n = issued < GEMM_STAGES ? issued : GEMM_STAGES;
+                const int n = issued < S ? issued : S;
                 for (int i = 1; i <= n; ++i) {
                     const int q = issued - i;
-                    mbar_wait(full_bar + (q % GEMM_STAGES), (uint32_t)((q / GEMM_STAGES) & 1), nullptr);
+                    mbar_wait(full_bar + (q % S), (uint32_t)((q / S) & 1), nullptr);
                 }
             }
         }
@@ -234,13 +252,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
                     if (!mbar_wait(full_bar + stage, phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t ad = smem_desc_k_sw128(sA + stage * GEMM_A_BYTES);
-                    const uint64_t bd = smem_desc_k_sw128(sB + stage * GEMM_B_BYTES);
+                    const uint64_t bd = smem_desc_k_sw128(sB + stage * p.b_slot);
 #pragma unroll
                     for (int kk = 0; kk < GEMM_BK / 16; ++kk)
                         umma_bf16(d_tmem, ad + 2ull * kk, bd + 2ull * kk, idesc, (kb | kk) != 0);
                     umma_commit(empty_bar + stage);
                     any = true;
-                    if (++stage == GEMM_STAGES) { stage = 0; phase ^= 1u; }
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
                 umma_commit(tfull_bar + acc);
@@ -316,8 +334,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
                             dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
                     }
                 }
-            } else {  // EPI_LOGITS
-                float* out = reinterpret_cast<float*>(c.out) + orow * c.ldo;
+            } else {  // EPI_LOGITS (K slice ks writes its partial sums split_stride further on)
+                float* out = reinterpret_cast<float*>(c.out) + ti.ks * c.split_stride + orow * c.ldo;
                 const bool vec_ok = (c.ldo & 3) == 0;
 #pragma unroll 1
                 for (int ch = 0; ch < c.mma_n / 32 + ((c.mma_n & 31) ? 1 : 0); ++ch) {

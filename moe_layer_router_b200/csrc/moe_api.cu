@@ -85,7 +85,7 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ER
 
 template <int EPI>
 int launch_gemm(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& b0b,
-                const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& b1b, const GemmParams& p,
+                const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& b1b, GemmParams p,
                 long long tiles_upper, cudaStream_t s) {
     {
         std::lock_guard<std::mutex> lock(g_mutex);
@@ -94,15 +94,38 @@ int launch_gemm(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b0, co
         cudaGetDevice(&dev);
         if (!attr_set[dev][EPI]) {
             if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     GEMM_SMEM_BYTES) != cudaSuccess)
+                                     GEMM_SMEM_MAX) != cudaSuccess)
                 return MOE_ERR_CUDA;
             attr_set[dev][EPI] = true;
         }
     }
     if (tiles_upper <= 0) return MOE_OK;
+    if (p.b_slot <= 0) p.b_slot = GEMM_B_BYTES;
+    if (p.stages <= 0) {   // as many ring slots as fit
+        p.stages = (GEMM_SMEM_MAX - 1024 - 256) / (GEMM_A_BYTES + p.b_slot);
+        if (p.stages > GEMM_MAX_STAGES) p.stages = GEMM_MAX_STAGES;
+    }
+    const int smem = gemm_smem_bytes(p.stages, p.b_slot);
     const int grid = (int)(tiles_upper < di->sms ? tiles_upper : di->sms);
-    grouped_gemm_kernel<EPI><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, s>>>(a0, b0, b0b, a1, b1, b1b, p);
+    grouped_gemm_kernel<EPI><<<grid, GEMM_THREADS, smem, s>>>(a0, b0, b0b, a1, b1, b1b, p);
     return launch_status();
+}
+
+// K slices of the router GEMM when it has too few output tiles to occupy the GPU: slices
+// double while the tile count stays under one CTA per SM of a B200 (148), each slice keeps
+// >= 256 of K and the partial sums stay under 16 MB.  A pure function of the shapes, so the
+// workspace size does not depend on the device.
+int router_ksplit(int T, int d, int E) {
+    const long long tiles = (long long)((T + GEMM_BM - 1) / GEMM_BM) * ((E + 255) / 256);
+    int ks = 1;
+    while (tiles * ks * 2 <= 148 && d % (GEMM_BK * ks * 2) == 0 && d / (ks * 2) >= 256 &&
+           (long long)ks * 2 * T * E * 4 <= (16ll << 20))
+        ks *= 2;
+    return ks;
+}
+size_t router_partial_bytes(int T, int d, int E) {
+    const int ks = router_ksplit(T, d, E);
+    return ks > 1 ? (size_t)ks * T * E * 4 : 0;
 }
 
 template <int EPI>
@@ -135,7 +158,7 @@ bool use_pair_tiles(long long rows, int E) { return rows >= 256ll * E; }
 
 struct LayerLayout {
     size_t off[12];
-    size_t blk_cnt, rank_local, mprefix, h_shared;
+    size_t blk_cnt, rank_local, mprefix, h_shared, router_part;
     size_t total;
 };
 
@@ -166,6 +189,7 @@ LayerLayout layer_layout(int T, int d, int E, int k, int f, int f_shared) {
     L.blk_cnt = take((size_t)permute_blocks(T) * E * 4);
     L.rank_local = take(Tk * 4);
     L.mprefix = take((size_t)(E + 1) * 4);
+    L.router_part = take(router_partial_bytes(T, d, E));
     L.total = cur;
     return L;
 }
@@ -184,8 +208,10 @@ size_t permute_scratch_bytes(int T, int E, int k, size_t* o_blk, size_t* o_rank,
 
 // ------------------------------------------------------------------ stage launchers
 
+// Router logits.  ks == 1: writes `logits` [T,E]; ks > 1: writes ks partial sums into
+// `partials` ([ks][T][E]), which the top-k kernel adds up.
 int run_router_gemm(DeviceInfo* di, const moe_bf16* x, const moe_bf16* Wg, int T, int d, int E, float* logits,
-                    cudaStream_t s) {
+                    float* partials, int ks, cudaStream_t s) {
     const int npad = E <= 256 ? ((E + 15) / 16) * 16 : 256;
     CUtensorMap a, b;
     int rc;
@@ -194,34 +220,44 @@ int run_router_gemm(DeviceInfo* di, const moe_bf16* x, const moe_bf16* Wg, int T
     GemmParams p;
     memset(&p, 0, sizeof(p));
     GemmClass& c = p.cls[1];
-    c.K = d;
+    c.K = d / ks;
     c.n_out = E;
     c.ntiles = (E + npad - 1) / npad;
     c.b_group_rows = 0;
     c.b_tile_rows = npad;
     c.mma_n = npad;
-    c.out = logits;
+    c.out = ks > 1 ? partials : logits;
     c.ldo = E;
     c.out_row0 = 0;
     c.out_rows = T;
+    c.ksplit = ks;
+    c.split_stride = (long long)T * E;
     p.cls[0] = c;
     p.offsets = nullptr;
     p.mprefix = nullptr;
     p.E = E;
     p.dense_rows = T;
-    const long long tiles = (long long)((T + GEMM_BM - 1) / GEMM_BM) * c.ntiles;
+    p.b_slot = npad * GEMM_BK * 2;      // a narrow B tile leaves room for more ring slots
+    p.stages = 0;
+    const long long tiles = (long long)((T + GEMM_BM - 1) / GEMM_BM) * c.ntiles * ks;
     return launch_gemm<EPI_LOGITS>(di, a, b, b, a, b, b, p, tiles, s);
 }
 
-int run_topk(const float* logits, const float* bias, int T, int E, int k, int32_t* idx, float* w, cudaStream_t s) {
+// Top-k on `logits` ([T,E]); with nsplit > 1 `logits` holds nsplit partial sums [nsplit][T][E]
+// that are added first (their sums go to logits_out).
+int run_topk(const float* logits, int nsplit, float* logits_out, const float* bias, int T, int E, int k,
+             int32_t* idx, float* w, cudaStream_t s) {
     const int blocks = (T + 7) / 8;
     const int epl = (E + 31) / 32;
-    if (epl <= 1) topk_softmax_kernel<1><<<blocks, 256, 0, s>>>(logits, bias, T, E, k, idx, w);
-    else if (epl <= 2) topk_softmax_kernel<2><<<blocks, 256, 0, s>>>(logits, bias, T, E, k, idx, w);
-    else if (epl <= 4) topk_softmax_kernel<4><<<blocks, 256, 0, s>>>(logits, bias, T, E, k, idx, w);
-    else if (epl <= 8) topk_softmax_kernel<8><<<blocks, 256, 0, s>>>(logits, bias, T, E, k, idx, w);
-    else if (epl <= 16) topk_softmax_kernel<16><<<blocks, 256, 0, s>>>(logits, bias, T, E, k, idx, w);
-    else topk_softmax_kernel<32><<<blocks, 256, 0, s>>>(logits, bias, T, E, k, idx, w);
+    const long long st = (long long)T * E;
+#define MOE_TOPK(EPL) topk_softmax_kernel<EPL><<<blocks, 256, 0, s>>>(logits, nsplit, st, logits_out, bias, T, E, k, idx, w)
+    if (epl <= 1) MOE_TOPK(1);
+    else if (epl <= 2) MOE_TOPK(2);
+    else if (epl <= 4) MOE_TOPK(4);
+    else if (epl <= 8) MOE_TOPK(8);
+    else if (epl <= 16) MOE_TOPK(16);
+    else MOE_TOPK(32);
+#undef MOE_TOPK
     return launch_status();
 }
 
@@ -245,8 +281,9 @@ int run_permute(DeviceInfo* di, const moe_bf16* x, const int32_t* idx, int T, in
     permute_scan_kernel<<<1, 1024, 0, s>>>(blk_cnt, nb, E, C, counts_raw, counts, offsets, mprefix, tile_rows);
     permute_scatter_kernel<<<nb, PERMUTE_TOKENS, 0, s>>>(idx, rank_local, blk_cnt, offsets, T, E, k, C, dest,
                                                           src_token);
-    gather_rows_kernel<<<(T + 7) / 8, 256, 0, s>>>(reinterpret_cast<const uint4*>(x), dest, T, d, k,
-                                                    reinterpret_cast<uint4*>(x_perm));
+    const long long chunks = (long long)T * (d / 8);
+    gather_rows_kernel<<<(unsigned)((chunks + 255) / 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(x), dest, T,
+                                                                         d, k, reinterpret_cast<uint4*>(x_perm));
     return launch_status();
 }
 
@@ -295,10 +332,13 @@ int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t
         c1.K = a.d; c1.n_out = a.f_shared; c1.ntiles = (a.f_shared + 127) / 128; c1.b_group_rows = 0;
         c1.b_tile_rows = 128; c1.mma_n = 256; c1.out = a.h_shared; c1.ldo = a.f_shared; c1.out_row0 = 0;
         c1.out_rows = a.T;
+        c0.ksplit = c1.ksplit = 1;
         p.offsets = routed ? a.offsets : nullptr;
         p.mprefix = a.mprefix;
         p.E = a.E;
         p.dense_rows = shared ? a.T : 0;
+        p.b_slot = GEMM_B_BYTES;
+        p.stages = GEMM_STAGES;
         long long tiles = 0;
         const int bm = a.pair ? PAIR_BM : GEMM_BM;
         if (routed) tiles += ((long long)(a.max_rows + bm - 1) / bm + a.E) * c0.ntiles;
@@ -329,10 +369,13 @@ int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t
         GemmClass& c1 = p.cls[1];
         c1.K = a.f_shared; c1.n_out = a.d; c1.ntiles = (a.d + 255) / 256; c1.b_group_rows = 0; c1.b_tile_rows = 256;
         c1.mma_n = 256; c1.out = a.y_shared; c1.ldo = a.d; c1.out_row0 = 0; c1.out_rows = a.T;
+        c0.ksplit = c1.ksplit = 1;
         p.offsets = routed ? a.offsets : nullptr;
         p.mprefix = a.mprefix;
         p.E = a.E;
         p.dense_rows = shared ? a.T : 0;
+        p.b_slot = GEMM_B_BYTES;
+        p.stages = GEMM_STAGES;
         long long tiles = 0;
         const int bm = a.pair ? PAIR_BM : GEMM_BM;
         if (routed) tiles += ((long long)(a.max_rows + bm - 1) / bm + a.E) * c0.ntiles;
@@ -346,9 +389,14 @@ int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t
 
 int run_combine(const moe_bf16* y_perm, const int32_t* dest, const float* w, const moe_bf16* y_shared, int T, int d,
                 int k, moe_bf16* out, cudaStream_t s) {
-    combine_kernel<<<(T + 7) / 8, 256, 0, s>>>(reinterpret_cast<const uint4*>(y_perm), dest, w,
-                                                reinterpret_cast<const uint4*>(y_shared), T, d, k,
-                                                reinterpret_cast<uint4*>(out));
+    // longest row segment per warp that still leaves >= 8192 warps (or one 32-chunk segment)
+    const int nvec = d / 8;
+    int seg = 1;
+    while (32 * seg * 2 <= nvec && (long long)T * ((nvec + 64 * seg - 1) / (64 * seg)) >= 8192) seg *= 2;
+    const long long warps = (long long)T * ((nvec + 32 * seg - 1) / (32 * seg));
+    combine_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(reinterpret_cast<const uint4*>(y_perm), dest, w,
+                                                                reinterpret_cast<const uint4*>(y_shared), T, d, k,
+                                                                seg, reinterpret_cast<uint4*>(out));
     return launch_status();
 }
 
@@ -401,24 +449,26 @@ int moe_route(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const fl
     int rc = device_info(&di);
     if (rc != MOE_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const float* logits = logits_in;
     if (!logits_in) {
         MOE_REQUIRE(x && Wg, MOE_ERR_INVALID_ARG);
         MOE_REQUIRE(d >= 64 && d % 64 == 0, MOE_ERR_SHAPE);
         MOE_REQUIRE(aligned16(x) && aligned16(Wg), MOE_ERR_ALIGN);
-        float* dst = logits_out;
-        if (!dst) {
-            MOE_REQUIRE(ws && ws_bytes >= (size_t)T * E * 4, MOE_ERR_WORKSPACE);
-            MOE_REQUIRE(aligned16(ws), MOE_ERR_ALIGN);
-            dst = static_cast<float*>(ws);
-        }
-        if ((rc = run_router_gemm(di, x, Wg, T, d, E, dst, s)) != MOE_OK) return rc;
-        logits = dst;
-    } else if (logits_out && logits_out != logits_in) {
+        const int ks = router_ksplit(T, d, E);
+        const size_t own = logits_out ? 0 : align256((size_t)T * E * 4);
+        const size_t need = own + (ks > 1 ? (size_t)ks * T * E * 4 : 0);
+        MOE_REQUIRE(need == 0 || (ws && ws_bytes >= need), MOE_ERR_WORKSPACE);
+        MOE_REQUIRE(aligned16(ws), MOE_ERR_ALIGN);
+        float* dst = logits_out ? logits_out : static_cast<float*>(ws);
+        float* part = ks > 1 ? reinterpret_cast<float*>(static_cast<char*>(ws) + own) : nullptr;
+        if ((rc = run_router_gemm(di, x, Wg, T, d, E, dst, part, ks, s)) != MOE_OK) return rc;
+        return ks > 1 ? run_topk(part, ks, dst, bias, T, E, k, idx, w, s)
+                      : run_topk(dst, 1, nullptr, bias, T, E, k, idx, w, s);
+    }
+    if (logits_out && logits_out != logits_in) {
         if (cudaMemcpyAsync(logits_out, logits_in, (size_t)T * E * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
-    return run_topk(logits, bias, T, E, k, idx, w, s);
+    return run_topk(logits_in, 1, nullptr, bias, T, E, k, idx, w, s);
 }
 
 int moe_permute(const moe_bf16* x, const int32_t* idx, int T, int d, int E, int k, int64_t capacity,
@@ -533,9 +583,13 @@ int moe_layer_forward_ex(const moe_bf16* x, const moe_bf16* Wg, const float* bia
 
     const long long C = moe_capacity(T, E, k, capacity_factor, cap_mode);
     if (!mark(ev.route)) return MOE_ERR_CUDA;
-    if ((rc = run_router_gemm(di, x, Wg, T, d, E, logits, s)) != MOE_OK) return rc;
+    const int ks = router_ksplit(T, d, E);
+    float* part = reinterpret_cast<float*>(base + L.router_part);
+    if ((rc = run_router_gemm(di, x, Wg, T, d, E, logits, part, ks, s)) != MOE_OK) return rc;
     if (!mark(ev.topk)) return MOE_ERR_CUDA;
-    if ((rc = run_topk(logits, bias, T, E, k, idx, w, s)) != MOE_OK) return rc;
+    rc = ks > 1 ? run_topk(part, ks, logits, bias, T, E, k, idx, w, s)
+                : run_topk(logits, 1, nullptr, bias, T, E, k, idx, w, s);
+    if (rc != MOE_OK) return rc;
     if (!mark(ev.permute)) return MOE_ERR_CUDA;
     const bool pair = use_pair_tiles((long long)T * k, E);
     if ((rc = run_permute(di, x, idx, T, d, E, k, C, counts_raw, counts, offsets, dest, src, x_perm, blk_cnt,

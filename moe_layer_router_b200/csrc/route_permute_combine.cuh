@@ -5,8 +5,8 @@
 //   permute_count_kernel  per-block expert histogram + stable rank of every assignment
 //   permute_scan_kernel   grid-wide scan: block bases, counts, capacity, offsets, m-tile prefix
 //   permute_scatter_kernel  dest / src_token from the ranks ([EP-KV] §8, [EP-DS3] §3.1)
-//   gather_rows_kernel    x_perm[dest] = x[t], one warp per token, 16-byte vectors
-//   combine_kernel        out[t] = sum_j w * y_perm[dest] (+ y_shared), one warp per token
+//   gather_rows_kernel    x_perm[dest] = x[t], one thread per 16-byte chunk
+//   combine_kernel        out[t] = sum_j w * y_perm[dest] (+ y_shared), one warp per row segment
 //                         ([EP-KV] §2, §7)
 //   tile_prefix_kernel    m-tile prefix of the grouped GEMM from offsets (with checks)
 #pragma once
@@ -58,9 +58,12 @@ __device__ __forceinline__ bool key_before(float ka, int ea, float kb, int eb) {
 }
 
 // EPL = logits held per lane (E <= 32*EPL).  One warp per token.
+// With nsplit > 1 the router GEMM left nsplit partial sums (split_stride floats apart); they
+// are added here in slice order 0, 1, ... and the sums are stored to logits_out.
 template <int EPL>
 __global__ void __launch_bounds__(256)
-topk_softmax_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k,
+topk_softmax_kernel(const float* __restrict__ logits, int nsplit, long long split_stride,
+                    float* __restrict__ logits_out, const float* __restrict__ bias, int T, int E, int k,
                     int32_t* __restrict__ idx, float* __restrict__ w) {
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -71,8 +74,20 @@ topk_softmax_kernel(const float* __restrict__ logits, const float* __restrict__ 
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         const int e = lane + 32 * i;
+        L[i] = e < E ? __ldg(row + e) : 0.0f;
+    }
+    for (int sp = 1; sp < nsplit; ++sp) {      // slice order; the EPL loads of a slice go out together
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E) L[i] = __fadd_rn(L[i], __ldg(row + sp * split_stride + e));
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
         if (e < E) {
-            L[i] = __ldg(row + e);
+            if (nsplit > 1 && logits_out) logits_out[(size_t)t * E + e] = L[i];
             key[i] = __fadd_rn(L[i], bias ? __ldg(bias + e) : 0.0f);   // fp32 add, no contraction
             bad |= !isfinite(key[i]) || !isfinite(L[i]);
         } else {
@@ -135,16 +150,18 @@ topk_softmax_kernel(const float* __restrict__ logits, const float* __restrict__ 
 // Block b owns tokens [256 b, 256 b + 256).  Writes blk_cnt[b, e] (assignments to e in the
 // block) and rank_local[t, j] = #{t' < t in the block : e = idx[t, j] is among idx[t', :]},
 // i.e. the stable (token-order) rank of (t, j) inside its block and expert.
-// Dynamic smem: (PERMUTE_WARPS * E + PERMUTE_TOKENS * k) ints.
+// Inside a warp (32 consecutive tokens) every lane sets its bit in a per-expert lane mask;
+// the rank is the number of lower lanes in the mask of its expert, plus the tokens of lower
+// warps routed to that expert.  Dynamic smem: (PERMUTE_WARPS * E + PERMUTE_TOKENS * k) ints.
 __global__ void __launch_bounds__(PERMUTE_TOKENS)
 permute_count_kernel(const int32_t* __restrict__ idx, int T, int E, int k, int32_t* __restrict__ blk_cnt,
                      int32_t* __restrict__ rank_local) {
     extern __shared__ int psm[];
-    int* wcnt = psm;                              // [PERMUTE_WARPS][E]
-    int* sidx = psm + PERMUTE_WARPS * E;          // [PERMUTE_TOKENS][k]
+    unsigned* lanes = reinterpret_cast<unsigned*>(psm);   // [PERMUTE_WARPS][E] lane masks, then warp bases
+    int* sidx = psm + PERMUTE_WARPS * E;                  // [PERMUTE_TOKENS][k]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int t0 = blockIdx.x * PERMUTE_TOKENS;
-    for (int i = threadIdx.x; i < PERMUTE_WARPS * E; i += blockDim.x) wcnt[i] = 0;
+    for (int i = threadIdx.x; i < PERMUTE_WARPS * E; i += blockDim.x) lanes[i] = 0u;
     for (int i = threadIdx.x; i < PERMUTE_TOKENS * k; i += blockDim.x) {
         const int t = t0 + i / k;
         int e = t < T ? __ldg(idx + (size_t)t0 * k + i) : -1;
@@ -157,28 +174,25 @@ permute_count_kernel(const int32_t* __restrict__ idx, int T, int E, int k, int32
     __syncthreads();
     const int me = warp * 32 + lane;              // token index inside the block
     const int t = t0 + me;
-    // rank inside the warp: lower lanes of this warp whose token routes to the same expert
+    unsigned* wl = lanes + warp * E;
     for (int j = 0; j < k; ++j) {
         const int e = sidx[me * k + j];
-        int r = 0;
-        for (int l = 0; l < 32; ++l) {
-            const int* other = sidx + (warp * 32 + l) * k;
-            int hit = 0;
-            for (int j2 = 0; j2 < k; ++j2) hit |= (other[j2] == e);
-            r += (l < lane) & hit;
-        }
-        if (e >= 0) {
-            atomicAdd(&wcnt[warp * E + e], 1);
-            rank_local[(size_t)t * k + j] = r;
-        }
+        if (e >= 0) atomicOr(wl + e, 1u << lane);
     }
     __syncthreads();
-    // per expert: exclusive prefix over warps, block total
+    // rank inside the warp: lower lanes whose token routes to the same expert
+    const unsigned lower = (1u << lane) - 1u;
+    for (int j = 0; j < k; ++j) {
+        const int e = sidx[me * k + j];
+        if (e >= 0) rank_local[(size_t)t * k + j] = __popc(wl[e] & lower);
+    }
+    __syncthreads();
+    // per expert: exclusive prefix over warps (replaces the masks), block total
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int run = 0;
         for (int w2 = 0; w2 < PERMUTE_WARPS; ++w2) {
-            const int c = wcnt[w2 * E + e];
-            wcnt[w2 * E + e] = run;
+            const int c = __popc(lanes[w2 * E + e]);
+            lanes[w2 * E + e] = (unsigned)run;
             run += c;
         }
         blk_cnt[(size_t)blockIdx.x * E + e] = run;
@@ -187,7 +201,7 @@ permute_count_kernel(const int32_t* __restrict__ idx, int T, int E, int k, int32
     if (t < T) {
         for (int j = 0; j < k; ++j) {
             const int e = sidx[me * k + j];
-            if (e >= 0) rank_local[(size_t)t * k + j] += wcnt[warp * E + e];
+            if (e >= 0) rank_local[(size_t)t * k + j] += (int)wl[e];
         }
     }
 }
@@ -269,25 +283,21 @@ permute_scatter_kernel(const int32_t* __restrict__ idx, const int32_t* __restric
     }
 }
 
-// x_perm[dest[t, j]] = x[t]; one warp per token reads the row once and writes it k times.
+// x_perm[dest[t, j]] = x[t].  One thread per 16-byte chunk of a token row: it reads the
+// chunk once and writes it to each kept destination (T*d/8 threads, so small batches still
+// spread over every SM).
 __global__ void __launch_bounds__(256)
 gather_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ dest, int T, int d, int k,
                    uint4* __restrict__ x_perm) {
-    const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (t >= T) return;
     const int nvec = d / 8;
-    const int dj = lane < k ? __ldg(dest + (size_t)t * k + lane) : -1;
-    const uint4* src = x + (size_t)t * nvec;
-    for (int base = 0; base < nvec; base += 32) {
-        const int c = base + lane;
-        const bool ok = c < nvec;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (ok) v = __ldg(src + c);
-        for (int j = 0; j < k; ++j) {
-            const int r = __shfl_sync(0xffffffffu, dj, j);
-            if (ok && r >= 0) x_perm[(size_t)r * nvec + c] = v;
-        }
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (long long)T * nvec) return;
+    const int t = (int)(i / nvec), c = (int)(i - (long long)t * nvec);
+    const uint4 v = __ldg(x + i);
+    const int32_t* dt = dest + (size_t)t * k;
+    for (int j = 0; j < k; ++j) {
+        const int r = __ldg(dt + j);
+        if (r >= 0) x_perm[(size_t)r * nvec + c] = v;
     }
 }
 
@@ -305,30 +315,49 @@ __device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// out[t] = bf16( sum_{j=0..k-1, dest>=0} w[t,j] * y_perm[dest[t,j]] + y_shared[t] ), fp32 FMA in j order.
+// out[t] = bf16( sum_{j=0..k-1, dest>=0} w[t,j] * y_perm[dest[t,j]] + y_shared[t] ), fp32 FMA in
+// j order.  One warp per (token, segment of 32*seg_chunks 16-byte chunks): lane j < k loads
+// slot j's row and weight once and shuffles them; loads of four slots are in flight at a
+// time.  seg_chunks is chosen on the host so that small batches still fill the GPU.
 __global__ void __launch_bounds__(256)
 combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ dest, const float* __restrict__ w,
-               const uint4* __restrict__ y_shared, int T, int d, int k, uint4* __restrict__ out) {
+               const uint4* __restrict__ y_shared, int T, int d, int k, int seg_chunks, uint4* __restrict__ out) {
     const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (t >= T) return;
     const int nvec = d / 8;
+    const int seg_len = 32 * seg_chunks;
+    const int nseg = (nvec + seg_len - 1) / seg_len;
+    const long long wid = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (wid >= (long long)T * nseg) return;
+    const int t = (int)(wid / nseg), sg = (int)(wid - (long long)t * nseg);
     const int dj = lane < k ? __ldg(dest + (size_t)t * k + lane) : -1;
     const float wj = lane < k ? __ldg(w + (size_t)t * k + lane) : 0.0f;
-    for (int base = 0; base < nvec; base += 32) {
-        const int c = base + lane;
-        const bool ok = c < nvec;
+    const int c_end = min(nvec, (sg + 1) * seg_len);
+    for (int c = sg * seg_len + lane; c - lane < c_end; c += 32) {
+        const bool ok = c < c_end;
         float acc[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-        for (int j = 0; j < k; ++j) {
-            const int r = __shfl_sync(0xffffffffu, dj, j);
-            const float wv = __shfl_sync(0xffffffffu, wj, j);
-            if (ok && r >= 0) {
-                float f[8];
-                bf16x8_to_f32(__ldg(y_perm + (size_t)r * nvec + c), f);
+        for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+        for (int j = 0; j < k; j += 4) {
+            int r[4];
+            float wv[4];
+            uint4 v[4];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(wv, f[i], acc[i]);
+            for (int q = 0; q < 4; ++q) {
+                r[q] = __shfl_sync(0xffffffffu, dj, (j + q) & 31);
+                wv[q] = __shfl_sync(0xffffffffu, wj, (j + q) & 31);
+                if (j + q >= k) r[q] = -1;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                v[q] = (ok && r[q] >= 0) ? __ldg(y_perm + (size_t)r[q] * nvec + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (r[q] >= 0) {
+                    float f[8];
+                    bf16x8_to_f32(v[q], f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[e] = fmaf(wv[q], f[e], acc[e]);
+                }
             }
         }
         if (ok) {
@@ -336,7 +365,7 @@ combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ des
                 float f[8];
                 bf16x8_to_f32(__ldg(y_shared + (size_t)t * nvec + c), f);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], f[i]);
+                for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], f[e]);
             }
             out[(size_t)t * nvec + c] = make_uint4(f32x2_to_bf16x2(acc[0], acc[1]), f32x2_to_bf16x2(acc[2], acc[3]),
                                                    f32x2_to_bf16x2(acc[4], acc[5]), f32x2_to_bf16x2(acc[6], acc[7]));
