@@ -243,6 +243,7 @@ def main():
     import torch
     import torch.distributed as dist
     import moe_layer_router_b200 as moe
+    from moe_layer_router_b200 import dp
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -252,7 +253,8 @@ def main():
     # inputs: replicated weights, a distinct token batch per rank
     tensors = synth.device_tensors(wl, dev, names=["wg", "w1", "w3", "w2", "w1s", "w3s", "w2s", "bias"])
     inp = synth.Inputs(wl)
-    x_host = torch.from_numpy(inp.x_rows(rank * wl.T, wl.T).view(np.int16)).view(torch.bfloat16).reshape(wl.T, wl.d)
+    row0, nrows = dp.token_rows(rank, world, wl.T)
+    x_host = torch.from_numpy(inp.x_rows(row0, nrows).view(np.int16)).view(torch.bfloat16).reshape(wl.T, wl.d)
     x = x_host.to(dev)
     T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
     ws = torch.empty(moe.moe_workspace_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device=dev)
@@ -288,11 +290,8 @@ def main():
     stage_ms = {}
     for a, b in zip(moe.STAGES[:-1], moe.STAGES[1:]):
         stage_ms[a] = float(np.mean([e[a].elapsed_time(e[b]) for e in evs]))
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
-    value = world * T * K / (total_ms / 1000.0)
+    total_ms = dp.max_over_ranks(total_ms, device=dev)
+    value = dp.job_throughput(T, world, K, total_ms)
 
     # kept rows and touched experts of the (deterministic) routing
     L = moe.moe_workspace_layout(T, d, E, k, f, fs)
@@ -322,11 +321,10 @@ def main():
         out_pin.copy_(out, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    e2e_ms = dp.max_over_ranks(e0.elapsed_time(e1), device=dev)
     if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
         dist.barrier()
-    e2e_value = world * T * K / (float(te.item()) / 1000.0)
+    e2e_value = dp.job_throughput(T, world, K, e2e_ms)
     rc = moe.moe_get_error()
     if rc != 0:
         raise RuntimeError(f"device error: {moe.strerror(rc)}")
