@@ -68,7 +68,7 @@ def load_peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for n in ("grouped_gemm.cuh", "ptx.cuh"):
+    for n in ("grouped_gemm.cuh", "grouped_gemm_pair.cuh", "ptx.cuh"):
         h.update(open(os.path.join(ROOT, "moe_layer_router_b200", "csrc", n), "rb").read())
     return h.hexdigest()[:16]
 
@@ -348,7 +348,9 @@ def main():
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"]}
     roof["traffic"] = recorded_traffic("gate_up", wl.name)
-    roof["kernel"] = "grouped_gemm_kernel<EPI_SWIGLU> (gate_up: W1/W3 + SwiGLU)"
+    pair = T * k >= 256 * E
+    roof["kernel"] = ("grouped_gemm_pair_kernel<EPI_SWIGLU>" if pair else "grouped_gemm_kernel<EPI_SWIGLU>") + \
+        " (gate_up: W1/W3 + SwiGLU)"
     roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if decode else 'bf16_tflops'}, burst)"
     roof["algorithmic_per_launch"] = alg
     lf, lb = layer_work(wl, N, touched)
