@@ -210,6 +210,7 @@ SMALL = [
     dict(name="single-expert", wl=synth.Workload("one", 200, 128, 1, 1, 256)),
     dict(name="pair-tiles-shared-cap", wl=synth.Workload("pairs", 1500, 256, 4, 2, 384, f_shared=256, bias_range=0.1,
                                                          cap_mode=synth.CAP_PER_TOKEN, capacity_factor=1.5)),
+    dict(name="pair-tail-tiles-shared", wl=synth.Workload("tails", 1400, 256, 4, 2, 448, f_shared=192, bias_range=0.1)),
 ]
 
 
