@@ -195,6 +195,43 @@ int moe_layer_forward_ex(const moe_bf16* x, const moe_bf16* Wg, const float* bia
                          const moe_stage_events* events);
 
 /*
+ * One global token batch sharded over G ranks (one process per GPU), with a capacity limit.
+ * Token-order dropping is global: rank r's tokens come after those of ranks 0..r-1, so an
+ * expert may keep only capacity - (its assignments on earlier ranks) of rank r's.  The one
+ * exchange this needs happens between two calls:
+ *   1. moe_layer_route_count(): router + top-k + per-expert histogram of this rank's batch;
+ *      counts_raw (workspace offset off[3] of moe_workspace_layout, [E] int32) is then valid.
+ *   2. the caller all-gathers every rank's counts_raw into all_counts [G, E] (rank-major),
+ *      e.g. with ncclAllGather, and moe_fill_base() turns it into this rank's
+ *      fill_base[e] = sum_{g < rank} all_counts[g, e].
+ *   3. moe_layer_finish(): permutation with the global capacity (e.g. moe_capacity(G*T, ...))
+ *      and fill_base, then experts (+ shared) and combine, on the same workspace.
+ * With fill_base = NULL, moe_layer_finish() after moe_layer_route_count() equals
+ * moe_layer_forward() with that capacity.  Same shapes, pointers and workspace rules as
+ * moe_layer_forward(); x must be the same tensor in both calls.
+ */
+int moe_layer_route_count(const moe_bf16* x, const moe_bf16* Wg, const float* bias, int f_shared,
+                          int T, int d, int E, int k, int f, void* ws, size_t ws_bytes, moe_stream_t stream);
+int moe_fill_base(const int32_t* all_counts, int G, int rank, int E, int32_t* fill_base, moe_stream_t stream);
+int moe_layer_finish(const moe_bf16* x, const moe_bf16* W1, const moe_bf16* W3, const moe_bf16* W2,
+                     const moe_bf16* W1s, const moe_bf16* W3s, const moe_bf16* W2s, int f_shared,
+                     int T, int d, int E, int k, int f, int64_t capacity, const int32_t* fill_base,
+                     moe_bf16* out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Selection bias from the overflow of the last batch ([EP-DS3] §2.1, the router's expert_bias
+ * update, applied between batches at inference):
+ *   bias[e] = -clamp((counts_raw[e] - capacity) / capacity, -1, 1)      (fp32, IEEE division)
+ * An expert routed more than `capacity` times gets a negative bias (fewer later tokens pick
+ * it), an idle one up to +1.  The page's comment states that sign; the formula it prints
+ * omits the minus.  Pass the result as `bias` of the next moe_route / moe_layer_forward.
+ *   counts_raw [E] int32 (device), e.g. the counts_raw that moe_permute wrote
+ *   capacity   > 0, e.g. moe_capacity(T, E, k, factor, MOE_CAP_PER_TOKEN)
+ *   bias       [E] fp32 (device), overwritten
+ */
+int moe_update_bias(const int32_t* counts_raw, int E, int64_t capacity, float* bias, moe_stream_t stream);
+
+/*
  * Byte offsets of the intermediates that moe_layer_forward() leaves in its workspace,
  * so that a caller (a test) can read them after the call:
  *   off[0] logits [T,E] fp32   off[1] idx [T,k] int32   off[2] w [T,k] fp32

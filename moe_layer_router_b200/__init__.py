@@ -63,6 +63,15 @@ _lib.moe_combine.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp]
 _lib.moe_layer_forward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                                    _i32, _i32, _i32, _i32, _i32, _dbl, _i32, _vp, _vp, _sz, _vp]
 _lib.moe_layer_forward_ex.argtypes = _lib.moe_layer_forward.argtypes + [_vp]
+_lib.moe_layer_route_count.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]
+_lib.moe_layer_route_count.restype = _i32
+_lib.moe_fill_base.argtypes = [_vp, _i32, _i32, _i32, _vp, _vp]
+_lib.moe_fill_base.restype = _i32
+_lib.moe_layer_finish.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i64, _vp,
+                                  _vp, _vp, _sz, _vp]
+_lib.moe_layer_finish.restype = _i32
+_lib.moe_update_bias.argtypes = [_vp, _i32, _i64, _vp, _vp]
+_lib.moe_update_bias.restype = _i32
 _lib.moe_get_error.argtypes = [_vp]
 _lib.moe_strerror.argtypes = [_i32]
 _lib.moe_strerror.restype = ctypes.c_char_p
@@ -183,6 +192,26 @@ def moe_layer_forward_ex(x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, f_shared, T, d,
                                      _ptr(W3s), _ptr(W2s), f_shared, T, d, E, k, f, float(capacity_factor),
                                      cap_mode, _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream),
                                      ctypes.byref(ev) if ev is not None else None), "moe_layer_forward_ex")
+
+
+def moe_layer_route_count(x, Wg, bias, f_shared, T, d, E, k, f, ws, stream=None) -> None:
+    _check(_lib.moe_layer_route_count(_ptr(x), _ptr(Wg), _ptr(bias), f_shared, T, d, E, k, f, _ptr(ws), _nbytes(ws),
+                                      _stream(stream)), "moe_layer_route_count")
+
+
+def moe_fill_base(all_counts, G, rank, E, fill_base, stream=None) -> None:
+    _check(_lib.moe_fill_base(_ptr(all_counts), G, rank, E, _ptr(fill_base), _stream(stream)), "moe_fill_base")
+
+
+def moe_layer_finish(x, W1, W3, W2, W1s, W3s, W2s, f_shared, T, d, E, k, f, capacity, fill_base, out, ws,
+                     stream=None) -> None:
+    _check(_lib.moe_layer_finish(_ptr(x), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(W1s), _ptr(W3s), _ptr(W2s), f_shared, T,
+                                 d, E, k, f, int(capacity), _ptr(fill_base), _ptr(out), _ptr(ws), _nbytes(ws),
+                                 _stream(stream)), "moe_layer_finish")
+
+
+def moe_update_bias(counts_raw, E, capacity, bias, stream=None) -> None:
+    _check(_lib.moe_update_bias(_ptr(counts_raw), E, int(capacity), _ptr(bias), _stream(stream)), "moe_update_bias")
 
 
 def moe_get_error(stream=None) -> int:

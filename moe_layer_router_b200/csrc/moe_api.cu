@@ -264,7 +264,7 @@ int run_topk(const float* logits, int nsplit, float* logits_out, const float* bi
 int run_permute(DeviceInfo* di, const moe_bf16* x, const int32_t* idx, int T, int d, int E, int k, long long C,
                 int32_t* counts_raw, int32_t* counts, int32_t* offsets, int32_t* dest, int32_t* src_token,
                 moe_bf16* x_perm, int32_t* blk_cnt, int32_t* rank_local, int32_t* mprefix, cudaStream_t s,
-                int tile_rows = GEMM_BM) {
+                int tile_rows = GEMM_BM, const int32_t* fill_base = nullptr, bool counts_only = false) {
     const int nb = permute_blocks(T);
     const size_t smem = (size_t)(PERMUTE_WARPS * E + PERMUTE_TOKENS * k) * sizeof(int);
     {
@@ -278,8 +278,10 @@ int run_permute(DeviceInfo* di, const moe_bf16* x, const int32_t* idx, int T, in
         }
     }
     permute_count_kernel<<<nb, PERMUTE_TOKENS, smem, s>>>(idx, T, E, k, blk_cnt, rank_local);
-    permute_scan_kernel<<<1, 1024, 0, s>>>(blk_cnt, nb, E, C, counts_raw, counts, offsets, mprefix, tile_rows);
-    permute_scatter_kernel<<<nb, PERMUTE_TOKENS, 0, s>>>(idx, rank_local, blk_cnt, offsets, T, E, k, C, dest,
+    permute_scan_kernel<<<1, 1024, 0, s>>>(blk_cnt, nb, E, C, fill_base, counts_raw, counts, offsets, mprefix,
+                                           tile_rows);
+    if (counts_only) return launch_status();
+    permute_scatter_kernel<<<nb, PERMUTE_TOKENS, 0, s>>>(idx, rank_local, blk_cnt, offsets, T, E, k, C, fill_base, dest,
                                                           src_token);
     const long long chunks = (long long)T * (d / 8);
     gather_rows_kernel<<<(unsigned)((chunks + 255) / 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(x), dest, T,
@@ -538,26 +540,39 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
                                 cap_mode, out, ws, ws_bytes, stream, nullptr);
 }
 
-int moe_layer_forward_ex(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const moe_bf16* W1,
-                         const moe_bf16* W3, const moe_bf16* W2, const moe_bf16* W1s, const moe_bf16* W3s,
-                         const moe_bf16* W2s, int f_shared, int T, int d, int E, int k, int f, double capacity_factor,
-                         int cap_mode, moe_bf16* out, void* ws, size_t ws_bytes, moe_stream_t stream,
-                         const moe_stage_events* events) {
+}  // extern "C"
+
+namespace moe {
+namespace {
+
+enum { LAYER_ROUTE = 1, LAYER_COUNT = 2, LAYER_FINISH = 4 };
+
+// The layer in phases over one workspace:
+//   LAYER_ROUTE  router GEMM + top-k                 (needs x, Wg, bias)
+//   LAYER_COUNT  histogram only: counts_raw          (no capacity)
+//   LAYER_FINISH histogram, capacity (with fill_base), permutation, experts, combine
+int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float* bias, const moe_bf16* W1,
+                 const moe_bf16* W3, const moe_bf16* W2, const moe_bf16* W1s, const moe_bf16* W3s, const moe_bf16* W2s,
+                 int f_shared, int T, int d, int E, int k, int f, long long C, const int32_t* fill_base,
+                 moe_bf16* out, void* ws, size_t ws_bytes, cudaStream_t s, const moe_stage_events* events) {
     int rc = check_shape(T, d, E, k, f);
     if (rc != MOE_OK) return rc;
     MOE_REQUIRE(f_shared >= 0 && f_shared % 64 == 0, MOE_ERR_SHAPE);
-    MOE_REQUIRE(cap_mode >= MOE_CAP_NONE && cap_mode <= MOE_CAP_PER_ASSIGNMENT, MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(x && Wg && W1 && W3 && W2 && out && ws, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(x && ws, MOE_ERR_INVALID_ARG);
+    if (phases & LAYER_ROUTE) MOE_REQUIRE(Wg, MOE_ERR_INVALID_ARG);
     const bool shared = f_shared > 0;
-    MOE_REQUIRE(!shared || (W1s && W3s && W2s), MOE_ERR_INVALID_ARG);
+    if (phases & LAYER_FINISH) {
+        MOE_REQUIRE(W1 && W3 && W2 && out, MOE_ERR_INVALID_ARG);
+        MOE_REQUIRE(!shared || (W1s && W3s && W2s), MOE_ERR_INVALID_ARG);
+    }
     MOE_REQUIRE(aligned16(x) && aligned16(Wg) && aligned16(bias) && aligned16(W1) && aligned16(W3) && aligned16(W2) &&
-                    aligned16(W1s) && aligned16(W3s) && aligned16(W2s) && aligned16(out) && aligned16(ws),
+                    aligned16(W1s) && aligned16(W3s) && aligned16(W2s) && aligned16(out) && aligned16(ws) &&
+                    aligned16(fill_base),
                 MOE_ERR_ALIGN);
     const LayerLayout L = layer_layout(T, d, E, k, f, f_shared);
     MOE_REQUIRE(ws_bytes >= L.total, MOE_ERR_WORKSPACE);
     DeviceInfo* di;
     if ((rc = device_info(&di)) != MOE_OK) return rc;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     char* base = static_cast<char*>(ws);
     float* logits = reinterpret_cast<float*>(base + L.off[0]);
     int32_t* idx = reinterpret_cast<int32_t*>(base + L.off[1]);
@@ -581,19 +596,26 @@ int moe_layer_forward_ex(const moe_bf16* x, const moe_bf16* Wg, const float* bia
     if (events) ev = *events;
     auto mark = [&](void* e) { return e == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(e), s) == cudaSuccess; };
 
-    const long long C = moe_capacity(T, E, k, capacity_factor, cap_mode);
-    if (!mark(ev.route)) return MOE_ERR_CUDA;
-    const int ks = router_ksplit(T, d, E);
-    float* part = reinterpret_cast<float*>(base + L.router_part);
-    if ((rc = run_router_gemm(di, x, Wg, T, d, E, logits, part, ks, s)) != MOE_OK) return rc;
-    if (!mark(ev.topk)) return MOE_ERR_CUDA;
-    rc = ks > 1 ? run_topk(part, ks, logits, bias, T, E, k, idx, w, s)
-                : run_topk(logits, 1, nullptr, bias, T, E, k, idx, w, s);
-    if (rc != MOE_OK) return rc;
-    if (!mark(ev.permute)) return MOE_ERR_CUDA;
+    if (phases & LAYER_ROUTE) {
+        if (!mark(ev.route)) return MOE_ERR_CUDA;
+        const int ks = router_ksplit(T, d, E);
+        float* part = reinterpret_cast<float*>(base + L.router_part);
+        if ((rc = run_router_gemm(di, x, Wg, T, d, E, logits, part, ks, s)) != MOE_OK) return rc;
+        if (!mark(ev.topk)) return MOE_ERR_CUDA;
+        rc = ks > 1 ? run_topk(part, ks, logits, bias, T, E, k, idx, w, s)
+                    : run_topk(logits, 1, nullptr, bias, T, E, k, idx, w, s);
+        if (rc != MOE_OK) return rc;
+    }
     const bool pair = use_pair_tiles((long long)T * k, E);
+    if (phases & LAYER_COUNT) {
+        if ((rc = run_permute(di, x, idx, T, d, E, k, -1, counts_raw, counts, offsets, dest, src, x_perm, blk_cnt,
+                              rank_local, mprefix, s, GEMM_BM, nullptr, true)) != MOE_OK)
+            return rc;
+    }
+    if (!(phases & LAYER_FINISH)) return MOE_OK;
+    if (!mark(ev.permute)) return MOE_ERR_CUDA;
     if ((rc = run_permute(di, x, idx, T, d, E, k, C, counts_raw, counts, offsets, dest, src, x_perm, blk_cnt,
-                          rank_local, mprefix, s, pair ? PAIR_BM : GEMM_BM)) != MOE_OK)
+                          rank_local, mprefix, s, pair ? PAIR_BM : GEMM_BM, fill_base)) != MOE_OK)
         return rc;
     if (!mark(ev.gate_up)) return MOE_ERR_CUDA;
     FfnArgs a;
@@ -607,6 +629,61 @@ int moe_layer_forward_ex(const moe_bf16* x, const moe_bf16* Wg, const float* bia
     if (!mark(ev.combine)) return MOE_ERR_CUDA;
     if ((rc = run_combine(y_perm, dest, w, y_shared, T, d, k, out, s)) != MOE_OK) return rc;
     return mark(ev.end) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" {
+
+int moe_layer_forward_ex(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const moe_bf16* W1,
+                         const moe_bf16* W3, const moe_bf16* W2, const moe_bf16* W1s, const moe_bf16* W3s,
+                         const moe_bf16* W2s, int f_shared, int T, int d, int E, int k, int f, double capacity_factor,
+                         int cap_mode, moe_bf16* out, void* ws, size_t ws_bytes, moe_stream_t stream,
+                         const moe_stage_events* events) {
+    MOE_REQUIRE(cap_mode >= MOE_CAP_NONE && cap_mode <= MOE_CAP_PER_ASSIGNMENT, MOE_ERR_INVALID_ARG);
+    const long long C = moe_capacity(T, E, k, capacity_factor, cap_mode);
+    return layer_phases(LAYER_ROUTE | LAYER_FINISH, x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, f_shared, T, d, E, k, f, C,
+                        nullptr, out, ws, ws_bytes, static_cast<cudaStream_t>(stream), events);
+}
+
+int moe_layer_route_count(const moe_bf16* x, const moe_bf16* Wg, const float* bias, int f_shared, int T, int d, int E,
+                          int k, int f, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    return layer_phases(LAYER_ROUTE | LAYER_COUNT, x, Wg, bias, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                        f_shared, T, d, E, k, f, -1, nullptr, nullptr, ws, ws_bytes, static_cast<cudaStream_t>(stream),
+                        nullptr);
+}
+
+int moe_fill_base(const int32_t* all_counts, int G, int rank, int E, int32_t* fill_base, moe_stream_t stream) {
+    MOE_REQUIRE(G >= 1 && rank >= 0 && rank < G && E >= 1 && E <= 1024, MOE_ERR_SHAPE);
+    MOE_REQUIRE(all_counts && fill_base, MOE_ERR_INVALID_ARG);
+    DeviceInfo* di;
+    int rc = device_info(&di);
+    if (rc != MOE_OK) return rc;
+    fill_base_kernel<<<(E + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(all_counts, G, rank, E,
+                                                                                    fill_base);
+    return launch_status();
+}
+
+int moe_layer_finish(const moe_bf16* x, const moe_bf16* W1, const moe_bf16* W3, const moe_bf16* W2,
+                     const moe_bf16* W1s, const moe_bf16* W3s, const moe_bf16* W2s, int f_shared, int T, int d, int E,
+                     int k, int f, int64_t capacity, const int32_t* fill_base, moe_bf16* out, void* ws,
+                     size_t ws_bytes, moe_stream_t stream) {
+    return layer_phases(LAYER_FINISH, x, nullptr, nullptr, W1, W3, W2, W1s, W3s, W2s, f_shared, T, d, E, k, f,
+                        capacity < 0 ? -1 : (long long)capacity, fill_base, out, ws, ws_bytes,
+                        static_cast<cudaStream_t>(stream), nullptr);
+}
+
+int moe_update_bias(const int32_t* counts_raw, int E, int64_t capacity, float* bias, moe_stream_t stream) {
+    MOE_REQUIRE(E >= 1 && E <= 1024, MOE_ERR_SHAPE);
+    MOE_REQUIRE(capacity > 0, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(counts_raw && bias, MOE_ERR_INVALID_ARG);
+    DeviceInfo* di;
+    int rc = device_info(&di);
+    if (rc != MOE_OK) return rc;
+    update_bias_kernel<<<(E + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(counts_raw, E,
+                                                                                      (long long)capacity, bias);
+    return launch_status();
 }
 
 int moe_get_error(moe_stream_t stream) {

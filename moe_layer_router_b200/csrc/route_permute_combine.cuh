@@ -207,12 +207,12 @@ permute_count_kernel(const int32_t* __restrict__ idx, int T, int E, int k, int32
 }
 
 // One block of 1024 threads.  In place, blk_cnt[b, e] becomes the number of assignments to
-// e in blocks before b.  Then counts_raw, counts = min(raw, C), offsets = exclusive scan
+// e in blocks before b.  Then counts_raw, counts = min(raw, C - fill_base), offsets = exclusive scan
 // of counts, and mprefix = exclusive scan of ceil(counts / tile_rows) (the GEMM m-tiles).
 __global__ void __launch_bounds__(1024)
-permute_scan_kernel(int32_t* __restrict__ blk_cnt, int nb, int E, long long C, int32_t* __restrict__ counts_raw,
-                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ mprefix,
-                    int tile_rows) {
+permute_scan_kernel(int32_t* __restrict__ blk_cnt, int nb, int E, long long C, const int32_t* __restrict__ fill_base,
+                    int32_t* __restrict__ counts_raw, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                    int32_t* __restrict__ mprefix, int tile_rows) {
     __shared__ int part[1024];
     __shared__ int tot[1024];
     const int P = blockDim.x / E;                 // partitions of the block range per expert
@@ -244,8 +244,11 @@ permute_scan_kernel(int32_t* __restrict__ blk_cnt, int nb, int E, long long C, i
             run += c;
         }
     }
+    // kept: the first C - fill_base[e] assignments in token order (fill_base: assignments of
+    // the same expert from tokens before this batch, on other ranks; 0 without sharding)
     const int raw = tid < E ? tot[tid] : 0;
-    const int kept = tid < E ? (C < 0 ? raw : (int)min((long long)raw, C)) : 0;
+    const long long room = tid < E ? C - (fill_base ? (long long)fill_base[tid] : 0ll) : 0;
+    const int kept = tid < E ? (C < 0 ? raw : (int)max(0ll, min((long long)raw, room))) : 0;
     int total;
     const int off = block_exclusive_scan(kept, &total);
     const int mt = (kept + tile_rows - 1) / tile_rows;
@@ -266,7 +269,8 @@ permute_scan_kernel(int32_t* __restrict__ blk_cnt, int nb, int E, long long C, i
 __global__ void __launch_bounds__(PERMUTE_TOKENS)
 permute_scatter_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ rank_local,
                        const int32_t* __restrict__ blk_base, const int32_t* __restrict__ offsets, int T, int E,
-                       int k, long long C, int32_t* __restrict__ dest, int32_t* __restrict__ src_token) {
+                       int k, long long C, const int32_t* __restrict__ fill_base, int32_t* __restrict__ dest,
+                       int32_t* __restrict__ src_token) {
     const int t = blockIdx.x * PERMUTE_TOKENS + threadIdx.x;
     if (t >= T) return;
     for (int j = 0; j < k; ++j) {
@@ -274,7 +278,8 @@ permute_scatter_kernel(const int32_t* __restrict__ idx, const int32_t* __restric
         int d = -1;
         if (e >= 0 && e < E) {
             const long long r = (long long)__ldg(blk_base + (size_t)blockIdx.x * E + e) + __ldg(rank_local + (size_t)t * k + j);
-            if (C < 0 || r < C) {
+            const long long base = fill_base ? (long long)__ldg(fill_base + e) : 0ll;
+            if (C < 0 || base + r < C) {
                 d = __ldg(offsets + e) + (int)r;
                 src_token[d] = t;
             }
@@ -371,6 +376,28 @@ combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ des
                                                    f32x2_to_bf16x2(acc[4], acc[5]), f32x2_to_bf16x2(acc[6], acc[7]));
         }
     }
+}
+
+// fill_base[e] = sum over ranks g < rank of all_counts[g, e]: the assignments to expert e
+// from the token batches before this rank's in global token order.
+__global__ void fill_base_kernel(const int32_t* __restrict__ all_counts, int G, int rank, int E,
+                                 int32_t* __restrict__ fill_base) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= E) return;
+    long long s = 0;
+    for (int g = 0; g < rank && g < G; ++g) s += all_counts[(size_t)g * E + e];
+    fill_base[e] = (int32_t)min(s, (long long)0x7fffffff);
+}
+
+// Selection bias from the overflow of the last batch ([EP-DS3] §2.1 expert_bias update):
+// bias_e = -clamp((counts_raw_e - C) / C, -1, 1) in fp32, IEEE division (C > 0).
+__global__ void update_bias_kernel(const int32_t* __restrict__ counts_raw, int E, long long C,
+                                   float* __restrict__ bias) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= E) return;
+    const float over = (float)((long long)counts_raw[e] - C);
+    const float r = fminf(fmaxf(__fdiv_rn(over, (float)C), -1.0f), 1.0f);
+    bias[e] = -r;
 }
 
 // mprefix = exclusive scan of ceil((offsets[e+1]-offsets[e]) / tile_rows).  If offsets are not a

@@ -55,6 +55,8 @@ def lib():
         L.oracle_dispatch.argtypes = [vp, i32, i32, i32, i64, vp, vp, vp, vp, vp]
         L.oracle_dispatch.restype = i32
         L.oracle_gather.argtypes = [vp, vp, i32, i32, i32, vp]
+        L.oracle_update_bias.argtypes = [vp, i32, i64, vp]
+        L.oracle_update_bias.restype = i32
         L.oracle_expert_ffn.argtypes = [vp, i32, vp, vp, vp, i32, i32, vp, vp]
         L.oracle_combine.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp]
         L.oracle_layer_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
@@ -114,6 +116,15 @@ def dispatch(idx: np.ndarray, E: int, C: int):
     dest = np.empty((T, k), np.int32); src = np.empty(max(T * k, 1), np.int32)
     N = lib().oracle_dispatch(_p(idx), T, E, k, int(C), _p(craw), _p(cnt), _p(off), _p(dest), _p(src))
     return dict(counts_raw=craw, counts=cnt, offsets=off, dest=dest, src_token=src[:N].copy(), N=N)
+
+
+def update_bias(counts_raw: np.ndarray, C: int) -> np.ndarray:
+    """Selection bias from the last batch's overflow: -clamp((c - C) / C, -1, 1), fp32."""
+    counts_raw = _c(counts_raw, np.int32)
+    out = np.empty(counts_raw.size, np.float32)
+    if lib().oracle_update_bias(_p(counts_raw), counts_raw.size, int(C), _p(out)) != 0:
+        raise ValueError("capacity must be positive")
+    return out
 
 
 def gather(x: np.ndarray, dest: np.ndarray, N: int) -> np.ndarray:

@@ -191,6 +191,27 @@ void oracle_gather(const uint16_t* x, const int32_t* dest, int T, int d, int k, 
         }
 }
 
+/*
+ * Overflow-driven selection bias ([EP-DS3] §2.1, the expert_bias update of the router code):
+ *   overflow_e = counts_raw_e - C,  bias_e = -clamp(overflow_e / C, -1, 1)
+ * computed in fp32 like the page's float tensors (the difference is exact; one division).
+ * Sign: the page's comment says an overloaded expert's bias is set negative so that later
+ * tokens avoid it; the formula it prints is positive for an overloaded expert.  The
+ * stated intent is taken: the bias is the negated clamped overflow ratio.
+ * Returns -1 for C <= 0 (no capacity: the update is undefined).
+ */
+int oracle_update_bias(const int32_t* counts_raw, int E, int64_t C, float* bias) {
+    if (C <= 0) return -1;
+    for (int e = 0; e < E; ++e) {
+        float over = (float)((int64_t)counts_raw[e] - C);
+        float r = over / (float)C;
+        if (r > 1.0f) r = 1.0f;
+        if (r < -1.0f) r = -1.0f;
+        bias[e] = -r;
+    }
+    return 0;
+}
+
 /* ---- experts ------------------------------------------------------------------------ */
 
 /*

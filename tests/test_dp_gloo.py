@@ -70,3 +70,59 @@ def test_single_process_helpers():
     assert dp.job_throughput(4096, 8, 10, 20.0) == pytest.approx(8 * 4096 * 10 / 0.02)
     with pytest.raises(ValueError):
         dp.token_rows(2, 2, 10)
+
+
+def _capacity_worker(rank, world, port, out):
+    """Each rank holds one shard of a global routing; the exchange of per-expert counts must
+    reproduce the global token-order capacity of the oracle on the whole batch."""
+    import datetime
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import oracle
+    from moe_layer_router_b200 import dp
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        T, E, k = 500, 12, 2
+        rng = np.random.default_rng(5)
+        logits = (rng.standard_normal((T * world, E)) + np.linspace(2, -2, E)).astype(np.float32)
+        idx, _ = oracle.route(logits, k)
+        C = oracle.capacity(T * world, E, k, 0.8, oracle.CAP_PER_ASSIGNMENT)
+        glob = oracle.dispatch(idx, E, C)
+        mine = idx[rank * T:(rank + 1) * T]
+        local = oracle.dispatch(mine, E, -1)["counts_raw"]
+        table = [torch.zeros(E, dtype=torch.int32) for _ in range(world)]
+        dist.all_gather(table, torch.from_numpy(local))
+        base = dp.fill_base_host(torch.stack(table).numpy(), rank)
+        # keep rule of one shard: position of the assignment among this shard's assignments to
+        # its expert, in token order, plus the base, below C
+        kept = np.zeros_like(mine, dtype=bool)
+        pos = np.zeros(E, np.int64)
+        for t in range(T):
+            for j in range(k):
+                e = mine[t, j]
+                kept[t, j] = base[e] + pos[e] < C
+                pos[e] += 1
+        want = glob["dest"][rank * T:(rank + 1) * T] >= 0
+        out[rank] = (bool(np.array_equal(kept, want)), int(kept.sum()), int(glob["N"]),
+                     bool((glob["counts_raw"] > C).any()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_global_capacity_exchange():
+    world = 2
+    manager = mp.Manager()
+    out = manager.dict()
+    mp.spawn(_capacity_worker, args=(world, _free_port(), out), nprocs=world, join=True)
+    assert all(out[r][0] for r in range(world))
+    assert out[0][1] + out[1][1] == out[0][2]          # kept over ranks = kept of the whole batch
+    assert out[0][3]                                   # the capacity did bind
+
+
+def test_fill_base_host():
+    from moe_layer_router_b200 import dp
+    t = np.array([[1, 2, 3], [4, 5, 6], [7, 8, 9]], np.int32)
+    assert list(dp.fill_base_host(t, 0)) == [0, 0, 0]
+    assert list(dp.fill_base_host(t, 2)) == [5, 7, 9]

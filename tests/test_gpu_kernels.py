@@ -259,3 +259,95 @@ def test_layer_small_all_intermediates(moe, case):
     assert np.mean(ulp_bf16(got, ref["out"]) <= 1) > 0.99
     if fs:
         assert_layer_close(bf16_bits(v("y_shared", (T, d), torch.bfloat16)), ref["y_shared"], "y_shared")
+
+
+# ----------------------------------------------------------------------------- overflow bias update
+
+def test_update_bias_bit_exact(moe):
+    E = 300
+    counts = (synth.uniform_f32(0, 120, 0, E, 0, 5000)).astype(np.int32)
+    for C in (1, 640, 1280, 4999):
+        ref = oracle.update_bias(counts, C)
+        b = torch.full((E,), 9.0, dtype=torch.float32, device="cuda")
+        moe.moe_update_bias(torch.from_numpy(counts).cuda(), E, C, b)
+        got = b.cpu().numpy()
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    with pytest.raises(moe.MoeError):
+        moe.moe_update_bias(torch.from_numpy(counts).cuda(), E, 0, b)
+
+
+def test_two_batches_with_overflow_bias_and_eval_capacity(moe):
+    # batch 1 routes without bias; its overflow sets the bias for batch 2 (eval factor 2.0)
+    wl = synth.Workload("bias", 1024, 256, 16, 2, 256, cap_mode=synth.CAP_PER_TOKEN, capacity_factor=2.0)
+    T, d, E, k, f = wl.T, wl.d, wl.E, wl.k, wl.f
+    inp = synth.Inputs(wl)
+    x1 = inp.x()
+    x2 = inp.x_rows(T, T).reshape(T, d)
+    wg = _bf16(E, d, 121, d ** -0.5)
+    wg[:4] = _bf16(4, d, 122, 3 * d ** -0.5)          # a few hot experts
+    W1, W3, W2 = inp.w1(), inp.w3(), inp.w2()
+    C = oracle.capacity(T, E, k, 2.0, oracle.CAP_PER_TOKEN)
+    dv = to_dev_bf16
+    ws = _ws(moe, T, d, E, k, f)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    bias = torch.zeros(E, dtype=torch.float32, device="cuda")
+    L = moe.moe_workspace_layout(T, d, E, k, f)
+    outs, logits = [], []
+    for xb, b in ((x1, None), (x2, bias)):
+        moe.moe_layer_forward(dv(xb), dv(wg), b, dv(W1), dv(W3), dv(W2), None, None, None, 0, T, d, E, k, f, 2.0,
+                              moe.MOE_CAP_PER_TOKEN, out, ws)
+        logits.append(moe.workspace_view(ws, L, "logits", (T, E), torch.float32).cpu().numpy())
+        outs.append(bf16_bits(out))
+        if b is None:     # bias for the next batch, from this batch's raw counts
+            craw = moe.workspace_view(ws, L, "counts_raw", (E,), torch.int32)
+            moe.moe_update_bias(craw, E, C, bias)
+    assert moe.moe_get_error() == 0
+    r1 = oracle.layer_forward(x1, wg, W1, W3, W2, k=k, C=C, logits_in=logits[0])
+    b_ref = oracle.update_bias(r1["counts_raw"], C)
+    assert np.array_equal(bias.cpu().numpy().view(np.uint32), b_ref.view(np.uint32))
+    assert r1["counts_raw"].max() > C                  # the first batch did overflow
+    r2 = oracle.layer_forward(x2, wg, W1, W3, W2, k=k, C=C, bias=b_ref, logits_in=logits[1])
+    assert_layer_close(outs[0], r1["out"])
+    assert_layer_close(outs[1], r2["out"])
+    assert np.array_equal(moe.workspace_view(ws, L, "idx", (T, k), torch.int32).cpu().numpy(), r2["idx"])
+
+
+# ----------------------------------------------------------------------------- one batch over two shards
+
+def test_sharded_batch_with_global_capacity_matches_whole_batch(moe):
+    # two shards of one batch run one after the other on this GPU (no kernel waits on another):
+    # shard 1's fill_base comes from shard 0's counts, exactly as the all-gather would give it
+    G, T, d, E, k, f = 2, 1024, 256, 16, 2, 256
+    wl = synth.Workload("shards", G * T, d, E, k, f)
+    inp = synth.Inputs(wl)
+    x = inp.x()
+    wg = _bf16(E, d, 131, d ** -0.5)
+    wg[:3] = _bf16(3, d, 132, 3 * d ** -0.5)                # hot experts: the capacity binds
+    W1, W3, W2 = inp.w1(), inp.w3(), inp.w2()
+    C = moe.moe_capacity(G * T, E, k, 1.0, moe.MOE_CAP_PER_ASSIGNMENT)
+    dv = to_dev_bf16
+    Wd = [dv(W1), dv(W3), dv(W2)]
+    ws = [_ws(moe, T, d, E, k, f) for _ in range(G)]
+    xs = [dv(x[g * T:(g + 1) * T]) for g in range(G)]
+    outs = [torch.empty((T, d), dtype=torch.bfloat16, device="cuda") for _ in range(G)]
+    L = moe.moe_workspace_layout(T, d, E, k, f)
+    for g in range(G):
+        moe.moe_layer_route_count(xs[g], dv(wg), None, 0, T, d, E, k, f, ws[g])
+    all_counts = torch.stack([moe.workspace_view(ws[g], L, "counts_raw", (E,), torch.int32) for g in range(G)])
+    fill = torch.empty((G, E), dtype=torch.int32, device="cuda")
+    for g in range(G):
+        moe.moe_fill_base(all_counts, G, g, E, fill[g])
+        moe.moe_layer_finish(xs[g], *Wd, None, None, None, 0, T, d, E, k, f, C, fill[g], outs[g], ws[g])
+    assert moe.moe_get_error() == 0
+    logits = np.concatenate([moe.workspace_view(ws[g], L, "logits", (T, E), torch.float32).cpu().numpy()
+                             for g in range(G)])
+    ref = oracle.layer_forward(x, wg, W1, W3, W2, k=k, C=C, logits_in=logits)
+    assert (ref["counts_raw"] > C).any()
+    assert np.array_equal(fill[1].cpu().numpy(), all_counts[0].cpu().numpy())
+    kept = 0
+    for g in range(G):
+        dest = moe.workspace_view(ws[g], L, "dest", (T, k), torch.int32).cpu().numpy()
+        assert np.array_equal(dest >= 0, ref["dest"][g * T:(g + 1) * T] >= 0)
+        kept += int((dest >= 0).sum())
+        assert_layer_close(bf16_bits(outs[g]), ref["out"][g * T:(g + 1) * T], f"shard {g}")
+    assert kept == ref["N"]

@@ -376,3 +376,34 @@ def test_layer_routes_supplied_logits():
     r = oracle.layer_forward(x, wg, W1, W3, W2, k=k, logits_in=logits)
     i2, _ = oracle.route(logits, k)
     assert np.array_equal(r["idx"], i2) and np.array_equal(r["logits"], logits)
+
+
+# --------------------------------------------------------------------------- overflow bias update
+
+def test_update_bias_closed_forms():
+    C = 200
+    counts = np.array([0, 100, 200, 300, 400, 1000, 50], np.int32)
+    b = oracle.update_bias(counts, C)
+    assert list(b) == [1.0, 0.5, 0.0, -0.5, -1.0, -1.0, 0.75]      # -clamp((c - C) / C, -1, 1)
+    assert np.signbit(b[2])                                          # -(+0) in fp32
+    with pytest.raises(ValueError):
+        oracle.update_bias(counts, 0)
+
+
+def test_update_bias_steers_load_away_from_overloaded_experts():
+    # route a batch, derive the bias from its overflow, route the next batch with it:
+    # the expert that overflowed most loses assignments, the idlest one gains
+    T, E, k = 4000, 16, 2
+    skew = np.linspace(1.0, -1.0, E).astype(np.float32)             # expert 0 popular, 15 idle
+    l1 = (RNG.standard_normal((T, E)) * 0.5 + skew).astype(np.float32)
+    l2 = (RNG.standard_normal((T, E)) * 0.5 + skew).astype(np.float32)
+    C = oracle.capacity(T, E, k, 2.0, oracle.CAP_PER_TOKEN)         # eval capacity factor 2.0
+    i1, _ = oracle.route(l1, k)
+    c1 = oracle.dispatch(i1, E, C)["counts_raw"]
+    bias = oracle.update_bias(c1, C)
+    i2, _ = oracle.route(l2, k, bias)
+    c2 = oracle.dispatch(i2, E, C)["counts_raw"]
+    i2n, _ = oracle.route(l2, k)
+    c2n = oracle.dispatch(i2n, E, C)["counts_raw"]
+    assert c1[0] > C and bias[0] < 0 and bias[-1] > 0
+    assert c2[0] < c2n[0] and c2[-1] > c2n[-1]
