@@ -49,7 +49,7 @@ DESCR = {
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="mixtral", choices=list(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -303,27 +303,29 @@ def main():
     N = int(counts.sum())
     touched = int((counts > 0).sum())
 
-    # end to end through the public API: pinned host input -> layer -> host output, every step
+    # end to end through the public API: every step copies its batch from pinned host memory to
+    # the device and its output back, in the library's host-buffer pipeline (the copies of the
+    # neighbouring batches overlap the layer); timed from the first copy in to the last copy out
     x_pin = x_host.pin_memory()
     out_pin = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
-    x_e2e = torch.empty_like(x)
-    for _ in range(2):
-        x_e2e.copy_(x_pin, non_blocking=True)
-        moe.moe_layer_forward(x_e2e, W["wg"], W["bias"], W["w1"], W["w3"], W["w2"], W.get("w1s"), W.get("w3s"),
-                              W.get("w2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, out, ws)
-        out_pin.copy_(out, non_blocking=True)
+    pmem = torch.empty(moe.moe_pipeline_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device=dev)
+    pl = moe.Pipeline(W["wg"], W["bias"], W["w1"], W["w3"], W["w2"], W.get("w1s"), W.get("w3s"), W.get("w2s"),
+                      fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, pmem)
+    s_h2d, _, s_d2h = pl.streams()
+    for _ in range(3):
+        pl.submit(x_pin, out_pin)
+    pl.sync()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    e0.record()
+    e0.record(torch.cuda.ExternalStream(s_h2d))
     for _ in range(K):
-        x_e2e.copy_(x_pin, non_blocking=True)
-        moe.moe_layer_forward(x_e2e, W["wg"], W["bias"], W["w1"], W["w3"], W["w2"], W.get("w1s"), W.get("w3s"),
-                              W.get("w2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, out, ws)
-        out_pin.copy_(out, non_blocking=True)
-    e1.record()
+        pl.submit(x_pin, out_pin)
+    e1.record(torch.cuda.ExternalStream(s_d2h))
+    pl.sync()
     torch.cuda.synchronize()
+    pl.close()
     e2e_ms = dp.max_over_ranks(e0.elapsed_time(e1), device=dev)
     if world > 1:
         dist.barrier()
@@ -350,6 +352,8 @@ def main():
         achieved = alg / (g1_ms / 1000.0) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"]}
+    if not decode:   # the same achieved rate against the power-capped sustained GEMM rate, for context
+        roof["frac_of_sustained"] = achieved / peaks["bf16_tflops_sustained"]
     roof["traffic"] = recorded_traffic("gate_up", wl.name)
     pair = T * k >= 256 * E
     roof["kernel"] = ("grouped_gemm_pair_kernel<EPI_SWIGLU>" if pair else "grouped_gemm_kernel<EPI_SWIGLU>") + \

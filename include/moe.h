@@ -232,6 +232,39 @@ int moe_layer_finish(const moe_bf16* x, const moe_bf16* W1, const moe_bf16* W3, 
 int moe_update_bias(const int32_t* counts_raw, int E, int64_t capacity, float* bias, moe_stream_t stream);
 
 /*
+ * Host-buffer pipeline: hidden-state batches in (pinned) host memory run through the layer
+ * with the copy of the next batch to the device and of the previous result back to the
+ * host overlapping the current batch's layer (two device slots, three streams: copy in,
+ * layer, copy out).  Layer parameters are fixed per pipeline; all pointers in the params
+ * are device pointers as for moe_layer_forward(), except nothing here is a batch.
+ *   moe_pipeline_bytes():   device memory the pipeline needs (2 input + 2 output slots of
+ *                           T*d bf16 and one layer workspace); the caller allocates it.
+ *   moe_pipeline_create():  binds the params and that memory; creates streams and events.
+ *   moe_pipeline_submit():  enqueues one batch: x_host [T,d] -> layer -> out_host [T,d].
+ *                           Returns at once; both host buffers must stay valid (and x_host
+ *                           unchanged) until moe_pipeline_sync().  Pinned memory makes the
+ *                           copies asynchronous.
+ *   moe_pipeline_sync():    waits for every submitted batch.
+ *   moe_pipeline_streams(): the three streams (e.g. to record timing events).
+ *   moe_pipeline_destroy(): syncs, then releases streams and events (not the caller's memory).
+ */
+typedef struct moe_pipeline_params {
+    const moe_bf16 *Wg, *W1, *W3, *W2;          /* routed experts and router */
+    const moe_bf16 *W1s, *W3s, *W2s;            /* shared expert, NULL if f_shared == 0 */
+    const float* bias;                          /* selection bias [E] or NULL */
+    int T, d, E, k, f, f_shared;
+    double capacity_factor;
+    int cap_mode;
+} moe_pipeline_params;
+typedef struct moe_pipeline moe_pipeline;
+int moe_pipeline_bytes(int T, int d, int E, int k, int f, int f_shared, size_t* bytes);
+int moe_pipeline_create(const moe_pipeline_params* params, void* dev_mem, size_t dev_bytes, moe_pipeline** out);
+int moe_pipeline_submit(moe_pipeline* pipeline, const moe_bf16* x_host, moe_bf16* out_host);
+int moe_pipeline_sync(moe_pipeline* pipeline);
+int moe_pipeline_streams(moe_pipeline* pipeline, moe_stream_t* h2d, moe_stream_t* compute, moe_stream_t* d2h);
+int moe_pipeline_destroy(moe_pipeline* pipeline);
+
+/*
  * Byte offsets of the intermediates that moe_layer_forward() leaves in its workspace,
  * so that a caller (a test) can read them after the call:
  *   off[0] logits [T,E] fp32   off[1] idx [T,k] int32   off[2] w [T,k] fp32

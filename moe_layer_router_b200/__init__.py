@@ -70,6 +70,15 @@ _lib.moe_fill_base.restype = _i32
 _lib.moe_layer_finish.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i64, _vp,
                                   _vp, _vp, _sz, _vp]
 _lib.moe_layer_finish.restype = _i32
+_lib.moe_pipeline_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(_sz)]
+_lib.moe_pipeline_create.argtypes = [_vp, _vp, _sz, ctypes.POINTER(_vp)]
+_lib.moe_pipeline_submit.argtypes = [_vp, _vp, _vp]
+_lib.moe_pipeline_sync.argtypes = [_vp]
+_lib.moe_pipeline_streams.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp)]
+_lib.moe_pipeline_destroy.argtypes = [_vp]
+for _n in ("moe_pipeline_bytes", "moe_pipeline_create", "moe_pipeline_submit", "moe_pipeline_sync",
+           "moe_pipeline_streams", "moe_pipeline_destroy"):
+    getattr(_lib, _n).restype = _i32
 _lib.moe_update_bias.argtypes = [_vp, _i32, _i64, _vp, _vp]
 _lib.moe_update_bias.restype = _i32
 _lib.moe_get_error.argtypes = [_vp]
@@ -212,6 +221,57 @@ def moe_layer_finish(x, W1, W3, W2, W1s, W3s, W2s, f_shared, T, d, E, k, f, capa
 
 def moe_update_bias(counts_raw, E, capacity, bias, stream=None) -> None:
     _check(_lib.moe_update_bias(_ptr(counts_raw), E, int(capacity), _ptr(bias), _stream(stream)), "moe_update_bias")
+
+
+class moe_pipeline_params(ctypes.Structure):
+    _fields_ = [("Wg", _vp), ("W1", _vp), ("W3", _vp), ("W2", _vp), ("W1s", _vp), ("W3s", _vp), ("W2s", _vp),
+                ("bias", _vp), ("T", _i32), ("d", _i32), ("E", _i32), ("k", _i32), ("f", _i32), ("f_shared", _i32),
+                ("capacity_factor", _dbl), ("cap_mode", _i32)]
+
+
+def moe_pipeline_bytes(T, d, E, k, f, f_shared=0) -> int:
+    out = _sz(0)
+    _check(_lib.moe_pipeline_bytes(T, d, E, k, f, f_shared, ctypes.byref(out)), "moe_pipeline_bytes")
+    return int(out.value)
+
+
+class Pipeline:
+    """moe_pipeline_* as an object: submit(x_host, out_host) per batch, sync() to wait.
+    dev_mem is a caller-owned device buffer of moe_pipeline_bytes() bytes; weights stay
+    referenced (keep the tensors alive)."""
+
+    def __init__(self, Wg, bias, W1, W3, W2, W1s, W3s, W2s, f_shared, T, d, E, k, f, capacity_factor, cap_mode,
+                 dev_mem):
+        self._keep = (Wg, bias, W1, W3, W2, W1s, W3s, W2s, dev_mem)
+        self.params = moe_pipeline_params(_ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(W1s), _ptr(W3s), _ptr(W2s),
+                                          _ptr(bias), T, d, E, k, f, f_shared, float(capacity_factor), cap_mode)
+        h = _vp()
+        _check(_lib.moe_pipeline_create(ctypes.byref(self.params), _ptr(dev_mem), _nbytes(dev_mem), ctypes.byref(h)),
+               "moe_pipeline_create")
+        self.handle = h
+
+    def submit(self, x_host, out_host) -> None:
+        _check(_lib.moe_pipeline_submit(self.handle, _ptr(x_host), _ptr(out_host)), "moe_pipeline_submit")
+
+    def sync(self) -> None:
+        _check(_lib.moe_pipeline_sync(self.handle), "moe_pipeline_sync")
+
+    def streams(self):
+        a, b, c = _vp(), _vp(), _vp()
+        _check(_lib.moe_pipeline_streams(self.handle, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
+               "moe_pipeline_streams")
+        return a.value, b.value, c.value
+
+    def close(self) -> None:
+        if self.handle:
+            _lib.moe_pipeline_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def moe_get_error(stream=None) -> int:

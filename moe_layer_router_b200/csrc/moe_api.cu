@@ -715,5 +715,7 @@ const char* moe_strerror(int code) {
 
 }  // extern "C"
 
-// The no-allocation variant of moe_permute shares this translation unit.
+// The host-buffer pipeline and the no-allocation variant of moe_permute share this
+// translation unit.
+#include "pipeline.cuh"
 #include "moe_noalloc.cu"

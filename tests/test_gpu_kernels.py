@@ -351,3 +351,33 @@ def test_sharded_batch_with_global_capacity_matches_whole_batch(moe):
         kept += int((dest >= 0).sum())
         assert_layer_close(bf16_bits(outs[g]), ref["out"][g * T:(g + 1) * T], f"shard {g}")
     assert kept == ref["N"]
+
+
+# ----------------------------------------------------------------------------- host-buffer pipeline
+
+def test_pipeline_matches_layer_forward_batch_by_batch(moe):
+    wl = synth.Workload("pipe", 512, 256, 8, 2, 384, f_shared=128, bias_range=0.1,
+                        cap_mode=synth.CAP_PER_TOKEN, capacity_factor=1.5)
+    T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
+    inp = synth.Inputs(wl)
+    dv = to_dev_bf16
+    Wg, W1, W3, W2 = dv(inp.wg()), dv(inp.w1()), dv(inp.w3()), dv(inp.w2())
+    W1s, W3s, W2s = dv(inp.shared("w1s")), dv(inp.shared("w3s")), dv(inp.shared("w2s"))
+    bias = torch.from_numpy(inp.bias()).cuda()
+    nb = 5
+    xs = [torch.from_numpy(inp.x_rows(b * T, T).view(np.int16)).view(torch.bfloat16).reshape(T, d).pin_memory()
+          for b in range(nb)]
+    outs = [torch.zeros((T, d), dtype=torch.bfloat16).pin_memory() for _ in range(nb)]
+    mem = torch.empty(moe.moe_pipeline_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device="cuda")
+    pl = moe.Pipeline(Wg, bias, W1, W3, W2, W1s, W3s, W2s, fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, mem)
+    for b in range(nb):
+        pl.submit(xs[b], outs[b])
+    pl.sync()
+    pl.close()
+    ws = _ws(moe, T, d, E, k, f, fs)
+    ref = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    for b in range(nb):
+        moe.moe_layer_forward(xs[b].cuda(), Wg, bias, W1, W3, W2, W1s, W3s, W2s, fs, T, d, E, k, f,
+                              wl.capacity_factor, wl.cap_mode, ref, ws)
+        assert torch.equal(outs[b].view(torch.int16), ref.cpu().view(torch.int16)), f"batch {b}"
+    assert moe.moe_get_error() == 0
