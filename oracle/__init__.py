@@ -59,6 +59,9 @@ def lib():
         L.oracle_update_bias.restype = i32
         L.oracle_expert_ffn.argtypes = [vp, i32, vp, vp, vp, i32, i32, vp, vp]
         L.oracle_combine.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp]
+        L.oracle_e4m3.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3.restype = dbl
+        L.oracle_expert_ffn_q8.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp]
         L.oracle_layer_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
                                            i32, i32, i32, i32, i32, i64,
                                            vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
@@ -145,6 +148,25 @@ def expert_ffn(x: np.ndarray, W1: np.ndarray, W3: np.ndarray, W2: np.ndarray):
     h = np.empty((rows, f), np.uint16)
     y = np.empty((rows, d), np.uint16)
     lib().oracle_expert_ffn(_p(x), rows, _p(W1), _p(W3), _p(W2), d, f, _p(h), _p(y))
+    return h, y
+
+
+def e4m3(b: int) -> float:
+    return float(lib().oracle_e4m3(int(b)))
+
+
+def expert_ffn_q8(x, W1q, s1, W3q, s3, W2q, s2):
+    """One expert with fp8 e4m3 weights and fp32 row scales: -> (h, y) bf16."""
+    x = _c(x, np.uint16)
+    W1q = _c(W1q, np.uint8); W3q = _c(W3q, np.uint8); W2q = _c(W2q, np.uint8)
+    s1 = _c(s1, np.float32); s3 = _c(s3, np.float32); s2 = _c(s2, np.float32)
+    rows, d = x.shape
+    f = W1q.shape[0]
+    assert W1q.shape == (f, d) and W3q.shape == (f, d) and W2q.shape == (d, f)
+    assert s1.shape == (f,) and s3.shape == (f,) and s2.shape == (d,)
+    h = np.empty((rows, f), np.uint16)
+    y = np.empty((rows, d), np.uint16)
+    lib().oracle_expert_ffn_q8(_p(x), rows, _p(W1q), _p(s1), _p(W3q), _p(s3), _p(W2q), _p(s2), d, f, _p(h), _p(y))
     return h, y
 
 

@@ -242,6 +242,47 @@ void oracle_expert_ffn(const uint16_t* x, int rows, const uint16_t* W1, const ui
     }
 }
 
+/*
+ * Low-bit expert weights (the "low-bit expert weights for decode" extension of the
+ * deployment page's quantization option): each weight is one fp8 e4m3 byte q and each
+ * output row n one fp32 scale s_n; the weight is e4m3(q) * s_n.
+ *   e4m3 ("fn"): sign | 4 exponent bits (bias 7) | 3 mantissa bits; exponent 0 is subnormal
+ *   (m * 2^-9); exponent 15 with mantissa 7 is NaN; no infinities.
+ */
+double oracle_e4m3(uint8_t b) {
+    int sgn = b >> 7, e = (b >> 3) & 15, m = b & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+/* oracle_expert_ffn with W1 = e4m3(W1q) * s1 (row scales [f]), W3 likewise, W2 = e4m3(W2q) * s2 ([d]). */
+void oracle_expert_ffn_q8(const uint16_t* x, int rows, const uint8_t* W1q, const float* s1, const uint8_t* W3q,
+                          const float* s3, const uint8_t* W2q, const float* s2, int d, int f, uint16_t* h, uint16_t* y) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < rows; ++r) {
+        const uint16_t* xr = x + (size_t)r * d;
+        uint16_t* hr = h + (size_t)r * f;
+        for (int n = 0; n < f; ++n) {
+            double g = 0.0, u = 0.0;
+            for (int i = 0; i < d; ++i) {
+                double xi = bf(xr[i]);
+                g += xi * (oracle_e4m3(W1q[(size_t)n * d + i]) * (double)s1[n]);
+                u += xi * (oracle_e4m3(W3q[(size_t)n * d + i]) * (double)s3[n]);
+            }
+            double silu = g / (1.0 + exp(-g));
+            hr[n] = bf16_round(silu * u);
+        }
+        for (int m = 0; m < d; ++m) {
+            double acc = 0.0;
+            for (int n = 0; n < f; ++n) acc += bf(hr[n]) * (oracle_e4m3(W2q[(size_t)m * f + n]) * (double)s2[m]);
+            y[(size_t)r * d + m] = bf16_round(acc);
+        }
+    }
+}
+
 /* ---- combine ------------------------------------------------------------------------ */
 
 /*

@@ -66,6 +66,7 @@ def lib():
         L.synth_uniform_f32.argtypes = [u32, u32, u64, u64, dbl, dbl, vp]
         L.synth_shifted_bf16.argtypes = [u32, u32, u64, u64, u64, dbl, vp, vp, vp]
         L.synth_zipf_shift.argtypes = [u32, u32, u32, i32, i32, dbl, dbl, vp, vp, i32, i32, vp]
+        L.synth_quantize_e4m3_rows.argtypes = [vp, u64, u64, vp, vp]
         _lib = L
     return _lib
 
@@ -112,6 +113,16 @@ def shifted_bf16(seed: int, tid: int, row0: int, nrows: int, ncols: int, std: fl
         out = np.empty(nrows * ncols, dtype=np.uint16)
     lib().synth_shifted_bf16(seed, tid, row0, nrows, ncols, float(std), _p(shift), _p(u), _p(out))
     return out
+
+
+def quantize_e4m3_rows(w: np.ndarray, K: int):
+    """bf16 rows [rows, K] -> (fp8 e4m3 bytes [rows, K] uint8, fp32 scale per row)."""
+    w = np.ascontiguousarray(w, dtype=np.uint16).reshape(-1, K)
+    rows = w.shape[0]
+    q = np.empty((rows, K), dtype=np.uint8)
+    s = np.empty(rows, dtype=np.float32)
+    lib().synth_quantize_e4m3_rows(_p(w), rows, K, _p(q), _p(s))
+    return q, s
 
 
 def bf16_bits_to_f32(a: np.ndarray) -> np.ndarray:

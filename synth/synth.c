@@ -187,3 +187,58 @@ void synth_zipf_shift(uint32_t seed, uint32_t tid_g, uint32_t tid_s, int E, int 
     }
     free(cnt); free(target); free(g); free(sv);
 }
+
+/*
+ * fp8 e4m3 ("fn" variant: no infinities, max 448) quantisation of bf16 weight rows, one fp32
+ * scale per row: s_r = max_i |w_ri| / 448 (1 for an all-zero row), q_ri = e4m3(w_ri / s_r)
+ * rounded to nearest even.  This turns the synthetic bf16 checkpoint into the low-bit one;
+ * the layer's arithmetic (dequantised weight = e4m3(q) * s) is defined elsewhere.
+ */
+static uint8_t f32_to_e4m3_rne(float v) {
+    uint32_t bits;
+    memcpy(&bits, &v, 4);
+    uint8_t sign = (uint8_t)((bits >> 24) & 0x80u);
+    float a = fabsf(v);
+    if (a != a) return 0x7F;                        /* NaN */
+    if (a >= 464.0f) return sign | 0x7E;            /* saturate to 448 */
+    if (a < 0x1p-10f) return sign;                  /* below half the smallest subnormal (2^-9) */
+    int ex;
+    frexpf(a, &ex);                                 /* a = m * 2^ex, 0.5 <= m < 1 */
+    int e = ex - 1;                                 /* a = 1.f * 2^e */
+    if (e < -6) e = -6;                             /* subnormal range: quantum 2^-9 */
+    float quantum = ldexpf(1.0f, e - 3);            /* 3 mantissa bits */
+    float r = nearbyintf(a / quantum) * quantum;    /* ties to even (exact division by 2^k) */
+    if (r >= 464.0f) return sign | 0x7E;
+    if (r == 0.0f) return sign;
+    int er;
+    float mr = frexpf(r, &er);
+    int E = er - 1;
+    if (E < -6) {                                   /* subnormal: r = m * 2^-9, m in 1..7 */
+        int m = (int)(r / 0x1p-9f);
+        return sign | (uint8_t)m;
+    }
+    int mant = (int)((mr * 2.0f - 1.0f) * 8.0f + 0.5f);
+    return sign | (uint8_t)(((E + 7) << 3) | mant);
+}
+
+void synth_quantize_e4m3_rows(const uint16_t* w, uint64_t rows, uint64_t K, uint8_t* q, float* scale) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < (int64_t)rows; ++r) {
+        const uint16_t* wr = w + (uint64_t)r * K;
+        float amax = 0.0f;
+        for (uint64_t i = 0; i < K; ++i) {
+            uint32_t b = (uint32_t)wr[i] << 16;
+            float f;
+            memcpy(&f, &b, 4);
+            if (fabsf(f) > amax) amax = fabsf(f);
+        }
+        float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+        scale[r] = s;
+        for (uint64_t i = 0; i < K; ++i) {
+            uint32_t b = (uint32_t)wr[i] << 16;
+            float f;
+            memcpy(&f, &b, 4);
+            q[(uint64_t)r * K + i] = f32_to_e4m3_rne(f / s);
+        }
+    }
+}

@@ -407,3 +407,52 @@ def test_update_bias_steers_load_away_from_overloaded_experts():
     c2n = oracle.dispatch(i2n, E, C)["counts_raw"]
     assert c1[0] > C and bias[0] < 0 and bias[-1] > 0
     assert c2[0] < c2n[0] and c2[-1] > c2n[-1]
+
+
+# --------------------------------------------------------------------------- fp8 e4m3 expert weights
+
+def test_e4m3_decode_matches_torch_for_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ours = np.array([oracle.e4m3(int(c)) for c in codes])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan) and nan.sum() == 2          # 0x7F, 0xFF
+    assert np.array_equal(ours[~nan], ref[~nan])
+    assert oracle.e4m3(0x7E) == 448.0 and oracle.e4m3(0x01) == 2.0 ** -9 and oracle.e4m3(0x38) == 1.0
+
+
+def test_q8_expert_equals_bf16_expert_on_representable_weights():
+    # scales that are powers of two make e4m3(q) * s exactly a bf16 value: the fp8 expert must
+    # then equal the (pinned) bf16 expert bit for bit
+    rows, d, f = 12, 64, 96
+    x = rand_bf16((rows, d))
+    q = lambda shape: RNG.integers(0, 256, shape).astype(np.uint8)
+    W1q, W3q, W2q = q((f, d)), q((f, d)), q((d, f))
+    for W in (W1q, W3q, W2q):
+        W[(W & 0x7F) == 0x7F] = 0x38                                       # no NaN codes
+    s1 = (2.0 ** RNG.integers(-12, -6, f)).astype(np.float32)
+    s3 = (2.0 ** RNG.integers(-12, -6, f)).astype(np.float32)
+    s2 = (2.0 ** RNG.integers(-12, -6, d)).astype(np.float32)
+    deq = lambda Wq, s: bf16_bits((torch.from_numpy(Wq).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+                                   * s[:, None]).astype(np.float32))
+    h_q, y_q = oracle.expert_ffn_q8(x, W1q, s1, W3q, s3, W2q, s2)
+    h_b, y_b = oracle.expert_ffn(x, deq(W1q, s1), deq(W3q, s3), deq(W2q, s2))
+    assert np.array_equal(h_q, h_b) and np.array_equal(y_q, y_b)
+
+
+def test_q8_expert_vs_textbook_dequantised():
+    rows, d, f = 10, 128, 64
+    x = rand_bf16((rows, d))
+    w = lambda shape, std: rand_bf16(shape, std)
+    import synth
+    W1q, s1 = synth.quantize_e4m3_rows(w((f, d), d ** -0.5), d)
+    W3q, s3 = synth.quantize_e4m3_rows(w((f, d), d ** -0.5), d)
+    W2q, s2 = synth.quantize_e4m3_rows(w((d, f), f ** -0.5), f)
+    h, y = oracle.expert_ffn_q8(x, W1q, s1, W3q, s3, W2q, s2)
+    deq = lambda Wq, s: torch.from_numpy(Wq).view(torch.float8_e4m3fn).to(torch.float64) * torch.from_numpy(s).double()[:, None]
+    X = torch.from_numpy(bf16_to_f64(x))
+    g, u = X @ deq(W1q, s1).T, X @ deq(W3q, s3).T
+    hh = torch_bf16_round_f64(torch.nn.functional.silu(g) * u)
+    yy = torch_bf16_round_f64(hh.double() @ deq(W2q, s2).T)
+    to_bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)
+    assert ulp_diff_bf16(h, to_bits(hh)).max() <= 1 and ulp_diff_bf16(y, to_bits(yy)).max() <= 1
