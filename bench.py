@@ -53,6 +53,13 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="mixtral", choices=list(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
+                    help="expert weight format: bf16, or fp8 e4m3 with fp32 row scales (moe_layer_forward_w8)")
+    ap.add_argument("--cache-slots", type=int, default=0,
+                    help="> 0: decode through the expert cache (moe_layer_forward_cached) with this many HBM "
+                         "slots; expert weights in page-locked host memory; a fresh token batch every step")
+    ap.add_argument("--cache-tokens", type=int, default=16, help="decode batch (tokens per step) with --cache-slots")
+    ap.add_argument("--cache-zipf", type=float, default=1.0, help="Zipf exponent of expert popularity (cache runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
@@ -217,21 +224,159 @@ def gemm1_work(wl, N):
     return flops
 
 
-def gemm1_bytes(wl, N, touched):
-    b = touched * 2.0 * wl.f * wl.d * 2            # W1, W3 of touched experts
+def gemm1_bytes(wl, N, touched, wbytes=2):
+    b = touched * 2.0 * wl.f * wl.d * wbytes        # W1, W3 of touched experts
+    if wbytes == 1:
+        b += touched * 2.0 * wl.f * 4                # row scales
     b += N * wl.d * 2 + N * wl.f * 2                # x_perm read, h write
     if wl.f_shared:
-        b += 2.0 * wl.f_shared * wl.d * 2 + wl.T * wl.d * 2 + wl.T * wl.f_shared * 2
+        b += 2.0 * wl.f_shared * wl.d * wbytes + wl.T * wl.d * 2 + wl.T * wl.f_shared * 2
     return b
 
 
-def layer_work(wl, N, touched):
+def layer_work(wl, N, touched, wbytes=2):
     flops = 6.0 * N * wl.d * wl.f + 2.0 * wl.T * wl.d * wl.E + 6.0 * wl.T * wl.d * wl.f_shared
-    b = touched * 3.0 * wl.f * wl.d * 2 + wl.E * wl.d * 2 + 3.0 * wl.f_shared * wl.d * 2
+    b = touched * 3.0 * wl.f * wl.d * wbytes + wl.E * wl.d * 2 + 3.0 * wl.f_shared * wl.d * wbytes
     b += wl.T * wl.d * 2 + 2 * N * wl.d * 2 + 2 * N * wl.f * 2 + 2 * N * wl.d * 2 + wl.T * wl.d * 2
     if wl.f_shared:
         b += 2 * wl.T * wl.f_shared * 2 + 2 * wl.T * wl.d * 2
     return flops, b
+
+
+def run_cached(args, base, rank, world, local):
+    """Decode with the routed experts in page-locked host memory and an LRU of S HBM slots.
+
+    One step = one moe_layer_forward_cached over a fresh batch of `--cache-tokens` tokens (the
+    router sees new tokens every step, so the cache sees real misses); the expert popularity
+    follows Zipf(`--cache-zipf`).  The dominant kernel is the copy of the missed experts over the
+    host link, so its roofline is that link: the bytes it moved over its event time, against a
+    pinned cudaMemcpyAsync host-to-device copy of 1 GiB measured in the same run."""
+    import dataclasses
+
+    import torch
+    import torch.distributed as dist
+    import moe_layer_router_b200 as moe
+    from moe_layer_router_b200 import dp
+
+    wl = dataclasses.replace(base, name=base.name + "_cached", T=args.cache_tokens, zipf_s=args.cache_zipf)
+    T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
+    S = args.cache_slots
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    W = synth.device_tensors(wl, dev, names=["wg", "w1", "w3", "w2", "w1s", "w3s", "w2s", "bias"])
+    host = {}
+    for n in ("w1", "w3", "w2"):          # the routed experts live in page-locked host memory
+        host[n] = torch.empty(W[n].shape, dtype=torch.bfloat16, pin_memory=True)
+        host[n].copy_(W[n])
+        del W[n]
+    torch.cuda.empty_cache()
+    slots = {n: torch.empty((S,) + tuple(host[n].shape[1:]), dtype=torch.bfloat16, device=dev)
+             for n in ("w1", "w3", "w2")}
+    state = torch.empty(moe.moe_cache_state_bytes(E, S), dtype=torch.uint8, device=dev)
+    moe.moe_cache_reset(state, E, S)
+    inp = synth.Inputs(wl)
+    nb = max(3, args.warmup) + args.steps
+    row0 = rank * nb * T
+    xs = torch.from_numpy(inp.x_rows(row0, nb * T).view(np.int16)).view(torch.bfloat16).reshape(nb, T, d).to(dev)
+    ws = torch.empty(moe.moe_workspace_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device=dev)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+
+    def fwd(i, events=None, xin=None):
+        moe.moe_layer_forward_cached(xs[i] if xin is None else xin, W["wg"], W["bias"], host["w1"], host["w3"], host["w2"], slots["w1"],
+                                     slots["w3"], slots["w2"], S, state, W.get("w1s"), W.get("w3s"), W.get("w2s"), fs,
+                                     T, d, E, k, f, wl.capacity_factor, wl.cap_mode, out, ws, events)
+
+    nw = max(3, args.warmup)
+    for i in range(nw):
+        fwd(i)
+    torch.cuda.synchronize()
+    if moe.moe_get_error() != 0:
+        raise RuntimeError("device error after warm-up")
+    c0 = moe.cache_counters(state)
+    K = args.steps
+    names = moe.STAGES + ["cache"]
+    evs = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(K)]
+    for e in evs:
+        for ev in e.values():
+            ev.record()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            fwd(nw + i, evs[i])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = dp.max_over_ranks(evs[0]["route"].elapsed_time(evs[K - 1]["end"]), device=dev)
+    order = ["route", "topk", "permute", "cache", "gate_up", "down", "combine", "end"]
+    stage_ms = {a: float(np.mean([e[a].elapsed_time(e[b]) for e in evs])) for a, b in zip(order[:-1], order[1:])}
+    c1 = moe.cache_counters(state)
+    expert_bytes = 3 * f * d * 2
+    hits, misses = c1["hits"] - c0["hits"], c1["misses"] - c0["misses"]
+    copy_ms = sum(e["cache"].elapsed_time(e["gate_up"]) for e in evs)   # plan + copy kernels, all steps
+    link_gbs = misses * expert_bytes / 1e9 / (copy_ms / 1e3)
+    # end to end: every step copies its tokens from page-locked host memory and its output back
+    x_pin = xs.cpu().pin_memory()
+    out_pin = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
+    xin = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(K):
+        xin.copy_(x_pin[nw + i], non_blocking=True)
+        fwd(0, None, xin)
+        out_pin.copy_(out, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = dp.max_over_ranks(e0.elapsed_time(e1), device=dev)
+    # the host link as a plain DMA copy sees it: 1 GiB page-locked -> device, 5 times
+    hsrc = torch.empty(1 << 30, dtype=torch.uint8, pin_memory=True)
+    ddst = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+    ddst.copy_(hsrc, non_blocking=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(5):
+        ddst.copy_(hsrc, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    dma_gbs = 5 * (1 << 30) / 1e9 / (e0.elapsed_time(e1) / 1e3)
+    if moe.moe_get_error() != 0:
+        raise RuntimeError("device error")
+    value = dp.job_throughput(T, world, K, total_ms)
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    line = {
+        "metric": "MoE-layer tokens/s on 1 B200, routed experts served from an HBM expert cache",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": nw,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded Philox4x32-10 + Box-Muller; random-init weights)",
+        "config": {"workload": f"DeepSeek-V3-like decode T={T} d={d} E={E} top-{k} f={f} + shared f={fs}, "
+                               f"Zipf({wl.zipf_s}) expert popularity, fresh tokens every step; routed experts in "
+                               f"page-locked host memory ({E * expert_bytes / 1e9:.1f} GB), {S} HBM slots",
+                   "global_batch": world * T, "seq_len": T, "parallelism": f"dp{world}", "cache_slots": S,
+                   "l2": "working set larger than L2 (expert weights streamed from host memory and HBM)"},
+        "roofline": {"bound": "host_link", "achieved": link_gbs, "peak": dma_gbs, "unit": "GB/s",
+                     "frac": link_gbs / dma_gbs if dma_gbs else None, "traffic": None,
+                     "kernel": "cache_load_kernel (missed experts' W1/W3/W2, host memory -> HBM slots)",
+                     "peak_source": "measured in this run (cudaMemcpyAsync page-locked -> device, 1 GiB x 5)",
+                     "algorithmic_per_launch": misses / K * expert_bytes},
+        "cache": {"hits": hits, "misses": misses, "hit_rate": hits / max(1, hits + misses),
+                  "loads_per_step": misses / K, "expert_mb": expert_bytes / 1e6},
+        "stages_ms": stage_ms,
+        "e2e": {"value": dp.job_throughput(T, world, K, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
+                "d2h_bytes_per_step": T * d * 2},
+        "gpu_launches": (KERNELS_PER_STEP + 2) * K,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
 
 
 def main():
@@ -242,6 +387,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, wl, rank, world)
+    if args.cache_slots > 0:
+        return run_cached(args, wl, rank, world, local)
 
     import torch
     import torch.distributed as dist
@@ -254,7 +401,11 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
     # inputs: replicated weights, a distinct token batch per rank
-    tensors = synth.device_tensors(wl, dev, names=["wg", "w1", "w3", "w2", "w1s", "w3s", "w2s", "bias"])
+    fp8 = args.weights == "fp8"
+    tensors = synth.device_tensors(wl, dev, names=["wg", "bias"] if fp8 else
+                                   ["wg", "w1", "w3", "w2", "w1s", "w3s", "w2s", "bias"])
+    if fp8:
+        tensors.update(synth.device_tensors_q8(wl, dev))
     inp = synth.Inputs(wl)
     row0, nrows = dp.token_rows(rank, world, wl.T)
     x_host = torch.from_numpy(inp.x_rows(row0, nrows).view(np.int16)).view(torch.bfloat16).reshape(wl.T, wl.d)
@@ -265,8 +416,13 @@ def main():
     W = tensors
 
     def fwd(xin, o, events=None):
-        moe.moe_layer_forward_ex(xin, W["wg"], W["bias"], W["w1"], W["w3"], W["w2"], W.get("w1s"), W.get("w3s"),
-                                 W.get("w2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, o, ws, events)
+        if fp8:
+            moe.moe_layer_forward_w8(xin, W["wg"], W["bias"], W["w1q"], W["s1"], W["w3q"], W["s3"], W["w2q"], W["s2"],
+                                     W.get("w1sq"), W.get("s1s"), W.get("w3sq"), W.get("s3s"), W.get("w2sq"),
+                                     W.get("s2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, o, ws, events)
+        else:
+            moe.moe_layer_forward_ex(xin, W["wg"], W["bias"], W["w1"], W["w3"], W["w2"], W.get("w1s"), W.get("w3s"),
+                                     W.get("w2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, o, ws, events)
 
     for _ in range(max(3, args.warmup)):
         fwd(x, out)
@@ -308,25 +464,40 @@ def main():
     # neighbouring batches overlap the layer); timed from the first copy in to the last copy out
     x_pin = x_host.pin_memory()
     out_pin = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
-    pmem = torch.empty(moe.moe_pipeline_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device=dev)
-    pl = moe.Pipeline(W["wg"], W["bias"], W["w1"], W["w3"], W["w2"], W.get("w1s"), W.get("w3s"), W.get("w2s"),
-                      fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, pmem)
-    s_h2d, _, s_d2h = pl.streams()
-    for _ in range(3):
-        pl.submit(x_pin, out_pin)
-    pl.sync()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0.record(torch.cuda.ExternalStream(s_h2d))
-    for _ in range(K):
-        pl.submit(x_pin, out_pin)
-    e1.record(torch.cuda.ExternalStream(s_d2h))
-    pl.sync()
-    torch.cuda.synchronize()
-    pl.close()
-    e2e_ms = dp.max_over_ranks(e0.elapsed_time(e1), device=dev)
+    if fp8:   # the pipeline object takes bf16 weights: copies around each call on one stream
+        x_e2e = torch.empty_like(x)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(K):
+            x_e2e.copy_(x_pin, non_blocking=True)
+            fwd(x_e2e, out)
+            out_pin.copy_(out, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        return_e2e = dp.max_over_ranks(e0.elapsed_time(e1), device=dev)
+    pmem = torch.empty(0 if fp8 else moe.moe_pipeline_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device=dev)
+    if fp8:
+        e2e_ms = return_e2e
+    else:
+        pl = moe.Pipeline(W["wg"], W["bias"], W["w1"], W["w3"], W["w2"], W.get("w1s"), W.get("w3s"), W.get("w2s"),
+                          fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, pmem)
+        s_h2d, _, s_d2h = pl.streams()
+        for _ in range(3):
+            pl.submit(x_pin, out_pin)
+        pl.sync()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(torch.cuda.ExternalStream(s_h2d))
+        for _ in range(K):
+            pl.submit(x_pin, out_pin)
+        e1.record(torch.cuda.ExternalStream(s_d2h))
+        pl.sync()
+        torch.cuda.synchronize()
+        pl.close()
+        e2e_ms = dp.max_over_ranks(e0.elapsed_time(e1), device=dev)
     if world > 1:
         dist.barrier()
     e2e_value = dp.job_throughput(T, world, K, e2e_ms)
@@ -343,7 +514,7 @@ def main():
     g1_ms = stage_ms["gate_up"]
     decode = wl.name.startswith("dsv3")
     if decode:
-        alg = gemm1_bytes(wl, N, touched)
+        alg = gemm1_bytes(wl, N, touched, 1 if fp8 else 2)
         achieved = alg / (g1_ms / 1000.0) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"]}
@@ -354,18 +525,20 @@ def main():
                 "frac": achieved / peaks["bf16_tflops"]}
     if not decode:   # the same achieved rate against the power-capped sustained GEMM rate, for context
         roof["frac_of_sustained"] = achieved / peaks["bf16_tflops_sustained"]
-    roof["traffic"] = recorded_traffic("gate_up", wl.name)
+    roof["traffic"] = recorded_traffic("gate_up" + ("_fp8" if fp8 else ""), wl.name)
     pair = T * k >= 256 * E
-    roof["kernel"] = ("grouped_gemm_pair_kernel<EPI_SWIGLU>" if pair else "grouped_gemm_kernel<EPI_SWIGLU>") + \
+    roof["kernel"] = ("grouped_gemm_w8_kernel<EPI_SWIGLU>" if fp8 else
+                      "grouped_gemm_pair_kernel<EPI_SWIGLU>" if pair else "grouped_gemm_kernel<EPI_SWIGLU>") + \
         " (gate_up: W1/W3 + SwiGLU)"
     roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if decode else 'bf16_tflops'}, burst)"
     roof["algorithmic_per_launch"] = alg
-    lf, lb = layer_work(wl, N, touched)
+    lf, lb = layer_work(wl, N, touched, 1 if fp8 else 2)
     step_s = total_ms / K / 1000.0
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic (seeded Philox4x32-10 + Box-Muller; random-init weights)",
+        "dtype": "bf16" if not fp8 else "bf16 activations, fp8 e4m3 expert weights",
+        "data": "synthetic (seeded Philox4x32-10 + Box-Muller; random-init weights)",
         "config": {"workload": DESCR[wl.name], "global_batch": world * T, "seq_len": T, "parallelism": f"dp{world}",
                    "l2": "working set larger than L2 (expert weights %.2f GB per step)" % (
                        touched * 3.0 * f * d * 2 / 1e9)},

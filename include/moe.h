@@ -184,12 +184,34 @@ typedef struct moe_stage_events {
     void* down;      /* before the second grouped GEMM (W2) */
     void* combine;   /* before the combine kernel */
     void* end;       /* after the combine kernel */
+    void* cache;     /* before the expert cache plan / copy kernels (moe_layer_forward_cached only) */
 } moe_stage_events;
 
 /* moe_layer_forward() with optional stage markers (events may be NULL). */
 int moe_layer_forward_ex(const moe_bf16* x, const moe_bf16* Wg, const float* bias,
                          const moe_bf16* W1, const moe_bf16* W3, const moe_bf16* W2,
                          const moe_bf16* W1s, const moe_bf16* W3s, const moe_bf16* W2s, int f_shared,
+                         int T, int d, int E, int k, int f, double capacity_factor, int cap_mode,
+                         moe_bf16* out, void* ws, size_t ws_bytes, moe_stream_t stream,
+                         const moe_stage_events* events);
+
+/*
+ * The layer with fp8 expert weights (the pages' low-bit quantization option for the expert
+ * weights, "low-bit expert weights for decode streaming"): every weight is one fp8 e4m3 byte
+ * q ("fn" encoding: no infinities, max 448) and every output row one fp32 scale, so the
+ * expert weight W[n, i] = e4m3(q[n, i]) * s[n].  The decode layer streams half the bytes of
+ * bf16 weights.  Everything else (router in bf16, routing, permutation, combine, rounding of
+ * h / y / out to bf16) is as in moe_layer_forward().
+ *   W1q, W3q [E, f, d] uint8, s1, s3 [E, f] fp32      gate / up
+ *   W2q [E, d, f] uint8, s2 [E, d] fp32                 down
+ *   W1sq, W3sq [f_shared, d], s1s, s3s [f_shared], W2sq [d, f_shared], s2s [d]: shared expert
+ *   (all NULL with f_shared = 0).  Same workspace as moe_layer_forward().
+ */
+int moe_layer_forward_w8(const moe_bf16* x, const moe_bf16* Wg, const float* bias,
+                         const uint8_t* W1q, const float* s1, const uint8_t* W3q, const float* s3,
+                         const uint8_t* W2q, const float* s2,
+                         const uint8_t* W1sq, const float* s1s, const uint8_t* W3sq, const float* s3s,
+                         const uint8_t* W2sq, const float* s2s, int f_shared,
                          int T, int d, int E, int k, int f, double capacity_factor, int cap_mode,
                          moe_bf16* out, void* ws, size_t ws_bytes, moe_stream_t stream,
                          const moe_stage_events* events);
@@ -263,6 +285,113 @@ int moe_pipeline_submit(moe_pipeline* pipeline, const moe_bf16* x_host, moe_bf16
 int moe_pipeline_sync(moe_pipeline* pipeline);
 int moe_pipeline_streams(moe_pipeline* pipeline, moe_stream_t* h2d, moe_stream_t* compute, moe_stream_t* d2h);
 int moe_pipeline_destroy(moe_pipeline* pipeline);
+
+/*
+ * The permutation alone, in the layer workspace (counts, offsets, dest, src_token, x_perm at
+ * their moe_workspace_layout() offsets): histogram, capacity with fill_base (as in
+ * moe_layer_finish), stable scatter and the gather of x_perm.  Needs the routing of
+ * moe_layer_route_count() in the same workspace.  Used by the expert-parallel path.
+ */
+int moe_layer_permute(const moe_bf16* x, int f_shared, int T, int d, int E, int k, int f, int64_t capacity,
+                      const int32_t* fill_base, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Expert parallelism: the E routed experts are split over R ranks, rank r holding experts
+ * [r El, (r + 1) El), El = E / R (uniform contiguous assignment).  [EP-KV] "MoE 推理中的 Expert
+ * Parallel、KV Cache 与大规模专家并行架构解析" sections 6-7: a layer sends each token's hidden
+ * state to the ranks of its experts and the expert outputs back to the token's rank, which
+ * combines them; all-to-all-v, point-to-point copies or fused kernels are all valid ways to move
+ * them.  [EP-DS3] section 3.1 (_assign_experts) gives the contiguous split.
+ *
+ * Per rank, per layer call (all asynchronous on `stream`):
+ *   1. moe_layer_route_count()                 routing and raw counts of the rank's T tokens
+ *   2. all-gather of counts_raw -> all_counts_raw [R, E] int32 on every rank (the caller's
+ *      collective; rank order = token order of the whole batch)
+ *   3. moe_fill_base() + moe_layer_permute()  global-capacity keep decisions, x_perm
+ *   4. moe_ep_plan()                           from all_counts_raw alone: the rows this rank
+ *      sends to / receives from every rank and the local GEMM segments (into ep_ws)
+ *      moe_ep_dispatch()                       puts this rank's x_perm rows into the receive
+ *      buffers of the experts' ranks; receive rows are in (source rank, local expert) order
+ *      (a caller with a collective library can move the same row ranges with an
+ *      all-to-all-v instead: rank r sends rows_kept(r, experts of q) to q, in q order)
+ *   5. a barrier (every rank's puts done before any rank reads its receive buffer)
+ *   6. moe_ep_expert_ffn()                     local experts over the received rows (one GEMM
+ *      segment per source rank and local expert) + the shared expert on the rank's own tokens
+ *   7. moe_ep_return()                         puts each result row back into the y_perm (layer
+ *      workspace) of the rank it came from, at the row it had in that rank's x_perm
+ *   8. a barrier, then moe_combine() with the rank's dest, w (layer workspace) and y_shared
+ * The output equals the single-GPU layer over the whole batch (capacity counted over all ranks).
+ *
+ * Buffers: recv_bufs / y_perm_bufs are host arrays of R device addresses, one per rank, that
+ * this device can write (peer-mapped buffers of other GPUs, or the same GPU's buffers when
+ * ranks share a device).  A receive buffer holds max_recv_rows rows of d bf16 (>= the rows the
+ * rank can receive: R * T * k bounds it).  ep_ws: moe_ep_workspace_bytes(E) bytes, 16-byte
+ * aligned, written by moe_ep_plan() and read by the later calls on the same rank.
+ * Errors: MOE_ERR_SHAPE unless 1 <= R <= 64, E % R == 0, E <= 1024, 0 <= rank < R.
+ */
+int moe_ep_workspace_bytes(int E, size_t* bytes);
+int moe_ep_plan(const int32_t* all_counts_raw, int R, int rank, int E, int64_t capacity, int max_recv_rows,
+                void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream);
+int moe_ep_dispatch(const moe_bf16* x_perm, int R, int rank, int E, int d, moe_bf16* const* recv_bufs,
+                    const void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream);
+int moe_ep_expert_ffn(const moe_bf16* recv_x, int max_recv_rows, int R, int rank, int E, int d, int f,
+                      const moe_bf16* W1_local, const moe_bf16* W3_local, const moe_bf16* W2_local, moe_bf16* h,
+                      moe_bf16* y_recv, const moe_bf16* x, int T, const moe_bf16* W1s, const moe_bf16* W3s,
+                      const moe_bf16* W2s, int f_shared, moe_bf16* h_shared, moe_bf16* y_shared, const void* ep_ws,
+                      size_t ep_ws_bytes, moe_stream_t stream);
+int moe_ep_return(const moe_bf16* y_recv, int R, int rank, int E, int d, moe_bf16* const* y_perm_bufs,
+                  const void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream);
+
+/*
+ * Expert cache: the routed experts' weights live in page-locked host memory and HBM holds S
+ * expert slots managed as an LRU.  [EP-DS3] "MoE 推理架构深度实战：从 Expert Parallelism 到
+ * DeepSeek-V3 的工程落地", section 3.2 (expert cache and preloading): inactive experts are
+ * kept in host memory, the experts a batch needs are loaded, the least recently used resident
+ * expert is evicted when the slots are full.  Readings where the page's sketch is open:
+ * recency is counted in batches (every expert a batch keeps at least one row for is stamped
+ * with the batch number, hit or miss); misses are filled in ascending expert order, each into
+ * the slot with the oldest stamp among the slots the batch does not use (empty slots first,
+ * then ties to the lower slot).  The decision and the copies run on the device after the
+ * batch's counts exist: no host round trip, capturable in a CUDA graph.
+ *
+ * State (caller-owned device memory, 16-byte aligned, moe_cache_state_bytes() bytes):
+ *   off[0] moe_cache_counters   off[1] slot_of [E] int32 (-1 = host only)
+ *   off[2] expert_in [S] int32 (-1 = empty)   off[3] stamp [S] int32 (batch of last use, -1)
+ *   off[4] load_expert [S] int32   off[5] load_slot [S] int32 (the last batch's loads, in order)
+ * moe_cache_reset() empties the cache (asynchronous on `stream`).
+ */
+typedef struct moe_cache_counters {
+    int64_t step;        /* batches run through the cache */
+    int64_t hits;        /* (batch, expert) pairs that found the expert resident */
+    int64_t misses;      /* (batch, expert) pairs that loaded it */
+    int64_t loads_last;  /* experts loaded by the last batch */
+    int64_t reserved[4];
+} moe_cache_counters;
+
+/* Bytes of the cache state; MOE_ERR_SHAPE unless 1 <= S <= E <= 1024. */
+int moe_cache_state_bytes(int E, int S, size_t* bytes);
+int moe_cache_layout(int E, int S, size_t off[6]);
+int moe_cache_reset(void* cache_state, int E, int S, moe_stream_t stream);
+
+/*
+ * moe_layer_forward() with the routed experts served from the cache.
+ *   W1_src, W3_src [E, f, d], W2_src [E, d, f]: the weights; page-locked host memory
+ *       (cudaHostAlloc / cudaHostRegister) read directly by the copy kernel, or device memory.
+ *       Pageable host memory is rejected (MOE_ERR_INVALID_ARG).
+ *   W1_slots, W3_slots [S, f, d], W2_slots [S, d, f]: device memory of the slots.
+ *   S: slots; must be >= min(E, T*k) so that one batch always fits (else MOE_ERR_SHAPE).
+ * Per batch, after the counts: the plan kernel updates the state and lists the loads, the copy
+ * kernel brings those experts into their slots, the grouped GEMMs read expert e from slot
+ * slot_of[e].  The output is the same as moe_layer_forward() with W1/W3/W2 = the sources.
+ * Device-side failure (a batch that needs more than S experts) sets MOE_ERR_CHECK.
+ */
+int moe_layer_forward_cached(const moe_bf16* x, const moe_bf16* Wg, const float* bias,
+                             const moe_bf16* W1_src, const moe_bf16* W3_src, const moe_bf16* W2_src,
+                             moe_bf16* W1_slots, moe_bf16* W3_slots, moe_bf16* W2_slots, int S,
+                             void* cache_state, const moe_bf16* W1s, const moe_bf16* W3s, const moe_bf16* W2s,
+                             int f_shared, int T, int d, int E, int k, int f, double capacity_factor,
+                             int cap_mode, moe_bf16* out, void* ws, size_t ws_bytes, moe_stream_t stream,
+                             const moe_stage_events* events);
 
 /*
  * Byte offsets of the intermediates that moe_layer_forward() leaves in its workspace,

@@ -63,6 +63,31 @@ _lib.moe_combine.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp]
 _lib.moe_layer_forward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
                                    _i32, _i32, _i32, _i32, _i32, _dbl, _i32, _vp, _vp, _sz, _vp]
 _lib.moe_layer_forward_ex.argtypes = _lib.moe_layer_forward.argtypes + [_vp]
+_lib.moe_layer_forward_w8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32,
+                                      _i32, _i32, _i32, _i32, _i32, _dbl, _i32, _vp, _vp, _sz, _vp, _vp]
+_lib.moe_layer_forward_w8.restype = _i32
+_lib.moe_cache_state_bytes.argtypes = [_i32, _i32, ctypes.POINTER(_sz)]
+_lib.moe_cache_state_bytes.restype = _i32
+_lib.moe_cache_layout.argtypes = [_i32, _i32, ctypes.POINTER(_sz)]
+_lib.moe_cache_layout.restype = _i32
+_lib.moe_cache_reset.argtypes = [_vp, _i32, _i32, _vp]
+_lib.moe_cache_reset.restype = _i32
+_lib.moe_layer_forward_cached.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i32,
+                                          _i32, _i32, _i32, _i32, _i32, _dbl, _i32, _vp, _vp, _sz, _vp, _vp]
+_lib.moe_layer_forward_cached.restype = _i32
+_lib.moe_layer_permute.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _i32, _i64, _vp, _vp, _sz, _vp]
+_lib.moe_layer_permute.restype = _i32
+_lib.moe_ep_workspace_bytes.argtypes = [_i32, ctypes.POINTER(_sz)]
+_lib.moe_ep_workspace_bytes.restype = _i32
+_lib.moe_ep_plan.argtypes = [_vp, _i32, _i32, _i32, _i64, _i32, _vp, _sz, _vp]
+_lib.moe_ep_plan.restype = _i32
+_lib.moe_ep_dispatch.argtypes = [_vp, _i32, _i32, _i32, _i32, ctypes.POINTER(_vp), _vp, _sz, _vp]
+_lib.moe_ep_dispatch.restype = _i32
+_lib.moe_ep_expert_ffn.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp,
+                                   _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]
+_lib.moe_ep_expert_ffn.restype = _i32
+_lib.moe_ep_return.argtypes = [_vp, _i32, _i32, _i32, _i32, ctypes.POINTER(_vp), _vp, _sz, _vp]
+_lib.moe_ep_return.restype = _i32
 _lib.moe_layer_route_count.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]
 _lib.moe_layer_route_count.restype = _i32
 _lib.moe_fill_base.argtypes = [_vp, _i32, _i32, _i32, _vp, _vp]
@@ -183,20 +208,26 @@ def moe_layer_forward(x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, f_shared, T, d, E,
                                   _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream)), "moe_layer_forward")
 
 
-STAGES = ["route", "topk", "permute", "gate_up", "down", "combine", "end"]
+STAGES = ["route", "topk", "permute", "gate_up", "down", "combine", "end"]   # timeline of one layer call
+_EVENT_FIELDS = STAGES + ["cache"]   # struct order; "cache" marks the expert cache kernels (between
+                                     # "permute" and "gate_up") in moe_layer_forward_cached
 
 
 class moe_stage_events(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in STAGES]
+    _fields_ = [(n, ctypes.c_void_p) for n in _EVENT_FIELDS]
+
+
+def _events(events: Optional[dict]):
+    if not events:
+        return None
+    return moe_stage_events(*[events[n].cuda_event if n in events and events[n] is not None else None
+                              for n in _EVENT_FIELDS])
 
 
 def moe_layer_forward_ex(x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, f_shared, T, d, E, k, f, capacity_factor,
                          cap_mode, out, ws, events: Optional[dict] = None, stream=None) -> None:
     """moe_layer_forward with optional stage markers: events = {stage name: torch.cuda.Event}."""
-    ev = None
-    if events:
-        ev = moe_stage_events(*[events[n].cuda_event if n in events and events[n] is not None else None
-                                for n in STAGES])
+    ev = _events(events)
     _check(_lib.moe_layer_forward_ex(_ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(W1s),
                                      _ptr(W3s), _ptr(W2s), f_shared, T, d, E, k, f, float(capacity_factor),
                                      cap_mode, _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream),
@@ -272,6 +303,99 @@ class Pipeline:
             self.close()
         except Exception:
             pass
+
+
+def moe_layer_forward_w8(x, Wg, bias, W1q, s1, W3q, s3, W2q, s2, W1sq, s1s, W3sq, s3s, W2sq, s2s, f_shared, T, d, E,
+                         k, f, capacity_factor, cap_mode, out, ws, events: Optional[dict] = None, stream=None) -> None:
+    """The layer with fp8 e4m3 expert weights (uint8 tensors) and fp32 per-row scales."""
+    ev = _events(events)
+    _check(_lib.moe_layer_forward_w8(_ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1q), _ptr(s1), _ptr(W3q), _ptr(s3),
+                                     _ptr(W2q), _ptr(s2), _ptr(W1sq), _ptr(s1s), _ptr(W3sq), _ptr(s3s), _ptr(W2sq),
+                                     _ptr(s2s), f_shared, T, d, E, k, f, float(capacity_factor), cap_mode, _ptr(out),
+                                     _ptr(ws), _nbytes(ws), _stream(stream), ctypes.byref(ev) if ev is not None else None),
+           "moe_layer_forward_w8")
+
+
+def moe_cache_state_bytes(E: int, S: int) -> int:
+    out = _sz(0)
+    _check(_lib.moe_cache_state_bytes(E, S, ctypes.byref(out)), "moe_cache_state_bytes")
+    return int(out.value)
+
+
+CACHE_FIELDS = ["counters", "slot_of", "expert_in", "stamp", "load_expert", "load_slot"]
+
+
+def moe_cache_layout(E: int, S: int) -> dict:
+    off = (_sz * 6)()
+    _check(_lib.moe_cache_layout(E, S, off), "moe_cache_layout")
+    return dict(zip(CACHE_FIELDS, [int(v) for v in off]))
+
+
+def moe_cache_reset(state, E: int, S: int, stream=None) -> None:
+    _check(_lib.moe_cache_reset(_ptr(state), E, S, _stream(stream)), "moe_cache_reset")
+
+
+def moe_layer_forward_cached(x, Wg, bias, W1_src, W3_src, W2_src, W1_slots, W3_slots, W2_slots, S, state, W1s, W3s,
+                             W2s, f_shared, T, d, E, k, f, capacity_factor, cap_mode, out, ws,
+                             events: Optional[dict] = None, stream=None) -> None:
+    """The layer with routed experts served from the expert cache.  W*_src: page-locked host
+    tensors (pin_memory) or device tensors; W*_slots: device tensors [S, ...]; state: a device
+    uint8 tensor of moe_cache_state_bytes(E, S) bytes, emptied once by moe_cache_reset."""
+    ev = _events(events)
+    _check(_lib.moe_layer_forward_cached(_ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1_src), _ptr(W3_src), _ptr(W2_src),
+                                         _ptr(W1_slots), _ptr(W3_slots), _ptr(W2_slots), S, _ptr(state), _ptr(W1s),
+                                         _ptr(W3s), _ptr(W2s), f_shared, T, d, E, k, f, float(capacity_factor),
+                                         cap_mode, _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream),
+                                         ctypes.byref(ev) if ev is not None else None), "moe_layer_forward_cached")
+
+
+def cache_counters(state) -> dict:
+    """The cache counters of a state tensor (copies 32 bytes to the host)."""
+    v = state[:32].view(__import__("torch").int64).cpu().tolist()
+    return dict(step=v[0], hits=v[1], misses=v[2], loads_last=v[3])
+
+
+def moe_layer_permute(x, f_shared, T, d, E, k, f, capacity, fill_base, ws, stream=None) -> None:
+    _check(_lib.moe_layer_permute(_ptr(x), f_shared, T, d, E, k, f, int(capacity), _ptr(fill_base), _ptr(ws),
+                                  _nbytes(ws), _stream(stream)), "moe_layer_permute")
+
+
+def moe_ep_workspace_bytes(E: int) -> int:
+    out = _sz(0)
+    _check(_lib.moe_ep_workspace_bytes(E, ctypes.byref(out)), "moe_ep_workspace_bytes")
+    return int(out.value)
+
+
+def _addr_array(bufs):
+    arr = (_vp * len(bufs))()
+    for i, b in enumerate(bufs):
+        arr[i] = _ptr(b)
+    return arr
+
+
+def moe_ep_plan(all_counts_raw, R, rank, E, capacity, max_recv_rows, ep_ws, stream=None) -> None:
+    _check(_lib.moe_ep_plan(_ptr(all_counts_raw), R, rank, E, int(capacity), max_recv_rows, _ptr(ep_ws),
+                            _nbytes(ep_ws), _stream(stream)), "moe_ep_plan")
+
+
+def moe_ep_dispatch(x_perm, R, rank, E, d, recv_bufs, ep_ws, stream=None) -> None:
+    """recv_bufs: R tensors (or device addresses), rank q's receive buffer [max_recv_rows, d] bf16."""
+    _check(_lib.moe_ep_dispatch(_ptr(x_perm), R, rank, E, d, _addr_array(recv_bufs), _ptr(ep_ws), _nbytes(ep_ws),
+                                _stream(stream)), "moe_ep_dispatch")
+
+
+def moe_ep_expert_ffn(recv_x, max_recv_rows, R, rank, E, d, f, W1_local, W3_local, W2_local, h, y_recv, x, T, W1s, W3s,
+                      W2s, f_shared, h_shared, y_shared, ep_ws, stream=None) -> None:
+    _check(_lib.moe_ep_expert_ffn(_ptr(recv_x), max_recv_rows, R, rank, E, d, f, _ptr(W1_local), _ptr(W3_local),
+                                  _ptr(W2_local), _ptr(h), _ptr(y_recv), _ptr(x), T, _ptr(W1s), _ptr(W3s), _ptr(W2s),
+                                  f_shared, _ptr(h_shared), _ptr(y_shared), _ptr(ep_ws), _nbytes(ep_ws),
+                                  _stream(stream)), "moe_ep_expert_ffn")
+
+
+def moe_ep_return(y_recv, R, rank, E, d, y_perm_bufs, ep_ws, stream=None) -> None:
+    """y_perm_bufs: R tensors (or device addresses), rank s's y_perm (in its layer workspace)."""
+    _check(_lib.moe_ep_return(_ptr(y_recv), R, rank, E, d, _addr_array(y_perm_bufs), _ptr(ep_ws), _nbytes(ep_ws),
+                              _stream(stream)), "moe_ep_return")
 
 
 def moe_get_error(stream=None) -> int:

@@ -73,7 +73,13 @@ struct GemmParams {
     int dense_rows;          // rows of class 1 (0 = no class 1)
     int stages;              // ring slots (<= GEMM_MAX_STAGES)
     int b_slot;              // bytes of one B slot (multiple of 1024)
+    const int32_t* group_map;  // [E] routed group -> weight group (expert cache slots); nullptr = identity
 };
+
+// Weight group that routed group g reads its B rows from.
+__device__ __forceinline__ int gemm_weight_group(const GemmParams& p, int g) {
+    return p.group_map ? __ldg(p.group_map + g) : g;
+}
 
 struct TileInfo {
     int cls;
@@ -111,7 +117,7 @@ __device__ __forceinline__ TileInfo gemm_decode_tile(const GemmParams& p, int t,
         ti.a_row = r0;
         ti.rows = min(GEMM_BM, __ldg(p.offsets + g + 1) - r0);
         ti.n_idx = n;
-        ti.b_row = g * c.b_group_rows + n * c.b_tile_rows;
+        ti.b_row = gemm_weight_group(p, g) * c.b_group_rows + n * c.b_tile_rows;
         ti.ks = 0;
     } else {
         const GemmClass& c = p.cls[1];

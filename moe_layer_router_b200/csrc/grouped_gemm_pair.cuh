@@ -151,13 +151,14 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                 const GemmClass& c = p.cls[ti.cls];
                 const CUtensorMap* mA = ti.cls ? &tmA1 : &tmA0;
                 const CUtensorMap* mB;
+                const int wg = ti.cls ? 0 : gemm_weight_group(p, ti.group);
                 int b_row;
                 if (EPI == EPI_SWIGLU) {       // CTA 0: W1 rows (gate), CTA 1: the same rows of W3 (up)
                     mB = ti.cls ? (leader ? &tmB1 : &tmB1b) : (leader ? &tmB0 : &tmB0b);
-                    b_row = ti.group * c.b_group_rows + ti.n_idx * 128;
+                    b_row = wg * c.b_group_rows + ti.n_idx * 128;
                 } else {                       // CTA r: rows [n0 + 128 r, n0 + 128 r + 128) of W2
                     mB = ti.cls ? &tmB1 : &tmB0;
-                    b_row = ti.group * c.b_group_rows + ti.n_idx * 256 + (int)rank * 128;
+                    b_row = wg * c.b_group_rows + ti.n_idx * 256 + (int)rank * 128;
                 }
                 const int a_row = ti.a_row + (int)rank * 128;
                 const int nk = c.K / GEMM_BK;

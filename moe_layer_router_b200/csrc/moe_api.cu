@@ -2,6 +2,7 @@
 //
 // The host side never allocates device memory and never synchronises (except
 // moe_get_error).  Every launch goes to the caller's stream.
+#include <algorithm>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -9,7 +10,10 @@
 #include "../../include/moe.h"
 #include "grouped_gemm.cuh"
 #include "grouped_gemm_pair.cuh"
+#include "grouped_gemm_w8.cuh"
 #include "route_permute_combine.cuh"
+#include "expert_cache.cuh"
+#include "expert_parallel.cuh"
 
 namespace moe {
 namespace {
@@ -77,6 +81,18 @@ int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, ui
     cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// 2-D fp8 (byte) tensor map [rows, inner], box [box_rows, 64 bytes], unswizzled, zero fill outside.
+int make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner};
+    cuuint32_t box[2] = {(cuuint32_t)GEMM_BK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -304,7 +320,11 @@ struct FfnArgs {
     const moe_bf16 *W1s, *W3s, *W2s;
     moe_bf16 *h_shared, *y_shared;
     bool pair;   // 2-SM tiles (mprefix counts 256-row tiles) instead of 1-SM tiles (128 rows)
+    const int32_t* group_map;   // routed group -> weight group (expert cache slots), nullptr = identity
+    int w_groups;               // weight groups in W1/W3/W2 (0 = E)
 };
+
+inline uint64_t weight_groups(const FfnArgs& a) { return (uint64_t)(a.w_groups ? a.w_groups : a.E); }
 
 int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t ev_down = nullptr) {
     const bool shared = a.f_shared > 0;
@@ -315,8 +335,8 @@ int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t
         CUtensorMap A0, B0, B0b, A1, B1, B1b;
         if (routed) {
             if ((rc = make_map(&A0, a.x_perm, a.d, a.max_rows, GEMM_BM)) != MOE_OK) return rc;
-            if ((rc = make_map(&B0, a.W1, a.d, (uint64_t)a.E * a.f, 128)) != MOE_OK) return rc;
-            if ((rc = make_map(&B0b, a.W3, a.d, (uint64_t)a.E * a.f, 128)) != MOE_OK) return rc;
+            if ((rc = make_map(&B0, a.W1, a.d, weight_groups(a) * a.f, 128)) != MOE_OK) return rc;
+            if ((rc = make_map(&B0b, a.W3, a.d, weight_groups(a) * a.f, 128)) != MOE_OK) return rc;
         }
         if (shared) {
             if ((rc = make_map(&A1, a.x, a.d, a.T, GEMM_BM)) != MOE_OK) return rc;
@@ -340,6 +360,7 @@ int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t
         p.E = a.E;
         p.dense_rows = shared ? a.T : 0;
         p.b_slot = GEMM_B_BYTES;
+        p.group_map = a.group_map;
         p.stages = GEMM_STAGES;
         long long tiles = 0;
         const int bm = a.pair ? PAIR_BM : GEMM_BM;
@@ -355,7 +376,7 @@ int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t
         CUtensorMap A0, B0, A1, B1;
         if (routed) {
             if ((rc = make_map(&A0, a.h, a.f, a.max_rows, GEMM_BM)) != MOE_OK) return rc;
-            if ((rc = make_map(&B0, a.W2, a.f, (uint64_t)a.E * a.d, a.pair ? 128 : 256)) != MOE_OK) return rc;
+            if ((rc = make_map(&B0, a.W2, a.f, weight_groups(a) * a.d, a.pair ? 128 : 256)) != MOE_OK) return rc;
         }
         if (shared) {
             if ((rc = make_map(&A1, a.h_shared, a.f_shared, a.T, GEMM_BM)) != MOE_OK) return rc;
@@ -377,6 +398,7 @@ int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t
         p.E = a.E;
         p.dense_rows = shared ? a.T : 0;
         p.b_slot = GEMM_B_BYTES;
+        p.group_map = a.group_map;
         p.stages = GEMM_STAGES;
         long long tiles = 0;
         const int bm = a.pair ? PAIR_BM : GEMM_BM;
@@ -385,6 +407,124 @@ int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t
         rc = a.pair ? launch_gemm_pair<EPI_STORE>(di, A0, B0, B0, A1, B1, B1, p, tiles, s)
                     : launch_gemm<EPI_STORE>(di, A0, B0, B0, A1, B1, B1, p, tiles, s);
         if (rc != MOE_OK) return rc;
+    }
+    return MOE_OK;
+}
+
+// fp8 e4m3 expert weights with fp32 row scales (routed: W1q/W3q [E,f,d], s1/s3 [E,f], W2q [E,d,f],
+// s2 [E,d]; shared: W1sq/W3sq [f_s,d], s1s/s3s [f_s], W2sq [d,f_s], s2s [d]).
+struct W8Weights {
+    const uint8_t *W1q, *W3q, *W2q, *W1sq, *W3sq, *W2sq;
+    const float *s1, *s3, *s2, *s1s, *s3s, *s2s;
+};
+
+template <int EPI>
+int launch_gemm_w8(DeviceInfo* di, const CUtensorMap* maps, const GemmParams& p, const W8Scales& sc,
+                   long long tiles_upper, cudaStream_t s) {
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        static bool attr_set[kMaxDevices][3] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (!attr_set[dev][EPI]) {
+            if (cudaFuncSetAttribute(grouped_gemm_w8_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     W8_SMEM_BYTES) != cudaSuccess)
+                return MOE_ERR_CUDA;
+            attr_set[dev][EPI] = true;
+        }
+    }
+    if (tiles_upper <= 0) return MOE_OK;
+    const int grid = (int)(tiles_upper < di->sms ? tiles_upper : di->sms);
+    grouped_gemm_w8_kernel<EPI><<<grid, W8_THREADS, W8_SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
+                                                                        maps[5], maps[6], maps[7], p, sc);
+    return launch_status();
+}
+
+int run_expert_ffn_w8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, cudaStream_t s, cudaEvent_t ev_down) {
+    const bool shared = a.f_shared > 0;
+    const bool routed = a.max_rows > 0;
+    int rc;
+    // ---- GEMM1 (maps: A, A32, W1q, W3q for routed, then shared)
+    {
+        CUtensorMap m[8];
+        if (routed) {
+            if ((rc = make_map(&m[0], a.x_perm, a.d, a.max_rows, GEMM_BM)) != MOE_OK) return rc;
+            if ((rc = make_map(&m[1], a.x_perm, a.d, a.max_rows, 32)) != MOE_OK) return rc;
+            if ((rc = make_map_u8(&m[2], q.W1q, a.d, (uint64_t)a.E * a.f, 128)) != MOE_OK) return rc;
+            if ((rc = make_map_u8(&m[3], q.W3q, a.d, (uint64_t)a.E * a.f, 128)) != MOE_OK) return rc;
+        }
+        if (shared) {
+            if ((rc = make_map(&m[4], a.x, a.d, a.T, GEMM_BM)) != MOE_OK) return rc;
+            if ((rc = make_map(&m[5], a.x, a.d, a.T, 32)) != MOE_OK) return rc;
+            if ((rc = make_map_u8(&m[6], q.W1sq, a.d, a.f_shared, 128)) != MOE_OK) return rc;
+            if ((rc = make_map_u8(&m[7], q.W3sq, a.d, a.f_shared, 128)) != MOE_OK) return rc;
+        }
+        for (int i = 0; i < 4; ++i) {
+            if (!routed) m[i] = m[i + 4];
+            if (!shared) m[i + 4] = m[i];
+        }
+        GemmParams p;
+        memset(&p, 0, sizeof(p));
+        GemmClass& c0 = p.cls[0];
+        c0.K = a.d; c0.n_out = a.f; c0.ntiles = (a.f + 127) / 128; c0.b_group_rows = a.f; c0.b_tile_rows = 128;
+        c0.mma_n = 256; c0.out = a.h; c0.ldo = a.f; c0.out_row0 = 0; c0.out_rows = a.max_rows; c0.ksplit = 1;
+        GemmClass& c1 = p.cls[1];
+        c1.K = a.d; c1.n_out = a.f_shared; c1.ntiles = (a.f_shared + 127) / 128; c1.b_group_rows = 0;
+        c1.b_tile_rows = 128; c1.mma_n = 256; c1.out = a.h_shared; c1.ldo = a.f_shared; c1.out_row0 = 0;
+        c1.out_rows = a.T; c1.ksplit = 1;
+        p.offsets = routed ? a.offsets : nullptr;
+        p.mprefix = a.mprefix;
+        p.E = a.E;
+        p.dense_rows = shared ? a.T : 0;
+        W8Scales sc;
+        memset(&sc, 0, sizeof(sc));
+        sc.s0[0] = q.s1; sc.s1[0] = q.s3; sc.group_stride[0] = a.f;
+        sc.s0[1] = shared ? q.s1s : q.s1; sc.s1[1] = shared ? q.s3s : q.s3; sc.group_stride[1] = 0;
+        long long tiles = 0;
+        if (routed) tiles += ((long long)(a.max_rows + GEMM_BM - 1) / GEMM_BM + a.E) * c0.ntiles;
+        if (shared) tiles += (long long)((a.T + GEMM_BM - 1) / GEMM_BM) * c1.ntiles;
+        if ((rc = launch_gemm_w8<EPI_SWIGLU>(di, m, p, sc, tiles, s)) != MOE_OK) return rc;
+    }
+    if (ev_down && cudaEventRecord(ev_down, s) != cudaSuccess) return MOE_ERR_CUDA;
+    // ---- GEMM2 (maps: A = h, A32, W2q; second W map unused)
+    {
+        CUtensorMap m[8];
+        if (routed) {
+            if ((rc = make_map(&m[0], a.h, a.f, a.max_rows, GEMM_BM)) != MOE_OK) return rc;
+            if ((rc = make_map(&m[1], a.h, a.f, a.max_rows, 32)) != MOE_OK) return rc;
+            if ((rc = make_map_u8(&m[2], q.W2q, a.f, (uint64_t)a.E * a.d, 256)) != MOE_OK) return rc;
+            m[3] = m[2];
+        }
+        if (shared) {
+            if ((rc = make_map(&m[4], a.h_shared, a.f_shared, a.T, GEMM_BM)) != MOE_OK) return rc;
+            if ((rc = make_map(&m[5], a.h_shared, a.f_shared, a.T, 32)) != MOE_OK) return rc;
+            if ((rc = make_map_u8(&m[6], q.W2sq, a.f_shared, a.d, 256)) != MOE_OK) return rc;
+            m[7] = m[6];
+        }
+        for (int i = 0; i < 4; ++i) {
+            if (!routed) m[i] = m[i + 4];
+            if (!shared) m[i + 4] = m[i];
+        }
+        GemmParams p;
+        memset(&p, 0, sizeof(p));
+        GemmClass& c0 = p.cls[0];
+        c0.K = a.f; c0.n_out = a.d; c0.ntiles = (a.d + 255) / 256; c0.b_group_rows = a.d; c0.b_tile_rows = 256;
+        c0.mma_n = 256; c0.out = a.y_perm; c0.ldo = a.d; c0.out_row0 = 0; c0.out_rows = a.max_rows; c0.ksplit = 1;
+        GemmClass& c1 = p.cls[1];
+        c1.K = a.f_shared; c1.n_out = a.d; c1.ntiles = (a.d + 255) / 256; c1.b_group_rows = 0; c1.b_tile_rows = 256;
+        c1.mma_n = 256; c1.out = a.y_shared; c1.ldo = a.d; c1.out_row0 = 0; c1.out_rows = a.T; c1.ksplit = 1;
+        p.offsets = routed ? a.offsets : nullptr;
+        p.mprefix = a.mprefix;
+        p.E = a.E;
+        p.dense_rows = shared ? a.T : 0;
+        W8Scales sc;
+        memset(&sc, 0, sizeof(sc));
+        sc.s0[0] = q.s2; sc.group_stride[0] = a.d;
+        sc.s0[1] = shared ? q.s2s : q.s2; sc.group_stride[1] = 0;
+        long long tiles = 0;
+        if (routed) tiles += ((long long)(a.max_rows + GEMM_BM - 1) / GEMM_BM + a.E) * c0.ntiles;
+        if (shared) tiles += (long long)((a.T + GEMM_BM - 1) / GEMM_BM) * c1.ntiles;
+        if ((rc = launch_gemm_w8<EPI_STORE>(di, m, p, sc, tiles, s)) != MOE_OK) return rc;
     }
     return MOE_OK;
 }
@@ -545,25 +685,44 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
 namespace moe {
 namespace {
 
-enum { LAYER_ROUTE = 1, LAYER_COUNT = 2, LAYER_FINISH = 4 };
+enum { LAYER_ROUTE = 1, LAYER_COUNT = 2, LAYER_FINISH = 4, LAYER_PERMUTE = 8 };
 
 // The layer in phases over one workspace:
-//   LAYER_ROUTE  router GEMM + top-k                 (needs x, Wg, bias)
-//   LAYER_COUNT  histogram only: counts_raw          (no capacity)
-//   LAYER_FINISH histogram, capacity (with fill_base), permutation, experts, combine
+//   LAYER_ROUTE   router GEMM + top-k                 (needs x, Wg, bias)
+//   LAYER_COUNT   histogram only: counts_raw          (no capacity)
+//   LAYER_PERMUTE histogram, capacity (with fill_base), permutation; stops there
+//   LAYER_FINISH  histogram, capacity (with fill_base), permutation, experts, combine
+// Routed expert weights served from the expert cache (moe_layer_forward_cached).
+struct CacheArgs {
+    const moe_bf16 *W1_src, *W3_src, *W2_src;   // device-usable addresses of the sources
+    moe_bf16 *W1_slots, *W3_slots, *W2_slots;
+    int S;
+    void* state;
+};
+
 int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float* bias, const moe_bf16* W1,
                  const moe_bf16* W3, const moe_bf16* W2, const moe_bf16* W1s, const moe_bf16* W3s, const moe_bf16* W2s,
                  int f_shared, int T, int d, int E, int k, int f, long long C, const int32_t* fill_base,
-                 moe_bf16* out, void* ws, size_t ws_bytes, cudaStream_t s, const moe_stage_events* events) {
+                 moe_bf16* out, void* ws, size_t ws_bytes, cudaStream_t s, const moe_stage_events* events,
+                 const W8Weights* w8 = nullptr, const CacheArgs* cache = nullptr) {
     int rc = check_shape(T, d, E, k, f);
     if (rc != MOE_OK) return rc;
     MOE_REQUIRE(f_shared >= 0 && f_shared % 64 == 0, MOE_ERR_SHAPE);
     MOE_REQUIRE(x && ws, MOE_ERR_INVALID_ARG);
     if (phases & LAYER_ROUTE) MOE_REQUIRE(Wg, MOE_ERR_INVALID_ARG);
     const bool shared = f_shared > 0;
-    if (phases & LAYER_FINISH) {
+    if ((phases & LAYER_FINISH) && !w8) {
         MOE_REQUIRE(W1 && W3 && W2 && out, MOE_ERR_INVALID_ARG);
         MOE_REQUIRE(!shared || (W1s && W3s && W2s), MOE_ERR_INVALID_ARG);
+    }
+    if ((phases & LAYER_FINISH) && w8) {
+        MOE_REQUIRE(w8->W1q && w8->W3q && w8->W2q && w8->s1 && w8->s3 && w8->s2 && out, MOE_ERR_INVALID_ARG);
+        MOE_REQUIRE(!shared || (w8->W1sq && w8->W3sq && w8->W2sq && w8->s1s && w8->s3s && w8->s2s),
+                    MOE_ERR_INVALID_ARG);
+        MOE_REQUIRE(aligned16(w8->W1q) && aligned16(w8->W3q) && aligned16(w8->W2q) && aligned16(w8->W1sq) &&
+                        aligned16(w8->W3sq) && aligned16(w8->W2sq) && aligned16(w8->s1) && aligned16(w8->s3) &&
+                        aligned16(w8->s2) && aligned16(w8->s1s) && aligned16(w8->s3s) && aligned16(w8->s2s),
+                    MOE_ERR_ALIGN);
     }
     MOE_REQUIRE(aligned16(x) && aligned16(Wg) && aligned16(bias) && aligned16(W1) && aligned16(W3) && aligned16(W2) &&
                     aligned16(W1s) && aligned16(W3s) && aligned16(W2s) && aligned16(out) && aligned16(ws) &&
@@ -606,26 +765,49 @@ int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float*
                     : run_topk(logits, 1, nullptr, bias, T, E, k, idx, w, s);
         if (rc != MOE_OK) return rc;
     }
-    const bool pair = use_pair_tiles((long long)T * k, E);
+    const bool pair = !w8 && use_pair_tiles((long long)T * k, E);    // fp8 weights: 1-SM tiles
     if (phases & LAYER_COUNT) {
         if ((rc = run_permute(di, x, idx, T, d, E, k, -1, counts_raw, counts, offsets, dest, src, x_perm, blk_cnt,
                               rank_local, mprefix, s, GEMM_BM, nullptr, true)) != MOE_OK)
             return rc;
     }
+    if (phases & LAYER_PERMUTE)
+        return run_permute(di, x, idx, T, d, E, k, C, counts_raw, counts, offsets, dest, src, x_perm, blk_cnt,
+                           rank_local, mprefix, s, GEMM_BM, fill_base);
     if (!(phases & LAYER_FINISH)) return MOE_OK;
     if (!mark(ev.permute)) return MOE_ERR_CUDA;
     if ((rc = run_permute(di, x, idx, T, d, E, k, C, counts_raw, counts, offsets, dest, src, x_perm, blk_cnt,
                           rank_local, mprefix, s, pair ? PAIR_BM : GEMM_BM, fill_base)) != MOE_OK)
         return rc;
+    CacheView cv{};
+    if (cache) {
+        if (!mark(ev.cache)) return MOE_ERR_CUDA;
+        cv = cache_view(cache->state, E, cache->S);
+        cache_plan_kernel<<<1, CACHE_MAX, 0, s>>>(counts, E, cache->S, cv);
+        if ((rc = launch_status()) != MOE_OK) return rc;
+        cache_load_kernel<<<2 * di->sms, CACHE_LOAD_THREADS, 0, s>>>(
+            cv.ctr, cv.load_expert, cv.load_slot, reinterpret_cast<const uint4*>(cache->W1_src),
+            reinterpret_cast<const uint4*>(cache->W3_src), reinterpret_cast<const uint4*>(cache->W2_src),
+            reinterpret_cast<uint4*>(cache->W1_slots), reinterpret_cast<uint4*>(cache->W3_slots),
+            reinterpret_cast<uint4*>(cache->W2_slots), (long long)f * d / 8);
+        if ((rc = launch_status()) != MOE_OK) return rc;
+    }
     if (!mark(ev.gate_up)) return MOE_ERR_CUDA;
     FfnArgs a;
     memset(&a, 0, sizeof(a));
     a.x_perm = x_perm; a.offsets = offsets; a.mprefix = mprefix; a.max_rows = T * k; a.E = E; a.d = d; a.f = f;
     a.W1 = W1; a.W3 = W3; a.W2 = W2; a.h = h; a.y_perm = y_perm;
+    if (cache) {
+        a.W1 = cache->W1_slots; a.W3 = cache->W3_slots; a.W2 = cache->W2_slots;
+        a.group_map = cv.slot_of;
+        a.w_groups = cache->S;
+    }
     a.x = x; a.T = T; a.f_shared = f_shared; a.W1s = W1s; a.W3s = W3s; a.W2s = W2s;
     a.h_shared = h_shared; a.y_shared = y_shared;
     a.pair = pair;
-    if ((rc = run_expert_ffn(di, a, s, static_cast<cudaEvent_t>(ev.down))) != MOE_OK) return rc;
+    rc = w8 ? run_expert_ffn_w8(di, a, *w8, s, static_cast<cudaEvent_t>(ev.down))
+            : run_expert_ffn(di, a, s, static_cast<cudaEvent_t>(ev.down));
+    if (rc != MOE_OK) return rc;
     if (!mark(ev.combine)) return MOE_ERR_CUDA;
     if ((rc = run_combine(y_perm, dest, w, y_shared, T, d, k, out, s)) != MOE_OK) return rc;
     return mark(ev.end) ? MOE_OK : MOE_ERR_CUDA;
@@ -645,6 +827,88 @@ int moe_layer_forward_ex(const moe_bf16* x, const moe_bf16* Wg, const float* bia
     const long long C = moe_capacity(T, E, k, capacity_factor, cap_mode);
     return layer_phases(LAYER_ROUTE | LAYER_FINISH, x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, f_shared, T, d, E, k, f, C,
                         nullptr, out, ws, ws_bytes, static_cast<cudaStream_t>(stream), events);
+}
+
+int moe_cache_state_bytes(int E, int S, size_t* bytes) {
+    MOE_REQUIRE(bytes, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(S >= 1 && S <= E && E <= moe::CACHE_MAX, MOE_ERR_SHAPE);
+    size_t off[6];
+    *bytes = moe::cache_layout(E, S, off);
+    return MOE_OK;
+}
+
+int moe_cache_layout(int E, int S, size_t off[6]) {
+    MOE_REQUIRE(off, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(S >= 1 && S <= E && E <= moe::CACHE_MAX, MOE_ERR_SHAPE);
+    moe::cache_layout(E, S, off);
+    return MOE_OK;
+}
+
+int moe_cache_reset(void* cache_state, int E, int S, moe_stream_t stream) {
+    using namespace moe;
+    MOE_REQUIRE(cache_state, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(cache_state), MOE_ERR_ALIGN);
+    MOE_REQUIRE(S >= 1 && S <= E && E <= CACHE_MAX, MOE_ERR_SHAPE);
+    DeviceInfo* di;
+    int rc = device_info(&di);
+    if (rc != MOE_OK) return rc;
+    cache_reset_kernel<<<1, CACHE_MAX, 0, static_cast<cudaStream_t>(stream)>>>(cache_view(cache_state, E, S), E, S);
+    return launch_status();
+}
+
+// Address the device uses for a cache source: page-locked host memory (mapped) or device memory.
+static int cache_source(const moe_bf16* p, const moe_bf16** dev) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_INVALID_ARG;
+    }
+    if (at.type == cudaMemoryTypeHost && at.devicePointer) *dev = static_cast<const moe_bf16*>(at.devicePointer);
+    else if (at.type == cudaMemoryTypeDevice) *dev = p;
+    else return MOE_ERR_INVALID_ARG;   // pageable host memory (or unknown)
+    return MOE_OK;
+}
+
+int moe_layer_forward_cached(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const moe_bf16* W1_src,
+                             const moe_bf16* W3_src, const moe_bf16* W2_src, moe_bf16* W1_slots, moe_bf16* W3_slots,
+                             moe_bf16* W2_slots, int S, void* cache_state, const moe_bf16* W1s, const moe_bf16* W3s,
+                             const moe_bf16* W2s, int f_shared, int T, int d, int E, int k, int f,
+                             double capacity_factor, int cap_mode, moe_bf16* out, void* ws, size_t ws_bytes,
+                             moe_stream_t stream, const moe_stage_events* events) {
+    using namespace moe;
+    MOE_REQUIRE(cap_mode >= MOE_CAP_NONE && cap_mode <= MOE_CAP_PER_ASSIGNMENT, MOE_ERR_INVALID_ARG);
+    int rc = check_shape(T, d, E, k, f);
+    if (rc != MOE_OK) return rc;
+    MOE_REQUIRE(S >= 1 && S <= E && (long long)S >= std::min<long long>(E, (long long)T * k), MOE_ERR_SHAPE);
+    MOE_REQUIRE(W1_src && W3_src && W2_src && W1_slots && W3_slots && W2_slots && cache_state, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(W1_src) && aligned16(W3_src) && aligned16(W2_src) && aligned16(W1_slots) &&
+                    aligned16(W3_slots) && aligned16(W2_slots) && aligned16(cache_state),
+                MOE_ERR_ALIGN);
+    CacheArgs ca;
+    if ((rc = cache_source(W1_src, &ca.W1_src)) != MOE_OK || (rc = cache_source(W3_src, &ca.W3_src)) != MOE_OK ||
+        (rc = cache_source(W2_src, &ca.W2_src)) != MOE_OK)
+        return rc;
+    ca.W1_slots = W1_slots; ca.W3_slots = W3_slots; ca.W2_slots = W2_slots;
+    ca.S = S;
+    ca.state = cache_state;
+    const long long C = moe_capacity(T, E, k, capacity_factor, cap_mode);
+    return layer_phases(LAYER_ROUTE | LAYER_FINISH, x, Wg, bias, W1_slots, W3_slots, W2_slots, W1s, W3s, W2s,
+                        f_shared, T, d, E, k, f, C, nullptr, out, ws, ws_bytes, static_cast<cudaStream_t>(stream),
+                        events, nullptr, &ca);
+}
+
+int moe_layer_forward_w8(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const uint8_t* W1q,
+                         const float* s1, const uint8_t* W3q, const float* s3, const uint8_t* W2q, const float* s2,
+                         const uint8_t* W1sq, const float* s1s, const uint8_t* W3sq, const float* s3s,
+                         const uint8_t* W2sq, const float* s2s, int f_shared, int T, int d, int E, int k, int f,
+                         double capacity_factor, int cap_mode, moe_bf16* out, void* ws, size_t ws_bytes,
+                         moe_stream_t stream, const moe_stage_events* events) {
+    MOE_REQUIRE(cap_mode >= MOE_CAP_NONE && cap_mode <= MOE_CAP_PER_ASSIGNMENT, MOE_ERR_INVALID_ARG);
+    const long long C = moe_capacity(T, E, k, capacity_factor, cap_mode);
+    W8Weights q = {W1q, W3q, W2q, W1sq, W3sq, W2sq, s1, s3, s2, s1s, s3s, s2s};
+    return layer_phases(LAYER_ROUTE | LAYER_FINISH, x, Wg, bias, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                        f_shared, T, d, E, k, f, C, nullptr, out, ws, ws_bytes, static_cast<cudaStream_t>(stream),
+                        events, &q);
 }
 
 int moe_layer_route_count(const moe_bf16* x, const moe_bf16* Wg, const float* bias, int f_shared, int T, int d, int E,
@@ -672,6 +936,153 @@ int moe_layer_finish(const moe_bf16* x, const moe_bf16* W1, const moe_bf16* W3, 
     return layer_phases(LAYER_FINISH, x, nullptr, nullptr, W1, W3, W2, W1s, W3s, W2s, f_shared, T, d, E, k, f,
                         capacity < 0 ? -1 : (long long)capacity, fill_base, out, ws, ws_bytes,
                         static_cast<cudaStream_t>(stream), nullptr);
+}
+
+int moe_layer_permute(const moe_bf16* x, int f_shared, int T, int d, int E, int k, int f, int64_t capacity,
+                      const int32_t* fill_base, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    return layer_phases(LAYER_PERMUTE, x, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                        f_shared, T, d, E, k, f, capacity < 0 ? -1 : (long long)capacity, fill_base, nullptr, ws,
+                        ws_bytes, static_cast<cudaStream_t>(stream), nullptr);
+}
+
+// ------------------------------------------------------------------ expert parallelism
+
+namespace {
+
+struct EpLayout {
+    size_t plan, seg_off, mprefix, group_map, total;
+};
+
+EpLayout ep_layout(int E) {
+    EpLayout L;
+    size_t o = 0;
+    L.plan = o; o += moe::align256(sizeof(moe::EpPlan));
+    L.seg_off = o; o += moe::align256((size_t)(E + 1) * 4);
+    L.mprefix = o; o += moe::align256((size_t)(E + 1) * 4);
+    L.group_map = o; o += moe::align256((size_t)E * 4);
+    L.total = o;
+    return L;
+}
+
+int ep_check(int R, int rank, int E, int d) {
+    MOE_REQUIRE(R >= 1 && R <= moe::EP_MAX_RANKS && rank >= 0 && rank < R, MOE_ERR_SHAPE);
+    MOE_REQUIRE(E >= 1 && E <= 1024 && E % R == 0, MOE_ERR_SHAPE);
+    MOE_REQUIRE(d >= 64 && d % 64 == 0, MOE_ERR_SHAPE);
+    return MOE_OK;
+}
+
+int ep_put(const void* src, int which, moe_bf16* const* dests, int R, int d, const void* ep_ws, cudaStream_t s) {
+    using namespace moe;
+    EpDests dst;
+    memset(&dst, 0, sizeof(dst));
+    for (int q = 0; q < R; ++q) {
+        MOE_REQUIRE(dests[q] && aligned16(dests[q]), MOE_ERR_INVALID_ARG);
+        dst.base[q] = reinterpret_cast<char*>(dests[q]);
+    }
+    DeviceInfo* di;
+    int rc = device_info(&di);
+    if (rc != MOE_OK) return rc;
+    const EpLayout L = ep_layout(1);
+    const EpPlan* plan = reinterpret_cast<const EpPlan*>(static_cast<const char*>(ep_ws) + L.plan);
+    const int bx = std::max(1, (2 * di->sms + R - 1) / R);
+    ep_put_rows_kernel<<<dim3(bx, R), 256, 0, s>>>(plan, which, static_cast<const uint4*>(src), dst, (long long)d / 8);
+    return launch_status();
+}
+
+}  // namespace
+
+int moe_ep_workspace_bytes(int E, size_t* bytes) {
+    MOE_REQUIRE(bytes, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(E >= 1 && E <= 1024, MOE_ERR_SHAPE);
+    *bytes = ep_layout(E).total;
+    return MOE_OK;
+}
+
+int moe_ep_plan(const int32_t* all_counts_raw, int R, int rank, int E, int64_t capacity, int max_recv_rows,
+                void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream) {
+    using namespace moe;
+    int rc = ep_check(R, rank, E, 64);
+    if (rc != MOE_OK) return rc;
+    MOE_REQUIRE(max_recv_rows >= 0, MOE_ERR_SHAPE);
+    MOE_REQUIRE(all_counts_raw && ep_ws, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(ep_ws), MOE_ERR_ALIGN);
+    const EpLayout L = ep_layout(E);
+    MOE_REQUIRE(ep_ws_bytes >= L.total, MOE_ERR_WORKSPACE);
+    DeviceInfo* di;
+    if ((rc = device_info(&di)) != MOE_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* b = static_cast<char*>(ep_ws);
+    const bool pair = use_pair_tiles(max_recv_rows, E);
+    ep_plan_kernel<<<1, 1024, 0, s>>>(all_counts_raw, R, E, rank, capacity < 0 ? -1 : (long long)capacity,
+                                      pair ? PAIR_BM : GEMM_BM, reinterpret_cast<EpPlan*>(b + L.plan),
+                                      reinterpret_cast<int32_t*>(b + L.seg_off), reinterpret_cast<int32_t*>(b + L.mprefix));
+    if ((rc = launch_status()) != MOE_OK) return rc;
+    ep_group_map_kernel<<<(E + 255) / 256, 256, 0, s>>>(R, E / R, reinterpret_cast<int32_t*>(b + L.group_map));
+    return launch_status();
+}
+
+int moe_ep_dispatch(const moe_bf16* x_perm, int R, int rank, int E, int d, moe_bf16* const* recv_bufs,
+                    const void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream) {
+    using namespace moe;
+    int rc = ep_check(R, rank, E, d);
+    if (rc != MOE_OK) return rc;
+    MOE_REQUIRE(x_perm && recv_bufs && ep_ws, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(x_perm) && aligned16(ep_ws), MOE_ERR_ALIGN);
+    MOE_REQUIRE(ep_ws_bytes >= ep_layout(E).total, MOE_ERR_WORKSPACE);
+    return ep_put(x_perm, 0, recv_bufs, R, d, ep_ws, static_cast<cudaStream_t>(stream));
+}
+
+int moe_ep_expert_ffn(const moe_bf16* recv_x, int max_recv_rows, int R, int rank, int E, int d, int f,
+                      const moe_bf16* W1_local, const moe_bf16* W3_local, const moe_bf16* W2_local, moe_bf16* h,
+                      moe_bf16* y_recv, const moe_bf16* x, int T, const moe_bf16* W1s, const moe_bf16* W3s,
+                      const moe_bf16* W2s, int f_shared, moe_bf16* h_shared, moe_bf16* y_shared, const void* ep_ws,
+                      size_t ep_ws_bytes, moe_stream_t stream) {
+    using namespace moe;
+    int rc = ep_check(R, rank, E, d);
+    if (rc != MOE_OK) return rc;
+    MOE_REQUIRE(max_recv_rows >= 0 && f >= 64 && f % 64 == 0 && f_shared >= 0 && f_shared % 64 == 0, MOE_ERR_SHAPE);
+    const bool shared = f_shared > 0;
+    MOE_REQUIRE(ep_ws && (max_recv_rows == 0 || (recv_x && W1_local && W3_local && W2_local && h && y_recv)),
+                MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(!shared || (x && T >= 1 && W1s && W3s && W2s && h_shared && y_shared), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(recv_x) && aligned16(W1_local) && aligned16(W3_local) && aligned16(W2_local) &&
+                    aligned16(h) && aligned16(y_recv) && aligned16(x) && aligned16(W1s) && aligned16(W3s) &&
+                    aligned16(W2s) && aligned16(h_shared) && aligned16(y_shared) && aligned16(ep_ws),
+                MOE_ERR_ALIGN);
+    const EpLayout L = ep_layout(E);
+    MOE_REQUIRE(ep_ws_bytes >= L.total, MOE_ERR_WORKSPACE);
+    DeviceInfo* di;
+    if ((rc = device_info(&di)) != MOE_OK) return rc;
+    const char* b = static_cast<const char*>(ep_ws);
+    FfnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x_perm = recv_x;
+    a.offsets = max_recv_rows > 0 ? reinterpret_cast<const int32_t*>(b + L.seg_off) : nullptr;
+    a.mprefix = reinterpret_cast<const int32_t*>(b + L.mprefix);
+    a.max_rows = max_recv_rows;
+    a.E = E;                       // R * El segments
+    a.d = d;
+    a.f = f;
+    a.W1 = W1_local; a.W3 = W3_local; a.W2 = W2_local;
+    a.h = h; a.y_perm = y_recv;
+    a.x = x; a.T = T; a.f_shared = f_shared; a.W1s = W1s; a.W3s = W3s; a.W2s = W2s;
+    a.h_shared = h_shared; a.y_shared = y_shared;
+    a.pair = use_pair_tiles(max_recv_rows, E);
+    a.group_map = reinterpret_cast<const int32_t*>(b + L.group_map);
+    a.w_groups = E / R;
+    if (max_recv_rows == 0 && !shared) return MOE_OK;
+    return run_expert_ffn(di, a, static_cast<cudaStream_t>(stream));
+}
+
+int moe_ep_return(const moe_bf16* y_recv, int R, int rank, int E, int d, moe_bf16* const* y_perm_bufs,
+                  const void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream) {
+    using namespace moe;
+    int rc = ep_check(R, rank, E, d);
+    if (rc != MOE_OK) return rc;
+    MOE_REQUIRE(y_recv && y_perm_bufs && ep_ws, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(y_recv) && aligned16(ep_ws), MOE_ERR_ALIGN);
+    MOE_REQUIRE(ep_ws_bytes >= ep_layout(E).total, MOE_ERR_WORKSPACE);
+    return ep_put(y_recv, 1, y_perm_bufs, R, d, ep_ws, static_cast<cudaStream_t>(stream));
 }
 
 int moe_update_bias(const int32_t* counts_raw, int E, int64_t capacity, float* bias, moe_stream_t stream) {

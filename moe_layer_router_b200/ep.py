@@ -1,0 +1,149 @@
+"""Expert parallelism around the C ABI: experts split over R ranks.
+
+Rank r holds the E / R experts [r El, (r + 1) El) (uniform contiguous split, [EP-DS3]
+section 3.1 _assign_experts).  A layer call per rank: route and count its own tokens, all-gather
+the raw counts [R, E], keep rows under the whole batch's capacity (token order over ranks in rank
+order), send each kept row to its expert's rank, run the local experts over the received rows,
+send the results back and combine ([EP-KV] sections 6-7).  Every step of the path runs in the
+library's kernels; this module only moves pointers, sizes and (for the NCCL path) the two
+all-to-all-v exchanges.
+
+Two drivers:
+  * ``EmulatedEP``: R ranks on one device in one process.  The row exchanges are the library's
+    put kernels writing into the other ranks' buffers; the all-gather is a device copy.
+  * ``ep_layer_forward_dist``: one process per GPU over ``torch.distributed``; counts are
+    all-gathered and rows moved with ``all_to_all_single`` (NCCL), whose split sizes
+    ``ep_row_splits`` computes on the host from the gathered counts.
+"""
+from __future__ import annotations
+
+from typing import List, Optional, Sequence
+
+import numpy as np
+
+
+def kept_counts(all_counts_raw: np.ndarray, capacity: int) -> np.ndarray:
+    """[R, E] rows each rank keeps per expert: the rows of rank r for expert e come after the
+    rows of ranks < r in token order, so r keeps min(c[r][e], max(0, C - sum_{s<r} c[s][e]))."""
+    c = np.asarray(all_counts_raw, dtype=np.int64)
+    if capacity < 0:
+        return c.copy()
+    before = np.cumsum(c, axis=0) - c
+    return np.clip(np.minimum(c, capacity - before), 0, None)
+
+
+def ep_row_splits(all_counts_raw: np.ndarray, capacity: int, rank: int):
+    """-> (send_rows [R], recv_rows [R]): rows `rank` sends to each rank (its kept rows of that
+    rank's experts, in rank order = x_perm order) and rows it receives from each rank."""
+    R, E = all_counts_raw.shape
+    if E % R:
+        raise ValueError("E must be a multiple of the number of ranks")
+    El = E // R
+    kept = kept_counts(all_counts_raw, capacity)
+    per_rank = kept.reshape(R, R, El).sum(axis=2)       # [src, dst]
+    return per_rank[rank].tolist(), per_rank[:, rank].tolist()
+
+
+def exchange_rows(src, send_rows: Sequence[int], recv_rows: Sequence[int], out, group=None) -> None:
+    """all_to_all_single over the leading (row) dimension: rows [sum(send[:q]), +send[q]) of `src`
+    go to rank q, rows from rank s land at [sum(recv[:s]), +recv[s]) of `out`."""
+    import torch.distributed as dist
+    ns, nr = int(sum(send_rows)), int(sum(recv_rows))
+    dist.all_to_all_single(out[:nr], src[:ns], output_split_sizes=[int(v) for v in recv_rows],
+                           input_split_sizes=[int(v) for v in send_rows], group=group)
+
+
+class _RankBuffers:
+    def __init__(self, moe, T, d, E, k, f, fs, max_recv, device):
+        import torch
+        self.ws = torch.empty(moe.moe_workspace_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device=device)
+        self.layout = moe.moe_workspace_layout(T, d, E, k, f, fs)
+        self.ep_ws = torch.empty(moe.moe_ep_workspace_bytes(E), dtype=torch.uint8, device=device)
+        self.fill_base = torch.empty(E, dtype=torch.int32, device=device)
+        rows = max(1, max_recv)
+        self.recv = torch.empty((rows, d), dtype=torch.bfloat16, device=device)
+        self.h = torch.empty((rows, f), dtype=torch.bfloat16, device=device)
+        self.y_recv = torch.empty((rows, d), dtype=torch.bfloat16, device=device)
+        self.h_shared = torch.empty((T, fs), dtype=torch.bfloat16, device=device) if fs else None
+        self.y_shared = torch.empty((T, d), dtype=torch.bfloat16, device=device) if fs else None
+
+    def view(self, moe, name, shape, dtype):
+        return moe.workspace_view(self.ws, self.layout, name, shape, dtype)
+
+
+class EmulatedEP:
+    """R expert-parallel ranks on one device (one process, one stream)."""
+
+    def __init__(self, R, T, d, E, k, f, f_shared=0, device="cuda"):
+        import moe_layer_router_b200 as moe
+        if E % R:
+            raise ValueError("E must be a multiple of R")
+        self.moe, self.R, self.T, self.d, self.E, self.k, self.f, self.fs = moe, R, T, d, E, k, f, f_shared
+        self.max_recv = R * T * k
+        self.ranks = [_RankBuffers(moe, T, d, E, k, f, f_shared, self.max_recv, device) for _ in range(R)]
+        import torch
+        self.all_counts = torch.empty((R, E), dtype=torch.int32, device=device)
+
+    def forward(self, xs: List, Wg, bias, W1, W3, W2, W1s, W3s, W2s, capacity_factor, cap_mode, outs: List) -> None:
+        """xs[r]: rank r's tokens [T, d]; W1/W3/W2: all experts (rank r uses its El-expert slice);
+        outs[r]: [T, d].  Capacity counts the whole batch of R * T tokens."""
+        moe, R, T, d, E, k, f, fs = self.moe, self.R, self.T, self.d, self.E, self.k, self.f, self.fs
+        El = E // R
+        C = moe.moe_capacity(R * T, E, k, capacity_factor, cap_mode)
+        for r, b in enumerate(self.ranks):
+            moe.moe_layer_route_count(xs[r], Wg, bias, fs, T, d, E, k, f, b.ws)
+        for r, b in enumerate(self.ranks):          # the all-gather of raw counts
+            self.all_counts[r].copy_(b.view(moe, "counts_raw", (E,), self.all_counts.dtype))
+        for r, b in enumerate(self.ranks):
+            moe.moe_fill_base(self.all_counts, R, r, E, b.fill_base)
+            moe.moe_layer_permute(xs[r], fs, T, d, E, k, f, C, b.fill_base, b.ws)
+            moe.moe_ep_plan(self.all_counts, R, r, E, C, self.max_recv, b.ep_ws)
+        recv = [b.recv for b in self.ranks]
+        for r, b in enumerate(self.ranks):
+            moe.moe_ep_dispatch(b.view(moe, "x_perm", (T * k, d), xs[r].dtype), R, r, E, d, recv, b.ep_ws)
+        for r, b in enumerate(self.ranks):
+            sl = slice(r * El, (r + 1) * El)
+            moe.moe_ep_expert_ffn(b.recv, self.max_recv, R, r, E, d, f, W1[sl], W3[sl], W2[sl], b.h, b.y_recv, xs[r],
+                                  T, W1s, W3s, W2s, fs, b.h_shared, b.y_shared, b.ep_ws)
+        y_perm = [b.view(moe, "y_perm", (T * k, d), xs[r].dtype) for r, b in enumerate(self.ranks)]
+        for r, b in enumerate(self.ranks):
+            moe.moe_ep_return(b.y_recv, R, r, E, d, y_perm, b.ep_ws)
+        for r, b in enumerate(self.ranks):
+            moe.moe_combine(y_perm[r], b.view(moe, "dest", (T, k), self.all_counts.dtype),
+                            b.view(moe, "w", (T, k), _f32()), b.y_shared, T, d, k, outs[r])
+
+
+def _f32():
+    import torch
+    return torch.float32
+
+
+def ep_layer_forward_dist(x, Wg, bias, W1_local, W3_local, W2_local, W1s, W3s, W2s, f_shared, T, d, E, k, f,
+                          capacity_factor, cap_mode, out, bufs: Optional[_RankBuffers] = None, group=None):
+    """One rank of an expert-parallel layer over torch.distributed (one process per GPU).
+    W*_local: this rank's El experts.  The collectives: an all-gather of the raw counts and two
+    all_to_all_single row exchanges; everything else runs in the library's kernels."""
+    import torch
+    import torch.distributed as dist
+    import moe_layer_router_b200 as moe
+
+    R, rank = dist.get_world_size(group), dist.get_rank(group)
+    if bufs is None:
+        bufs = _RankBuffers(moe, T, d, E, k, f, f_shared, R * T * k, x.device)
+    C = moe.moe_capacity(R * T, E, k, capacity_factor, cap_mode)
+    moe.moe_layer_route_count(x, Wg, bias, f_shared, T, d, E, k, f, bufs.ws)
+    all_counts = torch.empty((R, E), dtype=torch.int32, device=x.device)
+    dist.all_gather_into_tensor(all_counts, bufs.view(moe, "counts_raw", (E,), torch.int32), group=group)
+    moe.moe_fill_base(all_counts, R, rank, E, bufs.fill_base)
+    moe.moe_layer_permute(x, f_shared, T, d, E, k, f, C, bufs.fill_base, bufs.ws)
+    moe.moe_ep_plan(all_counts, R, rank, E, C, R * T * k, bufs.ep_ws)
+    send_rows, recv_rows = ep_row_splits(all_counts.cpu().numpy(), C, rank)
+    x_perm = bufs.view(moe, "x_perm", (T * k, d), x.dtype)
+    y_perm = bufs.view(moe, "y_perm", (T * k, d), x.dtype)
+    exchange_rows(x_perm, send_rows, recv_rows, bufs.recv, group)
+    moe.moe_ep_expert_ffn(bufs.recv, R * T * k, R, rank, E, d, f, W1_local, W3_local, W2_local, bufs.h, bufs.y_recv,
+                          x, T, W1s, W3s, W2s, f_shared, bufs.h_shared, bufs.y_shared, bufs.ep_ws)
+    exchange_rows(bufs.y_recv, recv_rows, send_rows, y_perm, group)
+    moe.moe_combine(y_perm, bufs.view(moe, "dest", (T, k), torch.int32), bufs.view(moe, "w", (T, k), torch.float32),
+                    bufs.y_shared, T, d, k, out)
+    return bufs

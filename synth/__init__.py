@@ -300,3 +300,35 @@ def device_tensors(wl: Workload, device, names=None, chunk_elems: int = 1 << 27)
         b = inp.bias()
         out["bias"] = torch.from_numpy(b).to(device) if b is not None else None
     return out
+
+
+def device_tensors_q8(wl: Workload, device, chunk_rows: int = 1 << 16) -> dict:
+    """fp8 e4m3 expert weights with fp32 row scales, quantised from the workload's bf16 weights
+    (quantize_e4m3_rows) chunk by chunk on the host and copied to `device`.
+    Keys: w1q, w3q [E,f,d] uint8, s1, s3 [E,f]; w2q [E,d,f], s2 [E,d]; w1sq, w3sq, w2sq, s1s,
+    s3s, s2s for the shared expert."""
+    import torch
+
+    inp = Inputs(wl)
+    out = {}
+    per = wl.f * wl.d
+    for name, K, rows_per_e in (("w1", wl.d, wl.f), ("w3", wl.d, wl.f), ("w2", wl.f, wl.d)):
+        q_dev = torch.empty((wl.E * rows_per_e, K), dtype=torch.uint8, device=device)
+        s_dev = torch.empty(wl.E * rows_per_e, dtype=torch.float32, device=device)
+        ne = max(1, min(wl.E, chunk_rows // rows_per_e))
+        for e0 in range(0, wl.E, ne):
+            n = min(ne, wl.E - e0)
+            w = inp.expert_rows(name, e0, n)
+            q, sc = quantize_e4m3_rows(w, K)
+            q_dev[e0 * rows_per_e:(e0 + n) * rows_per_e].copy_(torch.from_numpy(q))
+            s_dev[e0 * rows_per_e:(e0 + n) * rows_per_e].copy_(torch.from_numpy(sc))
+        out[name + "q"] = q_dev.view(wl.E, rows_per_e, K)
+        out["s" + name[1]] = s_dev.view(wl.E, rows_per_e)
+    if wl.has_shared:
+        for name in ("w1s", "w3s", "w2s"):
+            a = inp.shared(name)
+            q, sc = quantize_e4m3_rows(a, a.shape[1])
+            out[name[:2] + "sq"] = torch.from_numpy(q).to(device)
+            out["s" + name[1] + "s"] = torch.from_numpy(sc).to(device)
+    return out
+

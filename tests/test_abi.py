@@ -88,3 +88,51 @@ def test_entry_points_validate_before_touching_the_device(lib):
     assert lib.moe_combine(16, 16, 16, None, 8, 64, 2, 17, None) == -3     # misaligned out
     lib.moe_strerror.restype = ctypes.c_char_p
     assert lib.moe_strerror(-4) == b"workspace too small"
+
+
+def test_expert_cache_host_checks(lib):
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.moe_cache_state_bytes.argtypes = [i32, i32, ctypes.POINTER(sz)]
+    lib.moe_cache_layout.argtypes = [i32, i32, ctypes.POINTER(sz)]
+    b = sz(0)
+    assert lib.moe_cache_state_bytes(256, 128, ctypes.byref(b)) == 0
+    # 64-byte counters, then slot_of [256] and four [128] int32 arrays
+    assert b.value == 64 + 256 * 4 + 4 * 128 * 4
+    off = (sz * 6)()
+    assert lib.moe_cache_layout(10, 3, off) == 0
+    assert list(off) == [0, 64, 64 + 48, 64 + 48 + 16, 64 + 48 + 32, 64 + 48 + 48]   # padded to 16 bytes
+    assert lib.moe_cache_state_bytes(8, 9, ctypes.byref(b)) == -2      # more slots than experts
+    assert lib.moe_cache_state_bytes(2048, 16, ctypes.byref(b)) == -2  # more than 1024 experts
+    assert lib.moe_cache_state_bytes(8, 0, ctypes.byref(b)) == -2
+    # the layer needs S >= min(E, T*k) slots; checked before any device call
+    lib.moe_layer_forward_cached.argtypes = [vp] * 9 + [i32, vp, vp, vp, vp] + [i32] * 6 + \
+        [ctypes.c_double, i32, vp, vp, sz, vp, vp]
+    args = [16] * 9
+    assert lib.moe_layer_forward_cached(*args, 15, 16, None, None, None, 0, 8, 128, 64, 2, 64, 1.0, 0,
+                                        16, 16, 1 << 20, None, None) == -2            # 15 < min(64, 16)
+    assert lib.moe_layer_forward_cached(*args, 65, 16, None, None, None, 0, 8, 128, 64, 2, 64, 1.0, 0,
+                                        16, 16, 1 << 20, None, None) == -2            # S > E
+    assert lib.moe_layer_forward_cached(*([16] * 8 + [None]), 16, 16, None, None, None, 0, 8, 128, 64, 2, 64,
+                                        1.0, 0, 16, 16, 1 << 20, None, None) == -1    # missing slots
+    assert lib.moe_layer_forward_cached(*([16] * 8 + [24]), 16, 16, None, None, None, 0, 8, 128, 64, 2, 64,
+                                        1.0, 0, 16, 16, 1 << 20, None, None) == -3    # misaligned slots
+
+
+def test_expert_parallel_host_checks(lib):
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    lib.moe_ep_workspace_bytes.argtypes = [i32, ctypes.POINTER(sz)]
+    b = sz(0)
+    assert lib.moe_ep_workspace_bytes(256, ctypes.byref(b)) == 0 and b.value > 3 * 257 * 4
+    assert lib.moe_ep_workspace_bytes(2048, ctypes.byref(b)) == -2
+    lib.moe_ep_plan.argtypes = [vp, i32, i32, i32, i64, i32, vp, sz, vp]
+    ws = 1 << 20
+    assert lib.moe_ep_plan(16, 3, 0, 16, -1, 100, 16, ws, None) == -2     # E not a multiple of R
+    assert lib.moe_ep_plan(16, 65, 0, 130, -1, 100, 16, ws, None) == -2   # more than 64 ranks
+    assert lib.moe_ep_plan(16, 4, 4, 16, -1, 100, 16, ws, None) == -2     # rank out of range
+    assert lib.moe_ep_plan(None, 4, 1, 16, -1, 100, 16, ws, None) == -1   # no counts
+    assert lib.moe_ep_plan(16, 4, 1, 16, -1, 100, 24, ws, None) == -3     # misaligned workspace
+    assert lib.moe_ep_plan(16, 4, 1, 16, -1, 100, 16, 64, None) == -4     # workspace too small
+    lib.moe_ep_dispatch.argtypes = [vp, i32, i32, i32, i32, vp, vp, sz, vp]
+    assert lib.moe_ep_dispatch(16, 2, 0, 8, 100, 16, 16, ws, None) == -2   # d not a multiple of 64
+    lib.moe_layer_permute.argtypes = [vp, i32, i32, i32, i32, i32, i32, i64, vp, vp, sz, vp]
+    assert lib.moe_layer_permute(16, 0, 8, 100, 8, 2, 64, -1, None, 16, ws, None) == -2

@@ -1,0 +1,83 @@
+"""Expert-parallel layer with R ranks emulated on one GPU (the library's put kernels move the rows
+between the ranks' buffers): the output of every rank against the layer oracle over the whole
+batch (capacity counted over all ranks), and bit for bit against the token-sharded layer that
+holds all experts on every rank."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from _util import assert_layer_close, bf16_bits, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def moe():
+    import moe_layer_router_b200 as m
+    assert torch.cuda.is_available()
+    return m
+
+
+# (R, T per rank, d, E, k, f, f_shared, cap_mode, cf, zipf)
+CASES = {
+    "r2": (2, 96, 256, 8, 2, 192, 0, synth.CAP_NONE, 1.0, 0.0),
+    "r4_shared_cap": (4, 64, 256, 16, 4, 128, 128, synth.CAP_PER_TOKEN, 1.25, 1.2),
+    "r4_decode": (4, 8, 448, 32, 8, 192, 0, synth.CAP_NONE, 1.0, 0.0),
+    "r2_pair_tiles": (2, 1024, 256, 4, 2, 256, 0, synth.CAP_PER_ASSIGNMENT, 1.1, 0.8),
+}
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_emulated_expert_parallel_layer(moe, case):
+    from moe_layer_router_b200.ep import EmulatedEP
+    R, T, d, E, k, f, fs, cap_mode, cf, zs = CASES[case]
+    wl = synth.Workload("ep_" + case, R * T, d, E, k, f, f_shared=fs, cap_mode=cap_mode, capacity_factor=cf,
+                        zipf_s=zs, seed=3)
+    inp = synth.Inputs(wl)
+    x = inp.x()
+    wg = inp.wg()
+    W1, W3, W2 = inp.w1(), inp.w3(), inp.w2()
+    sh = [inp.shared(n) for n in ("w1s", "w3s", "w2s")] if fs else [None] * 3
+    dv = to_dev_bf16
+    dW1, dW3, dW2, dwg = dv(W1), dv(W3), dv(W2), dv(wg)
+    dsh = [dv(a) if a is not None else None for a in sh]
+    xs = [dv(x[r * T:(r + 1) * T]) for r in range(R)]
+    outs = [torch.empty((T, d), dtype=torch.bfloat16, device="cuda") for _ in range(R)]
+    ep = EmulatedEP(R, T, d, E, k, f, fs)
+    ep.forward(xs, dwg, None, dW1, dW3, dW2, *dsh, cf, cap_mode, outs)
+    assert moe.moe_get_error() == 0
+
+    # the token-sharded layer, all experts on every rank, same global capacity
+    C = moe.moe_capacity(R * T, E, k, cf, cap_mode)
+    wss = [torch.empty(moe.moe_workspace_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device="cuda")
+           for _ in range(R)]
+    L = moe.moe_workspace_layout(T, d, E, k, f, fs)
+    for r in range(R):
+        moe.moe_layer_route_count(xs[r], dwg, None, fs, T, d, E, k, f, wss[r])
+    allc = torch.stack([moe.workspace_view(wss[r], L, "counts_raw", (E,), torch.int32) for r in range(R)])
+    outs_dp = []
+    for r in range(R):
+        fb = torch.empty(E, dtype=torch.int32, device="cuda")
+        moe.moe_fill_base(allc, R, r, E, fb)
+        o = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+        moe.moe_layer_finish(xs[r], dW1, dW3, dW2, *dsh, fs, T, d, E, k, f, C, fb, o, wss[r])
+        outs_dp.append(o)
+    assert moe.moe_get_error() == 0
+
+    # oracle over the whole batch, routing the GPU's logits
+    logits = np.concatenate([moe.workspace_view(b.ws, b.layout, "logits", (T, E), torch.float32).cpu().numpy()
+                             for b in ep.ranks])
+    ref = oracle.layer_forward(x, wg, W1, W3, W2, k=k, C=C, logits_in=logits, W1s=sh[0], W3s=sh[1], W2s=sh[2])
+    got = np.concatenate([bf16_bits(o) for o in outs])
+    assert_layer_close(got, ref["out"], "expert-parallel layer")
+    # every rank kept exactly the rows the whole-batch dispatch keeps
+    kept = sum(int(moe.workspace_view(b.ws, b.layout, "counts", (E,), torch.int32).sum()) for b in ep.ranks)
+    assert kept == ref["N"]
+    if cap_mode != synth.CAP_NONE:
+        assert kept < R * T * k          # capacity dropped rows
+    same_tiles = (R * T * k >= 256 * E) == (T * k >= 256 * E)
+    if same_tiles:   # same tile kind in both paths: each row's arithmetic is the same
+        for r in range(R):
+            assert torch.equal(outs[r].view(torch.int16), outs_dp[r].view(torch.int16)), f"rank {r}"

@@ -381,3 +381,55 @@ def test_pipeline_matches_layer_forward_batch_by_batch(moe):
                               wl.capacity_factor, wl.cap_mode, ref, ws)
         assert torch.equal(outs[b].view(torch.int16), ref.cpu().view(torch.int16)), f"batch {b}"
     assert moe.moe_get_error() == 0
+
+
+# ----------------------------------------------------------------------------- fp8 expert weights
+
+def _q8_reference(wl, x, logits, inp, k, C):
+    """Oracle layer with fp8 experts: route the GPU's logits, dispatch, fp8 experts, combine."""
+    E, d, f = wl.E, wl.d, wl.f
+    idx, w = oracle.route(logits, k, inp.bias())
+    r = oracle.dispatch(idx, E, C)
+    y_perm = np.zeros((max(r["N"], 1), d), np.uint16)
+    for e in range(E):
+        a, b = r["offsets"][e], r["offsets"][e + 1]
+        if a == b:
+            continue
+        q1, s1 = synth.quantize_e4m3_rows(inp.expert_rows("w1", e, 1), d)
+        q3, s3 = synth.quantize_e4m3_rows(inp.expert_rows("w3", e, 1), d)
+        q2, s2 = synth.quantize_e4m3_rows(inp.expert_rows("w2", e, 1), f)
+        _, y_perm[a:b] = oracle.expert_ffn_q8(oracle.gather(x, r["dest"], r["N"])[a:b], q1, s1, q3, s3, q2, s2)
+    ysh = None
+    if wl.has_shared:
+        qs = {n: synth.quantize_e4m3_rows(inp.shared(n), inp.shared(n).shape[1]) for n in ("w1s", "w3s", "w2s")}
+        _, ysh = oracle.expert_ffn_q8(x, qs["w1s"][0], qs["w1s"][1], qs["w3s"][0], qs["w3s"][1], qs["w2s"][0],
+                                      qs["w2s"][1])
+    return idx, r, oracle.combine(y_perm, r["dest"], w, ysh)
+
+
+@pytest.mark.parametrize("wl", [synth.Workload("q8", 300, 256, 16, 4, 320, f_shared=192, bias_range=0.1,
+                                               cap_mode=synth.CAP_PER_TOKEN, capacity_factor=1.5),
+                                synth.Workload("q8dec", 40, 448, 32, 8, 192, f_shared=128, bias_range=0.1),
+                                synth.Workload("q8mix", 512, 256, 16, 2, 192, zipf_s=1.2)],
+                         ids=["shared-cap-bias", "decode-shaped", "skewed-mixed-tiles"])
+def test_layer_fp8_weights(moe, wl):
+    T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
+    inp = synth.Inputs(wl)
+    x = inp.x()
+    Q = synth.device_tensors_q8(wl, "cuda")
+    ws = _ws(moe, T, d, E, k, f, fs)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    bias = torch.from_numpy(inp.bias()).cuda() if inp.bias() is not None else None
+    moe.moe_layer_forward_w8(to_dev_bf16(x), to_dev_bf16(inp.wg()), bias, Q["w1q"], Q["s1"], Q["w3q"], Q["s3"],
+                             Q["w2q"], Q["s2"], Q.get("w1sq"), Q.get("s1s"), Q.get("w3sq"), Q.get("s3s"),
+                             Q.get("w2sq"), Q.get("s2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, out, ws)
+    assert moe.moe_get_error() == 0
+    L = moe.moe_workspace_layout(T, d, E, k, f, fs)
+    logits = moe.workspace_view(ws, L, "logits", (T, E), torch.float32).cpu().numpy()
+    C = oracle.capacity(T, E, k, wl.capacity_factor, wl.cap_mode)
+    idx, r, ref = _q8_reference(wl, x, logits, inp, k, C)
+    assert np.array_equal(moe.workspace_view(ws, L, "idx", (T, k), torch.int32).cpu().numpy(), idx)
+    assert np.array_equal(moe.workspace_view(ws, L, "dest", (T, k), torch.int32).cpu().numpy(), r["dest"])
+    got = bf16_bits(out)
+    assert_layer_close(got, ref, "fp8-weight layer")
+    assert np.mean(ulp_bf16(got, ref) <= 1) > 0.98
