@@ -60,6 +60,9 @@ def parse():
                          "slots; expert weights in page-locked host memory; a fresh token batch every step")
     ap.add_argument("--cache-tokens", type=int, default=16, help="decode batch (tokens per step) with --cache-slots")
     ap.add_argument("--cache-zipf", type=float, default=1.0, help="Zipf exponent of expert popularity (cache runs)")
+    ap.add_argument("--ep-ranks", type=int, default=0,
+                    help="> 0: expert parallelism with this many ranks emulated on one GPU (the workload's batch "
+                         "split over the ranks, experts split contiguously); prints its own line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
@@ -379,6 +382,94 @@ def run_cached(args, base, rank, world, local):
         dist.destroy_process_group()
 
 
+def run_ep(args, wl, local):
+    """The workload's batch split over R expert-parallel ranks emulated on one GPU (ep.EmulatedEP):
+    every rank routes its T / R tokens, the row ranges move between the ranks' buffers by the
+    library's put kernels, each rank runs its E / R experts.  Timed beside the single-GPU layer
+    on the same batch.  The exchange kernels' roofline is the HBM copy bandwidth here (on several
+    GPUs it would be the NVLink bandwidth); bytes = rows moved x d x 2 B, read + written, both ways."""
+    import torch
+    import moe_layer_router_b200 as moe
+    from moe_layer_router_b200.ep import EmulatedEP
+
+    R = args.ep_ranks
+    T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
+    if T % R or E % R:
+        raise SystemExit("--ep-ranks must divide T and E")
+    Tr = T // R
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    W = synth.device_tensors(wl, dev, names=["x", "wg", "w1", "w3", "w2", "w1s", "w3s", "w2s", "bias"])
+    xs = [W["x"][r * Tr:(r + 1) * Tr] for r in range(R)]
+    outs = [torch.empty((Tr, d), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+    ep = EmulatedEP(R, Tr, d, E, k, f, fs, device=dev)
+
+    def step(events=None):
+        ep.forward(xs, W["wg"], W["bias"], W["w1"], W["w3"], W["w2"], W.get("w1s"), W.get("w3s"), W.get("w2s"),
+                   wl.capacity_factor, wl.cap_mode, outs, events)
+
+    ws = torch.empty(moe.moe_workspace_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device=dev)
+    out1 = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+
+    def single():
+        moe.moe_layer_forward(W["x"], W["wg"], W["bias"], W["w1"], W["w3"], W["w2"], W.get("w1s"), W.get("w3s"),
+                              W.get("w2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, out1, ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+        single()
+    torch.cuda.synchronize()
+    if moe.moe_get_error() != 0:
+        raise RuntimeError("device error after warm-up")
+    K = args.steps
+    evs = [{n: torch.cuda.Event(enable_timing=True) for n in EmulatedEP.STAGES} for _ in range(K)]
+    for e in evs:
+        for ev in e.values():
+            ev.record()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            step(evs[i])
+        torch.cuda.synchronize()
+    total_ms = evs[0]["route"].elapsed_time(evs[K - 1]["end"])
+    st = EmulatedEP.STAGES
+    stage_ms = {a: float(np.mean([e[a].elapsed_time(e[b]) for e in evs])) for a, b in zip(st[:-1], st[1:])}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K):
+        single()
+    e1.record()
+    torch.cuda.synchronize()
+    single_ms = e0.elapsed_time(e1)
+    if moe.moe_get_error() != 0:
+        raise RuntimeError("device error")
+    N = sum(int(moe.workspace_view(b.ws, b.layout, "counts", (E,), torch.int32).sum()) for b in ep.ranks)
+    moved = 2 * N * d * 2                       # rows out and back, bf16
+    put_ms = stage_ms["dispatch"] + stage_ms["return"]
+    achieved = 2 * moved / 1e9 / (put_ms / 1e3)  # read + write
+    peaks, peak_src = load_peaks()
+    line = {
+        "metric": "MoE-layer tokens/s on 1 B200, experts split over R expert-parallel ranks emulated on the GPU",
+        "value": T * K / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": K, "warmup": max(3, args.warmup),
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded Philox4x32-10 + Box-Muller; random-init weights)",
+        "config": {"workload": DESCR.get(wl.name, wl.name) + f", split over {R} emulated expert-parallel ranks "
+                               f"({Tr} tokens and {E // R} experts each)",
+                   "global_batch": T, "seq_len": T, "parallelism": f"ep{R} (emulated on one GPU)",
+                   "l2": "working set larger than L2 (expert weights streamed every step)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "kernel": "ep_put_rows_kernel (dispatch + return row ranges between the ranks' buffers)",
+                     "peak_source": f"{peak_src} (hbm_gbs, burst)", "algorithmic_per_launch": 2 * moved / (2 * R)},
+        "single_gpu_layer_ms": single_ms / K,
+        "stages_ms": stage_ms,
+        "e2e": None,
+        "gpu_launches": None,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     wl = synth.WORKLOADS[args.workload]
@@ -389,6 +480,8 @@ def main():
         return run_reference(args, wl, rank, world)
     if args.cache_slots > 0:
         return run_cached(args, wl, rank, world, local)
+    if args.ep_ranks > 0:
+        return run_ep(args, wl, local)
 
     import torch
     import torch.distributed as dist

@@ -12,12 +12,12 @@
 //
 // Roles (448 threads, one CTA per SM): warp 0 TMA producer, warp 1 TMEM allocator + MMA
 // issuer, warps 2-5 epilogue, warps 6-13 converters.  Two rings:
-//   load ring (5 stages)  A [128 x 64] bf16, 128-byte swizzle (only the first 32 rows are loaded
+//   load ring (4 stages)  A [128 x 64] bf16, 128-byte swizzle (only the first 32 rows are loaded
 //                         when the tile has <= 32 rows: the other rows only feed accumulator rows
 //                         that are never stored), and Q [256 x 64] fp8, unswizzled rows of 64
 //                         bytes; both by TMA, so the A tile of a k-block is requested as early as
 //                         its weights
-//   B ring (2 stages)     [256 x 64] bf16, 128-byte swizzle, written by the converters
+//   B ring (3 stages)     [256 x 64] bf16, 128-byte swizzle, written by the converters
 // Barriers: full (TMA bytes of A + Q), load_empty (MMA commit), b_full (8 converter warps),
 // b_empty (MMA commit).
 #pragma once
@@ -28,8 +28,8 @@
 
 namespace moe {
 
-constexpr int W8_LSTAGES = 5;
-constexpr int W8_BSTAGES = 2;
+constexpr int W8_LSTAGES = 4;     // 4 + 3 measured best of {5+2, 4+3} x {8, 12, 16} converter warps
+constexpr int W8_BSTAGES = 3;
 constexpr int W8_THREADS = 448;
 constexpr int W8_A_BYTES = GEMM_BM * GEMM_BK * 2;   // 16 KB
 constexpr int W8_Q_BYTES = 256 * GEMM_BK;           // 16 KB

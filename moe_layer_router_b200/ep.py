@@ -84,14 +84,25 @@ class EmulatedEP:
         import torch
         self.all_counts = torch.empty((R, E), dtype=torch.int32, device=device)
 
-    def forward(self, xs: List, Wg, bias, W1, W3, W2, W1s, W3s, W2s, capacity_factor, cap_mode, outs: List) -> None:
+    STAGES = ["route", "permute", "dispatch", "experts", "return", "combine", "end"]
+
+    def forward(self, xs: List, Wg, bias, W1, W3, W2, W1s, W3s, W2s, capacity_factor, cap_mode, outs: List,
+                events: Optional[dict] = None) -> None:
         """xs[r]: rank r's tokens [T, d]; W1/W3/W2: all experts (rank r uses its El-expert slice);
-        outs[r]: [T, d].  Capacity counts the whole batch of R * T tokens."""
+        outs[r]: [T, d].  Capacity counts the whole batch of R * T tokens.  events: optional
+        {stage: torch.cuda.Event} recorded on the current stream before each phase (STAGES)."""
         moe, R, T, d, E, k, f, fs = self.moe, self.R, self.T, self.d, self.E, self.k, self.f, self.fs
         El = E // R
+
+        def mark(name):
+            if events and events.get(name) is not None:
+                events[name].record()
+
         C = moe.moe_capacity(R * T, E, k, capacity_factor, cap_mode)
+        mark("route")
         for r, b in enumerate(self.ranks):
             moe.moe_layer_route_count(xs[r], Wg, bias, fs, T, d, E, k, f, b.ws)
+        mark("permute")
         for r, b in enumerate(self.ranks):          # the all-gather of raw counts
             self.all_counts[r].copy_(b.view(moe, "counts_raw", (E,), self.all_counts.dtype))
         for r, b in enumerate(self.ranks):
@@ -99,18 +110,23 @@ class EmulatedEP:
             moe.moe_layer_permute(xs[r], fs, T, d, E, k, f, C, b.fill_base, b.ws)
             moe.moe_ep_plan(self.all_counts, R, r, E, C, self.max_recv, b.ep_ws)
         recv = [b.recv for b in self.ranks]
+        mark("dispatch")
         for r, b in enumerate(self.ranks):
             moe.moe_ep_dispatch(b.view(moe, "x_perm", (T * k, d), xs[r].dtype), R, r, E, d, recv, b.ep_ws)
+        mark("experts")
         for r, b in enumerate(self.ranks):
             sl = slice(r * El, (r + 1) * El)
             moe.moe_ep_expert_ffn(b.recv, self.max_recv, R, r, E, d, f, W1[sl], W3[sl], W2[sl], b.h, b.y_recv, xs[r],
                                   T, W1s, W3s, W2s, fs, b.h_shared, b.y_shared, b.ep_ws)
         y_perm = [b.view(moe, "y_perm", (T * k, d), xs[r].dtype) for r, b in enumerate(self.ranks)]
+        mark("return")
         for r, b in enumerate(self.ranks):
             moe.moe_ep_return(b.y_recv, R, r, E, d, y_perm, b.ep_ws)
+        mark("combine")
         for r, b in enumerate(self.ranks):
             moe.moe_combine(y_perm[r], b.view(moe, "dest", (T, k), self.all_counts.dtype),
                             b.view(moe, "w", (T, k), _f32()), b.y_shared, T, d, k, outs[r])
+        mark("end")
 
 
 def _f32():
