@@ -76,9 +76,11 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(fp8: bool = False) -> str:
+    """Hash of the sources of the grouped GEMM kernels (bf16, or the fp8-weight one)."""
     h = hashlib.sha256()
-    for n in ("grouped_gemm.cuh", "grouped_gemm_pair.cuh", "ptx.cuh"):
+    files = ("grouped_gemm.cuh", "grouped_gemm_pair.cuh", "ptx.cuh") + (("grouped_gemm_w8.cuh",) if fp8 else ())
+    for n in files:
         h.update(open(os.path.join(ROOT, "moe_layer_router_b200", "csrc", n), "rb").read())
     return h.hexdigest()[:16]
 
@@ -88,7 +90,7 @@ def recorded_traffic(kernel: str, workload: str):
     p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(p):
         return None
-    src = kernel_source_hash()
+    src = kernel_source_hash(kernel.endswith("_fp8"))
     for line in open(p):
         parts = line.split()
         if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload \
