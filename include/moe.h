@@ -308,15 +308,18 @@ int moe_layer_permute(const moe_bf16* x, int f_shared, int T, int d, int E, int 
  *   2. all-gather of counts_raw -> all_counts_raw [R, E] int32 on every rank (the caller's
  *      collective; rank order = token order of the whole batch)
  *   3. moe_fill_base() + moe_layer_permute()  global-capacity keep decisions, x_perm
- *   4. moe_ep_plan()                           from all_counts_raw alone: the rows this rank
- *      sends to / receives from every rank and the local GEMM segments (into ep_ws)
- *      moe_ep_dispatch()                       puts this rank's x_perm rows into the receive
- *      buffers of the experts' ranks; receive rows are in (source rank, local expert) order
- *      (a caller with a collective library can move the same row ranges with an
- *      all-to-all-v instead: rank r sends rows_kept(r, experts of q) to q, in q order)
+ *   4. moe_ep_plan()                           from all_counts_raw alone: the row ranges this
+ *      rank sends and returns, and the groups of its local GEMM (into ep_ws)
+ *      moe_ep_dispatch()                       puts this rank's x_perm rows of each expert into
+ *      the receive buffer of the expert's rank, in expert-major order there (the rows of one
+ *      local expert from all ranks are contiguous, in rank order), so each local expert is one
+ *      GEMM group and its weights are read once
+ *      (a caller with a collective library can move the rows with an all-to-all-v instead:
+ *      rank r sends its rows of q's experts to q; they arrive source-major, and
+ *      moe_ep_expert_ffn(source_major = 1) runs one segment per (source rank, local expert))
  *   5. a barrier (every rank's puts done before any rank reads its receive buffer)
- *   6. moe_ep_expert_ffn()                     local experts over the received rows (one GEMM
- *      segment per source rank and local expert) + the shared expert on the rank's own tokens
+ *   6. moe_ep_expert_ffn()                     local experts over the received rows + the
+ *      shared expert on the rank's own tokens
  *   7. moe_ep_return()                         puts each result row back into the y_perm (layer
  *      workspace) of the rank it came from, at the row it had in that rank's x_perm
  *   8. a barrier, then moe_combine() with the rank's dest, w (layer workspace) and y_shared
@@ -326,15 +329,18 @@ int moe_layer_permute(const moe_bf16* x, int f_shared, int T, int d, int E, int 
  * this device can write (peer-mapped buffers of other GPUs, or the same GPU's buffers when
  * ranks share a device).  A receive buffer holds max_recv_rows rows of d bf16 (>= the rows the
  * rank can receive: R * T * k bounds it).  ep_ws: moe_ep_workspace_bytes(E) bytes, 16-byte
- * aligned, written by moe_ep_plan() and read by the later calls on the same rank.
+ * aligned (moe_ep_workspace_bytes(R, E)), written by moe_ep_plan() and read by the later calls
+ * on the same rank.
  * Errors: MOE_ERR_SHAPE unless 1 <= R <= 64, E % R == 0, E <= 1024, 0 <= rank < R.
+ * moe_ep_expert_ffn: source_major = 0 after moe_ep_dispatch(), 1 after an all-to-all-v.
  */
-int moe_ep_workspace_bytes(int E, size_t* bytes);
+int moe_ep_workspace_bytes(int R, int E, size_t* bytes);
 int moe_ep_plan(const int32_t* all_counts_raw, int R, int rank, int E, int64_t capacity, int max_recv_rows,
                 void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream);
 int moe_ep_dispatch(const moe_bf16* x_perm, int R, int rank, int E, int d, moe_bf16* const* recv_bufs,
                     const void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream);
-int moe_ep_expert_ffn(const moe_bf16* recv_x, int max_recv_rows, int R, int rank, int E, int d, int f,
+int moe_ep_expert_ffn(const moe_bf16* recv_x, int max_recv_rows, int source_major, int R, int rank, int E, int d,
+                      int f,
                       const moe_bf16* W1_local, const moe_bf16* W3_local, const moe_bf16* W2_local, moe_bf16* h,
                       moe_bf16* y_recv, const moe_bf16* x, int T, const moe_bf16* W1s, const moe_bf16* W3s,
                       const moe_bf16* W2s, int f_shared, moe_bf16* h_shared, moe_bf16* y_shared, const void* ep_ws,

@@ -77,13 +77,13 @@ _lib.moe_layer_forward_cached.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp
 _lib.moe_layer_forward_cached.restype = _i32
 _lib.moe_layer_permute.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _i32, _i64, _vp, _vp, _sz, _vp]
 _lib.moe_layer_permute.restype = _i32
-_lib.moe_ep_workspace_bytes.argtypes = [_i32, ctypes.POINTER(_sz)]
+_lib.moe_ep_workspace_bytes.argtypes = [_i32, _i32, ctypes.POINTER(_sz)]
 _lib.moe_ep_workspace_bytes.restype = _i32
 _lib.moe_ep_plan.argtypes = [_vp, _i32, _i32, _i32, _i64, _i32, _vp, _sz, _vp]
 _lib.moe_ep_plan.restype = _i32
 _lib.moe_ep_dispatch.argtypes = [_vp, _i32, _i32, _i32, _i32, ctypes.POINTER(_vp), _vp, _sz, _vp]
 _lib.moe_ep_dispatch.restype = _i32
-_lib.moe_ep_expert_ffn.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp,
+_lib.moe_ep_expert_ffn.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp,
                                    _vp, _vp, _i32, _vp, _vp, _vp, _sz, _vp]
 _lib.moe_ep_expert_ffn.restype = _i32
 _lib.moe_ep_return.argtypes = [_vp, _i32, _i32, _i32, _i32, ctypes.POINTER(_vp), _vp, _sz, _vp]
@@ -360,9 +360,9 @@ def moe_layer_permute(x, f_shared, T, d, E, k, f, capacity, fill_base, ws, strea
                                   _nbytes(ws), _stream(stream)), "moe_layer_permute")
 
 
-def moe_ep_workspace_bytes(E: int) -> int:
+def moe_ep_workspace_bytes(R: int, E: int) -> int:
     out = _sz(0)
-    _check(_lib.moe_ep_workspace_bytes(E, ctypes.byref(out)), "moe_ep_workspace_bytes")
+    _check(_lib.moe_ep_workspace_bytes(R, E, ctypes.byref(out)), "moe_ep_workspace_bytes")
     return int(out.value)
 
 
@@ -385,8 +385,11 @@ def moe_ep_dispatch(x_perm, R, rank, E, d, recv_bufs, ep_ws, stream=None) -> Non
 
 
 def moe_ep_expert_ffn(recv_x, max_recv_rows, R, rank, E, d, f, W1_local, W3_local, W2_local, h, y_recv, x, T, W1s, W3s,
-                      W2s, f_shared, h_shared, y_shared, ep_ws, stream=None) -> None:
-    _check(_lib.moe_ep_expert_ffn(_ptr(recv_x), max_recv_rows, R, rank, E, d, f, _ptr(W1_local), _ptr(W3_local),
+                      W2s, f_shared, h_shared, y_shared, ep_ws, source_major=False, stream=None) -> None:
+    """source_major: the received rows came by an all-to-all-v (source-major) rather than by
+    moe_ep_dispatch (expert-major)."""
+    _check(_lib.moe_ep_expert_ffn(_ptr(recv_x), max_recv_rows, int(bool(source_major)), R, rank, E, d, f,
+                                  _ptr(W1_local), _ptr(W3_local),
                                   _ptr(W2_local), _ptr(h), _ptr(y_recv), _ptr(x), T, _ptr(W1s), _ptr(W3s), _ptr(W2s),
                                   f_shared, _ptr(h_shared), _ptr(y_shared), _ptr(ep_ws), _nbytes(ep_ws),
                                   _stream(stream)), "moe_ep_expert_ffn")

@@ -86,13 +86,14 @@ int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, ui
 }
 
 // 2-D fp8 (byte) tensor map [rows, inner], box [box_rows, 64 bytes], unswizzled, zero fill outside.
+// fp8 weights [rows, inner] bytes: boxes of box_rows rows x 64 bytes, 64-byte swizzle.
 int make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
     cuuint64_t dims[2] = {inner, rows};
     cuuint64_t strides[1] = {inner};
     cuuint32_t box[2] = {(cuuint32_t)GEMM_BK, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -949,29 +950,19 @@ int moe_layer_permute(const moe_bf16* x, int f_shared, int T, int d, int E, int 
 
 namespace {
 
-struct EpLayout {
-    size_t plan, seg_off, mprefix, group_map, total;
-};
-
-EpLayout ep_layout(int E) {
-    EpLayout L;
-    size_t o = 0;
-    L.plan = o; o += moe::align256(sizeof(moe::EpPlan));
-    L.seg_off = o; o += moe::align256((size_t)(E + 1) * 4);
-    L.mprefix = o; o += moe::align256((size_t)(E + 1) * 4);
-    L.group_map = o; o += moe::align256((size_t)E * 4);
-    L.total = o;
-    return L;
-}
-
 int ep_check(int R, int rank, int E, int d) {
     MOE_REQUIRE(R >= 1 && R <= moe::EP_MAX_RANKS && rank >= 0 && rank < R, MOE_ERR_SHAPE);
-    MOE_REQUIRE(E >= 1 && E <= 1024 && E % R == 0, MOE_ERR_SHAPE);
+    MOE_REQUIRE(E >= 1 && E <= moe::EP_MAX_EXPERTS && E % R == 0, MOE_ERR_SHAPE);
     MOE_REQUIRE(d >= 64 && d % 64 == 0, MOE_ERR_SHAPE);
     return MOE_OK;
 }
 
-int ep_put(const void* src, int which, moe_bf16* const* dests, int R, int d, const void* ep_ws, cudaStream_t s) {
+size_t ep_bytes(int R, int E) {
+    size_t off[8];
+    return moe::ep_layout_bytes(R, E, off);
+}
+
+int ep_put(const void* src, const int32_t* table, moe_bf16* const* dests, int R, int E, int d, cudaStream_t s) {
     using namespace moe;
     EpDests dst;
     memset(&dst, 0, sizeof(dst));
@@ -982,19 +973,19 @@ int ep_put(const void* src, int which, moe_bf16* const* dests, int R, int d, con
     DeviceInfo* di;
     int rc = device_info(&di);
     if (rc != MOE_OK) return rc;
-    const EpLayout L = ep_layout(1);
-    const EpPlan* plan = reinterpret_cast<const EpPlan*>(static_cast<const char*>(ep_ws) + L.plan);
-    const int bx = std::max(1, (2 * di->sms + R - 1) / R);
-    ep_put_rows_kernel<<<dim3(bx, R), 256, 0, s>>>(plan, which, static_cast<const uint4*>(src), dst, (long long)d / 8);
+    const int bx = std::max(1, std::min(8, (2 * di->sms + E - 1) / E));
+    ep_put_rows_kernel<<<dim3(bx, E), 256, 0, s>>>(table, E, E / R, static_cast<const uint4*>(src), dst,
+                                                    (long long)d / 8);
     return launch_status();
 }
 
 }  // namespace
 
-int moe_ep_workspace_bytes(int E, size_t* bytes) {
+int moe_ep_workspace_bytes(int R, int E, size_t* bytes) {
     MOE_REQUIRE(bytes, MOE_ERR_INVALID_ARG);
-    MOE_REQUIRE(E >= 1 && E <= 1024, MOE_ERR_SHAPE);
-    *bytes = ep_layout(E).total;
+    int rc = ep_check(R, 0, E, 64);
+    if (rc != MOE_OK) return rc;
+    *bytes = ep_bytes(R, E);
     return MOE_OK;
 }
 
@@ -1006,18 +997,13 @@ int moe_ep_plan(const int32_t* all_counts_raw, int R, int rank, int E, int64_t c
     MOE_REQUIRE(max_recv_rows >= 0, MOE_ERR_SHAPE);
     MOE_REQUIRE(all_counts_raw && ep_ws, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(aligned16(ep_ws), MOE_ERR_ALIGN);
-    const EpLayout L = ep_layout(E);
-    MOE_REQUIRE(ep_ws_bytes >= L.total, MOE_ERR_WORKSPACE);
+    MOE_REQUIRE(ep_ws_bytes >= ep_bytes(R, E), MOE_ERR_WORKSPACE);
     DeviceInfo* di;
     if ((rc = device_info(&di)) != MOE_OK) return rc;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    char* b = static_cast<char*>(ep_ws);
-    const bool pair = use_pair_tiles(max_recv_rows, E);
-    ep_plan_kernel<<<1, 1024, 0, s>>>(all_counts_raw, R, E, rank, capacity < 0 ? -1 : (long long)capacity,
-                                      pair ? PAIR_BM : GEMM_BM, reinterpret_cast<EpPlan*>(b + L.plan),
-                                      reinterpret_cast<int32_t*>(b + L.seg_off), reinterpret_cast<int32_t*>(b + L.mprefix));
-    if ((rc = launch_status()) != MOE_OK) return rc;
-    ep_group_map_kernel<<<(E + 255) / 256, 256, 0, s>>>(R, E / R, reinterpret_cast<int32_t*>(b + L.group_map));
+    const bool pair = use_pair_tiles(max_recv_rows, E / R);
+    ep_plan_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
+        all_counts_raw, R, E, rank, capacity < 0 ? -1 : (long long)capacity, pair ? PAIR_BM : GEMM_BM,
+        ep_view(ep_ws, R, E));
     return launch_status();
 }
 
@@ -1028,12 +1014,13 @@ int moe_ep_dispatch(const moe_bf16* x_perm, int R, int rank, int E, int d, moe_b
     if (rc != MOE_OK) return rc;
     MOE_REQUIRE(x_perm && recv_bufs && ep_ws, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(aligned16(x_perm) && aligned16(ep_ws), MOE_ERR_ALIGN);
-    MOE_REQUIRE(ep_ws_bytes >= ep_layout(E).total, MOE_ERR_WORKSPACE);
-    return ep_put(x_perm, 0, recv_bufs, R, d, ep_ws, static_cast<cudaStream_t>(stream));
+    MOE_REQUIRE(ep_ws_bytes >= ep_bytes(R, E), MOE_ERR_WORKSPACE);
+    const EpView v = ep_view(const_cast<void*>(ep_ws), R, E);
+    return ep_put(x_perm, v.send, recv_bufs, R, E, d, static_cast<cudaStream_t>(stream));
 }
 
-int moe_ep_expert_ffn(const moe_bf16* recv_x, int max_recv_rows, int R, int rank, int E, int d, int f,
-                      const moe_bf16* W1_local, const moe_bf16* W3_local, const moe_bf16* W2_local, moe_bf16* h,
+int moe_ep_expert_ffn(const moe_bf16* recv_x, int max_recv_rows, int source_major, int R, int rank, int E, int d,
+                      int f, const moe_bf16* W1_local, const moe_bf16* W3_local, const moe_bf16* W2_local, moe_bf16* h,
                       moe_bf16* y_recv, const moe_bf16* x, int T, const moe_bf16* W1s, const moe_bf16* W3s,
                       const moe_bf16* W2s, int f_shared, moe_bf16* h_shared, moe_bf16* y_shared, const void* ep_ws,
                       size_t ep_ws_bytes, moe_stream_t stream) {
@@ -1049,27 +1036,34 @@ int moe_ep_expert_ffn(const moe_bf16* recv_x, int max_recv_rows, int R, int rank
                     aligned16(h) && aligned16(y_recv) && aligned16(x) && aligned16(W1s) && aligned16(W3s) &&
                     aligned16(W2s) && aligned16(h_shared) && aligned16(y_shared) && aligned16(ep_ws),
                 MOE_ERR_ALIGN);
-    const EpLayout L = ep_layout(E);
-    MOE_REQUIRE(ep_ws_bytes >= L.total, MOE_ERR_WORKSPACE);
+    MOE_REQUIRE(ep_ws_bytes >= ep_bytes(R, E), MOE_ERR_WORKSPACE);
     DeviceInfo* di;
     if ((rc = device_info(&di)) != MOE_OK) return rc;
-    const char* b = static_cast<const char*>(ep_ws);
+    const EpView v = ep_view(const_cast<void*>(ep_ws), R, E);
+    const int El = E / R;
     FfnArgs a;
     memset(&a, 0, sizeof(a));
     a.x_perm = recv_x;
-    a.offsets = max_recv_rows > 0 ? reinterpret_cast<const int32_t*>(b + L.seg_off) : nullptr;
-    a.mprefix = reinterpret_cast<const int32_t*>(b + L.mprefix);
     a.max_rows = max_recv_rows;
-    a.E = E;                       // R * El segments
+    if (source_major) {            // one segment per (source rank, local expert)
+        a.offsets = v.seg_off;
+        a.mprefix = v.seg_tiles;
+        a.E = E;
+        a.group_map = v.group_map;
+        a.w_groups = El;
+    } else {                       // expert-major: one group per local expert
+        a.offsets = v.exp_off;
+        a.mprefix = v.exp_tiles;
+        a.E = El;
+    }
+    if (max_recv_rows == 0) a.offsets = nullptr;
     a.d = d;
     a.f = f;
     a.W1 = W1_local; a.W3 = W3_local; a.W2 = W2_local;
     a.h = h; a.y_perm = y_recv;
     a.x = x; a.T = T; a.f_shared = f_shared; a.W1s = W1s; a.W3s = W3s; a.W2s = W2s;
     a.h_shared = h_shared; a.y_shared = y_shared;
-    a.pair = use_pair_tiles(max_recv_rows, E);
-    a.group_map = reinterpret_cast<const int32_t*>(b + L.group_map);
-    a.w_groups = E / R;
+    a.pair = use_pair_tiles(max_recv_rows, El);
     if (max_recv_rows == 0 && !shared) return MOE_OK;
     return run_expert_ffn(di, a, static_cast<cudaStream_t>(stream));
 }
@@ -1081,8 +1075,9 @@ int moe_ep_return(const moe_bf16* y_recv, int R, int rank, int E, int d, moe_bf1
     if (rc != MOE_OK) return rc;
     MOE_REQUIRE(y_recv && y_perm_bufs && ep_ws, MOE_ERR_INVALID_ARG);
     MOE_REQUIRE(aligned16(y_recv) && aligned16(ep_ws), MOE_ERR_ALIGN);
-    MOE_REQUIRE(ep_ws_bytes >= ep_layout(E).total, MOE_ERR_WORKSPACE);
-    return ep_put(y_recv, 1, y_perm_bufs, R, d, ep_ws, static_cast<cudaStream_t>(stream));
+    MOE_REQUIRE(ep_ws_bytes >= ep_bytes(R, E), MOE_ERR_WORKSPACE);
+    const EpView v = ep_view(const_cast<void*>(ep_ws), R, E);
+    return ep_put(y_recv, v.back, y_perm_bufs, R, E, d, static_cast<cudaStream_t>(stream));
 }
 
 int moe_update_bias(const int32_t* counts_raw, int E, int64_t capacity, float* bias, moe_stream_t stream) {

@@ -10,10 +10,12 @@ all-to-all-v exchanges.
 
 Two drivers:
   * ``EmulatedEP``: R ranks on one device in one process.  The row exchanges are the library's
-    put kernels writing into the other ranks' buffers; the all-gather is a device copy.
+    put kernels writing into the other ranks' buffers (expert-major receive order, one GEMM group
+    per local expert); the all-gather is a device copy.
   * ``ep_layer_forward_dist``: one process per GPU over ``torch.distributed``; counts are
     all-gathered and rows moved with ``all_to_all_single`` (NCCL), whose split sizes
-    ``ep_row_splits`` computes on the host from the gathered counts.
+    ``ep_row_splits`` computes on the host from the gathered counts; rows arrive source-major and
+    the local GEMM runs one segment per (source rank, local expert).
 """
 from __future__ import annotations
 
@@ -54,11 +56,11 @@ def exchange_rows(src, send_rows: Sequence[int], recv_rows: Sequence[int], out, 
 
 
 class _RankBuffers:
-    def __init__(self, moe, T, d, E, k, f, fs, max_recv, device):
+    def __init__(self, moe, R, T, d, E, k, f, fs, max_recv, device):
         import torch
         self.ws = torch.empty(moe.moe_workspace_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device=device)
         self.layout = moe.moe_workspace_layout(T, d, E, k, f, fs)
-        self.ep_ws = torch.empty(moe.moe_ep_workspace_bytes(E), dtype=torch.uint8, device=device)
+        self.ep_ws = torch.empty(moe.moe_ep_workspace_bytes(R, E), dtype=torch.uint8, device=device)
         self.fill_base = torch.empty(E, dtype=torch.int32, device=device)
         rows = max(1, max_recv)
         self.recv = torch.empty((rows, d), dtype=torch.bfloat16, device=device)
@@ -74,13 +76,19 @@ class _RankBuffers:
 class EmulatedEP:
     """R expert-parallel ranks on one device (one process, one stream)."""
 
-    def __init__(self, R, T, d, E, k, f, f_shared=0, device="cuda"):
+    def __init__(self, R, T, d, E, k, f, f_shared=0, device="cuda", exchange="put"):
+        """exchange: "put" moves rows with the library's put kernels (expert-major receive order);
+        "a2a" moves them like an all-to-all-v would (source-major, device copies sized on the
+        host from the gathered counts) and runs the source-major GEMM segments."""
         import moe_layer_router_b200 as moe
         if E % R:
             raise ValueError("E must be a multiple of R")
+        if exchange not in ("put", "a2a"):
+            raise ValueError("exchange must be 'put' or 'a2a'")
+        self.exchange = exchange
         self.moe, self.R, self.T, self.d, self.E, self.k, self.f, self.fs = moe, R, T, d, E, k, f, f_shared
         self.max_recv = R * T * k
-        self.ranks = [_RankBuffers(moe, T, d, E, k, f, f_shared, self.max_recv, device) for _ in range(R)]
+        self.ranks = [_RankBuffers(moe, R, T, d, E, k, f, f_shared, self.max_recv, device) for _ in range(R)]
         import torch
         self.all_counts = torch.empty((R, E), dtype=torch.int32, device=device)
 
@@ -110,23 +118,49 @@ class EmulatedEP:
             moe.moe_layer_permute(xs[r], fs, T, d, E, k, f, C, b.fill_base, b.ws)
             moe.moe_ep_plan(self.all_counts, R, r, E, C, self.max_recv, b.ep_ws)
         recv = [b.recv for b in self.ranks]
+        x_perm = [b.view(moe, "x_perm", (T * k, d), xs[r].dtype) for r, b in enumerate(self.ranks)]
+        y_perm = [b.view(moe, "y_perm", (T * k, d), xs[r].dtype) for r, b in enumerate(self.ranks)]
+        a2a = self.exchange == "a2a"
+        if a2a:     # split sizes on the host, as an all-to-all-v caller has them
+            counts = self.all_counts.cpu().numpy()
+            splits = [ep_row_splits(counts, C, r) for r in range(R)]
         mark("dispatch")
-        for r, b in enumerate(self.ranks):
-            moe.moe_ep_dispatch(b.view(moe, "x_perm", (T * k, d), xs[r].dtype), R, r, E, d, recv, b.ep_ws)
+        if a2a:
+            self._a2a([x_perm[r] for r in range(R)], recv, [sp[0] for sp in splits], [sp[1] for sp in splits])
+        else:
+            for r, b in enumerate(self.ranks):
+                moe.moe_ep_dispatch(x_perm[r], R, r, E, d, recv, b.ep_ws)
         mark("experts")
         for r, b in enumerate(self.ranks):
             sl = slice(r * El, (r + 1) * El)
             moe.moe_ep_expert_ffn(b.recv, self.max_recv, R, r, E, d, f, W1[sl], W3[sl], W2[sl], b.h, b.y_recv, xs[r],
-                                  T, W1s, W3s, W2s, fs, b.h_shared, b.y_shared, b.ep_ws)
-        y_perm = [b.view(moe, "y_perm", (T * k, d), xs[r].dtype) for r, b in enumerate(self.ranks)]
+                                  T, W1s, W3s, W2s, fs, b.h_shared, b.y_shared, b.ep_ws, source_major=a2a)
         mark("return")
-        for r, b in enumerate(self.ranks):
-            moe.moe_ep_return(b.y_recv, R, r, E, d, y_perm, b.ep_ws)
+        if a2a:
+            self._a2a([b.y_recv for b in self.ranks], y_perm, [sp[1] for sp in splits], [sp[0] for sp in splits])
+        else:
+            for r, b in enumerate(self.ranks):
+                moe.moe_ep_return(b.y_recv, R, r, E, d, y_perm, b.ep_ws)
         mark("combine")
         for r, b in enumerate(self.ranks):
             moe.moe_combine(y_perm[r], b.view(moe, "dest", (T, k), self.all_counts.dtype),
                             b.view(moe, "w", (T, k), _f32()), b.y_shared, T, d, k, outs[r])
         mark("end")
+
+
+    @staticmethod
+    def _a2a(srcs, dsts, send, recv):
+        """What all_to_all_single does, on one device: rank s's rows for rank q (send[s][q], in q
+        order) land in q's buffer after the rows of ranks < s (recv[q][s])."""
+        R = len(srcs)
+        for s in range(R):
+            o = 0
+            for q in range(R):
+                n = int(send[s][q])
+                if n:
+                    at = int(sum(recv[q][:s]))
+                    dsts[q][at:at + n].copy_(srcs[s][o:o + n])
+                o += n
 
 
 def _f32():
@@ -145,7 +179,7 @@ def ep_layer_forward_dist(x, Wg, bias, W1_local, W3_local, W2_local, W1s, W3s, W
 
     R, rank = dist.get_world_size(group), dist.get_rank(group)
     if bufs is None:
-        bufs = _RankBuffers(moe, T, d, E, k, f, f_shared, R * T * k, x.device)
+        bufs = _RankBuffers(moe, R, T, d, E, k, f, f_shared, R * T * k, x.device)
     C = moe.moe_capacity(R * T, E, k, capacity_factor, cap_mode)
     moe.moe_layer_route_count(x, Wg, bias, f_shared, T, d, E, k, f, bufs.ws)
     all_counts = torch.empty((R, E), dtype=torch.int32, device=x.device)
@@ -158,7 +192,7 @@ def ep_layer_forward_dist(x, Wg, bias, W1_local, W3_local, W2_local, W1s, W3s, W
     y_perm = bufs.view(moe, "y_perm", (T * k, d), x.dtype)
     exchange_rows(x_perm, send_rows, recv_rows, bufs.recv, group)
     moe.moe_ep_expert_ffn(bufs.recv, R * T * k, R, rank, E, d, f, W1_local, W3_local, W2_local, bufs.h, bufs.y_recv,
-                          x, T, W1s, W3s, W2s, f_shared, bufs.h_shared, bufs.y_shared, bufs.ep_ws)
+                          x, T, W1s, W3s, W2s, f_shared, bufs.h_shared, bufs.y_shared, bufs.ep_ws, source_major=True)
     exchange_rows(bufs.y_recv, recv_rows, send_rows, y_perm, group)
     moe.moe_combine(y_perm, bufs.view(moe, "dest", (T, k), torch.int32), bufs.view(moe, "w", (T, k), torch.float32),
                     bufs.y_shared, T, d, k, out)

@@ -120,10 +120,11 @@ def test_expert_cache_host_checks(lib):
 
 def test_expert_parallel_host_checks(lib):
     vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
-    lib.moe_ep_workspace_bytes.argtypes = [i32, ctypes.POINTER(sz)]
+    lib.moe_ep_workspace_bytes.argtypes = [i32, i32, ctypes.POINTER(sz)]
     b = sz(0)
-    assert lib.moe_ep_workspace_bytes(256, ctypes.byref(b)) == 0 and b.value > 3 * 257 * 4
-    assert lib.moe_ep_workspace_bytes(2048, ctypes.byref(b)) == -2
+    assert lib.moe_ep_workspace_bytes(8, 256, ctypes.byref(b)) == 0 and b.value >= 8 * 256 * 4 + 6 * 256 * 4
+    assert lib.moe_ep_workspace_bytes(8, 2048, ctypes.byref(b)) == -2
+    assert lib.moe_ep_workspace_bytes(3, 256, ctypes.byref(b)) == -2
     lib.moe_ep_plan.argtypes = [vp, i32, i32, i32, i64, i32, vp, sz, vp]
     ws = 1 << 20
     assert lib.moe_ep_plan(16, 3, 0, 16, -1, 100, 16, ws, None) == -2     # E not a multiple of R

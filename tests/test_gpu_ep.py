@@ -1,7 +1,8 @@
-"""Expert-parallel layer with R ranks emulated on one GPU (the library's put kernels move the rows
-between the ranks' buffers): the output of every rank against the layer oracle over the whole
-batch (capacity counted over all ranks), and bit for bit against the token-sharded layer that
-holds all experts on every rank."""
+"""Expert-parallel layer with R ranks emulated on one GPU, rows moved either by the library's put
+kernels (expert-major receive buffers) or the way an all-to-all-v moves them (source-major,
+one GEMM segment per source rank and local expert): the output of every rank against the layer
+oracle over the whole batch (capacity counted over all ranks), and bit for bit against the
+token-sharded layer that holds all experts on every rank."""
 import numpy as np
 import pytest
 import torch
@@ -29,8 +30,9 @@ CASES = {
 }
 
 
+@pytest.mark.parametrize("exchange", ["put", "a2a"])
 @pytest.mark.parametrize("case", list(CASES))
-def test_emulated_expert_parallel_layer(moe, case):
+def test_emulated_expert_parallel_layer(moe, case, exchange):
     from moe_layer_router_b200.ep import EmulatedEP
     R, T, d, E, k, f, fs, cap_mode, cf, zs = CASES[case]
     wl = synth.Workload("ep_" + case, R * T, d, E, k, f, f_shared=fs, cap_mode=cap_mode, capacity_factor=cf,
@@ -45,7 +47,7 @@ def test_emulated_expert_parallel_layer(moe, case):
     dsh = [dv(a) if a is not None else None for a in sh]
     xs = [dv(x[r * T:(r + 1) * T]) for r in range(R)]
     outs = [torch.empty((T, d), dtype=torch.bfloat16, device="cuda") for _ in range(R)]
-    ep = EmulatedEP(R, T, d, E, k, f, fs)
+    ep = EmulatedEP(R, T, d, E, k, f, fs, exchange=exchange)
     ep.forward(xs, dwg, None, dW1, dW3, dW2, *dsh, cf, cap_mode, outs)
     assert moe.moe_get_error() == 0
 
@@ -77,7 +79,8 @@ def test_emulated_expert_parallel_layer(moe, case):
     assert kept == ref["N"]
     if cap_mode != synth.CAP_NONE:
         assert kept < R * T * k          # capacity dropped rows
-    same_tiles = (R * T * k >= 256 * E) == (T * k >= 256 * E)
+    # tile kind: pair (2-SM) tiles when the rows per expert average >= 256 (local experts for EP)
+    same_tiles = (R * T * k >= 256 * (E // R)) == (T * k >= 256 * E)
     if same_tiles:   # same tile kind in both paths: each row's arithmetic is the same
         for r in range(R):
             assert torch.equal(outs[r].view(torch.int16), outs_dp[r].view(torch.int16)), f"rank {r}"
