@@ -270,15 +270,26 @@ def run_cached(args, base, rank, world, local):
     dev = torch.device("cuda", local)
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
-    W = synth.device_tensors(wl, dev, names=["wg", "w1", "w3", "w2", "w1s", "w3s", "w2s", "bias"])
+    fp8 = args.weights == "fp8"
+    if fp8:
+        W = synth.device_tensors(wl, dev, names=["wg", "bias"])
+        Q = synth.device_tensors_q8(wl, dev)
+        routed = {"W1q": "w1q", "W3q": "w3q", "W2q": "w2q", "s1": "s1", "s3": "s3", "s2": "s2"}
+        shared = {"W1q": Q["w1sq"], "W3q": Q["w3sq"], "W2q": Q["w2sq"], "s1": Q["s1s"], "s3": Q["s3s"], "s2": Q["s2s"]}
+        W.update({n: Q[q] for n, q in routed.items()})
+        names = list(routed)
+    else:
+        W = synth.device_tensors(wl, dev, names=["wg", "w1", "w3", "w2", "w1s", "w3s", "w2s", "bias"])
+        names = ["w1", "w3", "w2"]
     host = {}
-    for n in ("w1", "w3", "w2"):          # the routed experts live in page-locked host memory
-        host[n] = torch.empty(W[n].shape, dtype=torch.bfloat16, pin_memory=True)
+    for n in names:                        # the routed experts live in page-locked host memory
+        host[n] = torch.empty(W[n].shape, dtype=W[n].dtype, pin_memory=True)
         host[n].copy_(W[n])
         del W[n]
+    if fp8:
+        del Q
     torch.cuda.empty_cache()
-    slots = {n: torch.empty((S,) + tuple(host[n].shape[1:]), dtype=torch.bfloat16, device=dev)
-             for n in ("w1", "w3", "w2")}
+    slots = {n: torch.empty((S,) + tuple(host[n].shape[1:]), dtype=host[n].dtype, device=dev) for n in names}
     state = torch.empty(moe.moe_cache_state_bytes(E, S), dtype=torch.uint8, device=dev)
     moe.moe_cache_reset(state, E, S)
     inp = synth.Inputs(wl)
@@ -289,9 +300,14 @@ def run_cached(args, base, rank, world, local):
     out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
 
     def fwd(i, events=None, xin=None):
-        moe.moe_layer_forward_cached(xs[i] if xin is None else xin, W["wg"], W["bias"], host["w1"], host["w3"], host["w2"], slots["w1"],
-                                     slots["w3"], slots["w2"], S, state, W.get("w1s"), W.get("w3s"), W.get("w2s"), fs,
-                                     T, d, E, k, f, wl.capacity_factor, wl.cap_mode, out, ws, events)
+        xi = xs[i] if xin is None else xin
+        if fp8:
+            moe.moe_layer_forward_cached_w8(xi, W["wg"], W["bias"], host, slots, S, state, shared, fs, T, d, E, k, f,
+                                            wl.capacity_factor, wl.cap_mode, out, ws, events)
+        else:
+            moe.moe_layer_forward_cached(xi, W["wg"], W["bias"], host["w1"], host["w3"], host["w2"], slots["w1"],
+                                         slots["w3"], slots["w2"], S, state, W.get("w1s"), W.get("w3s"), W.get("w2s"),
+                                         fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, out, ws, events)
 
     nw = max(3, args.warmup)
     for i in range(nw):
@@ -319,7 +335,7 @@ def run_cached(args, base, rank, world, local):
     order = ["route", "topk", "permute", "cache", "gate_up", "down", "combine", "end"]
     stage_ms = {a: float(np.mean([e[a].elapsed_time(e[b]) for e in evs])) for a, b in zip(order[:-1], order[1:])}
     c1 = moe.cache_counters(state)
-    expert_bytes = 3 * f * d * 2
+    expert_bytes = 3 * f * d + 4 * (2 * f + d) if fp8 else 3 * f * d * 2
     hits, misses = c1["hits"] - c0["hits"], c1["misses"] - c0["misses"]
     copy_ms = sum(e["cache"].elapsed_time(e["gate_up"]) for e in evs)   # plan + copy kernels, all steps
     link_gbs = misses * expert_bytes / 1e9 / (copy_ms / 1e3)
@@ -360,7 +376,8 @@ def run_cached(args, base, rank, world, local):
         "metric": "MoE-layer tokens/s on 1 B200, routed experts served from an HBM expert cache",
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": nw,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic (seeded Philox4x32-10 + Box-Muller; random-init weights)",
+        "dtype": "bf16 activations, fp8 e4m3 expert weights" if fp8 else "bf16",
+        "data": "synthetic (seeded Philox4x32-10 + Box-Muller; random-init weights)",
         "config": {"workload": f"DeepSeek-V3-like decode T={T} d={d} E={E} top-{k} f={f} + shared f={fs}, "
                                f"Zipf({wl.zipf_s}) expert popularity, fresh tokens every step; routed experts in "
                                f"page-locked host memory ({E * expert_bytes / 1e9:.1f} GB), {S} HBM slots",

@@ -400,6 +400,31 @@ int moe_layer_forward_cached(const moe_bf16* x, const moe_bf16* Wg, const float*
                              const moe_stage_events* events);
 
 /*
+ * The cached layer with fp8 expert weights (moe_layer_forward_w8's format): the sources hold
+ * every expert's codes and row scales, the slots S experts' worth of each.  A miss copies half
+ * the bytes of a bf16 expert over the host link.
+ *   src:    W1q, W3q [E, f, d] uint8, W2q [E, d, f] uint8, s1, s3 [E, f], s2 [E, d] fp32;
+ *           page-locked host memory or device memory
+ *   slots:  the same arrays with S in place of E, device memory
+ *   shared: the shared expert (W1q, W3q [f_shared, d], W2q [d, f_shared], s1, s3 [f_shared],
+ *           s2 [d]), device memory, or NULL with f_shared = 0
+ * Same state, workspace and checks as moe_layer_forward_cached().
+ */
+typedef struct moe_w8_experts {
+    const uint8_t *W1q, *W3q, *W2q;
+    const float *s1, *s3, *s2;
+} moe_w8_experts;
+typedef struct moe_w8_slots {
+    uint8_t *W1q, *W3q, *W2q;
+    float *s1, *s3, *s2;
+} moe_w8_slots;
+int moe_layer_forward_cached_w8(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const moe_w8_experts* src,
+                                const moe_w8_slots* slots, int S, void* cache_state, const moe_w8_experts* shared,
+                                int f_shared, int T, int d, int E, int k, int f, double capacity_factor, int cap_mode,
+                                moe_bf16* out, void* ws, size_t ws_bytes, moe_stream_t stream,
+                                const moe_stage_events* events);
+
+/*
  * Byte offsets of the intermediates that moe_layer_forward() leaves in its workspace,
  * so that a caller (a test) can read them after the call:
  *   off[0] logits [T,E] fp32   off[1] idx [T,k] int32   off[2] w [T,k] fp32

@@ -75,6 +75,15 @@ _lib.moe_cache_reset.restype = _i32
 _lib.moe_layer_forward_cached.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i32,
                                           _i32, _i32, _i32, _i32, _i32, _dbl, _i32, _vp, _vp, _sz, _vp, _vp]
 _lib.moe_layer_forward_cached.restype = _i32
+class moe_w8_experts(ctypes.Structure):
+    _fields_ = [("W1q", _vp), ("W3q", _vp), ("W2q", _vp), ("s1", _vp), ("s3", _vp), ("s2", _vp)]
+
+
+_lib.moe_layer_forward_cached_w8.argtypes = [_vp, _vp, _vp, ctypes.POINTER(moe_w8_experts),
+                                             ctypes.POINTER(moe_w8_experts), _i32, _vp,
+                                             ctypes.POINTER(moe_w8_experts), _i32, _i32, _i32, _i32, _i32, _i32,
+                                             _dbl, _i32, _vp, _vp, _sz, _vp, _vp]
+_lib.moe_layer_forward_cached_w8.restype = _i32
 _lib.moe_layer_permute.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _i32, _i64, _vp, _vp, _sz, _vp]
 _lib.moe_layer_permute.restype = _i32
 _lib.moe_ep_workspace_bytes.argtypes = [_i32, _i32, ctypes.POINTER(_sz)]
@@ -347,6 +356,27 @@ def moe_layer_forward_cached(x, Wg, bias, W1_src, W3_src, W2_src, W1_slots, W3_s
                                          _ptr(W3s), _ptr(W2s), f_shared, T, d, E, k, f, float(capacity_factor),
                                          cap_mode, _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream),
                                          ctypes.byref(ev) if ev is not None else None), "moe_layer_forward_cached")
+
+
+def _w8(d):
+    """dict with W1q, W3q, W2q, s1, s3, s2 tensors (or None) -> moe_w8_experts."""
+    if d is None:
+        return None
+    return moe_w8_experts(*[_ptr(d[n]) for n in ("W1q", "W3q", "W2q", "s1", "s3", "s2")])
+
+
+def moe_layer_forward_cached_w8(x, Wg, bias, src: dict, slots: dict, S, state, shared: Optional[dict], f_shared, T, d,
+                                E, k, f, capacity_factor, cap_mode, out, ws, events: Optional[dict] = None,
+                                stream=None) -> None:
+    """The cached layer with fp8 experts.  src / slots / shared: dicts of W1q, W3q, W2q (uint8)
+    and s1, s3, s2 (fp32) tensors; src may be page-locked host tensors."""
+    ev = _events(events)
+    a, b, c = _w8(src), _w8(slots), _w8(shared)
+    _check(_lib.moe_layer_forward_cached_w8(_ptr(x), _ptr(Wg), _ptr(bias), ctypes.byref(a), ctypes.byref(b), S,
+                                            _ptr(state), ctypes.byref(c) if c is not None else None, f_shared, T, d,
+                                            E, k, f, float(capacity_factor), cap_mode, _ptr(out), _ptr(ws),
+                                            _nbytes(ws), _stream(stream), ctypes.byref(ev) if ev is not None else None),
+           "moe_layer_forward_cached_w8")
 
 
 def cache_counters(state) -> dict:

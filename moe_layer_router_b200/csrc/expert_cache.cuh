@@ -8,8 +8,9 @@
 //   cache_plan_kernel   one CTA: stamps the hits, ranks the misses (ascending expert) and the
 //                       free-able slots (oldest stamp first, then lower slot), pairs them rank by
 //                       rank and writes the load list
-//   cache_load_kernel   every SM streams the listed experts' W1, W3, W2 from page-locked host
-//                       memory (read directly over the host link) into their slots
+//   cache_load_kernel   every SM streams the listed experts' weights (W1, W3, W2; or their fp8
+//                       codes and row scales) from page-locked host memory (read directly over
+//                       the host link) into their slots
 // The grouped GEMMs then read weight group slot_of[e] for routed group e.
 //
 // Pairing the r-th miss with the r-th candidate slot is the same as taking misses one at a time
@@ -148,37 +149,46 @@ __global__ void __launch_bounds__(CACHE_MAX) cache_plan_kernel(const int32_t* __
     }
 }
 
-// Copy the listed experts' three matrices (each `per_mat` uint4 per expert) into their slots.
-// Every CTA takes a strided share of every matrix, so all SMs keep requests in flight.
+// The per-expert arrays one cache load copies: for expert e and slot v, array i moves
+// per[i] 16-byte chunks from src[i] + e per[i] to dst[i] + v per[i].  bf16 experts: W1, W3, W2;
+// fp8 experts: W1q, W3q, W2q and the scales s1, s3, s2.
+constexpr int CACHE_MAX_ARRAYS = 6;
+struct CacheCopy {
+    const uint4* src[CACHE_MAX_ARRAYS];
+    uint4* dst[CACHE_MAX_ARRAYS];
+    long long per[CACHE_MAX_ARRAYS];
+    int n;
+};
+
+// Copy the listed experts' arrays into their slots.  Every CTA takes a strided share of every
+// array, so all SMs keep requests in flight.
 constexpr int CACHE_LOAD_THREADS = 512;
 constexpr int CACHE_LOAD_UNROLL = 8;
 
 __global__ void __launch_bounds__(CACHE_LOAD_THREADS) cache_load_kernel(
     const moe_cache_counters* __restrict__ ctr, const int32_t* __restrict__ load_expert,
-    const int32_t* __restrict__ load_slot, const uint4* __restrict__ src0, const uint4* __restrict__ src1,
-    const uint4* __restrict__ src2, uint4* __restrict__ dst0, uint4* __restrict__ dst1, uint4* __restrict__ dst2,
-    long long per_mat) {
+    const int32_t* __restrict__ load_slot, const CacheCopy cp) {
     const int n = (int)ctr->loads_last;
     const long long stride = (long long)gridDim.x * CACHE_LOAD_THREADS * CACHE_LOAD_UNROLL;
     for (int l = 0; l < n; ++l) {
-        const long long se = (long long)load_expert[l] * per_mat;
-        const long long ds = (long long)load_slot[l] * per_mat;
+        const long long e = load_expert[l], v = load_slot[l];
 #pragma unroll 1
-        for (int m = 0; m < 3; ++m) {
-            const uint4* src = (m == 0 ? src0 : m == 1 ? src1 : src2) + se;
-            uint4* dst = (m == 0 ? dst0 : m == 1 ? dst1 : dst2) + ds;
+        for (int m = 0; m < cp.n; ++m) {
+            const long long per = cp.per[m];
+            const uint4* src = cp.src[m] + e * per;
+            uint4* dst = cp.dst[m] + v * per;
             for (long long base = (long long)blockIdx.x * CACHE_LOAD_THREADS * CACHE_LOAD_UNROLL + threadIdx.x;
-                 base < per_mat; base += stride) {
+                 base < per; base += stride) {
                 uint4 r[CACHE_LOAD_UNROLL];
 #pragma unroll
                 for (int u = 0; u < CACHE_LOAD_UNROLL; ++u) {
                     const long long i = base + (long long)u * CACHE_LOAD_THREADS;
-                    if (i < per_mat) r[u] = src[i];
+                    if (i < per) r[u] = src[i];
                 }
 #pragma unroll
                 for (int u = 0; u < CACHE_LOAD_UNROLL; ++u) {
                     const long long i = base + (long long)u * CACHE_LOAD_THREADS;
-                    if (i < per_mat) dst[i] = r[u];
+                    if (i < per) dst[i] = r[u];
                 }
             }
         }

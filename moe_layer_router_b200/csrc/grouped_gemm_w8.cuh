@@ -11,20 +11,21 @@
 // token count.  The converted weights never touch shared memory: the converters store them into
 // tensor memory with tcgen05.st and the MMAs read their A operand from there.
 //
-// Roles (448 threads, one CTA per SM): warp 0 TMA producer, warp 1 TMEM allocator + MMA
-// issuer, warps 2-5 epilogue, warps 6-13 converters (warp w owns TMEM lanes 32 (w % 4) ..
-// +31 of weight half (w - 6) / 4, one weight row per thread).
-//   shared ring (6 stages)  A [128 x 64] bf16 token rows, 128-byte swizzle (only the first 32
-//                           rows when the tile has <= 32 rows: the other rows only feed
-//                           accumulator columns that are never stored), and Q [256 x 64] fp8,
-//                           64-byte rows with 64-byte swizzle (conflict-free row reads); freed
-//                           when the MMAs have read A and the converters have read Q
-//   TMEM columns            [0, 192): 3 stages of converted weights, 64 columns each (half h
-//                           at +32 h, two bf16 per column); [192, 320) and [320, 448): two
-//                           accumulator slots of 128 columns; a tile of <= 32 rows takes one
-//                           slot (2 x 32 columns), a wider tile both (2 x 128 columns)
-// Barriers: full (TMA bytes), empty (MMA commit + 8 converter warps), w_full (8 converter warps),
-// w_empty (MMA commit), acc_full / acc_empty per slot.
+// Roles (480 threads, one CTA per SM): warp 0 loads the fp8 weights, warp 14 loads the token
+// rows, warp 1 allocates TMEM and issues the MMAs, warps 2-5 run the epilogue, warps 6-13 convert
+// (warp w owns TMEM lanes 32 (w % 4) .. +31 of weight half (w - 6) / 4, one weight row per thread).
+//   fp8 ring (8 stages)     Q [256 x 64] fp8, 64-byte rows with 64-byte swizzle (conflict-free row
+//                           reads); a slot is free again as soon as the converters have read it,
+//                           so up to 128 KB of weights per SM stay in flight
+//   token ring (4 stages)   A [128 x 64] bf16 token rows, 128-byte swizzle (only the first 32 rows
+//                           when the tile has <= 32 rows: the other rows only feed accumulator
+//                           columns that are never stored); freed by the MMA commit
+//   TMEM columns            [0, 192): 3 stages of converted weights, 64 columns each (half h at
+//                           +32 h, two bf16 per column); [192, 320) and [320, 448): two accumulator
+//                           slots of 128 columns; a tile of <= 32 rows takes one slot (2 x 32
+//                           columns), a wider tile both (2 x 128 columns)
+// Barriers: q_full / a_full (TMA bytes), q_empty / w_full (8 converter warps), a_empty / w_empty
+// (MMA commit), acc_full / acc_empty per slot.
 #pragma once
 
 #include <cuda_fp8.h>
@@ -33,14 +34,14 @@
 
 namespace moe {
 
-constexpr int W8_STAGES = 6;
+constexpr int W8_QSTAGES = 8;
+constexpr int W8_ASTAGES = 4;
 constexpr int W8_TSTAGES = 3;
 constexpr int W8_CONV_WARPS = 8;
-constexpr int W8_THREADS = (6 + W8_CONV_WARPS) * 32;
+constexpr int W8_THREADS = (7 + W8_CONV_WARPS) * 32;
 constexpr int W8_A_BYTES = GEMM_BM * GEMM_BK * 2;   // 16 KB
 constexpr int W8_Q_BYTES = 256 * GEMM_BK;           // 16 KB
-constexpr int W8_STAGE_BYTES = W8_A_BYTES + W8_Q_BYTES;
-constexpr int W8_RING_BYTES = W8_STAGES * W8_STAGE_BYTES;
+constexpr int W8_RING_BYTES = W8_QSTAGES * W8_Q_BYTES + W8_ASTAGES * W8_A_BYTES;
 constexpr int W8_SMEM_BYTES = W8_RING_BYTES + 1024 + 512;
 constexpr uint32_t W8_TCOL_W = 0;                    // converted weights
 constexpr uint32_t W8_TCOL_ACC = 64 * W8_TSTAGES;    // accumulator slots
@@ -116,25 +117,31 @@ grouped_gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
     static_assert(EPI == EPI_SWIGLU || EPI == EPI_STORE, "expert GEMMs only");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + W8_RING_BYTES);
-    uint64_t* empty_bar = full_bar + W8_STAGES;
-    uint64_t* w_full = empty_bar + W8_STAGES;
+    uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + W8_RING_BYTES);
+    uint64_t* q_empty = q_full + W8_QSTAGES;
+    uint64_t* a_full = q_empty + W8_QSTAGES;
+    uint64_t* a_empty = a_full + W8_ASTAGES;
+    uint64_t* w_full = a_empty + W8_ASTAGES;
     uint64_t* w_empty = w_full + W8_TSTAGES;
     uint64_t* acc_full = w_empty + W8_TSTAGES;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain_bar = acc_empty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    auto sA = [&](int s) { return smem + s * W8_STAGE_BYTES; };
-    auto sQ = [&](int s) { return smem + s * W8_STAGE_BYTES + W8_A_BYTES; };
+    auto sQ = [&](int s) { return smem + s * W8_Q_BYTES; };
+    auto sA = [&](int s) { return smem + W8_QSTAGES * W8_Q_BYTES + s * W8_A_BYTES; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < W8_STAGES; ++s) {
-            mbar_init(full_bar + s, 1);
-            mbar_init(empty_bar + s, 1 + W8_CONV_WARPS);
+        for (int s = 0; s < W8_QSTAGES; ++s) {
+            mbar_init(q_full + s, 1);
+            mbar_init(q_empty + s, W8_CONV_WARPS);
+        }
+        for (int s = 0; s < W8_ASTAGES; ++s) {
+            mbar_init(a_full + s, 1);
+            mbar_init(a_empty + s, 1);
         }
         for (int s = 0; s < W8_TSTAGES; ++s) {
             mbar_init(w_full + s, W8_CONV_WARPS);
@@ -149,16 +156,18 @@ grouped_gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&tmA0);
-        prefetch_tensormap(&tmA0s);
         prefetch_tensormap(&tmQ0);
-        prefetch_tensormap(&tmA1);
-        prefetch_tensormap(&tmA1s);
         prefetch_tensormap(&tmQ1);
         if (EPI == EPI_SWIGLU) {
             prefetch_tensormap(&tmQ0b);
             prefetch_tensormap(&tmQ1b);
         }
+    }
+    if (warp == 14 && lane == 0) {
+        prefetch_tensormap(&tmA0);
+        prefetch_tensormap(&tmA0s);
+        prefetch_tensormap(&tmA1);
+        prefetch_tensormap(&tmA1s);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, GEMM_TMEM_COLS);
@@ -173,10 +182,41 @@ grouped_gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
     const int total = gemm_total_tiles(p, routed_tiles);
 
     if (warp == 0) {
-        // ------------------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------------ fp8 weight producer
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first();   // weights are read once
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                const TileInfo ti = gemm_decode_tile(p, t, routed_tiles);
+                const GemmClass& c = p.cls[ti.cls];
+                const CUtensorMap* mQ = ti.cls ? &tmQ1 : &tmQ0;
+                const CUtensorMap* mQb = ti.cls ? &tmQ1b : &tmQ0b;
+                const int nk = c.K / GEMM_BK;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(q_empty + stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+                    mbar_arrive_expect_tx(q_full + stage, (uint32_t)W8_Q_BYTES);
+                    tma_load_2d(sQ(stage), mQ, q_full + stage, kb * GEMM_BK, ti.b_row, pol_w);
+                    if (EPI == EPI_SWIGLU)
+                        tma_load_2d(sQ(stage) + 128 * GEMM_BK, mQb, q_full + stage, kb * GEMM_BK, ti.b_row, pol_w);
+                    ++issued;
+                    if (++stage == W8_QSTAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok) {   // let the copies in flight land before the CTA exits
+                const int n = issued < W8_QSTAGES ? issued : W8_QSTAGES;
+                for (int i = 1; i <= n; ++i) {
+                    const int q = issued - i;
+                    mbar_wait(q_full + (q % W8_QSTAGES), (uint32_t)((q / W8_QSTAGES) & 1), nullptr);
+                }
+            }
+        }
+    } else if (warp == 14) {
+        // ------------------------------------------------------------------ token-row producer
         if (lane == 0) {
             const uint64_t pol_a = policy_evict_last();
-            const uint64_t pol_w = policy_evict_first();   // weights are read once
             int stage = 0;
             uint32_t phase = 0;
             int issued = 0;
@@ -186,26 +226,21 @@ grouped_gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
                 const GemmClass& c = p.cls[ti.cls];
                 const bool narrow = ti.rows <= 32;
                 const CUtensorMap* mA = ti.cls ? (narrow ? &tmA1s : &tmA1) : (narrow ? &tmA0s : &tmA0);
-                const CUtensorMap* mQ = ti.cls ? &tmQ1 : &tmQ0;
-                const CUtensorMap* mQb = ti.cls ? &tmQ1b : &tmQ0b;
-                const uint32_t bytes = (narrow ? 32u : 128u) * GEMM_BK * 2u + (uint32_t)W8_Q_BYTES;
+                const uint32_t bytes = (narrow ? 32u : 128u) * GEMM_BK * 2u;
                 const int nk = c.K / GEMM_BK;
                 for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(empty_bar + stage, phase ^ 1u, abort_flag)) { ok = false; break; }
-                    mbar_arrive_expect_tx(full_bar + stage, bytes);
-                    tma_load_2d(sQ(stage), mQ, full_bar + stage, kb * GEMM_BK, ti.b_row, pol_w);
-                    if (EPI == EPI_SWIGLU)
-                        tma_load_2d(sQ(stage) + 128 * GEMM_BK, mQb, full_bar + stage, kb * GEMM_BK, ti.b_row, pol_w);
-                    tma_load_2d(sA(stage), mA, full_bar + stage, kb * GEMM_BK, ti.a_row, pol_a);
+                    if (!mbar_wait(a_empty + stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+                    mbar_arrive_expect_tx(a_full + stage, bytes);
+                    tma_load_2d(sA(stage), mA, a_full + stage, kb * GEMM_BK, ti.a_row, pol_a);
                     ++issued;
-                    if (++stage == W8_STAGES) { stage = 0; phase ^= 1u; }
+                    if (++stage == W8_ASTAGES) { stage = 0; phase ^= 1u; }
                 }
             }
-            if (!ok) {   // let the copies in flight land before the CTA exits
-                const int n = issued < W8_STAGES ? issued : W8_STAGES;
+            if (!ok) {
+                const int n = issued < W8_ASTAGES ? issued : W8_ASTAGES;
                 for (int i = 1; i <= n; ++i) {
                     const int q = issued - i;
-                    mbar_wait(full_bar + (q % W8_STAGES), (uint32_t)((q / W8_STAGES) & 1), nullptr);
+                    mbar_wait(a_full + (q % W8_ASTAGES), (uint32_t)((q / W8_ASTAGES) & 1), nullptr);
                 }
             }
         }
@@ -235,7 +270,7 @@ grouped_gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
                 const uint32_t d0 = tmem_base + W8_TCOL_ACC + (wide ? 0u : 128u * (uint32_t)slot);
                 const uint32_t d1 = d0 + (uint32_t)nN;
                 for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(full_bar + stage, phase, abort_flag) || !mbar_wait(w_full + wstage, wphase, abort_flag)) {
+                    if (!mbar_wait(a_full + stage, phase, abort_flag) || !mbar_wait(w_full + wstage, wphase, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -247,10 +282,10 @@ grouped_gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
                         umma_bf16_ts(d0, w0 + 8u * kk, xd + 2ull * kk, idesc, (kb | kk) != 0);
                         umma_bf16_ts(d1, w0 + 32u + 8u * kk, xd + 2ull * kk, idesc, (kb | kk) != 0);
                     }
-                    umma_commit(empty_bar + stage);
+                    umma_commit(a_empty + stage);
                     umma_commit(w_empty + wstage);
                     any = true;
-                    if (++stage == W8_STAGES) { stage = 0; phase ^= 1u; }
+                    if (++stage == W8_ASTAGES) { stage = 0; phase ^= 1u; }
                     if (++wstage == W8_TSTAGES) { wstage = 0; wphase ^= 1u; }
                 }
                 if (!ok) break;
@@ -287,7 +322,7 @@ grouped_gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
             const int nk = p.cls[ti.cls].K / GEMM_BK;
             bool ok = true;
             for (int kb = 0; kb < nk; ++kb) {
-                const bool ready = mbar_wait(full_bar + stage, phase, abort_flag) &&
+                const bool ready = mbar_wait(q_full + stage, phase, abort_flag) &&
                                    mbar_wait(w_empty + wstage, wphase ^ 1u, abort_flag);
                 if (!__all_sync(0xffffffffu, ready)) { ok = false; break; }
                 tc_fence_after();
@@ -300,13 +335,13 @@ grouped_gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
 #pragma unroll
                 for (int g = 0; g < 4; ++g) e4m3x16_to_bf16(v[g], o + 8 * g);
                 __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar + stage);     // the fp8 slot has been read
+                if (lane == 0) mbar_arrive(q_empty + stage);     // the fp8 slot has been read
                 tmem_st_32cols(tmem_base + lane_addr + W8_TCOL_W + 64u * (uint32_t)wstage + 32u * (uint32_t)half, o);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(w_full + wstage);
-                if (++stage == W8_STAGES) { stage = 0; phase ^= 1u; }
+                if (++stage == W8_QSTAGES) { stage = 0; phase ^= 1u; }
                 if (++wstage == W8_TSTAGES) { wstage = 0; wphase ^= 1u; }
             }
             if (!ok) break;

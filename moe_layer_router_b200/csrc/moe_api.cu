@@ -451,8 +451,8 @@ int run_expert_ffn_w8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, cuda
         if (routed) {
             if ((rc = make_map(&m[0], a.x_perm, a.d, a.max_rows, GEMM_BM)) != MOE_OK) return rc;
             if ((rc = make_map(&m[1], a.x_perm, a.d, a.max_rows, 32)) != MOE_OK) return rc;
-            if ((rc = make_map_u8(&m[2], q.W1q, a.d, (uint64_t)a.E * a.f, 128)) != MOE_OK) return rc;
-            if ((rc = make_map_u8(&m[3], q.W3q, a.d, (uint64_t)a.E * a.f, 128)) != MOE_OK) return rc;
+            if ((rc = make_map_u8(&m[2], q.W1q, a.d, weight_groups(a) * a.f, 128)) != MOE_OK) return rc;
+            if ((rc = make_map_u8(&m[3], q.W3q, a.d, weight_groups(a) * a.f, 128)) != MOE_OK) return rc;
         }
         if (shared) {
             if ((rc = make_map(&m[4], a.x, a.d, a.T, GEMM_BM)) != MOE_OK) return rc;
@@ -477,6 +477,7 @@ int run_expert_ffn_w8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, cuda
         p.mprefix = a.mprefix;
         p.E = a.E;
         p.dense_rows = shared ? a.T : 0;
+        p.group_map = a.group_map;   // scales follow: the epilogue finds them by the mapped weight row
         W8Scales sc;
         memset(&sc, 0, sizeof(sc));
         sc.s0[0] = q.s1; sc.s1[0] = q.s3; sc.group_stride[0] = a.f;
@@ -493,7 +494,7 @@ int run_expert_ffn_w8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, cuda
         if (routed) {
             if ((rc = make_map(&m[0], a.h, a.f, a.max_rows, GEMM_BM)) != MOE_OK) return rc;
             if ((rc = make_map(&m[1], a.h, a.f, a.max_rows, 32)) != MOE_OK) return rc;
-            if ((rc = make_map_u8(&m[2], q.W2q, a.f, (uint64_t)a.E * a.d, 256)) != MOE_OK) return rc;
+            if ((rc = make_map_u8(&m[2], q.W2q, a.f, weight_groups(a) * a.d, 256)) != MOE_OK) return rc;
             m[3] = m[2];
         }
         if (shared) {
@@ -518,6 +519,7 @@ int run_expert_ffn_w8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, cuda
         p.mprefix = a.mprefix;
         p.E = a.E;
         p.dense_rows = shared ? a.T : 0;
+        p.group_map = a.group_map;   // scales follow: the epilogue finds them by the mapped weight row
         W8Scales sc;
         memset(&sc, 0, sizeof(sc));
         sc.s0[0] = q.s2; sc.group_stride[0] = a.d;
@@ -693,10 +695,11 @@ enum { LAYER_ROUTE = 1, LAYER_COUNT = 2, LAYER_FINISH = 4, LAYER_PERMUTE = 8 };
 //   LAYER_COUNT   histogram only: counts_raw          (no capacity)
 //   LAYER_PERMUTE histogram, capacity (with fill_base), permutation; stops there
 //   LAYER_FINISH  histogram, capacity (with fill_base), permutation, experts, combine
-// Routed expert weights served from the expert cache (moe_layer_forward_cached).
+// Routed expert weights served from the expert cache (moe_layer_forward_cached[_w8]).  cp lists
+// the per-expert arrays to copy (device-usable source addresses, slot arrays); the GEMMs then
+// read the slots (bf16: W1/W3/W2 arguments of layer_phases; fp8: its W8Weights) through slot_of.
 struct CacheArgs {
-    const moe_bf16 *W1_src, *W3_src, *W2_src;   // device-usable addresses of the sources
-    moe_bf16 *W1_slots, *W3_slots, *W2_slots;
+    CacheCopy cp;
     int S;
     void* state;
 };
@@ -786,11 +789,7 @@ int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float*
         cv = cache_view(cache->state, E, cache->S);
         cache_plan_kernel<<<1, CACHE_MAX, 0, s>>>(counts, E, cache->S, cv);
         if ((rc = launch_status()) != MOE_OK) return rc;
-        cache_load_kernel<<<2 * di->sms, CACHE_LOAD_THREADS, 0, s>>>(
-            cv.ctr, cv.load_expert, cv.load_slot, reinterpret_cast<const uint4*>(cache->W1_src),
-            reinterpret_cast<const uint4*>(cache->W3_src), reinterpret_cast<const uint4*>(cache->W2_src),
-            reinterpret_cast<uint4*>(cache->W1_slots), reinterpret_cast<uint4*>(cache->W3_slots),
-            reinterpret_cast<uint4*>(cache->W2_slots), (long long)f * d / 8);
+        cache_load_kernel<<<2 * di->sms, CACHE_LOAD_THREADS, 0, s>>>(cv.ctr, cv.load_expert, cv.load_slot, cache->cp);
         if ((rc = launch_status()) != MOE_OK) return rc;
     }
     if (!mark(ev.gate_up)) return MOE_ERR_CUDA;
@@ -798,8 +797,7 @@ int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float*
     memset(&a, 0, sizeof(a));
     a.x_perm = x_perm; a.offsets = offsets; a.mprefix = mprefix; a.max_rows = T * k; a.E = E; a.d = d; a.f = f;
     a.W1 = W1; a.W3 = W3; a.W2 = W2; a.h = h; a.y_perm = y_perm;
-    if (cache) {
-        a.W1 = cache->W1_slots; a.W3 = cache->W3_slots; a.W2 = cache->W2_slots;
+    if (cache) {     // W1/W3/W2 (or w8) already point at the slots
         a.group_map = cv.slot_of;
         a.w_groups = cache->S;
     }
@@ -858,14 +856,14 @@ int moe_cache_reset(void* cache_state, int E, int S, moe_stream_t stream) {
 }
 
 // Address the device uses for a cache source: page-locked host memory (mapped) or device memory.
-static int cache_source(const moe_bf16* p, const moe_bf16** dev) {
+static int cache_source(const void* p, const uint4** dev) {
     cudaPointerAttributes at;
     if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
         cudaGetLastError();
         return MOE_ERR_INVALID_ARG;
     }
-    if (at.type == cudaMemoryTypeHost && at.devicePointer) *dev = static_cast<const moe_bf16*>(at.devicePointer);
-    else if (at.type == cudaMemoryTypeDevice) *dev = p;
+    if (at.type == cudaMemoryTypeHost && at.devicePointer) *dev = static_cast<const uint4*>(at.devicePointer);
+    else if (at.type == cudaMemoryTypeDevice) *dev = static_cast<const uint4*>(p);
     else return MOE_ERR_INVALID_ARG;   // pageable host memory (or unknown)
     return MOE_OK;
 }
@@ -886,16 +884,60 @@ int moe_layer_forward_cached(const moe_bf16* x, const moe_bf16* Wg, const float*
                     aligned16(W3_slots) && aligned16(W2_slots) && aligned16(cache_state),
                 MOE_ERR_ALIGN);
     CacheArgs ca;
-    if ((rc = cache_source(W1_src, &ca.W1_src)) != MOE_OK || (rc = cache_source(W3_src, &ca.W3_src)) != MOE_OK ||
-        (rc = cache_source(W2_src, &ca.W2_src)) != MOE_OK)
-        return rc;
-    ca.W1_slots = W1_slots; ca.W3_slots = W3_slots; ca.W2_slots = W2_slots;
+    memset(&ca, 0, sizeof(ca));
+    const void* srcs[3] = {W1_src, W3_src, W2_src};
+    void* dsts[3] = {W1_slots, W3_slots, W2_slots};
+    for (int i = 0; i < 3; ++i) {
+        if ((rc = cache_source(srcs[i], &ca.cp.src[i])) != MOE_OK) return rc;
+        ca.cp.dst[i] = static_cast<uint4*>(dsts[i]);
+        ca.cp.per[i] = (long long)f * d / 8;
+    }
+    ca.cp.n = 3;
     ca.S = S;
     ca.state = cache_state;
     const long long C = moe_capacity(T, E, k, capacity_factor, cap_mode);
     return layer_phases(LAYER_ROUTE | LAYER_FINISH, x, Wg, bias, W1_slots, W3_slots, W2_slots, W1s, W3s, W2s,
                         f_shared, T, d, E, k, f, C, nullptr, out, ws, ws_bytes, static_cast<cudaStream_t>(stream),
                         events, nullptr, &ca);
+}
+
+int moe_layer_forward_cached_w8(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const moe_w8_experts* src,
+                                const moe_w8_slots* slots, int S, void* cache_state, const moe_w8_experts* shared,
+                                int f_shared, int T, int d, int E, int k, int f, double capacity_factor, int cap_mode,
+                                moe_bf16* out, void* ws, size_t ws_bytes, moe_stream_t stream,
+                                const moe_stage_events* events) {
+    using namespace moe;
+    MOE_REQUIRE(cap_mode >= MOE_CAP_NONE && cap_mode <= MOE_CAP_PER_ASSIGNMENT, MOE_ERR_INVALID_ARG);
+    int rc = check_shape(T, d, E, k, f);
+    if (rc != MOE_OK) return rc;
+    MOE_REQUIRE(S >= 1 && S <= E && (long long)S >= std::min<long long>(E, (long long)T * k), MOE_ERR_SHAPE);
+    MOE_REQUIRE(src && slots && cache_state && (f_shared == 0 || shared), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(src->W1q && src->W3q && src->W2q && src->s1 && src->s3 && src->s2, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(slots->W1q && slots->W3q && slots->W2q && slots->s1 && slots->s3 && slots->s2, MOE_ERR_INVALID_ARG);
+    const void* sp[6] = {src->W1q, src->W3q, src->W2q, src->s1, src->s3, src->s2};
+    void* dp[6] = {slots->W1q, slots->W3q, slots->W2q, slots->s1, slots->s3, slots->s2};
+    for (int i = 0; i < 6; ++i) MOE_REQUIRE(aligned16(sp[i]) && aligned16(dp[i]), MOE_ERR_ALIGN);
+    MOE_REQUIRE(aligned16(cache_state), MOE_ERR_ALIGN);
+    CacheArgs ca;
+    memset(&ca, 0, sizeof(ca));
+    const long long per[6] = {(long long)f * d / 16, (long long)f * d / 16, (long long)d * f / 16,
+                              (long long)f * 4 / 16, (long long)f * 4 / 16, (long long)d * 4 / 16};
+    for (int i = 0; i < 6; ++i) {
+        if ((rc = cache_source(sp[i], &ca.cp.src[i])) != MOE_OK) return rc;
+        ca.cp.dst[i] = static_cast<uint4*>(dp[i]);
+        ca.cp.per[i] = per[i];
+    }
+    ca.cp.n = 6;
+    ca.S = S;
+    ca.state = cache_state;
+    W8Weights q = {slots->W1q, slots->W3q, slots->W2q,
+                   shared ? shared->W1q : nullptr, shared ? shared->W3q : nullptr, shared ? shared->W2q : nullptr,
+                   slots->s1, slots->s3, slots->s2,
+                   shared ? shared->s1 : nullptr, shared ? shared->s3 : nullptr, shared ? shared->s2 : nullptr};
+    const long long C = moe_capacity(T, E, k, capacity_factor, cap_mode);
+    return layer_phases(LAYER_ROUTE | LAYER_FINISH, x, Wg, bias, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                        f_shared, T, d, E, k, f, C, nullptr, out, ws, ws_bytes, static_cast<cudaStream_t>(stream),
+                        events, &q, &ca);
 }
 
 int moe_layer_forward_w8(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const uint8_t* W1q,

@@ -137,3 +137,21 @@ def test_expert_parallel_host_checks(lib):
     assert lib.moe_ep_dispatch(16, 2, 0, 8, 100, 16, 16, ws, None) == -2   # d not a multiple of 64
     lib.moe_layer_permute.argtypes = [vp, i32, i32, i32, i32, i32, i32, i64, vp, vp, sz, vp]
     assert lib.moe_layer_permute(16, 0, 8, 100, 8, 2, 64, -1, None, 16, ws, None) == -2
+
+
+def test_cached_fp8_entry_host_checks(lib):
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+
+    class W8(ctypes.Structure):
+        _fields_ = [(n, vp) for n in ("W1q", "W3q", "W2q", "s1", "s3", "s2")]
+
+    lib.moe_layer_forward_cached_w8.argtypes = [vp, vp, vp, ctypes.POINTER(W8), ctypes.POINTER(W8), i32, vp,
+                                                ctypes.POINTER(W8), i32, i32, i32, i32, i32, i32,
+                                                ctypes.c_double, i32, vp, vp, sz, vp, vp]
+    src, slots = W8(*([16] * 6)), W8(*([32] * 6))
+    call = lambda S, a, b, T=8, k=2, E=64: lib.moe_layer_forward_cached_w8(
+        16, 16, None, a, b, S, 16, None, 0, T, 128, E, k, 64, 1.0, 0, 16, 16, 1 << 20, None, None)
+    assert call(15, ctypes.byref(src), ctypes.byref(slots)) == -2          # S < min(E, T*k)
+    assert call(16, None, ctypes.byref(slots)) == -1                        # no sources
+    bad = W8(16, 16, 16, 16, 16, 24)
+    assert call(16, ctypes.byref(src), ctypes.byref(bad)) == -3             # misaligned slot array

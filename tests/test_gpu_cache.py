@@ -134,3 +134,46 @@ def test_cached_layer_rejects_pageable_source(moe):
         moe.moe_layer_forward_cached(x, wg, None, W1, W1, W1.transpose(1, 2).contiguous(), *slots, S, state,
                                      None, None, None, 0, T, d, E, k, f, 1.0, moe.MOE_CAP_NONE, out, ws)
     assert ei.value.code == moe.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("src", ["pinned", "device"])
+def test_cached_layer_fp8_experts(moe, src):
+    """fp8 experts through the cache: state against the cache oracle, output bit-identical to the
+    uncached fp8 layer, slots equal to their source experts."""
+    T, d, E, k, f, S, fs = 8, 256, 48, 4, 192, 32, 128
+    wl = synth.Workload("cache_q8", T, d, E, k, f, f_shared=fs, zipf_s=1.1, seed=9)
+    inp = synth.Inputs(wl)
+    Q = synth.device_tensors_q8(wl, "cuda")
+    names = {"W1q": "w1q", "W3q": "w3q", "W2q": "w2q", "s1": "s1", "s3": "s3", "s2": "s2"}
+    dev_src = {n: Q[q] for n, q in names.items()}
+    srcs = {n: (t.cpu().pin_memory() if src == "pinned" else t) for n, t in dev_src.items()}
+    slots = {n: torch.empty((S,) + tuple(t.shape[1:]), dtype=t.dtype, device="cuda") for n, t in dev_src.items()}
+    shared = {"W1q": Q["w1sq"], "W3q": Q["w3sq"], "W2q": Q["w2sq"], "s1": Q["s1s"], "s3": Q["s3s"], "s2": Q["s2s"]}
+    state = torch.empty(moe.moe_cache_state_bytes(E, S), dtype=torch.uint8, device="cuda")
+    moe.moe_cache_reset(state, E, S)
+    ws = torch.empty(moe.moe_workspace_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device="cuda")
+    ws2 = torch.empty_like(ws)
+    L = moe.moe_workspace_layout(T, d, E, k, f, fs)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    out_plain = torch.empty_like(out)
+    wg = to_dev_bf16(inp.wg())
+    ref_cache = ExpertCacheOracle(E, S)
+    for b in range(8):
+        x = to_dev_bf16(inp.x_rows(b * T, T).reshape(T, d))
+        moe.moe_layer_forward_cached_w8(x, wg, None, srcs, slots, S, state, shared, fs, T, d, E, k, f, 1.0,
+                                        moe.MOE_CAP_NONE, out, ws)
+        moe.moe_layer_forward_w8(x, wg, None, Q["w1q"], Q["s1"], Q["w3q"], Q["s3"], Q["w2q"], Q["s2"], Q["w1sq"],
+                                 Q["s1s"], Q["w3sq"], Q["s3s"], Q["w2sq"], Q["s2s"], fs, T, d, E, k, f, 1.0,
+                                 moe.MOE_CAP_NONE, out_plain, ws2)
+        assert moe.moe_get_error() == 0
+        counts = moe.workspace_view(ws, L, "counts", (E,), torch.int32).cpu().numpy()
+        loads = ref_cache.batch(np.nonzero(counts > 0)[0])
+        st = _state(moe, state, E, S)
+        assert list(zip(st["load_expert"][:len(loads)].tolist(), st["load_slot"][:len(loads)].tolist())) == loads
+        assert st["slot_of"].tolist() == ref_cache.slot_of
+        assert torch.equal(out.view(torch.int16), out_plain.view(torch.int16))
+    assert ref_cache.misses > 0 and ref_cache.hits > 0
+    for e, v in enumerate(ref_cache.slot_of):
+        if v >= 0:
+            for n in names:
+                assert torch.equal(slots[n][v], dev_src[n][e]), n
