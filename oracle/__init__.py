@@ -62,6 +62,10 @@ def lib():
         L.oracle_e4m3.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3.restype = dbl
         L.oracle_expert_ffn_q8.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp]
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_quantize_rows_e4m3.argtypes = [vp, i32, i32, vp, vp]
+        L.oracle_expert_ffn_w8a8.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp]
         L.oracle_layer_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
                                            i32, i32, i32, i32, i32, i64,
                                            vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
@@ -167,6 +171,33 @@ def expert_ffn_q8(x, W1q, s1, W3q, s3, W2q, s2):
     h = np.empty((rows, f), np.uint16)
     y = np.empty((rows, d), np.uint16)
     lib().oracle_expert_ffn_q8(_p(x), rows, _p(W1q), _p(s1), _p(W3q), _p(s3), _p(W2q), _p(s2), d, f, _p(h), _p(y))
+    return h, y
+
+
+def e4m3_encode(v: float) -> int:
+    return int(lib().oracle_e4m3_encode(float(v)))
+
+
+def quantize_rows_e4m3(x: np.ndarray):
+    """bf16 rows [rows, K] -> (e4m3 codes uint8 [rows, K], fp32 scale per row): s = amax / 448."""
+    x = _c(x, np.uint16)
+    rows, K = x.shape
+    q = np.empty((rows, K), np.uint8)
+    s = np.empty(rows, np.float32)
+    lib().oracle_quantize_rows_e4m3(_p(x), rows, K, _p(q), _p(s))
+    return q, s
+
+
+def expert_ffn_w8a8(x, W1q, s1, W3q, s3, W2q, s2):
+    """One expert with fp8 weights and fp8 activations (rows quantised per row): -> (h, y) bf16."""
+    x = _c(x, np.uint16)
+    W1q = _c(W1q, np.uint8); W3q = _c(W3q, np.uint8); W2q = _c(W2q, np.uint8)
+    s1 = _c(s1, np.float32); s3 = _c(s3, np.float32); s2 = _c(s2, np.float32)
+    rows, d = x.shape
+    f = W1q.shape[0]
+    h = np.empty((rows, f), np.uint16)
+    y = np.empty((rows, d), np.uint16)
+    lib().oracle_expert_ffn_w8a8(_p(x), rows, _p(W1q), _p(s1), _p(W3q), _p(s3), _p(W2q), _p(s2), d, f, _p(h), _p(y))
     return h, y
 
 

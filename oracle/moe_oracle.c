@@ -283,6 +283,99 @@ void oracle_expert_ffn_q8(const uint16_t* x, int rows, const uint8_t* W1q, const
     }
 }
 
+/*
+ * fp8 activations ("w4afp8" on the deployment page: low-bit weights with fp8 activations; here
+ * fp8 weights and fp8 activations).  Every activation row (a token's hidden state before the
+ * first expert GEMM, its h before the second) is quantised on its own:
+ *   s = amax(|x|) / 448 in fp32 (1 for an all-zero row), q_i = e4m3(fp32(x_i) / s) rounded to
+ *   nearest, ties to even, saturating at 448;
+ * the expert GEMMs then multiply fp8 by fp8 and scale the sum by s_row * s_col.
+ */
+
+/* fp32 -> e4m3 ("fn") code by the format's definition: sign | 4 exponent bits (bias 7) | 3
+ * mantissa bits, subnormals m * 2^-9, round to nearest even, values beyond 448 saturate to 448. */
+uint8_t oracle_e4m3_encode(float v) {
+    if (v != v) return 0x7F;
+    uint8_t sgn = signbit(v) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+    if (a >= 448.0) return sgn | 0x7E;
+    /* candidates are multiples of the code spacing at a's binade: 2^-9 below 2^-6 */
+    int e;
+    frexp(a, &e);              /* a = f * 2^e, f in [0.5, 1) -> binade exponent e - 1 */
+    int be = e - 1;
+    if (be < -6) be = -6;      /* subnormal range shares the spacing of [2^-6, 2^-5) */
+    double step = ldexp(1.0, be - 3);
+    double k = a / step;       /* exact: a is an fp32 value, step a power of two */
+    double kf = floor(k);
+    double rem = k - kf;
+    if (rem > 0.5 || (rem == 0.5 && fmod(kf, 2.0) != 0.0)) kf += 1.0;
+    double r = kf * step;      /* the rounded magnitude */
+    if (r >= 448.0) return sgn | 0x7E;
+    if (r == 0.0) return sgn;
+    /* encode r */
+    if (r < ldexp(1.0, -6)) return sgn | (uint8_t)(int)(r / ldexp(1.0, -9));        /* subnormal */
+    int re;
+    double rf = frexp(r, &re);                 /* r = rf * 2^re, rf in [0.5, 1) */
+    int ex = re - 1 + 7;
+    int m = (int)((rf * 2.0 - 1.0) * 8.0);
+    return sgn | (uint8_t)((ex << 3) | m);
+}
+
+/* bf16 rows [rows, K] -> e4m3 codes [rows, K] and one fp32 scale per row (see above). */
+void oracle_quantize_rows_e4m3(const uint16_t* x, int rows, int K, uint8_t* q, float* scale) {
+#pragma omp parallel for schedule(static)
+    for (int r = 0; r < rows; ++r) {
+        const uint16_t* xr = x + (size_t)r * K;
+        float amax = 0.0f;
+        for (int i = 0; i < K; ++i) {
+            float a = fabsf((float)bf(xr[i]));
+            if (a > amax) amax = a;
+        }
+        float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+        scale[r] = s;
+        for (int i = 0; i < K; ++i) q[(size_t)r * K + i] = oracle_e4m3_encode((float)bf(xr[i]) / s);
+    }
+}
+
+/* One expert with fp8 weights (row scales s1, s3, s2) and fp8 activations: x rows quantised,
+ * G = s_x s1 (xq . W1q), U likewise, h = bf16(silu(G) U); h rows quantised, y = bf16(s_h s2 (hq . W2q)). */
+void oracle_expert_ffn_w8a8(const uint16_t* x, int rows, const uint8_t* W1q, const float* s1, const uint8_t* W3q,
+                            const float* s3, const uint8_t* W2q, const float* s2, int d, int f, uint16_t* h,
+                            uint16_t* y) {
+    uint8_t* xq = (uint8_t*)malloc((size_t)(rows > 0 ? rows : 1) * d);
+    float* sx = (float*)malloc(sizeof(float) * (size_t)(rows > 0 ? rows : 1));
+    uint8_t* hq = (uint8_t*)malloc((size_t)(rows > 0 ? rows : 1) * f);
+    float* sh = (float*)malloc(sizeof(float) * (size_t)(rows > 0 ? rows : 1));
+    oracle_quantize_rows_e4m3(x, rows, d, xq, sx);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < rows; ++r) {
+        const uint8_t* xr = xq + (size_t)r * d;
+        uint16_t* hr = h + (size_t)r * f;
+        for (int n = 0; n < f; ++n) {
+            double g = 0.0, u = 0.0;
+            for (int i = 0; i < d; ++i) {
+                double xi = oracle_e4m3(xr[i]);
+                g += xi * oracle_e4m3(W1q[(size_t)n * d + i]);
+                u += xi * oracle_e4m3(W3q[(size_t)n * d + i]);
+            }
+            g *= (double)sx[r] * (double)s1[n];
+            u *= (double)sx[r] * (double)s3[n];
+            hr[n] = bf16_round(g / (1.0 + exp(-g)) * u);
+        }
+    }
+    oracle_quantize_rows_e4m3(h, rows, f, hq, sh);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < rows; ++r) {
+        const uint8_t* hr = hq + (size_t)r * f;
+        for (int m = 0; m < d; ++m) {
+            double acc = 0.0;
+            for (int n = 0; n < f; ++n) acc += oracle_e4m3(hr[n]) * oracle_e4m3(W2q[(size_t)m * f + n]);
+            y[(size_t)r * d + m] = bf16_round(acc * (double)sh[r] * (double)s2[m]);
+        }
+    }
+    free(xq); free(sx); free(hq); free(sh);
+}
+
 /* ---- combine ------------------------------------------------------------------------ */
 
 /*

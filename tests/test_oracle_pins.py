@@ -456,3 +456,68 @@ def test_q8_expert_vs_textbook_dequantised():
     yy = torch_bf16_round_f64(hh.double() @ deq(W2q, s2).T)
     to_bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)
     assert ulp_diff_bf16(h, to_bits(hh)).max() <= 1 and ulp_diff_bf16(y, to_bits(yy)).max() <= 1
+
+
+# --------------------------------------------------------------------------- fp8 activations
+
+
+def test_e4m3_encode_matches_torch_rne():
+    # every code, every midpoint between neighbouring codes (ties go to the even code), random
+    # fp32 values across the range, and saturation beyond 448
+    pos = np.array([oracle.e4m3(c) for c in range(0x7F)], np.float64)          # 0 .. 448
+    mids = (pos[:-1] + pos[1:]) / 2
+    rng = np.random.default_rng(3)
+    rand = np.exp(rng.uniform(np.log(2.0 ** -12), np.log(400.0), 4000))
+    vals = np.concatenate([pos, mids, rand, [0.0, 2.0 ** -11, 2.0 ** -10, 460.0, 1e6]]).astype(np.float32)
+    vals = np.concatenate([vals, -vals])
+    ours = np.array([oracle.e4m3_encode(float(v)) for v in vals], np.uint8)
+    clipped = np.clip(vals, -448.0, 448.0)               # saturating conversion
+    ref = torch.from_numpy(clipped).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+    # ties: the midpoint of codes 0x38 (1.0) and 0x39 (1.125) goes to the even code 0x38
+    assert oracle.e4m3_encode(1.0625) == 0x38 and oracle.e4m3_encode(1.1875) == 0x3A
+
+
+def test_quantize_rows_matches_torch_fp32_recipe():
+    # rows across magnitudes, one row scaled into the tiny range, and an all-zero row
+    x = np.concatenate([rand_bf16((1, 512), std) for std in (1e-6, 1e-3, 1.0, 37.0, 3e4)]
+                       + [np.zeros((1, 512), np.uint16)])
+    q, s = oracle.quantize_rows_e4m3(x)
+    xf = torch.from_numpy((x.astype(np.uint32) << 16).view(np.float32))
+    amax = xf.abs().amax(dim=1)
+    s_ref = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    assert np.array_equal(s.view(np.uint32), s_ref.numpy().view(np.uint32))
+    q_ref = (xf / s_ref[:, None]).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(q, q_ref)
+    assert (q[-1] == 0).all() and s[-1] == 1.0
+    # the largest magnitude of each nonzero row lands on +-448
+    for r in range(len(x) - 1):
+        assert np.abs(np.array([oracle.e4m3(c) for c in q[r]])).max() == 448.0
+
+
+def test_w8a8_expert_equals_weight_only_expert_when_activations_are_exact():
+    # x rows made of e4m3 values times a power of two, each row reaching 448 * 2^k: quantising them
+    # is exact, so the first GEMM (h) must equal the weight-only fp8 expert's h bit for bit
+    import synth
+    rng = np.random.default_rng(11)
+    d, f, rows = 128, 64, 5
+    codes = rng.integers(0, 0x7F, size=(rows, d)).astype(np.uint8)
+    codes[rng.random((rows, d)) < 0.5] |= 0x80
+    codes[:, 0] = 0x7E                                              # amax = 448 in every row
+    vals = np.array([[oracle.e4m3(c) for c in row] for row in codes]) * (2.0 ** rng.integers(-8, 4, (rows, 1)))
+    x = bf16_bits(vals.astype(np.float32))
+    assert np.array_equal((x.astype(np.uint32) << 16).view(np.float32), vals.astype(np.float32))   # exact in bf16
+    W1q, s1 = synth.quantize_e4m3_rows(rand_bf16((f, d), d ** -0.5), d)
+    W3q, s3 = synth.quantize_e4m3_rows(rand_bf16((f, d), d ** -0.5), d)
+    W2q, s2 = synth.quantize_e4m3_rows(rand_bf16((d, f), f ** -0.5), f)
+    h_a8, y_a8 = oracle.expert_ffn_w8a8(x, W1q, s1, W3q, s3, W2q, s2)
+    h_w8, _ = oracle.expert_ffn_q8(x, W1q, s1, W3q, s3, W2q, s2)
+    assert np.array_equal(h_a8, h_w8)
+    # the second GEMM: dequantise h with the pinned quantiser and multiply in float64 (torch)
+    hq, sh = oracle.quantize_rows_e4m3(h_a8)
+    deq = lambda qq: torch.from_numpy(qq).view(torch.float8_e4m3fn).to(torch.float64)
+    hd = deq(hq) * torch.from_numpy(sh.astype(np.float64))[:, None]
+    Wd = deq(W2q) * torch.from_numpy(s2.astype(np.float64))[:, None]
+    y_ref = bf16_bits((hd @ Wd.T).numpy().astype(np.float32))
+    assert np.max(ulp_diff_bf16(y_a8, y_ref)) <= 1
+    assert np.mean(y_a8 == y_ref) > 0.95
