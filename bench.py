@@ -53,8 +53,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="mixtral", choices=list(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
-                    help="expert weight format: bf16, or fp8 e4m3 with fp32 row scales (moe_layer_forward_w8)")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8", "fp8a8"],
+                    help="expert weight format: bf16; fp8 e4m3 with fp32 row scales (moe_layer_forward_w8); "
+                         "fp8a8: fp8 weights and fp8 activations with per-row scales (moe_layer_forward_w8a8)")
     ap.add_argument("--cache-slots", type=int, default=0,
                     help="> 0: decode through the expert cache (moe_layer_forward_cached) with this many HBM "
                          "slots; expert weights in page-locked host memory; a fresh token batch every step")
@@ -90,7 +91,7 @@ def recorded_traffic(kernel: str, workload: str):
     p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(p):
         return None
-    src = kernel_source_hash(kernel.endswith("_fp8"))
+    src = kernel_source_hash(kernel.endswith("_fp8"))   # "_fp8a8" kernels live in the bf16 sources
     for line in open(p):
         parts = line.split()
         if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload \
@@ -513,7 +514,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
     # inputs: replicated weights, a distinct token batch per rank
-    fp8 = args.weights == "fp8"
+    fp8 = args.weights in ("fp8", "fp8a8")
+    a8 = args.weights == "fp8a8"
     tensors = synth.device_tensors(wl, dev, names=["wg", "bias"] if fp8 else
                                    ["wg", "w1", "w3", "w2", "w1s", "w3s", "w2s", "bias"])
     if fp8:
@@ -523,15 +525,17 @@ def main():
     x_host = torch.from_numpy(inp.x_rows(row0, nrows).view(np.int16)).view(torch.bfloat16).reshape(wl.T, wl.d)
     x = x_host.to(dev)
     T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
-    ws = torch.empty(moe.moe_workspace_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device=dev)
+    ws_bytes = moe.moe_workspace_bytes_a8(T, d, E, k, f, fs) if a8 else moe.moe_workspace_bytes(T, d, E, k, f, fs)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
     W = tensors
 
     def fwd(xin, o, events=None):
         if fp8:
-            moe.moe_layer_forward_w8(xin, W["wg"], W["bias"], W["w1q"], W["s1"], W["w3q"], W["s3"], W["w2q"], W["s2"],
-                                     W.get("w1sq"), W.get("s1s"), W.get("w3sq"), W.get("s3s"), W.get("w2sq"),
-                                     W.get("s2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, o, ws, events)
+            call = moe.moe_layer_forward_w8a8 if a8 else moe.moe_layer_forward_w8
+            call(xin, W["wg"], W["bias"], W["w1q"], W["s1"], W["w3q"], W["s3"], W["w2q"], W["s2"], W.get("w1sq"),
+                 W.get("s1s"), W.get("w3sq"), W.get("s3s"), W.get("w2sq"), W.get("s2s"), fs, T, d, E, k, f,
+                 wl.capacity_factor, wl.cap_mode, o, ws, events)
         else:
             moe.moe_layer_forward_ex(xin, W["wg"], W["bias"], W["w1"], W["w3"], W["w2"], W.get("w1s"), W.get("w3s"),
                                      W.get("w2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, o, ws, events)
@@ -631,25 +635,29 @@ def main():
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"]}
     else:
+        tc_ratio = 2.0 if a8 else 1.0     # fp8 tensor peak = measured bf16 peak x the nominal 4.5 / 2.25
         alg = gemm1_work(wl, N)
         achieved = alg / (g1_ms / 1000.0) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"]}
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"] * tc_ratio, "unit": "TFLOP/s",
+                "frac": achieved / (peaks["bf16_tflops"] * tc_ratio)}
     if not decode:   # the same achieved rate against the power-capped sustained GEMM rate, for context
-        roof["frac_of_sustained"] = achieved / peaks["bf16_tflops_sustained"]
-    roof["traffic"] = recorded_traffic("gate_up" + ("_fp8" if fp8 else ""), wl.name)
+        roof["frac_of_sustained"] = achieved / (peaks["bf16_tflops_sustained"] * tc_ratio)
+    roof["traffic"] = recorded_traffic("gate_up" + ("_fp8a8" if a8 else "_fp8" if fp8 else ""), wl.name)
     pair = T * k >= 256 * E
-    roof["kernel"] = ("grouped_gemm_w8_kernel<EPI_SWIGLU>" if fp8 else
+    roof["kernel"] = ("grouped_gemm_kernel<EPI_SWIGLU, F8> (fp8 x fp8)" if a8 else
+                      "grouped_gemm_w8_kernel<EPI_SWIGLU>" if fp8 else
                       "grouped_gemm_pair_kernel<EPI_SWIGLU>" if pair else "grouped_gemm_kernel<EPI_SWIGLU>") + \
         " (gate_up: W1/W3 + SwiGLU)"
-    roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if decode else 'bf16_tflops'}, burst)"
+    roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if decode else 'bf16_tflops'}, burst)" + \
+        ("" if decode or not a8 else " x 2 (nominal fp8 / bf16 dense ratio)")
     roof["algorithmic_per_launch"] = alg
     lf, lb = layer_work(wl, N, touched, 1 if fp8 else 2)
     step_s = total_ms / K / 1000.0
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if not fp8 else "bf16 activations, fp8 e4m3 expert weights",
+        "dtype": ("fp8 e4m3 activations and expert weights (per-row scales), bf16 in/out" if a8 else
+                  "bf16 activations, fp8 e4m3 expert weights" if fp8 else "bf16"),
         "data": "synthetic (seeded Philox4x32-10 + Box-Muller; random-init weights)",
         "config": {"workload": DESCR[wl.name], "global_batch": world * T, "seq_len": T, "parallelism": f"dp{world}",
                    "l2": "working set larger than L2 (expert weights %.2f GB per step)" % (

@@ -349,6 +349,27 @@ int moe_ep_return(const moe_bf16* y_recv, int R, int rank, int E, int d, moe_bf1
                   const void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream);
 
 /*
+ * The layer with fp8 e4m3 weights AND fp8 activations: the weights as in moe_layer_forward_w8();
+ * every activation row entering an expert GEMM (the token's hidden state, then h) is quantised
+ * on its own, s_row = amax(|row|) / 448 in fp32 (1 for an all-zero row), codes
+ * e4m3(fp32(x) / s_row) rounded to nearest even, saturating at 448 (the deployment page's
+ * "w4afp8" option: low-bit weights with fp8 activations).  The expert GEMMs run fp8 x fp8 on
+ * the tensor cores (tcgen05 kind::f8f6f4) with fp32 accumulation and scale each sum by
+ * s_row * s_col before SwiGLU / the bf16 store.  Router, routing, permutation and combine as in
+ * moe_layer_forward().  Workspace: moe_workspace_bytes_a8() (the layer workspace followed by the
+ * quantised rows and their scales).  Shapes: d, f, f_shared multiples of 128 (MOE_ERR_SHAPE).
+ */
+int moe_workspace_bytes_a8(int T, int d, int E, int k, int f, int f_shared, size_t* bytes);
+int moe_layer_forward_w8a8(const moe_bf16* x, const moe_bf16* Wg, const float* bias,
+                           const uint8_t* W1q, const float* s1, const uint8_t* W3q, const float* s3,
+                           const uint8_t* W2q, const float* s2,
+                           const uint8_t* W1sq, const float* s1s, const uint8_t* W3sq, const float* s3s,
+                           const uint8_t* W2sq, const float* s2s, int f_shared,
+                           int T, int d, int E, int k, int f, double capacity_factor, int cap_mode,
+                           moe_bf16* out, void* ws, size_t ws_bytes, moe_stream_t stream,
+                           const moe_stage_events* events);
+
+/*
  * Expert cache: the routed experts' weights live in page-locked host memory and HBM holds S
  * expert slots managed as an LRU.  [EP-DS3] "MoE 推理架构深度实战：从 Expert Parallelism 到
  * DeepSeek-V3 的工程落地", section 3.2 (expert cache and preloading): inactive experts are

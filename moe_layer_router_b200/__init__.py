@@ -84,6 +84,10 @@ _lib.moe_layer_forward_cached_w8.argtypes = [_vp, _vp, _vp, ctypes.POINTER(moe_w
                                              ctypes.POINTER(moe_w8_experts), _i32, _i32, _i32, _i32, _i32, _i32,
                                              _dbl, _i32, _vp, _vp, _sz, _vp, _vp]
 _lib.moe_layer_forward_cached_w8.restype = _i32
+_lib.moe_workspace_bytes_a8.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(_sz)]
+_lib.moe_workspace_bytes_a8.restype = _i32
+_lib.moe_layer_forward_w8a8.argtypes = _lib.moe_layer_forward_w8.argtypes
+_lib.moe_layer_forward_w8a8.restype = _i32
 _lib.moe_layer_permute.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _i32, _i64, _vp, _vp, _sz, _vp]
 _lib.moe_layer_permute.restype = _i32
 _lib.moe_ep_workspace_bytes.argtypes = [_i32, _i32, ctypes.POINTER(_sz)]
@@ -429,6 +433,25 @@ def moe_ep_return(y_recv, R, rank, E, d, y_perm_bufs, ep_ws, stream=None) -> Non
     """y_perm_bufs: R tensors (or device addresses), rank s's y_perm (in its layer workspace)."""
     _check(_lib.moe_ep_return(_ptr(y_recv), R, rank, E, d, _addr_array(y_perm_bufs), _ptr(ep_ws), _nbytes(ep_ws),
                               _stream(stream)), "moe_ep_return")
+
+
+def moe_workspace_bytes_a8(T: int, d: int, E: int, k: int, f: int, f_shared: int = 0) -> int:
+    out = _sz(0)
+    _check(_lib.moe_workspace_bytes_a8(T, d, E, k, f, f_shared, ctypes.byref(out)), "moe_workspace_bytes_a8")
+    return int(out.value)
+
+
+def moe_layer_forward_w8a8(x, Wg, bias, W1q, s1, W3q, s3, W2q, s2, W1sq, s1s, W3sq, s3s, W2sq, s2s, f_shared, T, d,
+                           E, k, f, capacity_factor, cap_mode, out, ws, events: Optional[dict] = None,
+                           stream=None) -> None:
+    """The layer with fp8 e4m3 weights and fp8 activations (per-row scales); ws: a uint8 tensor of
+    moe_workspace_bytes_a8() bytes."""
+    ev = _events(events)
+    _check(_lib.moe_layer_forward_w8a8(_ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1q), _ptr(s1), _ptr(W3q), _ptr(s3),
+                                       _ptr(W2q), _ptr(s2), _ptr(W1sq), _ptr(s1s), _ptr(W3sq), _ptr(s3s),
+                                       _ptr(W2sq), _ptr(s2s), f_shared, T, d, E, k, f, float(capacity_factor),
+                                       cap_mode, _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream),
+                                       ctypes.byref(ev) if ev is not None else None), "moe_layer_forward_w8a8")
 
 
 def moe_get_error(stream=None) -> int:

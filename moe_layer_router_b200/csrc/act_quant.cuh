@@ -1,0 +1,58 @@
+// act_quant.cuh - fp8 e4m3 activations for the fp8 x fp8 expert GEMMs.
+//
+// Every activation row is quantised on its own ([EP-DS3] deployment section, w4afp8: low-bit
+// weights with fp8 activations): s = amax(|x|) / 448 in fp32 (1 for an all-zero row), and each
+// element becomes e4m3(fp32(x) / s), rounded to nearest even and saturating at 448 (the
+// hardware conversion with .satfinite).  One warp per row; 16-byte loads, 8-byte stores.
+#pragma once
+
+#include <cuda_fp8.h>
+
+namespace moe {
+
+// rows of src (bf16, K per row; row r of the output reads src row gather[r] when gather is
+// given) -> dst (e4m3, K bytes per row) and scale[r].  Rows r >= *n_rows (when n_rows is given)
+// are skipped.  K % 8 == 0.
+__global__ void __launch_bounds__(256) quant_rows_e4m3_kernel(const uint4* __restrict__ src,
+                                                              const int32_t* __restrict__ gather,
+                                                              const int32_t* __restrict__ n_rows, int rows, int K,
+                                                              uint2* __restrict__ dst, float* __restrict__ scale) {
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    if (n_rows && row >= __ldg(n_rows)) return;
+    const long long srow = gather ? __ldg(gather + row) : row;
+    const int chunks = K / 8;                     // 8 bf16 per uint4
+    const uint4* s = src + srow * chunks;
+    float amax = 0.f;
+    for (int c = lane; c < chunks; c += 32) {
+        const uint4 v = __ldg(s + c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            amax = fmaxf(amax, fabsf(__uint_as_float(w[i] << 16)));
+            amax = fmaxf(amax, fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    if (lane == 0) scale[row] = sc;
+    uint2* d = dst + (long long)row * chunks;
+    for (int c = lane; c < chunks; c += 32) {
+        const uint4 v = __ldg(s + c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t out[2] = {0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float lo = __fdiv_rn(__uint_as_float(w[i] << 16), sc);
+            const float hi = __fdiv_rn(__uint_as_float(w[i] & 0xFFFF0000u), sc);
+            const uint32_t b0 = __nv_cvt_float_to_fp8(lo, __NV_SATFINITE, __NV_E4M3);
+            const uint32_t b1 = __nv_cvt_float_to_fp8(hi, __NV_SATFINITE, __NV_E4M3);
+            out[i >> 1] |= (b0 | (b1 << 8)) << (16 * (i & 1));
+        }
+        d[c] = make_uint2(out[0], out[1]);
+    }
+}
+
+}  // namespace moe

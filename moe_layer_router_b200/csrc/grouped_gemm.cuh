@@ -63,6 +63,13 @@ struct GemmClass {
     long long out_rows; // output rows available (stores at or beyond are dropped)
     int ksplit;         // dense class: K is cut into ksplit slices of K each (>= 1)
     long long split_stride;  // output elements between the partial results of two slices
+    // fp8 operands (F8 kernels): the fp32 accumulator of A row r, output column n of weight
+    // group g is multiplied by a_scale[r] * b_scale[g * b_scale_stride + n] (b_scale2: the up
+    // projection of a SwiGLU tile)
+    const float* a_scale;
+    const float* b_scale;
+    const float* b_scale2;
+    long long b_scale_stride;
 };
 
 struct GemmParams {
@@ -140,7 +147,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int EPI>
+// F8: A and B are e4m3 (one byte per element, 128 K-elements per stage row of 128 bytes),
+// tcgen05.mma kind::f8f6f4, and the epilogue applies the row and column scales.
+template <int EPI, bool F8 = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB0b, const __grid_constant__ CUtensorMap tmA1,
@@ -212,7 +221,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
                 const CUtensorMap* mA = ti.cls ? &tmA1 : &tmA0;
                 const CUtensorMap* mB = ti.cls ? &tmB1 : &tmB0;
                 const CUtensorMap* mBb = ti.cls ? &tmB1b : &tmB0b;
-                const int nk = c.K / GEMM_BK;
+                constexpr int KB = F8 ? 2 * GEMM_BK : GEMM_BK;   // K elements per 128-byte stage row
+                const int nk = c.K / KB;
                 const int k0 = ti.ks * c.K;
                 const uint32_t bytes =
                     GEMM_A_BYTES + (EPI == EPI_SWIGLU ? 2u : 1u) * (uint32_t)c.b_tile_rows * GEMM_BK * 2u;
@@ -221,10 +231,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
                     mbar_arrive_expect_tx(full_bar + stage, bytes);
                     uint8_t* a_dst = sA + stage * GEMM_A_BYTES;
                     uint8_t* b_dst = sB + stage * p.b_slot;
-                    tma_load_2d(a_dst, mA, full_bar + stage, k0 + kb * GEMM_BK, ti.a_row, pol_a);
-                    tma_load_2d(b_dst, mB, full_bar + stage, k0 + kb * GEMM_BK, ti.b_row, pol_b);
+                    tma_load_2d(a_dst, mA, full_bar + stage, k0 + kb * KB, ti.a_row, pol_a);
+                    tma_load_2d(b_dst, mB, full_bar + stage, k0 + kb * KB, ti.b_row, pol_b);
                     if (EPI == EPI_SWIGLU)
-                        tma_load_2d(b_dst + 128 * 128, mBb, full_bar + stage, k0 + kb * GEMM_BK, ti.b_row, pol_b);
+                        tma_load_2d(b_dst + 128 * 128, mBb, full_bar + stage, k0 + kb * KB, ti.b_row, pol_b);
                     ++issued;
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
@@ -249,8 +259,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
                 const TileInfo ti = gemm_decode_tile(p, t, routed_tiles);
                 const GemmClass& c = p.cls[ti.cls];
-                const uint32_t idesc = idesc_bf16_f32(GEMM_BM, c.mma_n);
-                const int nk = c.K / GEMM_BK;
+                const uint32_t idesc = F8 ? idesc_e4m3_f32(GEMM_BM, c.mma_n) : idesc_bf16_f32(GEMM_BM, c.mma_n);
+                const int nk = c.K / (F8 ? 2 * GEMM_BK : GEMM_BK);
                 if (!mbar_wait(tempty_bar + acc, acc_phase ^ 1u, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * GEMM_ACC_COLS);
@@ -260,8 +270,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
                     const uint64_t ad = smem_desc_k_sw128(sA + stage * GEMM_A_BYTES);
                     const uint64_t bd = smem_desc_k_sw128(sB + stage * p.b_slot);
 #pragma unroll
-                    for (int kk = 0; kk < GEMM_BK / 16; ++kk)
-                        umma_bf16(d_tmem, ad + 2ull * kk, bd + 2ull * kk, idesc, (kb | kk) != 0);
+                    for (int kk = 0; kk < 4; ++kk) {   // 32 bytes of K per instruction (16 bf16 or 32 e4m3)
+                        if (F8) umma_e4m3(d_tmem, ad + 2ull * kk, bd + 2ull * kk, idesc, (kb | kk) != 0);
+                        else umma_bf16(d_tmem, ad + 2ull * kk, bd + 2ull * kk, idesc, (kb | kk) != 0);
+                    }
                     umma_commit(empty_bar + stage);
                     any = true;
                     if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -294,6 +306,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
             const long long orow = c.out_row0 + ti.a_row + row_in_tile;
             const bool row_ok = row_in_tile < ti.rows && orow >= 0 && orow < c.out_rows;
 
+            // fp8: the A row's scale and the weight group's column scales
+            float sa = 1.f;
+            const float *sb = nullptr, *sb2 = nullptr;
+            if (F8) {
+                if (row_ok) sa = __ldg(c.a_scale + ti.a_row + row_in_tile);
+                const long long wg = c.b_group_rows > 0 ? ti.b_row / c.b_group_rows : 0;
+                sb = c.b_scale + wg * c.b_scale_stride;
+                if (EPI == EPI_SWIGLU) sb2 = c.b_scale2 + wg * c.b_scale_stride;
+            }
             if (EPI == EPI_SWIGLU) {
                 __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(c.out) + orow * c.ldo;
 #pragma unroll 1
@@ -305,6 +326,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
                     tmem_ld_wait();
                     const int col0 = ti.n_idx * 128 + ch * 32;
                     if (row_ok && col0 < c.n_out) {
+                        if (F8) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) {
+                                const bool in = col0 + i < c.n_out;
+                                g[i] = __float_as_uint(__uint_as_float(g[i]) * sa * (in ? __ldg(sb + col0 + i) : 0.f));
+                                u[i] = __float_as_uint(__uint_as_float(u[i]) * sa * (in ? __ldg(sb2 + col0 + i) : 0.f));
+                            }
+                        }
                         uint32_t packed[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
@@ -330,6 +359,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
                     tmem_ld_wait();
                     const int col0 = ti.n_idx * c.b_tile_rows + ch * 32;
                     if (row_ok && col0 < c.n_out) {
+                        if (F8) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                v[i] = __float_as_uint(__uint_as_float(v[i]) * sa *
+                                                       (col0 + i < c.n_out ? __ldg(sb + col0 + i) : 0.f));
+                        }
                         uint32_t packed[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i)

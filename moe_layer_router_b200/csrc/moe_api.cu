@@ -14,6 +14,7 @@
 #include "route_permute_combine.cuh"
 #include "expert_cache.cuh"
 #include "expert_parallel.cuh"
+#include "act_quant.cuh"
 
 namespace moe {
 namespace {
@@ -98,9 +99,22 @@ int make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// e4m3 operands [rows, inner] bytes for the fp8 x fp8 GEMMs: boxes of box_rows rows x 128 bytes,
+// 128-byte swizzle (the layout the K-major tcgen05 descriptors read).
+int make_map_e4m3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
 int launch_status() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-template <int EPI>
+template <int EPI, bool F8 = false>
 int launch_gemm(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& b0b,
                 const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& b1b, GemmParams p,
                 long long tiles_upper, cudaStream_t s) {
@@ -110,7 +124,7 @@ int launch_gemm(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b0, co
         int dev = 0;
         cudaGetDevice(&dev);
         if (!attr_set[dev][EPI]) {
-            if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      GEMM_SMEM_MAX) != cudaSuccess)
                 return MOE_ERR_CUDA;
             attr_set[dev][EPI] = true;
@@ -124,7 +138,7 @@ int launch_gemm(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b0, co
     }
     const int smem = gemm_smem_bytes(p.stages, p.b_slot);
     const int grid = (int)(tiles_upper < di->sms ? tiles_upper : di->sms);
-    grouped_gemm_kernel<EPI><<<grid, GEMM_THREADS, smem, s>>>(a0, b0, b0b, a1, b1, b1b, p);
+    grouped_gemm_kernel<EPI, F8><<<grid, GEMM_THREADS, smem, s>>>(a0, b0, b0b, a1, b1, b1b, p);
     return launch_status();
 }
 
@@ -209,6 +223,33 @@ LayerLayout layer_layout(int T, int d, int E, int k, int f, int f_shared) {
     L.router_part = take(router_partial_bytes(T, d, E));
     L.total = cur;
     return L;
+}
+
+// fp8 activations of the fp8 x fp8 layer, after the layer workspace: the permuted rows and h
+// (routed), x and h of the shared expert, each as e4m3 codes plus one fp32 scale per row.
+struct A8Layout {
+    size_t xq, sx, hq, sh, xqs, sxs, hqs, shs, total;
+};
+
+A8Layout a8_layout(size_t base, int T, int d, int k, int f, int f_shared) {
+    A8Layout A;
+    const size_t Tk = (size_t)T * k;
+    size_t cur = align256(base);
+    auto take = [&](size_t bytes) {
+        size_t o = cur;
+        cur = align256(cur + bytes);
+        return o;
+    };
+    A.xq = take(Tk * d);
+    A.sx = take(Tk * 4);
+    A.hq = take(Tk * f);
+    A.sh = take(Tk * 4);
+    A.xqs = take(f_shared > 0 ? (size_t)T * d : 0);
+    A.sxs = take(f_shared > 0 ? (size_t)T * 4 : 0);
+    A.hqs = take(f_shared > 0 ? (size_t)T * f_shared : 0);
+    A.shs = take(f_shared > 0 ? (size_t)T * 4 : 0);
+    A.total = cur;
+    return A;
 }
 
 // scratch used by moe_permute: blk_cnt + rank_local + mprefix
@@ -532,6 +573,114 @@ int run_expert_ffn_w8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, cuda
     return MOE_OK;
 }
 
+// Both expert GEMMs with fp8 weights and fp8 activations: x_perm rows are quantised straight
+// from x (gathered by src_token), h rows after GEMM1; the 1-SM grouped GEMM runs kind::f8f6f4
+// and scales each accumulator by its activation row scale and weight row scale.
+struct A8Bufs {
+    uint8_t *xq, *hq, *xqs, *hqs;
+    float *sx, *sh, *sxs, *shs;
+    const int32_t* src_token;
+};
+
+int run_quant_rows(const void* src, const int32_t* gather, const int32_t* n_rows, int rows, int K, uint8_t* dst,
+                   float* scale, cudaStream_t s) {
+    if (rows <= 0) return MOE_OK;
+    quant_rows_e4m3_kernel<<<(rows + 7) / 8, 256, 0, s>>>(static_cast<const uint4*>(src), gather, n_rows, rows, K,
+                                                          reinterpret_cast<uint2*>(dst), scale);
+    return launch_status();
+}
+
+int run_expert_ffn_a8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, const A8Bufs& b, cudaStream_t s,
+                      cudaEvent_t ev_down) {
+    const bool shared = a.f_shared > 0;
+    const bool routed = a.max_rows > 0;
+    const int32_t* n_routed = routed ? a.offsets + a.E : nullptr;   // kept rows (device)
+    int rc;
+    if (routed && (rc = run_quant_rows(a.x, b.src_token, n_routed, a.max_rows, a.d, b.xq, b.sx, s)) != MOE_OK)
+        return rc;
+    if (shared && (rc = run_quant_rows(a.x, nullptr, nullptr, a.T, a.d, b.xqs, b.sxs, s)) != MOE_OK) return rc;
+    // ---- GEMM1: h = silu(s_x s1 (xq W1q^T)) * (s_x s3 (xq W3q^T))
+    {
+        CUtensorMap A0, B0, B0b, A1, B1, B1b;
+        if (routed) {
+            if ((rc = make_map_e4m3(&A0, b.xq, a.d, a.max_rows, GEMM_BM)) != MOE_OK) return rc;
+            if ((rc = make_map_e4m3(&B0, q.W1q, a.d, weight_groups(a) * a.f, 128)) != MOE_OK) return rc;
+            if ((rc = make_map_e4m3(&B0b, q.W3q, a.d, weight_groups(a) * a.f, 128)) != MOE_OK) return rc;
+        }
+        if (shared) {
+            if ((rc = make_map_e4m3(&A1, b.xqs, a.d, a.T, GEMM_BM)) != MOE_OK) return rc;
+            if ((rc = make_map_e4m3(&B1, q.W1sq, a.d, a.f_shared, 128)) != MOE_OK) return rc;
+            if ((rc = make_map_e4m3(&B1b, q.W3sq, a.d, a.f_shared, 128)) != MOE_OK) return rc;
+        }
+        if (!routed) { A0 = A1; B0 = B1; B0b = B1b; }
+        if (!shared) { A1 = A0; B1 = B0; B1b = B0b; }
+        GemmParams p;
+        memset(&p, 0, sizeof(p));
+        GemmClass& c0 = p.cls[0];
+        c0.K = a.d; c0.n_out = a.f; c0.ntiles = (a.f + 127) / 128; c0.b_group_rows = a.f; c0.b_tile_rows = 128;
+        c0.mma_n = 256; c0.out = a.h; c0.ldo = a.f; c0.out_row0 = 0; c0.out_rows = a.max_rows;
+        c0.a_scale = b.sx; c0.b_scale = q.s1; c0.b_scale2 = q.s3; c0.b_scale_stride = a.f;
+        GemmClass& c1 = p.cls[1];
+        c1.K = a.d; c1.n_out = a.f_shared; c1.ntiles = (a.f_shared + 127) / 128; c1.b_group_rows = 0;
+        c1.b_tile_rows = 128; c1.mma_n = 256; c1.out = a.h_shared; c1.ldo = a.f_shared; c1.out_row0 = 0;
+        c1.out_rows = a.T;
+        c1.a_scale = b.sxs; c1.b_scale = q.s1s; c1.b_scale2 = q.s3s; c1.b_scale_stride = 0;
+        c0.ksplit = c1.ksplit = 1;
+        p.offsets = routed ? a.offsets : nullptr;
+        p.mprefix = a.mprefix;
+        p.E = a.E;
+        p.dense_rows = shared ? a.T : 0;
+        p.b_slot = GEMM_B_BYTES;
+        p.stages = GEMM_STAGES;
+        p.group_map = a.group_map;
+        long long tiles = 0;
+        if (routed) tiles += ((long long)(a.max_rows + GEMM_BM - 1) / GEMM_BM + a.E) * c0.ntiles;
+        if (shared) tiles += (long long)((a.T + GEMM_BM - 1) / GEMM_BM) * c1.ntiles;
+        if ((rc = launch_gemm<EPI_SWIGLU, true>(di, A0, B0, B0b, A1, B1, B1b, p, tiles, s)) != MOE_OK) return rc;
+    }
+    if (ev_down && cudaEventRecord(ev_down, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (routed && (rc = run_quant_rows(a.h, nullptr, n_routed, a.max_rows, a.f, b.hq, b.sh, s)) != MOE_OK) return rc;
+    if (shared && (rc = run_quant_rows(a.h_shared, nullptr, nullptr, a.T, a.f_shared, b.hqs, b.shs, s)) != MOE_OK)
+        return rc;
+    // ---- GEMM2: y = s_h s2 (hq W2q^T)
+    {
+        CUtensorMap A0, B0, A1, B1;
+        if (routed) {
+            if ((rc = make_map_e4m3(&A0, b.hq, a.f, a.max_rows, GEMM_BM)) != MOE_OK) return rc;
+            if ((rc = make_map_e4m3(&B0, q.W2q, a.f, weight_groups(a) * a.d, 256)) != MOE_OK) return rc;
+        }
+        if (shared) {
+            if ((rc = make_map_e4m3(&A1, b.hqs, a.f_shared, a.T, GEMM_BM)) != MOE_OK) return rc;
+            if ((rc = make_map_e4m3(&B1, q.W2sq, a.f_shared, a.d, 256)) != MOE_OK) return rc;
+        }
+        if (!routed) { A0 = A1; B0 = B1; }
+        if (!shared) { A1 = A0; B1 = B0; }
+        GemmParams p;
+        memset(&p, 0, sizeof(p));
+        GemmClass& c0 = p.cls[0];
+        c0.K = a.f; c0.n_out = a.d; c0.ntiles = (a.d + 255) / 256; c0.b_group_rows = a.d; c0.b_tile_rows = 256;
+        c0.mma_n = 256; c0.out = a.y_perm; c0.ldo = a.d; c0.out_row0 = 0; c0.out_rows = a.max_rows;
+        c0.a_scale = b.sh; c0.b_scale = q.s2; c0.b_scale_stride = a.d;
+        GemmClass& c1 = p.cls[1];
+        c1.K = a.f_shared; c1.n_out = a.d; c1.ntiles = (a.d + 255) / 256; c1.b_group_rows = 0; c1.b_tile_rows = 256;
+        c1.mma_n = 256; c1.out = a.y_shared; c1.ldo = a.d; c1.out_row0 = 0; c1.out_rows = a.T;
+        c1.a_scale = b.shs; c1.b_scale = q.s2s; c1.b_scale_stride = 0;
+        c0.ksplit = c1.ksplit = 1;
+        p.offsets = routed ? a.offsets : nullptr;
+        p.mprefix = a.mprefix;
+        p.E = a.E;
+        p.dense_rows = shared ? a.T : 0;
+        p.b_slot = GEMM_B_BYTES;
+        p.stages = GEMM_STAGES;
+        p.group_map = a.group_map;
+        long long tiles = 0;
+        if (routed) tiles += ((long long)(a.max_rows + GEMM_BM - 1) / GEMM_BM + a.E) * c0.ntiles;
+        if (shared) tiles += (long long)((a.T + GEMM_BM - 1) / GEMM_BM) * c1.ntiles;
+        if ((rc = launch_gemm<EPI_STORE, true>(di, A0, B0, B0, A1, B1, B1, p, tiles, s)) != MOE_OK) return rc;
+    }
+    return MOE_OK;
+}
+
 int run_combine(const moe_bf16* y_perm, const int32_t* dest, const float* w, const moe_bf16* y_shared, int T, int d,
                 int k, moe_bf16* out, cudaStream_t s) {
     // longest row segment per warp that still leaves >= 8192 warps (or one 32-chunk segment)
@@ -708,7 +857,7 @@ int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float*
                  const moe_bf16* W3, const moe_bf16* W2, const moe_bf16* W1s, const moe_bf16* W3s, const moe_bf16* W2s,
                  int f_shared, int T, int d, int E, int k, int f, long long C, const int32_t* fill_base,
                  moe_bf16* out, void* ws, size_t ws_bytes, cudaStream_t s, const moe_stage_events* events,
-                 const W8Weights* w8 = nullptr, const CacheArgs* cache = nullptr) {
+                 const W8Weights* w8 = nullptr, const CacheArgs* cache = nullptr, bool act8 = false) {
     int rc = check_shape(T, d, E, k, f);
     if (rc != MOE_OK) return rc;
     MOE_REQUIRE(f_shared >= 0 && f_shared % 64 == 0, MOE_ERR_SHAPE);
@@ -734,6 +883,8 @@ int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float*
                 MOE_ERR_ALIGN);
     const LayerLayout L = layer_layout(T, d, E, k, f, f_shared);
     MOE_REQUIRE(ws_bytes >= L.total, MOE_ERR_WORKSPACE);
+    const A8Layout A8 = a8_layout(L.total, T, d, k, f, f_shared);
+    if (act8) MOE_REQUIRE(ws_bytes >= A8.total, MOE_ERR_WORKSPACE);
     DeviceInfo* di;
     if ((rc = device_info(&di)) != MOE_OK) return rc;
     char* base = static_cast<char*>(ws);
@@ -804,8 +955,22 @@ int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float*
     a.x = x; a.T = T; a.f_shared = f_shared; a.W1s = W1s; a.W3s = W3s; a.W2s = W2s;
     a.h_shared = h_shared; a.y_shared = y_shared;
     a.pair = pair;
-    rc = w8 ? run_expert_ffn_w8(di, a, *w8, s, static_cast<cudaEvent_t>(ev.down))
-            : run_expert_ffn(di, a, s, static_cast<cudaEvent_t>(ev.down));
+    if (w8 && act8) {
+        A8Bufs b;
+        b.xq = reinterpret_cast<uint8_t*>(base + A8.xq);
+        b.hq = reinterpret_cast<uint8_t*>(base + A8.hq);
+        b.xqs = shared ? reinterpret_cast<uint8_t*>(base + A8.xqs) : nullptr;
+        b.hqs = shared ? reinterpret_cast<uint8_t*>(base + A8.hqs) : nullptr;
+        b.sx = reinterpret_cast<float*>(base + A8.sx);
+        b.sh = reinterpret_cast<float*>(base + A8.sh);
+        b.sxs = shared ? reinterpret_cast<float*>(base + A8.sxs) : nullptr;
+        b.shs = shared ? reinterpret_cast<float*>(base + A8.shs) : nullptr;
+        b.src_token = src;
+        rc = run_expert_ffn_a8(di, a, *w8, b, s, static_cast<cudaEvent_t>(ev.down));
+    } else {
+        rc = w8 ? run_expert_ffn_w8(di, a, *w8, s, static_cast<cudaEvent_t>(ev.down))
+                : run_expert_ffn(di, a, s, static_cast<cudaEvent_t>(ev.down));
+    }
     if (rc != MOE_OK) return rc;
     if (!mark(ev.combine)) return MOE_ERR_CUDA;
     if ((rc = run_combine(y_perm, dest, w, y_shared, T, d, k, out, s)) != MOE_OK) return rc;
@@ -938,6 +1103,31 @@ int moe_layer_forward_cached_w8(const moe_bf16* x, const moe_bf16* Wg, const flo
     return layer_phases(LAYER_ROUTE | LAYER_FINISH, x, Wg, bias, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                         f_shared, T, d, E, k, f, C, nullptr, out, ws, ws_bytes, static_cast<cudaStream_t>(stream),
                         events, &q, &ca);
+}
+
+int moe_workspace_bytes_a8(int T, int d, int E, int k, int f, int f_shared, size_t* bytes) {
+    using namespace moe;
+    MOE_REQUIRE(bytes, MOE_ERR_INVALID_ARG);
+    int rc = check_shape(T, d, E, k, f);
+    if (rc != MOE_OK) return rc;
+    MOE_REQUIRE(f_shared >= 0 && f_shared % 64 == 0, MOE_ERR_SHAPE);
+    *bytes = a8_layout(layer_layout(T, d, E, k, f, f_shared).total, T, d, k, f, f_shared).total;
+    return MOE_OK;
+}
+
+int moe_layer_forward_w8a8(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const uint8_t* W1q,
+                           const float* s1, const uint8_t* W3q, const float* s3, const uint8_t* W2q, const float* s2,
+                           const uint8_t* W1sq, const float* s1s, const uint8_t* W3sq, const float* s3s,
+                           const uint8_t* W2sq, const float* s2s, int f_shared, int T, int d, int E, int k, int f,
+                           double capacity_factor, int cap_mode, moe_bf16* out, void* ws, size_t ws_bytes,
+                           moe_stream_t stream, const moe_stage_events* events) {
+    MOE_REQUIRE(cap_mode >= MOE_CAP_NONE && cap_mode <= MOE_CAP_PER_ASSIGNMENT, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(d % 128 == 0 && f % 128 == 0 && f_shared % 128 == 0, MOE_ERR_SHAPE);   // 128-byte fp8 K rows
+    const long long C = moe_capacity(T, E, k, capacity_factor, cap_mode);
+    moe::W8Weights q = {W1q, W3q, W2q, W1sq, W3sq, W2sq, s1, s3, s2, s1s, s3s, s2s};
+    return moe::layer_phases(moe::LAYER_ROUTE | moe::LAYER_FINISH, x, Wg, bias, nullptr, nullptr, nullptr, nullptr,
+                             nullptr, nullptr, f_shared, T, d, E, k, f, C, nullptr, out, ws, ws_bytes,
+                             static_cast<cudaStream_t>(stream), events, &q, nullptr, true);
 }
 
 int moe_layer_forward_w8(const moe_bf16* x, const moe_bf16* Wg, const float* bias, const uint8_t* W1q,

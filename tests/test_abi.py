@@ -155,3 +155,19 @@ def test_cached_fp8_entry_host_checks(lib):
     assert call(16, None, ctypes.byref(slots)) == -1                        # no sources
     bad = W8(16, 16, 16, 16, 16, 24)
     assert call(16, ctypes.byref(src), ctypes.byref(bad)) == -3             # misaligned slot array
+
+
+def test_fp8_activation_entry_needs_128_byte_k(lib):
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.moe_layer_forward_w8a8.argtypes = [vp] * 15 + [i32] * 6 + [ctypes.c_double, i32, vp, vp, sz, vp, vp]
+    args = [16] * 15
+    # d = 192 is a multiple of 64 but not of 128: the fp8 stage rows are 128 K-elements
+    assert lib.moe_layer_forward_w8a8(*args, 0, 8, 192, 8, 2, 256, 1.0, 0, 16, 16, 1 << 20, None, None) == -2
+    assert lib.moe_layer_forward_w8a8(*args, 64, 8, 256, 8, 2, 256, 1.0, 0, 16, 16, 1 << 20, None, None) == -2
+    lib.moe_workspace_bytes_a8.argtypes = [i32] * 6 + [ctypes.POINTER(sz)]
+    lib.moe_workspace_bytes.argtypes = [i32] * 6 + [ctypes.POINTER(sz)]
+    a, b = sz(0), sz(0)
+    assert lib.moe_workspace_bytes_a8(256, 7168, 256, 8, 2048, 2048, ctypes.byref(a)) == 0
+    assert lib.moe_workspace_bytes(256, 7168, 256, 8, 2048, 2048, ctypes.byref(b)) == 0
+    # plus fp8 copies of the permuted rows and of h (routed and shared) and their scales
+    assert a.value >= b.value + 2048 * (7168 + 2048) + 256 * (7168 + 2048)

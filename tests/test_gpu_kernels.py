@@ -433,3 +433,87 @@ def test_layer_fp8_weights(moe, wl):
     got = bf16_bits(out)
     assert_layer_close(got, ref, "fp8-weight layer")
     assert np.mean(ulp_bf16(got, ref) <= 1) > 0.98
+
+
+def _a8_reference(wl, x, logits, inp, k, C):
+    """Oracle layer with fp8 weights and fp8 activations: route the GPU's logits, dispatch,
+    fp8 x fp8 experts, combine."""
+    E, d, f = wl.E, wl.d, wl.f
+    idx, w = oracle.route(logits, k, inp.bias())
+    r = oracle.dispatch(idx, E, C)
+    xp = oracle.gather(x, r["dest"], r["N"])
+    y_perm = np.zeros((max(r["N"], 1), d), np.uint16)
+    for e in range(E):
+        a, b = r["offsets"][e], r["offsets"][e + 1]
+        if a == b:
+            continue
+        q1, s1 = synth.quantize_e4m3_rows(inp.expert_rows("w1", e, 1), d)
+        q3, s3 = synth.quantize_e4m3_rows(inp.expert_rows("w3", e, 1), d)
+        q2, s2 = synth.quantize_e4m3_rows(inp.expert_rows("w2", e, 1), f)
+        _, y_perm[a:b] = oracle.expert_ffn_w8a8(xp[a:b], q1, s1, q3, s3, q2, s2)
+    ysh = None
+    if wl.has_shared:
+        qs = {n: synth.quantize_e4m3_rows(inp.shared(n), inp.shared(n).shape[1]) for n in ("w1s", "w3s", "w2s")}
+        _, ysh = oracle.expert_ffn_w8a8(x, qs["w1s"][0], qs["w1s"][1], qs["w3s"][0], qs["w3s"][1], qs["w2s"][0],
+                                        qs["w2s"][1])
+    return idx, r, xp, oracle.combine(y_perm, r["dest"], w, ysh)
+
+
+@pytest.mark.parametrize("wl", [synth.Workload("a8", 300, 256, 16, 4, 384, f_shared=256, bias_range=0.1,
+                                               cap_mode=synth.CAP_PER_TOKEN, capacity_factor=1.5),
+                                synth.Workload("a8dec", 40, 512, 32, 8, 256, f_shared=128, bias_range=0.1),
+                                synth.Workload("a8mix", 512, 256, 16, 2, 128, zipf_s=1.2)],
+                         ids=["shared-cap-bias", "decode-shaped", "skewed-mixed-tiles"])
+def test_layer_fp8_weights_and_activations(moe, wl):
+    T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
+    inp = synth.Inputs(wl)
+    x = inp.x()
+    Q = synth.device_tensors_q8(wl, "cuda")
+    ws = torch.empty(moe.moe_workspace_bytes_a8(T, d, E, k, f, fs), dtype=torch.uint8, device="cuda")
+    out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    bias = torch.from_numpy(inp.bias()).cuda() if inp.bias() is not None else None
+    moe.moe_layer_forward_w8a8(to_dev_bf16(x), to_dev_bf16(inp.wg()), bias, Q["w1q"], Q["s1"], Q["w3q"], Q["s3"],
+                               Q["w2q"], Q["s2"], Q.get("w1sq"), Q.get("s1s"), Q.get("w3sq"), Q.get("s3s"),
+                               Q.get("w2sq"), Q.get("s2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode,
+                               out, ws)
+    assert moe.moe_get_error() == 0
+    L = moe.moe_workspace_layout(T, d, E, k, f, fs)
+    logits = moe.workspace_view(ws, L, "logits", (T, E), torch.float32).cpu().numpy()
+    C = oracle.capacity(T, E, k, wl.capacity_factor, wl.cap_mode)
+    idx, r, xp, ref = _a8_reference(wl, x, logits, inp, k, C)
+    assert np.array_equal(moe.workspace_view(ws, L, "idx", (T, k), torch.int32).cpu().numpy(), idx)
+    xq_ref, sx_ref = oracle.quantize_rows_e4m3(xp)
+    got = bf16_bits(out)
+    assert_layer_close(got, ref, "fp8 x fp8 layer")
+    g64, r64 = bits_to_f64(got), bits_to_f64(ref)
+    assert np.sqrt(np.mean((g64 - r64) ** 2) / max(np.mean(r64 ** 2), 1e-30)) < 5e-3
+    assert xq_ref.shape[0] == r["N"] and np.isfinite(sx_ref).all()
+
+
+def test_quantised_rows_bit_exact(moe):
+    """The layer's activation quantiser against the oracle's on the permuted rows: the workspace's
+    fp8 region follows the layer workspace (moe_workspace_bytes_a8 - ...), so it is read through a
+    layer call on a shape whose routed rows fill the region from its start."""
+    wl = synth.Workload("a8q", 64, 256, 4, 2, 128)
+    T, d, E, k, f = wl.T, wl.d, wl.E, wl.k, wl.f
+    inp = synth.Inputs(wl)
+    x = inp.x()
+    Q = synth.device_tensors_q8(wl, "cuda")
+    ws = torch.zeros(moe.moe_workspace_bytes_a8(T, d, E, k, f, 0), dtype=torch.uint8, device="cuda")
+    out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_layer_forward_w8a8(to_dev_bf16(x), to_dev_bf16(inp.wg()), None, Q["w1q"], Q["s1"], Q["w3q"], Q["s3"],
+                               Q["w2q"], Q["s2"], None, None, None, None, None, None, 0, T, d, E, k, f, 1.0,
+                               moe.MOE_CAP_NONE, out, ws)
+    assert moe.moe_get_error() == 0
+    L = moe.moe_workspace_layout(T, d, E, k, f, 0)
+    base = moe.moe_workspace_bytes(T, d, E, k, f, 0)
+    start = (base + 255) // 256 * 256
+    N = T * k
+    xq = ws[start:start + N * d].cpu().numpy().reshape(N, d)
+    so = (start + N * d + 255) // 256 * 256
+    sx = ws[so:so + 4 * N].view(torch.float32).cpu().numpy()
+    dest = moe.workspace_view(ws, L, "dest", (T, k), torch.int32).cpu().numpy()
+    xp = oracle.gather(x, dest, N)
+    xq_ref, sx_ref = oracle.quantize_rows_e4m3(xp)
+    assert np.array_equal(sx.view(np.uint32), sx_ref.view(np.uint32))
+    assert np.array_equal(xq, xq_ref)
