@@ -644,7 +644,8 @@ def main():
         roof["frac_of_sustained"] = achieved / (peaks["bf16_tflops_sustained"] * tc_ratio)
     roof["traffic"] = recorded_traffic("gate_up" + ("_fp8a8" if a8 else "_fp8" if fp8 else ""), wl.name)
     pair = T * k >= 256 * E
-    roof["kernel"] = ("grouped_gemm_kernel<EPI_SWIGLU, F8> (fp8 x fp8)" if a8 else
+    roof["kernel"] = (("grouped_gemm_pair_kernel" if pair else "grouped_gemm_kernel") + "<EPI_SWIGLU, F8> (fp8 x fp8)"
+                      if a8 else
                       "grouped_gemm_w8_kernel<EPI_SWIGLU>" if fp8 else
                       "grouped_gemm_pair_kernel<EPI_SWIGLU>" if pair else "grouped_gemm_kernel<EPI_SWIGLU>") + \
         " (gate_up: W1/W3 + SwiGLU)"

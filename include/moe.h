@@ -452,9 +452,10 @@ int moe_layer_forward_cached_w8(const moe_bf16* x, const moe_bf16* Wg, const flo
  *   off[3] counts_raw [E]      off[4] counts [E]        off[5] offsets [E+1]
  *   off[6] dest [T,k]          off[7] src_token [T*k]   off[8] x_perm [T*k,d] bf16
  *   off[9] h [T*k,f] bf16      off[10] y_perm [T*k,d]   off[11] y_shared [T,d] bf16
+ *   off[12] h_shared [T,f_shared] bf16
  * Returns MOE_OK or a shape error.
  */
-int moe_workspace_layout(int T, int d, int E, int k, int f, int f_shared, size_t off[12]);
+int moe_workspace_layout(int T, int d, int E, int k, int f, int f_shared, size_t off[13]);
 
 /*
  * Synchronises `stream`, returns the first device-side error recorded on the current

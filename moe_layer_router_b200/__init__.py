@@ -34,7 +34,7 @@ MOE_CAP_NONE, MOE_CAP_PER_TOKEN, MOE_CAP_PER_ASSIGNMENT = 0, 1, 2
 
 # Names of the intermediates moe_layer_forward leaves in its workspace (moe_workspace_layout order).
 WS_NAMES = ["logits", "idx", "w", "counts_raw", "counts", "offsets", "dest", "src_token",
-            "x_perm", "h", "y_perm", "y_shared"]
+            "x_perm", "h", "y_perm", "y_shared", "h_shared"]
 
 
 class MoeError(RuntimeError):
@@ -175,7 +175,7 @@ def moe_workspace_bytes(T: int, d: int, E: int, k: int, f: int, f_shared: int = 
 
 
 def moe_workspace_layout(T: int, d: int, E: int, k: int, f: int, f_shared: int = 0) -> dict:
-    arr = (_sz * 12)()
+    arr = (_sz * 13)()
     _check(_lib.moe_workspace_layout(T, d, E, k, f, f_shared, arr), "moe_workspace_layout")
     return {n: int(arr[i]) for i, n in enumerate(WS_NAMES)}
 

@@ -76,7 +76,9 @@ __device__ __forceinline__ PairTile pair_decode_tile(const GemmParams& p, int t,
     return ti;
 }
 
-template <int EPI>
+// F8: e4m3 operands (128 K-elements per 128-byte stage row, kind::f8f6f4) and the epilogue
+// applies the row and column scales of GemmClass.
+template <int EPI, bool F8 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                          const __grid_constant__ CUtensorMap tmB0b, const __grid_constant__ CUtensorMap tmA1,
@@ -161,13 +163,14 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                     b_row = wg * c.b_group_rows + ti.n_idx * 256 + (int)rank * 128;
                 }
                 const int a_row = ti.a_row + (int)rank * 128;
-                const int nk = c.K / GEMM_BK;
+                constexpr int KB = F8 ? 2 * GEMM_BK : GEMM_BK;
+                const int nk = c.K / KB;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(empty_bar + stage, phase ^ 1u, abort_flag)) { ok = false; break; }
                     const uint32_t fb = full_leader0 + (uint32_t)stage * 8u;
                     if (leader) mbar_arrive_expect_tx(full_bar + stage, 2u * (PAIR_A_BYTES + PAIR_B_BYTES));
-                    tma_load_2d_pair(sA + stage * PAIR_A_BYTES, mA, fb, kb * GEMM_BK, a_row, pol_a);
-                    tma_load_2d_pair(sB + stage * PAIR_B_BYTES, mB, fb, kb * GEMM_BK, b_row, pol_b);
+                    tma_load_2d_pair(sA + stage * PAIR_A_BYTES, mA, fb, kb * KB, a_row, pol_a);
+                    tma_load_2d_pair(sB + stage * PAIR_B_BYTES, mB, fb, kb * KB, b_row, pol_b);
                     ++issued;
                     if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -184,7 +187,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer (leader only)
         if (lane == 0 && leader) {
-            const uint32_t idesc = idesc_bf16_f32(PAIR_BM, 256);
+            const uint32_t idesc = F8 ? idesc_e4m3_f32(PAIR_BM, 256) : idesc_bf16_f32(PAIR_BM, 256);
             int stage = 0;
             uint32_t phase = 0;
             int acc = 0;
@@ -193,7 +196,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
             for (int t = pair_id; t < total && ok; t += npairs) {
                 const PairTile ti = pair_decode_tile(p, t, routed_tiles);
                 const GemmClass& c = p.cls[ti.cls];
-                const int nk = c.K / GEMM_BK;
+                const int nk = c.K / (F8 ? 2 * GEMM_BK : GEMM_BK);
                 if (!mbar_wait(tempty_bar + acc, acc_phase ^ 1u, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * GEMM_ACC_COLS);
@@ -203,8 +206,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                     const uint64_t ad = smem_desc_k_sw128(sA + stage * PAIR_A_BYTES);
                     const uint64_t bd = smem_desc_k_sw128(sB + stage * PAIR_B_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < GEMM_BK / 16; ++kk)
-                        umma_bf16_pair(d_tmem, ad + 2ull * kk, bd + 2ull * kk, idesc, (kb | kk) != 0);
+                    for (int kk = 0; kk < 4; ++kk) {   // 32 bytes of K per instruction
+                        if (F8) umma_e4m3_pair(d_tmem, ad + 2ull * kk, bd + 2ull * kk, idesc, (kb | kk) != 0);
+                        else umma_bf16_pair(d_tmem, ad + 2ull * kk, bd + 2ull * kk, idesc, (kb | kk) != 0);
+                    }
                     umma_commit_pair(empty_bar + stage, 0x3);
                     any = true;
                     if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
@@ -237,6 +242,14 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
             const long long orow = c.out_row0 + ti.a_row + row_in_tile;
             const bool row_ok = row_in_tile < ti.rows && orow >= 0 && orow < c.out_rows;
             __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(c.out) + orow * c.ldo;
+            float sa = 1.f;                        // fp8: activation row scale, weight column scales
+            const float *sb = nullptr, *sb2 = nullptr;
+            if (F8) {
+                if (row_ok) sa = __ldg(c.a_scale + ti.a_row + row_in_tile);
+                const long long wg = ti.cls ? 0 : gemm_weight_group(p, ti.group);
+                sb = c.b_scale + wg * c.b_scale_stride;
+                if (EPI == EPI_SWIGLU) sb2 = c.b_scale2 + wg * c.b_scale_stride;
+            }
             if (EPI == EPI_SWIGLU) {
 #pragma unroll 1
                 for (int ch = 0; ch < 4; ++ch) {
@@ -247,6 +260,14 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                     tmem_ld_wait();
                     const int col0 = ti.n_idx * 128 + ch * 32;
                     if (row_ok && col0 < c.n_out) {
+                        if (F8) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) {
+                                const bool in = col0 + i < c.n_out;
+                                g[i] = __float_as_uint(__uint_as_float(g[i]) * sa * (in ? __ldg(sb + col0 + i) : 0.f));
+                                u[i] = __float_as_uint(__uint_as_float(u[i]) * sa * (in ? __ldg(sb2 + col0 + i) : 0.f));
+                            }
+                        }
                         uint32_t packed[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
@@ -271,6 +292,12 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                     tmem_ld_wait();
                     const int col0 = ti.n_idx * 256 + ch * 32;
                     if (row_ok && col0 < c.n_out) {
+                        if (F8) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                v[i] = __float_as_uint(__uint_as_float(v[i]) * sa *
+                                                       (col0 + i < c.n_out ? __ldg(sb + col0 + i) : 0.f));
+                        }
                         uint32_t packed[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i)

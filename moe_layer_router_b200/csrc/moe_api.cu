@@ -159,7 +159,7 @@ size_t router_partial_bytes(int T, int d, int E) {
     return ks > 1 ? (size_t)ks * T * E * 4 : 0;
 }
 
-template <int EPI>
+template <int EPI, bool F8 = false>
 int launch_gemm_pair(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& b0b,
                      const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& b1b, const GemmParams& p,
                      long long tiles_upper, cudaStream_t s) {
@@ -169,7 +169,7 @@ int launch_gemm_pair(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b
         int dev = 0;
         cudaGetDevice(&dev);
         if (!attr_set[dev][EPI]) {
-            if (cudaFuncSetAttribute(grouped_gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            if (cudaFuncSetAttribute(grouped_gemm_pair_kernel<EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      PAIR_SMEM_BYTES) != cudaSuccess)
                 return MOE_ERR_CUDA;
             attr_set[dev][EPI] = true;
@@ -178,7 +178,7 @@ int launch_gemm_pair(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b
     if (tiles_upper <= 0) return MOE_OK;
     const long long pairs = di->sms / 2;
     const int grid = 2 * (int)(tiles_upper < pairs ? tiles_upper : pairs);
-    grouped_gemm_pair_kernel<EPI><<<grid, GEMM_THREADS, PAIR_SMEM_BYTES, s>>>(a0, b0, b0b, a1, b1, b1b, p);
+    grouped_gemm_pair_kernel<EPI, F8><<<grid, GEMM_THREADS, PAIR_SMEM_BYTES, s>>>(a0, b0, b0b, a1, b1, b1b, p);
     return launch_status();
 }
 
@@ -634,9 +634,12 @@ int run_expert_ffn_a8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, cons
         p.stages = GEMM_STAGES;
         p.group_map = a.group_map;
         long long tiles = 0;
-        if (routed) tiles += ((long long)(a.max_rows + GEMM_BM - 1) / GEMM_BM + a.E) * c0.ntiles;
-        if (shared) tiles += (long long)((a.T + GEMM_BM - 1) / GEMM_BM) * c1.ntiles;
-        if ((rc = launch_gemm<EPI_SWIGLU, true>(di, A0, B0, B0b, A1, B1, B1b, p, tiles, s)) != MOE_OK) return rc;
+        const int bm = a.pair ? PAIR_BM : GEMM_BM;
+        if (routed) tiles += ((long long)(a.max_rows + bm - 1) / bm + a.E) * c0.ntiles;
+        if (shared) tiles += (long long)((a.T + bm - 1) / bm) * c1.ntiles;
+        rc = a.pair ? launch_gemm_pair<EPI_SWIGLU, true>(di, A0, B0, B0b, A1, B1, B1b, p, tiles, s)
+                    : launch_gemm<EPI_SWIGLU, true>(di, A0, B0, B0b, A1, B1, B1b, p, tiles, s);
+        if (rc != MOE_OK) return rc;
     }
     if (ev_down && cudaEventRecord(ev_down, s) != cudaSuccess) return MOE_ERR_CUDA;
     if (routed && (rc = run_quant_rows(a.h, nullptr, n_routed, a.max_rows, a.f, b.hq, b.sh, s)) != MOE_OK) return rc;
@@ -647,11 +650,11 @@ int run_expert_ffn_a8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, cons
         CUtensorMap A0, B0, A1, B1;
         if (routed) {
             if ((rc = make_map_e4m3(&A0, b.hq, a.f, a.max_rows, GEMM_BM)) != MOE_OK) return rc;
-            if ((rc = make_map_e4m3(&B0, q.W2q, a.f, weight_groups(a) * a.d, 256)) != MOE_OK) return rc;
+            if ((rc = make_map_e4m3(&B0, q.W2q, a.f, weight_groups(a) * a.d, a.pair ? 128 : 256)) != MOE_OK) return rc;
         }
         if (shared) {
             if ((rc = make_map_e4m3(&A1, b.hqs, a.f_shared, a.T, GEMM_BM)) != MOE_OK) return rc;
-            if ((rc = make_map_e4m3(&B1, q.W2sq, a.f_shared, a.d, 256)) != MOE_OK) return rc;
+            if ((rc = make_map_e4m3(&B1, q.W2sq, a.f_shared, a.d, a.pair ? 128 : 256)) != MOE_OK) return rc;
         }
         if (!routed) { A0 = A1; B0 = B1; }
         if (!shared) { A1 = A0; B1 = B0; }
@@ -674,9 +677,12 @@ int run_expert_ffn_a8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, cons
         p.stages = GEMM_STAGES;
         p.group_map = a.group_map;
         long long tiles = 0;
-        if (routed) tiles += ((long long)(a.max_rows + GEMM_BM - 1) / GEMM_BM + a.E) * c0.ntiles;
-        if (shared) tiles += (long long)((a.T + GEMM_BM - 1) / GEMM_BM) * c1.ntiles;
-        if ((rc = launch_gemm<EPI_STORE, true>(di, A0, B0, B0, A1, B1, B1, p, tiles, s)) != MOE_OK) return rc;
+        const int bm = a.pair ? PAIR_BM : GEMM_BM;
+        if (routed) tiles += ((long long)(a.max_rows + bm - 1) / bm + a.E) * c0.ntiles;
+        if (shared) tiles += (long long)((a.T + bm - 1) / bm) * c1.ntiles;
+        rc = a.pair ? launch_gemm_pair<EPI_STORE, true>(di, A0, B0, B0, A1, B1, B1, p, tiles, s)
+                    : launch_gemm<EPI_STORE, true>(di, A0, B0, B0, A1, B1, B1, p, tiles, s);
+        if (rc != MOE_OK) return rc;
     }
     return MOE_OK;
 }
@@ -722,13 +728,14 @@ int moe_workspace_bytes(int T, int d, int E, int k, int f, int f_shared, size_t*
     return MOE_OK;
 }
 
-int moe_workspace_layout(int T, int d, int E, int k, int f, int f_shared, size_t off[12]) {
+int moe_workspace_layout(int T, int d, int E, int k, int f, int f_shared, size_t off[13]) {
     MOE_REQUIRE(off != nullptr, MOE_ERR_INVALID_ARG);
     int rc = check_shape(T, d, E, k, f);
     if (rc != MOE_OK) return rc;
     MOE_REQUIRE(f_shared >= 0 && f_shared % 64 == 0, MOE_ERR_SHAPE);
     LayerLayout L = layer_layout(T, d, E, k, f, f_shared);
     for (int i = 0; i < 12; ++i) off[i] = L.off[i];
+    off[12] = L.h_shared;
     return MOE_OK;
 }
 
@@ -920,7 +927,8 @@ int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float*
                     : run_topk(logits, 1, nullptr, bias, T, E, k, idx, w, s);
         if (rc != MOE_OK) return rc;
     }
-    const bool pair = !w8 && use_pair_tiles((long long)T * k, E);    // fp8 weights: 1-SM tiles
+    // weight-only fp8: 1-SM tiles (its own kernel); bf16 and fp8 x fp8: 2-SM tiles for big experts
+    const bool pair = (!w8 || act8) && use_pair_tiles((long long)T * k, E);
     if (phases & LAYER_COUNT) {
         if ((rc = run_permute(di, x, idx, T, d, E, k, -1, counts_raw, counts, offsets, dest, src, x_perm, blk_cnt,
                               rank_local, mprefix, s, GEMM_BM, nullptr, true)) != MOE_OK)

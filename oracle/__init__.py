@@ -66,6 +66,8 @@ def lib():
         L.oracle_e4m3_encode.restype = ctypes.c_uint8
         L.oracle_quantize_rows_e4m3.argtypes = [vp, i32, i32, vp, vp]
         L.oracle_expert_ffn_w8a8.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp]
+        L.oracle_expert_gate_up_w8a8.argtypes = [vp, i32, vp, vp, vp, vp, i32, i32, vp]
+        L.oracle_expert_down_w8a8.argtypes = [vp, i32, vp, vp, i32, i32, vp]
         L.oracle_layer_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
                                            i32, i32, i32, i32, i32, i64,
                                            vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
@@ -199,6 +201,27 @@ def expert_ffn_w8a8(x, W1q, s1, W3q, s3, W2q, s2):
     y = np.empty((rows, d), np.uint16)
     lib().oracle_expert_ffn_w8a8(_p(x), rows, _p(W1q), _p(s1), _p(W3q), _p(s3), _p(W2q), _p(s2), d, f, _p(h), _p(y))
     return h, y
+
+
+def expert_gate_up_w8a8(x, W1q, s1, W3q, s3):
+    """First GEMM of the fp8 x fp8 expert: -> h bf16 [rows, f]."""
+    x = _c(x, np.uint16); W1q = _c(W1q, np.uint8); W3q = _c(W3q, np.uint8)
+    s1 = _c(s1, np.float32); s3 = _c(s3, np.float32)
+    rows, d = x.shape
+    f = W1q.shape[0]
+    h = np.empty((rows, f), np.uint16)
+    lib().oracle_expert_gate_up_w8a8(_p(x), rows, _p(W1q), _p(s1), _p(W3q), _p(s3), d, f, _p(h))
+    return h
+
+
+def expert_down_w8a8(h, W2q, s2):
+    """Second GEMM of the fp8 x fp8 expert on given bf16 h rows: -> y bf16 [rows, d]."""
+    h = _c(h, np.uint16); W2q = _c(W2q, np.uint8); s2 = _c(s2, np.float32)
+    rows, f = h.shape
+    d = W2q.shape[0]
+    y = np.empty((rows, d), np.uint16)
+    lib().oracle_expert_down_w8a8(_p(h), rows, _p(W2q), _p(s2), d, f, _p(y))
+    return y
 
 
 def combine(y_perm: np.ndarray, dest: np.ndarray, w: np.ndarray, y_shared: Optional[np.ndarray] = None) -> np.ndarray:

@@ -337,15 +337,12 @@ void oracle_quantize_rows_e4m3(const uint16_t* x, int rows, int K, uint8_t* q, f
     }
 }
 
-/* One expert with fp8 weights (row scales s1, s3, s2) and fp8 activations: x rows quantised,
- * G = s_x s1 (xq . W1q), U likewise, h = bf16(silu(G) U); h rows quantised, y = bf16(s_h s2 (hq . W2q)). */
-void oracle_expert_ffn_w8a8(const uint16_t* x, int rows, const uint8_t* W1q, const float* s1, const uint8_t* W3q,
-                            const float* s3, const uint8_t* W2q, const float* s2, int d, int f, uint16_t* h,
-                            uint16_t* y) {
+/* First GEMM of an expert with fp8 weights and fp8 activations: x rows quantised,
+ * G = s_x s1 (xq . W1q), U likewise, h = bf16(silu(G) U). */
+void oracle_expert_gate_up_w8a8(const uint16_t* x, int rows, const uint8_t* W1q, const float* s1,
+                                const uint8_t* W3q, const float* s3, int d, int f, uint16_t* h) {
     uint8_t* xq = (uint8_t*)malloc((size_t)(rows > 0 ? rows : 1) * d);
     float* sx = (float*)malloc(sizeof(float) * (size_t)(rows > 0 ? rows : 1));
-    uint8_t* hq = (uint8_t*)malloc((size_t)(rows > 0 ? rows : 1) * f);
-    float* sh = (float*)malloc(sizeof(float) * (size_t)(rows > 0 ? rows : 1));
     oracle_quantize_rows_e4m3(x, rows, d, xq, sx);
 #pragma omp parallel for schedule(dynamic, 1)
     for (int r = 0; r < rows; ++r) {
@@ -363,6 +360,14 @@ void oracle_expert_ffn_w8a8(const uint16_t* x, int rows, const uint8_t* W1q, con
             hr[n] = bf16_round(g / (1.0 + exp(-g)) * u);
         }
     }
+    free(xq); free(sx);
+}
+
+/* Second GEMM: h rows quantised, y = bf16(s_h s2 (hq . W2q)). */
+void oracle_expert_down_w8a8(const uint16_t* h, int rows, const uint8_t* W2q, const float* s2, int d, int f,
+                             uint16_t* y) {
+    uint8_t* hq = (uint8_t*)malloc((size_t)(rows > 0 ? rows : 1) * f);
+    float* sh = (float*)malloc(sizeof(float) * (size_t)(rows > 0 ? rows : 1));
     oracle_quantize_rows_e4m3(h, rows, f, hq, sh);
 #pragma omp parallel for schedule(dynamic, 1)
     for (int r = 0; r < rows; ++r) {
@@ -373,7 +378,15 @@ void oracle_expert_ffn_w8a8(const uint16_t* x, int rows, const uint8_t* W1q, con
             y[(size_t)r * d + m] = bf16_round(acc * (double)sh[r] * (double)s2[m]);
         }
     }
-    free(xq); free(sx); free(hq); free(sh);
+    free(hq); free(sh);
+}
+
+/* One expert with fp8 weights (row scales s1, s3, s2) and fp8 activations: the two GEMMs above. */
+void oracle_expert_ffn_w8a8(const uint16_t* x, int rows, const uint8_t* W1q, const float* s1, const uint8_t* W3q,
+                            const float* s3, const uint8_t* W2q, const float* s2, int d, int f, uint16_t* h,
+                            uint16_t* y) {
+    oracle_expert_gate_up_w8a8(x, rows, W1q, s1, W3q, s3, d, f, h);
+    oracle_expert_down_w8a8(h, rows, W2q, s2, d, f, y);
 }
 
 /* ---- combine ------------------------------------------------------------------------ */

@@ -62,12 +62,16 @@ def test_workspace_sizes_and_layout(lib):
     T, d, E, k, f = 4096, 4096, 8, 2, 14336
     big = T * k * d * 2 * 2 + T * k * f * 2
     assert big < sz.value < big * 1.05
-    off = (ctypes.c_size_t * 12)()
-    lib.moe_workspace_layout.argtypes = [ctypes.c_int] * 6 + [ctypes.c_size_t * 12]
+    off = (ctypes.c_size_t * 13)()
+    lib.moe_workspace_layout.argtypes = [ctypes.c_int] * 6 + [ctypes.c_size_t * 13]
     assert lib.moe_workspace_layout(T, d, E, k, f, 0, off) == 0
     offs = list(off)
     assert all(o % 256 == 0 for o in offs)
     assert offs[:11] == sorted(offs[:11]) and offs[10] + T * k * d * 2 <= sz.value
+    # with a shared expert: y_shared [T, d] then h_shared [T, f_s] follow y_perm
+    assert lib.moe_workspace_layout(T, d, E, k, f, 2048, off) == 0
+    offs = list(off)
+    assert offs[10] < offs[11] < offs[12] and offs[11] + T * d * 2 <= offs[12]
     # shape checks: d % 64, k <= 32, k <= E, E <= 1024
     for args in [(128, 100, 8, 2, 512), (128, 256, 8, 33, 512), (128, 256, 4, 8, 512), (128, 256, 2000, 2, 512),
                  (0, 256, 8, 2, 512), (128, 256, 8, 2, 500)]:

@@ -435,13 +435,16 @@ def test_layer_fp8_weights(moe, wl):
     assert np.mean(ulp_bf16(got, ref) <= 1) > 0.98
 
 
-def _a8_reference(wl, x, logits, inp, k, C):
-    """Oracle layer with fp8 weights and fp8 activations: route the GPU's logits, dispatch,
-    fp8 x fp8 experts, combine."""
+def _a8_reference(wl, x, logits, inp, k, C, g_h, g_hs):
+    """Oracle layer with fp8 weights and fp8 activations on the GPU's logits.  The first expert
+    GEMM runs on the oracle's own quantised x; the second on the GPU's h (g_h, g_hs), so that
+    both sides quantise the same h rows (h itself is checked against the oracle's h).
+    -> idx, dispatch, permuted x, oracle h, oracle h of the shared expert, output."""
     E, d, f = wl.E, wl.d, wl.f
     idx, w = oracle.route(logits, k, inp.bias())
     r = oracle.dispatch(idx, E, C)
     xp = oracle.gather(x, r["dest"], r["N"])
+    h_ref = np.zeros((max(r["N"], 1), f), np.uint16)
     y_perm = np.zeros((max(r["N"], 1), d), np.uint16)
     for e in range(E):
         a, b = r["offsets"][e], r["offsets"][e + 1]
@@ -450,20 +453,30 @@ def _a8_reference(wl, x, logits, inp, k, C):
         q1, s1 = synth.quantize_e4m3_rows(inp.expert_rows("w1", e, 1), d)
         q3, s3 = synth.quantize_e4m3_rows(inp.expert_rows("w3", e, 1), d)
         q2, s2 = synth.quantize_e4m3_rows(inp.expert_rows("w2", e, 1), f)
-        _, y_perm[a:b] = oracle.expert_ffn_w8a8(xp[a:b], q1, s1, q3, s3, q2, s2)
-    ysh = None
+        h_ref[a:b] = oracle.expert_gate_up_w8a8(xp[a:b], q1, s1, q3, s3)
+        y_perm[a:b] = oracle.expert_down_w8a8(g_h[a:b], q2, s2)
+    hs_ref, ysh = None, None
     if wl.has_shared:
         qs = {n: synth.quantize_e4m3_rows(inp.shared(n), inp.shared(n).shape[1]) for n in ("w1s", "w3s", "w2s")}
-        _, ysh = oracle.expert_ffn_w8a8(x, qs["w1s"][0], qs["w1s"][1], qs["w3s"][0], qs["w3s"][1], qs["w2s"][0],
-                                        qs["w2s"][1])
-    return idx, r, xp, oracle.combine(y_perm, r["dest"], w, ysh)
+        hs_ref = oracle.expert_gate_up_w8a8(x, qs["w1s"][0], qs["w1s"][1], qs["w3s"][0], qs["w3s"][1])
+        ysh = oracle.expert_down_w8a8(g_hs, qs["w2s"][0], qs["w2s"][1])
+    return idx, r, xp, h_ref[:r["N"]], hs_ref, oracle.combine(y_perm, r["dest"], w, ysh)
+
+
+def _assert_h_close(g, r, what):
+    """h bar: |d| <= 1e-3 + 8e-3 |ref| (one bf16 ulp plus a floor for cancellation in g, u)."""
+    g64, r64 = bits_to_f64(g), bits_to_f64(r)
+    bad = np.abs(g64 - r64) > 1e-3 + 8e-3 * np.abs(r64)
+    assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} outside 1e-3 + 8e-3|ref|"
 
 
 @pytest.mark.parametrize("wl", [synth.Workload("a8", 300, 256, 16, 4, 384, f_shared=256, bias_range=0.1,
                                                cap_mode=synth.CAP_PER_TOKEN, capacity_factor=1.5),
                                 synth.Workload("a8dec", 40, 512, 32, 8, 256, f_shared=128, bias_range=0.1),
-                                synth.Workload("a8mix", 512, 256, 16, 2, 128, zipf_s=1.2)],
-                         ids=["shared-cap-bias", "decode-shaped", "skewed-mixed-tiles"])
+                                synth.Workload("a8mix", 512, 256, 16, 2, 128, zipf_s=1.2),
+                                synth.Workload("a8pair", 1024, 256, 4, 2, 256, f_shared=128,
+                                               cap_mode=synth.CAP_PER_ASSIGNMENT, capacity_factor=1.1)],
+                         ids=["shared-cap-bias", "decode-shaped", "skewed-mixed-tiles", "pair-tiles-shared-cap"])
 def test_layer_fp8_weights_and_activations(moe, wl):
     T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
     inp = synth.Inputs(wl)
@@ -480,8 +493,13 @@ def test_layer_fp8_weights_and_activations(moe, wl):
     L = moe.moe_workspace_layout(T, d, E, k, f, fs)
     logits = moe.workspace_view(ws, L, "logits", (T, E), torch.float32).cpu().numpy()
     C = oracle.capacity(T, E, k, wl.capacity_factor, wl.cap_mode)
-    idx, r, xp, ref = _a8_reference(wl, x, logits, inp, k, C)
+    g_h = bf16_bits(moe.workspace_view(ws, L, "h", (T * k, f), torch.bfloat16))
+    g_hs = bf16_bits(moe.workspace_view(ws, L, "h_shared", (T, fs), torch.bfloat16)) if fs else None
+    idx, r, xp, h_ref, hs_ref, ref = _a8_reference(wl, x, logits, inp, k, C, g_h, g_hs)
     assert np.array_equal(moe.workspace_view(ws, L, "idx", (T, k), torch.int32).cpu().numpy(), idx)
+    _assert_h_close(g_h[:r["N"]], h_ref, "fp8 x fp8 h")
+    if fs:
+        _assert_h_close(g_hs, hs_ref, "fp8 x fp8 shared h")
     xq_ref, sx_ref = oracle.quantize_rows_e4m3(xp)
     got = bf16_bits(out)
     assert_layer_close(got, ref, "fp8 x fp8 layer")

@@ -180,3 +180,71 @@ def test_full_size_decode_fp8_weights(moe):
     assert_layer_close(got, ref_out, "dsv3 fp8 sampled outputs")
     g64, r64 = bits_to_f64(got), bits_to_f64(ref_out)
     assert np.sqrt(np.mean((g64 - r64) ** 2) / np.mean(r64 ** 2)) < 5e-3
+
+
+@pytest.mark.parametrize("name", ["dsv3", "mixtral"])
+def test_full_size_fp8_weights_and_activations(moe, name):
+    """bench.py --weights fp8a8 at full size (decode on 1-SM tiles, prefill on 2-SM tiles): routing
+    bit-exact for every token, sampled outputs against the oracle's fp8 x fp8 experts on weights
+    regenerated and quantised on the host."""
+    wl = synth.WORKLOADS[name]
+    T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
+    W = synth.device_tensors(wl, "cuda", names=["x", "wg", "bias"])
+    Q = synth.device_tensors_q8(wl, "cuda")
+    ws = torch.empty(moe.moe_workspace_bytes_a8(T, d, E, k, f, fs), dtype=torch.uint8, device="cuda")
+    out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_layer_forward_w8a8(W["x"], W["wg"], W.get("bias"), Q["w1q"], Q["s1"], Q["w3q"], Q["s3"], Q["w2q"],
+                               Q["s2"], Q.get("w1sq"), Q.get("s1s"), Q.get("w3sq"), Q.get("s3s"), Q.get("w2sq"),
+                               Q.get("s2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, out, ws)
+    assert moe.moe_get_error() == 0
+    del Q
+    L = moe.moe_workspace_layout(T, d, E, k, f, fs)
+    v = lambda n, s, dt: moe.workspace_view(ws, L, n, s, dt).cpu()
+    g_logits = v("logits", (T, E), torch.float32).numpy()
+    g_idx = v("idx", (T, k), torch.int32).numpy()
+    inp = synth.Inputs(wl)
+    idx_o, w_o = oracle.route(g_logits, k, inp.bias())
+    assert np.array_equal(g_idx, idx_o)
+    g_dest = v("dest", (T, k), torch.int32).numpy()
+    rng = np.random.default_rng(13)
+    toks = sorted(set([0, T - 1] + list(rng.choice(T, 4, replace=False))))
+    xs = np.stack([inp.x_rows(t, 1) for t in toks])
+    h_all = moe.workspace_view(ws, L, "h", (T * k, f), torch.bfloat16)
+    # the first GEMM against the oracle; the second on the GPU's h, so both sides quantise the
+    # same h rows
+    by_expert = {}
+    for i, t in enumerate(toks):
+        for j in range(k):
+            if g_dest[t, j] >= 0:
+                by_expert.setdefault(int(g_idx[t, j]), []).append((i, j, int(g_dest[t, j])))
+    y = {}
+    for e, items in by_expert.items():
+        q1, s1 = synth.quantize_e4m3_rows(inp.expert_rows("w1", e, 1), d)
+        q3, s3 = synth.quantize_e4m3_rows(inp.expert_rows("w3", e, 1), d)
+        q2, s2 = synth.quantize_e4m3_rows(inp.expert_rows("w2", e, 1), f)
+        h_ref = oracle.expert_gate_up_w8a8(np.stack([xs[i] for i, _, _ in items]), q1, s1, q3, s3)
+        g_h = np.stack([bf16_bits(h_all[r]) for _, _, r in items])
+        g64, r64 = bits_to_f64(g_h), bits_to_f64(h_ref)
+        assert not (np.abs(g64 - r64) > 1e-3 + 8e-3 * np.abs(r64)).any(), f"h of expert {e}"
+        ye = oracle.expert_down_w8a8(g_h, q2, s2)
+        for (i, j, _), row in zip(items, ye):
+            y[(i, j)] = row
+    ysh = None
+    if fs:
+        qs = {n: synth.quantize_e4m3_rows(inp.shared(n), inp.shared(n).shape[1]) for n in ("w1s", "w3s", "w2s")}
+        g_hs = bf16_bits(moe.workspace_view(ws, L, "h_shared", (T, fs), torch.bfloat16)[toks])
+        hs_ref = oracle.expert_gate_up_w8a8(xs, qs["w1s"][0], qs["w1s"][1], qs["w3s"][0], qs["w3s"][1])
+        g64, r64 = bits_to_f64(g_hs), bits_to_f64(hs_ref)
+        assert not (np.abs(g64 - r64) > 1e-3 + 8e-3 * np.abs(r64)).any(), "shared h"
+        ysh = oracle.expert_down_w8a8(g_hs, qs["w2s"][0], qs["w2s"][1])
+    S = len(toks)
+    mini_y = np.zeros((S * k, d), np.uint16)
+    mini_dest = np.full((S, k), -1, np.int32)
+    for (i, j), row in y.items():
+        mini_y[i * k + j] = row
+        mini_dest[i, j] = i * k + j
+    ref_out = oracle.combine(mini_y, mini_dest, w_o[toks], ysh)
+    got = bf16_bits(out[toks])
+    assert_layer_close(got, ref_out, f"{name} fp8 x fp8 sampled outputs")
+    g64, r64 = bits_to_f64(got), bits_to_f64(ref_out)
+    assert np.sqrt(np.mean((g64 - r64) ** 2) / np.mean(r64 ** 2)) < 5e-3
