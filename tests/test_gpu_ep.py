@@ -84,3 +84,39 @@ def test_emulated_expert_parallel_layer(moe, case, exchange):
     if same_tiles:   # same tile kind in both paths: each row's arithmetic is the same
         for r in range(R):
             assert torch.equal(outs[r].view(torch.int16), outs_dp[r].view(torch.int16)), f"rank {r}"
+
+
+def test_nccl_driver_single_rank_matches_layer(moe):
+    """ep_layer_forward_dist on one NCCL rank (the all-gather and both all_to_all_single calls run,
+    rows arrive source-major, the GEMMs run the source-major segments): bit-identical to the
+    single-GPU layer."""
+    import os
+    import socket
+    import torch.distributed as dist
+    from moe_layer_router_b200.ep import ep_layer_forward_dist
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        wl = synth.Workload("ep_nccl", 64, 256, 8, 2, 128, f_shared=128, cap_mode=synth.CAP_PER_TOKEN,
+                            capacity_factor=1.0, seed=5)
+        inp = synth.Inputs(wl)
+        T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
+        dv = to_dev_bf16
+        x, wg = dv(inp.x()), dv(inp.wg())
+        W1, W3, W2 = dv(inp.w1()), dv(inp.w3()), dv(inp.w2())
+        sh = [dv(inp.shared(n)) for n in ("w1s", "w3s", "w2s")]
+        out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+        ep_layer_forward_dist(x, wg, None, W1, W3, W2, *sh, fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, out)
+        ref = torch.empty_like(out)
+        ws = torch.empty(moe.moe_workspace_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device="cuda")
+        moe.moe_layer_forward(x, wg, None, W1, W3, W2, *sh, fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode,
+                              ref, ws)
+        torch.cuda.synchronize()
+        assert moe.moe_get_error() == 0
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    finally:
+        dist.destroy_process_group()

@@ -535,3 +535,30 @@ def test_quantised_rows_bit_exact(moe):
     xq_ref, sx_ref = oracle.quantize_rows_e4m3(xp)
     assert np.array_equal(sx.view(np.uint32), sx_ref.view(np.uint32))
     assert np.array_equal(xq, xq_ref)
+
+
+@pytest.mark.parametrize("wl", [synth.Workload("a8c0", 64, 256, 16, 4, 128, f_shared=128, cap_mode=synth.CAP_PER_TOKEN,
+                                               capacity_factor=0.2),
+                                synth.Workload("a8t1", 1, 256, 8, 2, 128)],
+                         ids=["capacity-zero-shared-only", "one-token"])
+def test_fp8_activation_layer_edge_cases(moe, wl):
+    T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
+    inp = synth.Inputs(wl)
+    x = inp.x()
+    Q = synth.device_tensors_q8(wl, "cuda")
+    ws = torch.empty(moe.moe_workspace_bytes_a8(T, d, E, k, f, fs), dtype=torch.uint8, device="cuda")
+    out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    moe.moe_layer_forward_w8a8(to_dev_bf16(x), to_dev_bf16(inp.wg()), None, Q["w1q"], Q["s1"], Q["w3q"], Q["s3"],
+                               Q["w2q"], Q["s2"], Q.get("w1sq"), Q.get("s1s"), Q.get("w3sq"), Q.get("s3s"),
+                               Q.get("w2sq"), Q.get("s2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode,
+                               out, ws)
+    assert moe.moe_get_error() == 0
+    L = moe.moe_workspace_layout(T, d, E, k, f, fs)
+    logits = moe.workspace_view(ws, L, "logits", (T, E), torch.float32).cpu().numpy()
+    C = oracle.capacity(T, E, k, wl.capacity_factor, wl.cap_mode)
+    g_h = bf16_bits(moe.workspace_view(ws, L, "h", (T * k, f), torch.bfloat16))
+    g_hs = bf16_bits(moe.workspace_view(ws, L, "h_shared", (T, fs), torch.bfloat16)) if fs else None
+    idx, r, xp, h_ref, hs_ref, ref = _a8_reference(wl, x, logits, inp, k, C, g_h, g_hs)
+    if wl.name == "a8c0":
+        assert C == 0 and r["N"] == 0          # every routed row dropped: the shared expert alone
+    assert_layer_close(bf16_bits(out), ref, "fp8 x fp8 edge case")
