@@ -35,6 +35,14 @@ METRIC = "MoE-layer tokens/s on 1 B200; % of BF16 tensor or HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS_PER_STEP = 9   # router GEMM, top-k, count, scan, scatter, gather, GEMM1, GEMM2, combine
 
+
+def launches_per_step(a8: bool, shared: bool) -> int:
+    """Kernels one layer call launches.  fp8 activations: no gather (the quantiser reads x through
+    src_token), one quantiser before each grouped GEMM, two more for the shared expert's rows."""
+    if not a8:
+        return KERNELS_PER_STEP
+    return KERNELS_PER_STEP - 1 + 2 + (2 if shared else 0)
+
 DESCR = {
     "tiny": "tiny MoE layer T=128 d=256 E=8 top-2 f=512",
     "mixtral": "Mixtral-like prefill T=4096 d=4096 E=8 top-2 SwiGLU f=14336",
@@ -43,6 +51,7 @@ DESCR = {
     "skew": "skewed routing T=32768 d=4096 E=64 top-2 f=2048 Zipf(1.2), capacity int(T*k/E*1.25)",
     "mixtral2e": "profiling case: Mixtral-like layer cut to T=2048, E=2 (same tile shapes)",
     "dsv3_32e": "profiling case: DeepSeek-V3-like decode cut to T=32, E=32 (same tile shapes)",
+    "qwen3_16e": "profiling case: Qwen3-like prefill cut to T=2048, E=16 (same tile shapes)",
 }
 
 
@@ -548,7 +557,8 @@ def main():
         raise RuntimeError(f"device error after warm-up: {moe.strerror(rc)}")
 
     K = args.steps
-    evs = [{n: torch.cuda.Event(enable_timing=True) for n in moe.STAGES} for _ in range(K)]
+    ev_names = moe.STAGES + (["gemm1", "gemm2"] if a8 else [])
+    evs = [{n: torch.cuda.Event(enable_timing=True) for n in ev_names} for _ in range(K)]
     for e in evs:               # torch creates the CUDA event on its first record
         for ev in e.values():
             ev.record()
@@ -565,6 +575,13 @@ def main():
     stage_ms = {}
     for a, b in zip(moe.STAGES[:-1], moe.STAGES[1:]):
         stage_ms[a] = float(np.mean([e[a].elapsed_time(e[b]) for e in evs]))
+    # the grouped GEMM kernels alone (fp8 activations: the stages also hold the row quantisers)
+    gemm_ms = {"gate_up": stage_ms["gate_up"], "down": stage_ms["down"]}
+    if a8:
+        gemm_ms = {"gate_up": float(np.mean([e["gemm1"].elapsed_time(e["down"]) for e in evs])),
+                   "down": float(np.mean([e["gemm2"].elapsed_time(e["combine"]) for e in evs]))}
+        stage_ms["quant_x"] = float(np.mean([e["gate_up"].elapsed_time(e["gemm1"]) for e in evs]))
+        stage_ms["quant_h"] = float(np.mean([e["down"].elapsed_time(e["gemm2"]) for e in evs]))
     total_ms = dp.max_over_ranks(total_ms, device=dev)
     value = dp.job_throughput(T, world, K, total_ms)
 
@@ -627,7 +644,7 @@ def main():
         return
 
     peaks, peak_src = load_peaks()
-    g1_ms = stage_ms["gate_up"]
+    g1_ms = gemm_ms["gate_up"]
     decode = wl.name.startswith("dsv3")
     if decode:
         alg = gemm1_bytes(wl, N, touched, 1 if fp8 else 2)
@@ -673,7 +690,8 @@ def main():
         "stages_ms": stage_ms,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
                 "d2h_bytes_per_step": T * d * 2},
-        "gpu_launches": KERNELS_PER_STEP * K,
+        "gemm_ms": gemm_ms,
+        "gpu_launches": launches_per_step(a8, wl.has_shared) * K,
         "clocks": clk.summary(),
     }
     if wl.zipf_s > 0:

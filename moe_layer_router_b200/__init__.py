@@ -222,8 +222,10 @@ def moe_layer_forward(x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, f_shared, T, d, E,
 
 
 STAGES = ["route", "topk", "permute", "gate_up", "down", "combine", "end"]   # timeline of one layer call
-_EVENT_FIELDS = STAGES + ["cache"]   # struct order; "cache" marks the expert cache kernels (between
-                                     # "permute" and "gate_up") in moe_layer_forward_cached
+# struct order; "cache" marks the expert cache kernels (between "permute" and "gate_up") in
+# moe_layer_forward_cached; "gemm1" / "gemm2" mark the grouped GEMM kernels themselves in the
+# fp8-activation layer (after the quantisation of their rows, inside "gate_up" / "down")
+_EVENT_FIELDS = STAGES + ["cache", "gemm1", "gemm2"]
 
 
 class moe_stage_events(ctypes.Structure):

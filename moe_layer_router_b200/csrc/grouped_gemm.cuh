@@ -147,6 +147,47 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// SwiGLU of one gate/up accumulator pair: silu(g) u with silu(g) = g / (1 + e^-g).  The fast
+// divide (two ulp) is ample for a value rounded to bf16 next; for g below about -87 the
+// denominator overflows and the result is the correct limit 0.
+__device__ __forceinline__ float swiglu_f32(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+
+// fp8 products: 32 accumulator columns times the A row's scale sa and the columns' weight
+// scales sb[0..32) (16-byte aligned; fp8 outputs come in whole 128-column tiles).
+__device__ __forceinline__ void scale_cols32(uint32_t (&v)[32], float sa, const float* sb) {
+    const float4* s4 = reinterpret_cast<const float4*>(sb);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float4 c = __ldg(s4 + q);
+        v[4 * q + 0] = __float_as_uint(__uint_as_float(v[4 * q + 0]) * sa * c.x);
+        v[4 * q + 1] = __float_as_uint(__uint_as_float(v[4 * q + 1]) * sa * c.y);
+        v[4 * q + 2] = __float_as_uint(__uint_as_float(v[4 * q + 2]) * sa * c.z);
+        v[4 * q + 3] = __float_as_uint(__uint_as_float(v[4 * q + 3]) * sa * c.w);
+    }
+}
+
+// 32 gate and 32 up columns -> 32 bf16 of h, stored at dst (16-byte aligned).
+__device__ __forceinline__ void swiglu_store32(const uint32_t (&g)[32], const uint32_t (&u)[32], __nv_bfloat16* dst) {
+    uint32_t packed[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        packed[i] = pack_bf16x2(swiglu_f32(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                                swiglu_f32(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+}
+
+// 32 accumulator columns -> 32 bf16 at dst (16-byte aligned).
+__device__ __forceinline__ void store32(const uint32_t (&v)[32], __nv_bfloat16* dst) {
+    uint32_t packed[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+}
+
 // F8: A and B are e4m3 (one byte per element, 128 K-elements per stage row of 128 bytes),
 // tcgen05.mma kind::f8f6f4, and the epilogue applies the row and column scales.
 template <int EPI, bool F8 = false>
@@ -327,26 +368,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
                     const int col0 = ti.n_idx * 128 + ch * 32;
                     if (row_ok && col0 < c.n_out) {
                         if (F8) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) {
-                                const bool in = col0 + i < c.n_out;
-                                g[i] = __float_as_uint(__uint_as_float(g[i]) * sa * (in ? __ldg(sb + col0 + i) : 0.f));
-                                u[i] = __float_as_uint(__uint_as_float(u[i]) * sa * (in ? __ldg(sb2 + col0 + i) : 0.f));
-                            }
+                            scale_cols32(g, sa, sb + col0);
+                            scale_cols32(u, sa, sb2 + col0);
                         }
-                        uint32_t packed[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-                            const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-                            const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
-                            const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
-                            packed[i] = pack_bf16x2(h0, h1);
-                        }
-                        uint4* dst = reinterpret_cast<uint4*>(out + col0);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                        swiglu_store32(g, u, out + col0);
                     }
                 }
             } else if (EPI == EPI_STORE) {
@@ -359,20 +384,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
                     tmem_ld_wait();
                     const int col0 = ti.n_idx * c.b_tile_rows + ch * 32;
                     if (row_ok && col0 < c.n_out) {
-                        if (F8) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                v[i] = __float_as_uint(__uint_as_float(v[i]) * sa *
-                                                       (col0 + i < c.n_out ? __ldg(sb + col0 + i) : 0.f));
-                        }
-                        uint32_t packed[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-                        uint4* dst = reinterpret_cast<uint4*>(out + col0);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                        if (F8) scale_cols32(v, sa, sb + col0);
+                        store32(v, out + col0);
                     }
                 }
             } else {  // EPI_LOGITS (K slice ks writes its partial sums split_stride further on)

@@ -10,7 +10,8 @@
 //     issues tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16), which reads both CTAs'
 //     halves and accumulates rows [128 r, 128 r + 128) into CTA r's tensor memory.
 //   - the leader's commits arrive on both CTAs' barriers (empty stage, accumulator full);
-//     every epilogue warp of both CTAs arrives on the leader's accumulator-empty barrier.
+//     every epilogue thread of both CTAs (eight warps each) arrives on the leader's
+//     accumulator-empty barrier.
 // Per SM this halves the B operand traffic of a 1-SM M = 128 tile and leaves room for a
 // 6-stage ring (A 16 KB + B 16 KB per stage per CTA).
 #pragma once
@@ -24,6 +25,11 @@ constexpr int PAIR_STAGES = 6;
 constexpr int PAIR_A_BYTES = 128 * GEMM_BK * 2;   // 16 KB per CTA
 constexpr int PAIR_B_BYTES = 128 * GEMM_BK * 2;   // 16 KB per CTA
 constexpr int PAIR_SMEM_BYTES = PAIR_STAGES * (PAIR_A_BYTES + PAIR_B_BYTES) + 1024 + 256;
+// warp 0 TMA, warp 1 MMA, warps 2..9 epilogue: two warps per TMEM lane quarter, each taking half
+// of the accumulator's columns, so that the epilogue of one tile stays shorter than the next
+// tile's MMAs even at the fp8 rate (twice the bf16 K per cycle).
+constexpr int PAIR_EPI_WARPS = 8;
+constexpr int PAIR_THREADS = 64 + 32 * PAIR_EPI_WARPS;
 
 // Tile walk with 256-row m-tiles (mprefix counts 256-row tiles per group).
 __device__ __forceinline__ int pair_total_tiles(const GemmParams& p, int& routed_tiles) {
@@ -79,7 +85,7 @@ __device__ __forceinline__ PairTile pair_decode_tile(const GemmParams& p, int t,
 // F8: e4m3 operands (128 K-elements per 128-byte stage row, kind::f8f6f4) and the epilogue
 // applies the row and column scales of GemmClass.
 template <int EPI, bool F8 = false>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                          const __grid_constant__ CUtensorMap tmB0b, const __grid_constant__ CUtensorMap tmA1,
                          const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB1b,
@@ -111,7 +117,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull_bar + a, 1);     // one multicast commit
-            mbar_init(tempty_bar + a, 256);  // leader: 128 epilogue threads x 2 CTAs
+            mbar_init(tempty_bar + a, 2 * 32 * PAIR_EPI_WARPS);  // leader: epilogue threads of 2 CTAs
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -226,7 +232,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
         }
     } else {
         // ------------------------------------------------------------------ epilogue (both CTAs)
-        const int sub = warp & 3;
+        const int sub = warp & 3;                 // TMEM lane quarter of this warp
+        const int half = (warp - 2) >> 2;         // which half of the columns it converts
         const int row_in_cta = sub * 32 + lane;
         const uint32_t tempty_leader0 = map_to_cta(tempty_bar, 0);
         int acc = 0;
@@ -252,7 +259,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
             }
             if (EPI == EPI_SWIGLU) {
 #pragma unroll 1
-                for (int ch = 0; ch < 4; ++ch) {
+                for (int ch = 2 * half; ch < 2 * half + 2; ++ch) {
                     uint32_t g[32], u[32];
                     __syncwarp();
                     tmem_ld_32cols(tbase + ch * 32, g);
@@ -261,51 +268,23 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                     const int col0 = ti.n_idx * 128 + ch * 32;
                     if (row_ok && col0 < c.n_out) {
                         if (F8) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) {
-                                const bool in = col0 + i < c.n_out;
-                                g[i] = __float_as_uint(__uint_as_float(g[i]) * sa * (in ? __ldg(sb + col0 + i) : 0.f));
-                                u[i] = __float_as_uint(__uint_as_float(u[i]) * sa * (in ? __ldg(sb2 + col0 + i) : 0.f));
-                            }
+                            scale_cols32(g, sa, sb + col0);
+                            scale_cols32(u, sa, sb2 + col0);
                         }
-                        uint32_t packed[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-                            const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-                            const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
-                            const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
-                            packed[i] = pack_bf16x2(h0, h1);
-                        }
-                        uint4* dst = reinterpret_cast<uint4*>(out + col0);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                        swiglu_store32(g, u, out + col0);
                     }
                 }
             } else {
 #pragma unroll 1
-                for (int ch = 0; ch < 8; ++ch) {
+                for (int ch = 4 * half; ch < 4 * half + 4; ++ch) {
                     uint32_t v[32];
                     __syncwarp();
                     tmem_ld_32cols(tbase + ch * 32, v);
                     tmem_ld_wait();
                     const int col0 = ti.n_idx * 256 + ch * 32;
                     if (row_ok && col0 < c.n_out) {
-                        if (F8) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                v[i] = __float_as_uint(__uint_as_float(v[i]) * sa *
-                                                       (col0 + i < c.n_out ? __ldg(sb + col0 + i) : 0.f));
-                        }
-                        uint32_t packed[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-                        uint4* dst = reinterpret_cast<uint4*>(out + col0);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+                        if (F8) scale_cols32(v, sa, sb + col0);
+                        store32(v, out + col0);
                     }
                 }
             }

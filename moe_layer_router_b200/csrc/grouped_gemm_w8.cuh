@@ -391,7 +391,7 @@ grouped_gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
                         if (n_ok && tok < ti.rows && orow >= 0 && orow < c.out_rows) {
                             const float gg = __uint_as_float(gv[j]) * sg;
                             const float uu = __uint_as_float(uv[j]) * su;
-                            out[orow * c.ldo + n] = __float2bfloat16_rn(gg / (1.0f + __expf(-gg)) * uu);
+                            out[orow * c.ldo + n] = __float2bfloat16_rn(swiglu_f32(gg, uu));
                         }
                     }
                 }

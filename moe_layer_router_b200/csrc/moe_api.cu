@@ -178,7 +178,7 @@ int launch_gemm_pair(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b
     if (tiles_upper <= 0) return MOE_OK;
     const long long pairs = di->sms / 2;
     const int grid = 2 * (int)(tiles_upper < pairs ? tiles_upper : pairs);
-    grouped_gemm_pair_kernel<EPI, F8><<<grid, GEMM_THREADS, PAIR_SMEM_BYTES, s>>>(a0, b0, b0b, a1, b1, b1b, p);
+    grouped_gemm_pair_kernel<EPI, F8><<<grid, PAIR_THREADS, PAIR_SMEM_BYTES, s>>>(a0, b0, b0b, a1, b1, b1b, p);
     return launch_status();
 }
 
@@ -322,7 +322,8 @@ int run_topk(const float* logits, int nsplit, float* logits_out, const float* bi
 int run_permute(DeviceInfo* di, const moe_bf16* x, const int32_t* idx, int T, int d, int E, int k, long long C,
                 int32_t* counts_raw, int32_t* counts, int32_t* offsets, int32_t* dest, int32_t* src_token,
                 moe_bf16* x_perm, int32_t* blk_cnt, int32_t* rank_local, int32_t* mprefix, cudaStream_t s,
-                int tile_rows = GEMM_BM, const int32_t* fill_base = nullptr, bool counts_only = false) {
+                int tile_rows = GEMM_BM, const int32_t* fill_base = nullptr, bool counts_only = false,
+                bool gather = true) {
     const int nb = permute_blocks(T);
     const size_t smem = (size_t)(PERMUTE_WARPS * E + PERMUTE_TOKENS * k) * sizeof(int);
     {
@@ -341,6 +342,7 @@ int run_permute(DeviceInfo* di, const moe_bf16* x, const int32_t* idx, int T, in
     if (counts_only) return launch_status();
     permute_scatter_kernel<<<nb, PERMUTE_TOKENS, 0, s>>>(idx, rank_local, blk_cnt, offsets, T, E, k, C, fill_base, dest,
                                                           src_token);
+    if (!gather) return launch_status();   // the caller reads x through src_token itself
     const long long chunks = (long long)T * (d / 8);
     gather_rows_kernel<<<(unsigned)((chunks + 255) / 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(x), dest, T,
                                                                          d, k, reinterpret_cast<uint4*>(x_perm));
@@ -591,7 +593,7 @@ int run_quant_rows(const void* src, const int32_t* gather, const int32_t* n_rows
 }
 
 int run_expert_ffn_a8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, const A8Bufs& b, cudaStream_t s,
-                      cudaEvent_t ev_down) {
+                      cudaEvent_t ev_down, cudaEvent_t ev_gemm1, cudaEvent_t ev_gemm2) {
     const bool shared = a.f_shared > 0;
     const bool routed = a.max_rows > 0;
     const int32_t* n_routed = routed ? a.offsets + a.E : nullptr;   // kept rows (device)
@@ -599,6 +601,7 @@ int run_expert_ffn_a8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, cons
     if (routed && (rc = run_quant_rows(a.x, b.src_token, n_routed, a.max_rows, a.d, b.xq, b.sx, s)) != MOE_OK)
         return rc;
     if (shared && (rc = run_quant_rows(a.x, nullptr, nullptr, a.T, a.d, b.xqs, b.sxs, s)) != MOE_OK) return rc;
+    if (ev_gemm1 && cudaEventRecord(ev_gemm1, s) != cudaSuccess) return MOE_ERR_CUDA;
     // ---- GEMM1: h = silu(s_x s1 (xq W1q^T)) * (s_x s3 (xq W3q^T))
     {
         CUtensorMap A0, B0, B0b, A1, B1, B1b;
@@ -645,6 +648,7 @@ int run_expert_ffn_a8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, cons
     if (routed && (rc = run_quant_rows(a.h, nullptr, n_routed, a.max_rows, a.f, b.hq, b.sh, s)) != MOE_OK) return rc;
     if (shared && (rc = run_quant_rows(a.h_shared, nullptr, nullptr, a.T, a.f_shared, b.hqs, b.shs, s)) != MOE_OK)
         return rc;
+    if (ev_gemm2 && cudaEventRecord(ev_gemm2, s) != cudaSuccess) return MOE_ERR_CUDA;
     // ---- GEMM2: y = s_h s2 (hq W2q^T)
     {
         CUtensorMap A0, B0, A1, B1;
@@ -939,8 +943,9 @@ int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float*
                            rank_local, mprefix, s, GEMM_BM, fill_base);
     if (!(phases & LAYER_FINISH)) return MOE_OK;
     if (!mark(ev.permute)) return MOE_ERR_CUDA;
+    // fp8 activations are quantised straight from x through src_token: no x_perm
     if ((rc = run_permute(di, x, idx, T, d, E, k, C, counts_raw, counts, offsets, dest, src, x_perm, blk_cnt,
-                          rank_local, mprefix, s, pair ? PAIR_BM : GEMM_BM, fill_base)) != MOE_OK)
+                          rank_local, mprefix, s, pair ? PAIR_BM : GEMM_BM, fill_base, false, !(w8 && act8))) != MOE_OK)
         return rc;
     CacheView cv{};
     if (cache) {
@@ -974,7 +979,8 @@ int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float*
         b.sxs = shared ? reinterpret_cast<float*>(base + A8.sxs) : nullptr;
         b.shs = shared ? reinterpret_cast<float*>(base + A8.shs) : nullptr;
         b.src_token = src;
-        rc = run_expert_ffn_a8(di, a, *w8, b, s, static_cast<cudaEvent_t>(ev.down));
+        rc = run_expert_ffn_a8(di, a, *w8, b, s, static_cast<cudaEvent_t>(ev.down), static_cast<cudaEvent_t>(ev.gemm1),
+                               static_cast<cudaEvent_t>(ev.gemm2));
     } else {
         rc = w8 ? run_expert_ffn_w8(di, a, *w8, s, static_cast<cudaEvent_t>(ev.down))
                 : run_expert_ffn(di, a, s, static_cast<cudaEvent_t>(ev.down));

@@ -162,6 +162,7 @@ WORKLOAD_ORDER = ["tiny", "mixtral", "qwen3", "dsv3", "skew"]
 PROFILE_WORKLOADS = {
     "mixtral2e": Workload("mixtral2e", 2048, 4096, 2, 2, 14336),
     "dsv3_32e": Workload("dsv3_32e", 32, 7168, 32, 8, 2048, f_shared=2048, bias_range=0.1),
+    "qwen3_16e": Workload("qwen3_16e", 2048, 4096, 16, 8, 1536),
 }
 WORKLOADS.update(PROFILE_WORKLOADS)
 
