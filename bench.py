@@ -37,11 +37,12 @@ KERNELS_PER_STEP = 9   # router GEMM, top-k, count, scan, scatter, gather, GEMM1
 
 
 def launches_per_step(a8: bool, shared: bool) -> int:
-    """Kernels one layer call launches.  fp8 activations: no gather (the quantiser reads x through
-    src_token), one quantiser before each grouped GEMM, two more for the shared expert's rows."""
+    """Kernels one layer call launches.  fp8 activations: no gather (one quantiser writes each x
+    row's codes to its permuted rows and, with a shared expert, its own row), a quantiser of h
+    before GEMM2 and one more for the shared expert's h."""
     if not a8:
         return KERNELS_PER_STEP
-    return KERNELS_PER_STEP - 1 + 2 + (2 if shared else 0)
+    return KERNELS_PER_STEP - 1 + 2 + (1 if shared else 0)
 
 DESCR = {
     "tiny": "tiny MoE layer T=128 d=256 E=8 top-2 f=512",

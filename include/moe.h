@@ -360,8 +360,8 @@ int moe_ep_return(const moe_bf16* y_recv, int R, int rank, int E, int d, moe_bf1
  * s_row * s_col before SwiGLU / the bf16 store.  Router, routing, permutation and combine as in
  * moe_layer_forward().  Workspace: moe_workspace_bytes_a8() (the layer workspace followed by the
  * quantised rows and their scales).  Shapes: d, f, f_shared multiples of 128 (MOE_ERR_SHAPE).
- * The routed rows are quantised straight from x through src_token, so the workspace's x_perm is
- * not written by this layer.
+ * Each token row of x is quantised once and its codes written to its permuted rows (dest), so
+ * the workspace's x_perm is not written by this layer.
  */
 int moe_workspace_bytes_a8(int T, int d, int E, int k, int f, int f_shared, size_t* bytes);
 int moe_layer_forward_w8a8(const moe_bf16* x, const moe_bf16* Wg, const float* bias,

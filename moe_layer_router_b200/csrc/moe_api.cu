@@ -342,7 +342,7 @@ int run_permute(DeviceInfo* di, const moe_bf16* x, const int32_t* idx, int T, in
     if (counts_only) return launch_status();
     permute_scatter_kernel<<<nb, PERMUTE_TOKENS, 0, s>>>(idx, rank_local, blk_cnt, offsets, T, E, k, C, fill_base, dest,
                                                           src_token);
-    if (!gather) return launch_status();   // the caller reads x through src_token itself
+    if (!gather) return launch_status();   // the caller moves x's rows itself (dest / src_token)
     const long long chunks = (long long)T * (d / 8);
     gather_rows_kernel<<<(unsigned)((chunks + 255) / 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(x), dest, T,
                                                                          d, k, reinterpret_cast<uint4*>(x_perm));
@@ -575,13 +575,16 @@ int run_expert_ffn_w8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, cuda
     return MOE_OK;
 }
 
-// Both expert GEMMs with fp8 weights and fp8 activations: x_perm rows are quantised straight
-// from x (gathered by src_token), h rows after GEMM1; the 1-SM grouped GEMM runs kind::f8f6f4
-// and scales each accumulator by its activation row scale and weight row scale.
+// Both expert GEMMs with fp8 weights and fp8 activations: each token row of x is quantised once
+// and its codes written to its k permuted rows (dest) and, with a shared expert, to its own row;
+// h rows after GEMM1; the grouped GEMMs run kind::f8f6f4 and scale each accumulator by its
+// activation row scale and weight row scale.
 struct A8Bufs {
     uint8_t *xq, *hq, *xqs, *hqs;
     float *sx, *sh, *sxs, *shs;
-    const int32_t* src_token;
+    const int32_t* dest;        // [T, k] permuted row of each assignment, -1 = dropped
+    const int32_t* src_token;   // [T k] token of each permuted row (for rows too long to hold)
+    int k;
 };
 
 int run_quant_rows(const void* src, const int32_t* gather, const int32_t* n_rows, int rows, int K, uint8_t* dst,
@@ -592,15 +595,49 @@ int run_quant_rows(const void* src, const int32_t* gather, const int32_t* n_rows
     return launch_status();
 }
 
+// The one-CTA-per-row quantiser for rows of up to 16384 elements (the row in registers);
+// returns false (nothing launched) for longer rows.
+bool run_quant_blk(const void* src, const int32_t* n_rows, int rows, int K, const int32_t* dest, int k, uint8_t* dst,
+                   float* scale, uint8_t* dst_tok, float* scale_tok, cudaStream_t s) {
+    const int cpt = (K / 8 + QUANT_THREADS - 1) / QUANT_THREADS;
+    const uint4* x = static_cast<const uint4*>(src);
+    uint2* d = reinterpret_cast<uint2*>(dst);
+    uint2* dt = reinterpret_cast<uint2*>(dst_tok);
+#define MOE_QUANT(C) quant_rows_e4m3_blk_kernel<C><<<rows, QUANT_THREADS, 0, s>>>(x, n_rows, K, dest, k, d, scale, dt, \
+                                                                                  scale_tok)
+    if (cpt <= 2) MOE_QUANT(2);
+    else if (cpt <= 4) MOE_QUANT(4);
+    else if (cpt <= 8) MOE_QUANT(8);
+    else if (cpt <= 16) MOE_QUANT(16);
+    else return false;
+#undef MOE_QUANT
+    return true;
+}
+
+// h rows [0, *n_rows) of a [rows, K] buffer -> e4m3 rows + scales.
+int run_quant_h(const void* h, const int32_t* n_rows, int rows, int K, uint8_t* dst, float* scale, cudaStream_t s) {
+    if (rows <= 0) return MOE_OK;
+    if (!run_quant_blk(h, n_rows, rows, K, nullptr, 0, dst, scale, nullptr, nullptr, s))
+        return run_quant_rows(h, nullptr, n_rows, rows, K, dst, scale, s);
+    return launch_status();
+}
+
 int run_expert_ffn_a8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, const A8Bufs& b, cudaStream_t s,
                       cudaEvent_t ev_down, cudaEvent_t ev_gemm1, cudaEvent_t ev_gemm2) {
     const bool shared = a.f_shared > 0;
     const bool routed = a.max_rows > 0;
     const int32_t* n_routed = routed ? a.offsets + a.E : nullptr;   // kept rows (device)
     int rc;
-    if (routed && (rc = run_quant_rows(a.x, b.src_token, n_routed, a.max_rows, a.d, b.xq, b.sx, s)) != MOE_OK)
-        return rc;
-    if (shared && (rc = run_quant_rows(a.x, nullptr, nullptr, a.T, a.d, b.xqs, b.sxs, s)) != MOE_OK) return rc;
+    // x: every token row quantised once, its codes written to its permuted rows (and its own
+    // row for the shared expert)
+    if (routed && run_quant_blk(a.x, nullptr, a.T, a.d, b.dest, b.k, b.xq, b.sx, shared ? b.xqs : nullptr,
+                                shared ? b.sxs : nullptr, s)) {
+        if ((rc = launch_status()) != MOE_OK) return rc;
+    } else {
+        if (routed && (rc = run_quant_rows(a.x, b.src_token, n_routed, a.max_rows, a.d, b.xq, b.sx, s)) != MOE_OK)
+            return rc;
+        if (shared && (rc = run_quant_h(a.x, nullptr, a.T, a.d, b.xqs, b.sxs, s)) != MOE_OK) return rc;
+    }
     if (ev_gemm1 && cudaEventRecord(ev_gemm1, s) != cudaSuccess) return MOE_ERR_CUDA;
     // ---- GEMM1: h = silu(s_x s1 (xq W1q^T)) * (s_x s3 (xq W3q^T))
     {
@@ -645,9 +682,8 @@ int run_expert_ffn_a8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, cons
         if (rc != MOE_OK) return rc;
     }
     if (ev_down && cudaEventRecord(ev_down, s) != cudaSuccess) return MOE_ERR_CUDA;
-    if (routed && (rc = run_quant_rows(a.h, nullptr, n_routed, a.max_rows, a.f, b.hq, b.sh, s)) != MOE_OK) return rc;
-    if (shared && (rc = run_quant_rows(a.h_shared, nullptr, nullptr, a.T, a.f_shared, b.hqs, b.shs, s)) != MOE_OK)
-        return rc;
+    if (routed && (rc = run_quant_h(a.h, n_routed, a.max_rows, a.f, b.hq, b.sh, s)) != MOE_OK) return rc;
+    if (shared && (rc = run_quant_h(a.h_shared, nullptr, a.T, a.f_shared, b.hqs, b.shs, s)) != MOE_OK) return rc;
     if (ev_gemm2 && cudaEventRecord(ev_gemm2, s) != cudaSuccess) return MOE_ERR_CUDA;
     // ---- GEMM2: y = s_h s2 (hq W2q^T)
     {
@@ -943,7 +979,7 @@ int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float*
                            rank_local, mprefix, s, GEMM_BM, fill_base);
     if (!(phases & LAYER_FINISH)) return MOE_OK;
     if (!mark(ev.permute)) return MOE_ERR_CUDA;
-    // fp8 activations are quantised straight from x through src_token: no x_perm
+    // fp8 activations: each x row is quantised once and written to its rows by dest: no x_perm
     if ((rc = run_permute(di, x, idx, T, d, E, k, C, counts_raw, counts, offsets, dest, src, x_perm, blk_cnt,
                           rank_local, mprefix, s, pair ? PAIR_BM : GEMM_BM, fill_base, false, !(w8 && act8))) != MOE_OK)
         return rc;
@@ -978,7 +1014,9 @@ int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float*
         b.sh = reinterpret_cast<float*>(base + A8.sh);
         b.sxs = shared ? reinterpret_cast<float*>(base + A8.sxs) : nullptr;
         b.shs = shared ? reinterpret_cast<float*>(base + A8.shs) : nullptr;
+        b.dest = dest;
         b.src_token = src;
+        b.k = k;
         rc = run_expert_ffn_a8(di, a, *w8, b, s, static_cast<cudaEvent_t>(ev.down), static_cast<cudaEvent_t>(ev.gemm1),
                                static_cast<cudaEvent_t>(ev.gemm2));
     } else {

@@ -508,33 +508,59 @@ def test_layer_fp8_weights_and_activations(moe, wl):
     assert xq_ref.shape[0] == r["N"] and np.isfinite(sx_ref).all()
 
 
-def test_quantised_rows_bit_exact(moe):
-    """The layer's activation quantiser against the oracle's on the permuted rows: the workspace's
-    fp8 region follows the layer workspace (moe_workspace_bytes_a8 - ...), so it is read through a
-    layer call on a shape whose routed rows fill the region from its start."""
-    wl = synth.Workload("a8q", 64, 256, 4, 2, 128)
-    T, d, E, k, f = wl.T, wl.d, wl.E, wl.k, wl.f
+def _a8_regions(T, d, k, f, fs, base):
+    """Byte offsets of the fp8 rows and scales that follow the layer workspace (256-byte aligned,
+    in the order xq, sx, hq, sh, xqs, sxs, hqs, shs)."""
+    al = lambda v: (v + 255) // 256 * 256
+    sizes = [("xq", T * k * d), ("sx", T * k * 4), ("hq", T * k * f), ("sh", T * k * 4),
+             ("xqs", T * d if fs else 0), ("sxs", T * 4 if fs else 0), ("hqs", T * fs), ("shs", T * 4 if fs else 0)]
+    off, cur = {}, al(base)
+    for n, b in sizes:
+        off[n] = cur
+        cur = al(cur + b)
+    return off
+
+
+@pytest.mark.parametrize("wl", [synth.Workload("a8q", 64, 256, 4, 2, 128),
+                                synth.Workload("a8qs", 24, 7168, 2, 2, 9216, f_shared=1536),
+                                synth.Workload("a8qm", 40, 4096, 16, 4, 2048, f_shared=128)],
+                         ids=["short-rows", "long-rows-shared", "mid-rows-shared"])
+def test_quantised_rows_bit_exact(moe, wl):
+    """The layer's activation quantisers against the oracle's: the routed rows (each token row
+    quantised once and written to its permuted rows), the shared expert's rows, and h before
+    GEMM2 (the kernel's own h, read back), bit for bit.  Row lengths take every
+    register tile of the one-CTA-per-row quantiser (256 .. 9216 here)."""
+    T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
     inp = synth.Inputs(wl)
     x = inp.x()
     Q = synth.device_tensors_q8(wl, "cuda")
-    ws = torch.zeros(moe.moe_workspace_bytes_a8(T, d, E, k, f, 0), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(moe.moe_workspace_bytes_a8(T, d, E, k, f, fs), dtype=torch.uint8, device="cuda")
     out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
     moe.moe_layer_forward_w8a8(to_dev_bf16(x), to_dev_bf16(inp.wg()), None, Q["w1q"], Q["s1"], Q["w3q"], Q["s3"],
-                               Q["w2q"], Q["s2"], None, None, None, None, None, None, 0, T, d, E, k, f, 1.0,
-                               moe.MOE_CAP_NONE, out, ws)
+                               Q["w2q"], Q["s2"], Q.get("w1sq"), Q.get("s1s"), Q.get("w3sq"), Q.get("s3s"),
+                               Q.get("w2sq"), Q.get("s2s"), fs, T, d, E, k, f, 1.0, moe.MOE_CAP_NONE, out, ws)
     assert moe.moe_get_error() == 0
-    L = moe.moe_workspace_layout(T, d, E, k, f, 0)
-    base = moe.moe_workspace_bytes(T, d, E, k, f, 0)
-    start = (base + 255) // 256 * 256
+    L = moe.moe_workspace_layout(T, d, E, k, f, fs)
+    o = _a8_regions(T, d, k, f, fs, moe.moe_workspace_bytes(T, d, E, k, f, fs))
     N = T * k
-    xq = ws[start:start + N * d].cpu().numpy().reshape(N, d)
-    so = (start + N * d + 255) // 256 * 256
-    sx = ws[so:so + 4 * N].view(torch.float32).cpu().numpy()
+    rows = lambda n, r, c: ws[o[n]:o[n] + r * c].cpu().numpy().reshape(r, c)
+    scales = lambda n, r: ws[o[n]:o[n] + 4 * r].view(torch.float32).cpu().numpy()
     dest = moe.workspace_view(ws, L, "dest", (T, k), torch.int32).cpu().numpy()
-    xp = oracle.gather(x, dest, N)
-    xq_ref, sx_ref = oracle.quantize_rows_e4m3(xp)
-    assert np.array_equal(sx.view(np.uint32), sx_ref.view(np.uint32))
-    assert np.array_equal(xq, xq_ref)
+    xq_ref, sx_ref = oracle.quantize_rows_e4m3(oracle.gather(x, dest, N))
+    assert np.array_equal(scales("sx", N).view(np.uint32), sx_ref.view(np.uint32))
+    assert np.array_equal(rows("xq", N, d), xq_ref)
+    h = bf16_bits(moe.workspace_view(ws, L, "h", (N, f), torch.bfloat16))
+    hq_ref, sh_ref = oracle.quantize_rows_e4m3(h)
+    assert np.array_equal(scales("sh", N).view(np.uint32), sh_ref.view(np.uint32))
+    assert np.array_equal(rows("hq", N, f), hq_ref)
+    if fs:
+        xqs_ref, sxs_ref = oracle.quantize_rows_e4m3(x)
+        assert np.array_equal(scales("sxs", T).view(np.uint32), sxs_ref.view(np.uint32))
+        assert np.array_equal(rows("xqs", T, d), xqs_ref)
+        hs = bf16_bits(moe.workspace_view(ws, L, "h_shared", (T, fs), torch.bfloat16))
+        hqs_ref, shs_ref = oracle.quantize_rows_e4m3(hs)
+        assert np.array_equal(scales("shs", T).view(np.uint32), shs_ref.view(np.uint32))
+        assert np.array_equal(rows("hqs", T, fs), hqs_ref)
 
 
 @pytest.mark.parametrize("wl", [synth.Workload("a8c0", 64, 256, 16, 4, 128, f_shared=128, cap_mode=synth.CAP_PER_TOKEN,
