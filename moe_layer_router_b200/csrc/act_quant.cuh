@@ -55,76 +55,94 @@ __global__ void __launch_bounds__(256) quant_rows_e4m3_kernel(const uint4* __res
     }
 }
 
-// The same recipe with one 128-thread CTA per source row, the row held in registers (MAXC
-// 16-byte chunks per thread, K <= 1024 MAXC): one HBM read of the row however long it is, and
-// every load of the row in flight at once.  Destinations:
+// The same recipe with each source row held in the registers of TPR threads (MAXC 16-byte
+// chunks per thread, K <= 8 TPR MAXC): one HBM read of the row however long it is, all of its
+// loads in flight at once.  A CTA of 256 threads takes 256 / TPR rows (TPR = 32: a warp per row,
+// for short rows; 128 or 256 for long ones).  Destinations:
 //   dest == nullptr: row r of src -> row r of dst / scale, rows r >= *n_rows (when given) skipped;
 //   dest != nullptr: token row t -> rows dest[t k + j] (j < k, dest >= 0) of dst / scale, and,
 //                    when dst_tok is given, row t of dst_tok / scale_tok (the shared expert's rows).
 // Each warp store instruction writes 256 contiguous bytes of one destination row.
-constexpr int QUANT_THREADS = 128;
+constexpr int QUANT_CTA = 256;
 
-template <int MAXC>
-__global__ void __launch_bounds__(QUANT_THREADS) quant_rows_e4m3_blk_kernel(
-    const uint4* __restrict__ src, const int32_t* __restrict__ n_rows, int K, const int32_t* __restrict__ dest, int k,
-    uint2* __restrict__ dst, float* __restrict__ scale, uint2* __restrict__ dst_tok, float* __restrict__ scale_tok) {
-    __shared__ float s_max[QUANT_THREADS / 32];
-    __shared__ int s_dest[32];
-    const int tid = threadIdx.x, lane = tid & 31;
-    const long long row = blockIdx.x;
-    if (!dest && n_rows && row >= __ldg(n_rows)) return;    // uniform over the CTA
+__device__ __forceinline__ float amax_bf16x8(float m, const uint4& v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        m = fmaxf(m, fabsf(__uint_as_float(w[e] << 16)));
+        m = fmaxf(m, fabsf(__uint_as_float(w[e] & 0xFFFF0000u)));
+    }
+    return m;
+}
+
+// 8 bf16 -> 8 e4m3 codes of e4m3(x / sc), round to nearest even, saturating
+__device__ __forceinline__ uint2 e4m3x8(const uint4& v, float sc) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[2] = {0u, 0u};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float lo = __fdiv_rn(__uint_as_float(w[e] << 16), sc);
+        const float hi = __fdiv_rn(__uint_as_float(w[e] & 0xFFFF0000u), sc);
+        const uint32_t b0 = __nv_cvt_float_to_fp8(lo, __NV_SATFINITE, __NV_E4M3);
+        const uint32_t b1 = __nv_cvt_float_to_fp8(hi, __NV_SATFINITE, __NV_E4M3);
+        out[e >> 1] |= (b0 | (b1 << 8)) << (16 * (e & 1));
+    }
+    return make_uint2(out[0], out[1]);
+}
+
+template <int TPR, int MAXC>
+__global__ void __launch_bounds__(QUANT_CTA) quant_rows_e4m3_reg_kernel(
+    const uint4* __restrict__ src, const int32_t* __restrict__ n_rows, long long rows, int K,
+    const int32_t* __restrict__ dest, int k, uint2* __restrict__ dst, float* __restrict__ scale,
+    uint2* __restrict__ dst_tok, float* __restrict__ scale_tok) {
+    static_assert(TPR == 32 || TPR == 128 || TPR == 256, "a warp, or whole warps of one CTA");
+    constexpr int RPC = QUANT_CTA / TPR;            // rows per CTA
+    __shared__ float s_max[QUANT_CTA / 32];
+    __shared__ int s_dest[RPC][32];
+    const int tid = threadIdx.x % TPR, grp = threadIdx.x / TPR, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * RPC + grp;
+    // rows past the end do no memory work but (TPR > 32) still meet the CTA barrier
+    const bool live = row < rows && (dest || !n_rows || row < __ldg(n_rows));
     const int chunks = K / 8;
     const uint4* s = src + row * chunks;
     uint4 v[MAXC];
 #pragma unroll
     for (int i = 0; i < MAXC; ++i) {
-        const int c = tid + i * QUANT_THREADS;
-        v[i] = c < chunks ? __ldg(s + c) : make_uint4(0u, 0u, 0u, 0u);
+        const int c = tid + i * TPR;
+        v[i] = live && c < chunks ? __ldg(s + c) : make_uint4(0u, 0u, 0u, 0u);
     }
-    if (dest && tid < 32) s_dest[tid] = tid < k ? __ldg(dest + row * k + tid) : -1;
+    if (dest && tid < 32) s_dest[grp][tid] = live && tid < k ? __ldg(dest + row * k + tid) : -1;
     float amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < MAXC; ++i) {
-        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            amax = fmaxf(amax, fabsf(__uint_as_float(w[e] << 16)));
-            amax = fmaxf(amax, fabsf(__uint_as_float(w[e] & 0xFFFF0000u)));
-        }
-    }
+    for (int i = 0; i < MAXC; ++i) amax = amax_bf16x8(amax, v[i]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if (lane == 0) s_max[tid >> 5] = amax;
-    __syncthreads();
+    if (TPR > 32) {
+        if (lane == 0) s_max[threadIdx.x >> 5] = amax;
+        __syncthreads();
 #pragma unroll
-    for (int w = 0; w < QUANT_THREADS / 32; ++w) amax = fmaxf(amax, s_max[w]);
+        for (int w = 0; w < TPR / 32; ++w) amax = fmaxf(amax, s_max[grp * (TPR / 32) + w]);
+    } else {
+        __syncwarp();
+    }
+    if (!live) return;
     const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
     if (!dest) {
         if (tid == 0) scale[row] = sc;
     } else {
-        if (tid < k && s_dest[tid] >= 0) scale[s_dest[tid]] = sc;
+        if (tid < k && s_dest[grp][tid] >= 0) scale[s_dest[grp][tid]] = sc;
         if (tid == 0 && dst_tok) scale_tok[row] = sc;
     }
 #pragma unroll
     for (int i = 0; i < MAXC; ++i) {
-        const int c = tid + i * QUANT_THREADS;
+        const int c = tid + i * TPR;
         if (c >= chunks) break;
-        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-        uint32_t out[2] = {0u, 0u};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float lo = __fdiv_rn(__uint_as_float(w[e] << 16), sc);
-            const float hi = __fdiv_rn(__uint_as_float(w[e] & 0xFFFF0000u), sc);
-            const uint32_t b0 = __nv_cvt_float_to_fp8(lo, __NV_SATFINITE, __NV_E4M3);
-            const uint32_t b1 = __nv_cvt_float_to_fp8(hi, __NV_SATFINITE, __NV_E4M3);
-            out[e >> 1] |= (b0 | (b1 << 8)) << (16 * (e & 1));
-        }
-        const uint2 q = make_uint2(out[0], out[1]);
+        const uint2 q = e4m3x8(v[i], sc);
         if (!dest) {
             dst[row * chunks + c] = q;
         } else {
             for (int j = 0; j < k; ++j) {
-                const int r = s_dest[j];
+                const int r = s_dest[grp][j];
                 if (r >= 0) dst[(long long)r * chunks + c] = q;
             }
             if (dst_tok) dst_tok[row * chunks + c] = q;

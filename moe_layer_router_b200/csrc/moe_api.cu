@@ -595,20 +595,23 @@ int run_quant_rows(const void* src, const int32_t* gather, const int32_t* n_rows
     return launch_status();
 }
 
-// The one-CTA-per-row quantiser for rows of up to 16384 elements (the row in registers);
-// returns false (nothing launched) for longer rows.
+// The register-held quantiser for rows of up to 16384 elements: a warp per row up to 2048
+// elements, 128 threads up to 8192, 256 beyond; returns false (nothing launched) for longer rows.
 bool run_quant_blk(const void* src, const int32_t* n_rows, int rows, int K, const int32_t* dest, int k, uint8_t* dst,
                    float* scale, uint8_t* dst_tok, float* scale_tok, cudaStream_t s) {
-    const int cpt = (K / 8 + QUANT_THREADS - 1) / QUANT_THREADS;
+    const int chunks = K / 8;
     const uint4* x = static_cast<const uint4*>(src);
     uint2* d = reinterpret_cast<uint2*>(dst);
     uint2* dt = reinterpret_cast<uint2*>(dst_tok);
-#define MOE_QUANT(C) quant_rows_e4m3_blk_kernel<C><<<rows, QUANT_THREADS, 0, s>>>(x, n_rows, K, dest, k, d, scale, dt, \
-                                                                                  scale_tok)
-    if (cpt <= 2) MOE_QUANT(2);
-    else if (cpt <= 4) MOE_QUANT(4);
-    else if (cpt <= 8) MOE_QUANT(8);
-    else if (cpt <= 16) MOE_QUANT(16);
+#define MOE_QUANT(TPR, C)                                                                                    \
+    quant_rows_e4m3_reg_kernel<TPR, C><<<(unsigned)(((long long)rows * TPR + QUANT_CTA - 1) / QUANT_CTA),      \
+                                         QUANT_CTA, 0, s>>>(x, n_rows, rows, K, dest, k, d, scale, dt, scale_tok)
+    if (chunks <= 32 * 2) MOE_QUANT(32, 2);
+    else if (chunks <= 32 * 4) MOE_QUANT(32, 4);
+    else if (chunks <= 32 * 8) MOE_QUANT(32, 8);
+    else if (chunks <= 128 * 4) MOE_QUANT(128, 4);
+    else if (chunks <= 128 * 8) MOE_QUANT(128, 8);
+    else if (chunks <= 256 * 8) MOE_QUANT(256, 8);
     else return false;
 #undef MOE_QUANT
     return true;

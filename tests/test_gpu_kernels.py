@@ -521,7 +521,7 @@ def _a8_regions(T, d, k, f, fs, base):
     return off
 
 
-@pytest.mark.parametrize("wl", [synth.Workload("a8q", 64, 256, 4, 2, 128),
+@pytest.mark.parametrize("wl", [synth.Workload("a8q", 64, 256, 4, 2, 768),
                                 synth.Workload("a8qs", 24, 7168, 2, 2, 9216, f_shared=1536),
                                 synth.Workload("a8qm", 40, 4096, 16, 4, 2048, f_shared=128)],
                          ids=["short-rows", "long-rows-shared", "mid-rows-shared"])
@@ -529,7 +529,7 @@ def test_quantised_rows_bit_exact(moe, wl):
     """The layer's activation quantisers against the oracle's: the routed rows (each token row
     quantised once and written to its permuted rows), the shared expert's rows, and h before
     GEMM2 (the kernel's own h, read back), bit for bit.  Row lengths take every
-    register tile of the one-CTA-per-row quantiser (256 .. 9216 here)."""
+    register-tile variant of the quantiser (rows of 256 .. 9216 elements)."""
     T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
     inp = synth.Inputs(wl)
     x = inp.x()
