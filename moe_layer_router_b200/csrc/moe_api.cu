@@ -617,10 +617,13 @@ bool run_quant_blk(const void* src, const int32_t* n_rows, int rows, int K, cons
     return true;
 }
 
-// h rows [0, *n_rows) of a [rows, K] buffer -> e4m3 rows + scales.
+// h rows [0, *n_rows) of a [rows, K] buffer -> e4m3 rows + scales.  Rows of up to 2048
+// elements take the two-pass warp-per-row kernel: its 28 registers keep 64 warps per SM busy
+// with the correctly rounded divisions, and its second pass over a row hits L2 (measured faster
+// than holding the row in registers for K = 1536 and 2048); longer rows are read once.
 int run_quant_h(const void* h, const int32_t* n_rows, int rows, int K, uint8_t* dst, float* scale, cudaStream_t s) {
     if (rows <= 0) return MOE_OK;
-    if (!run_quant_blk(h, n_rows, rows, K, nullptr, 0, dst, scale, nullptr, nullptr, s))
+    if (K <= 2048 || !run_quant_blk(h, n_rows, rows, K, nullptr, 0, dst, scale, nullptr, nullptr, s))
         return run_quant_rows(h, nullptr, n_rows, rows, K, dst, scale, s);
     return launch_status();
 }

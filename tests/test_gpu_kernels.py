@@ -521,15 +521,18 @@ def _a8_regions(T, d, k, f, fs, base):
     return off
 
 
-@pytest.mark.parametrize("wl", [synth.Workload("a8q", 64, 256, 4, 2, 768),
-                                synth.Workload("a8qs", 24, 7168, 2, 2, 9216, f_shared=1536),
-                                synth.Workload("a8qm", 40, 4096, 16, 4, 2048, f_shared=128)],
-                         ids=["short-rows", "long-rows-shared", "mid-rows-shared"])
+@pytest.mark.parametrize("wl", [synth.Workload("a8q", 64, 512, 4, 2, 768),
+                                synth.Workload("a8q1", 32, 1024, 8, 3, 256),
+                                synth.Workload("a8q2", 48, 2048, 8, 2, 6144),
+                                synth.Workload("a8qm", 40, 4096, 16, 4, 2048, f_shared=128),
+                                synth.Workload("a8qs", 24, 7168, 2, 2, 9216, f_shared=1536)],
+                         ids=["d512", "d1024", "d2048-f6144", "d4096-shared", "d7168-f9216-shared"])
 def test_quantised_rows_bit_exact(moe, wl):
     """The layer's activation quantisers against the oracle's: the routed rows (each token row
     quantised once and written to its permuted rows), the shared expert's rows, and h before
-    GEMM2 (the kernel's own h, read back), bit for bit.  Row lengths take every
-    register-tile variant of the quantiser (rows of 256 .. 9216 elements)."""
+    GEMM2 (the kernel's own h, read back), bit for bit.  The row lengths reach every variant:
+    a warp per row with 2, 4 or 8 chunks a lane (d = 512, 1024, 2048), 128 threads with 4 or 8
+    (d = 4096, 7168; h of 6144), 256 threads (h of 9216), and the two-pass kernel (h <= 2048)."""
     T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
     inp = synth.Inputs(wl)
     x = inp.x()
