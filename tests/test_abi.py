@@ -175,3 +175,33 @@ def test_fp8_activation_entry_needs_128_byte_k(lib):
     assert lib.moe_workspace_bytes(256, 7168, 256, 8, 2048, 2048, ctypes.byref(b)) == 0
     # plus fp8 copies of the permuted rows and of h (routed and shared) and their scales
     assert a.value >= b.value + 2048 * (7168 + 2048) + 256 * (7168 + 2048)
+
+
+def header_struct_fields(name):
+    """Field names of a `typedef struct name { ... } name;` in the header, in order."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    m = re.search(r"typedef struct %s \{(.*?)\} %s;" % (name, name), src, flags=re.S)
+    assert m, name
+    names = []
+    for decl in m.group(1).split(";"):
+        for part in decl.split(","):
+            ids = re.findall(r"[A-Za-z_][A-Za-z0-9_]*", part)
+            if ids:
+                names.append(ids[-1])
+    return names
+
+
+def test_binding_stage_events_match_the_header():
+    """The ctypes mirror of moe_stage_events has the header's members in the header's order
+    (the library reads the whole struct, so a missing trailing member would be read past)."""
+    import moe_layer_router_b200 as moe
+    fields = header_struct_fields("moe_stage_events")
+    assert [n for n, _ in moe.moe_stage_events._fields_] == fields
+    assert ctypes.sizeof(moe.moe_stage_events) == len(fields) * ctypes.sizeof(ctypes.c_void_p)
+    assert fields[:len(moe.STAGES)] == moe.STAGES
+
+
+@pytest.mark.parametrize("name", ["moe_pipeline_params", "moe_w8_experts"])
+def test_binding_structs_match_the_header(name):
+    import moe_layer_router_b200 as moe
+    assert [n for n, _ in getattr(moe, name)._fields_] == header_struct_fields(name)
