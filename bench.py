@@ -240,14 +240,28 @@ def gemm1_work(wl, N):
     return flops
 
 
-def gemm1_bytes(wl, N, touched, wbytes=2):
+def gemm1_bytes(wl, N, touched, wbytes=2, abytes=2):
+    """Algorithmic bytes of one launch of the first grouped GEMM: weights of the touched experts
+    (wbytes per element, + fp32 row scales for fp8), its A rows (abytes per element, + a row
+    scale for fp8 activations), h written in bf16; the same for the shared expert."""
     b = touched * 2.0 * wl.f * wl.d * wbytes        # W1, W3 of touched experts
     if wbytes == 1:
         b += touched * 2.0 * wl.f * 4                # row scales
-    b += N * wl.d * 2 + N * wl.f * 2                # x_perm read, h write
+    b += N * wl.d * abytes + N * wl.f * 2           # A rows read, h write
+    if abytes == 1:
+        b += N * 4.0
     if wl.f_shared:
-        b += 2.0 * wl.f_shared * wl.d * wbytes + wl.T * wl.d * 2 + wl.T * wl.f_shared * 2
+        b += 2.0 * wl.f_shared * wl.d * wbytes + wl.T * wl.d * abytes + wl.T * wl.f_shared * 2
+        if wbytes == 1:
+            b += 2.0 * wl.f_shared * 4
+        if abytes == 1:
+            b += wl.T * 4.0
     return b
+
+
+def gemms_work(wl, N):
+    """FLOPs of both grouped GEMMs of one layer call (routed + shared)."""
+    return 6.0 * N * wl.d * wl.f + 6.0 * wl.T * wl.d * wl.f_shared
 
 
 def layer_work(wl, N, touched, wbytes=2):
@@ -648,7 +662,7 @@ def main():
     g1_ms = gemm_ms["gate_up"]
     decode = wl.name.startswith("dsv3")
     if decode:
-        alg = gemm1_bytes(wl, N, touched, 1 if fp8 else 2)
+        alg = gemm1_bytes(wl, N, touched, 1 if fp8 else 2, 1 if a8 else 2)
         achieved = alg / (g1_ms / 1000.0) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"]}
@@ -683,6 +697,10 @@ def main():
                        touched * 3.0 * f * d * 2 / 1e9)},
         "roofline": roof,
         "layer": {"tflops": lf / step_s / 1e12, "gbs": lb / step_s / 1e9,
+                  # both grouped GEMMs' FLOPs over their kernel times, against the tensor peak
+                  # of their operand type (bf16, or fp8 = measured bf16 x 2)
+                  "gemms_tensor_frac": gemms_work(wl, N) / ((gemm_ms["gate_up"] + gemm_ms["down"]) / 1e3) / 1e12
+                  / (peaks["bf16_tflops"] * (2.0 if a8 else 1.0)),
                   "tensor_frac": lf / step_s / 1e12 / peaks["bf16_tflops"],
                   "hbm_frac": lb / step_s / 1e9 / peaks["hbm_gbs"], "kept_rows": N, "touched_experts": touched,
                   "drop_rate": 1.0 - N / float(T * k), "load_var_raw": float(np.var(craw)),
