@@ -166,6 +166,42 @@ __device__ __forceinline__ void scale_cols32(uint32_t (&v)[32], float sa, const 
     }
 }
 
+// 32 gate and 32 up columns -> 32 bf16 of h, packed in pairs.
+__device__ __forceinline__ void swiglu_pack32(const uint32_t (&g)[32], const uint32_t (&u)[32], uint32_t (&packed)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        packed[i] = pack_bf16x2(swiglu_f32(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                                swiglu_f32(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
+}
+
+// 32 accumulator columns -> 32 bf16, packed in pairs.
+__device__ __forceinline__ void pack32(const uint32_t (&v)[32], uint32_t (&packed)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+}
+
+// A warp's 32 consecutive output rows x 32 bf16 (lane = row, 16 packed words each) stored through
+// 2 KB of shared memory, so that a store instruction writes the 64 bytes of 8 whole rows (full
+// 32-byte sectors) instead of 16 bytes of each of 32 rows (half sectors).  Lane l first writes
+// its row to `stage` (its four 16-byte pieces XOR-swizzled by row: no bank conflicts either way),
+// then stores piece l % 4 of row 8 j + l / 4 for j = 0..3; rows whose bit in `valid` is clear
+// are skipped.  out0 = row 0, first column.  Warp-collective.
+__device__ __forceinline__ void store_rows_staged(const uint32_t (&packed)[16], uint4* stage, int lane,
+                                                  __nv_bfloat16* out0, long long ldo, uint32_t valid) {
+    __syncwarp();                                   // the previous chunk's reads of stage are done
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        stage[lane * 4 + (q ^ ((lane >> 1) & 3))] =
+            make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int r = 8 * j + (lane >> 2), q = lane & 3;
+        const uint4 w = stage[r * 4 + (q ^ ((r >> 1) & 3))];
+        if ((valid >> r) & 1u) reinterpret_cast<uint4*>(out0 + r * ldo)[q] = w;
+    }
+}
+
 // 32 gate and 32 up columns -> 32 bf16 of h, stored at dst (16-byte aligned).
 __device__ __forceinline__ void swiglu_store32(const uint32_t (&g)[32], const uint32_t (&u)[32], __nv_bfloat16* dst) {
     uint32_t packed[16];

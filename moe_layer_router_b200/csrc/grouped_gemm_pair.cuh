@@ -24,12 +24,14 @@ constexpr int PAIR_BM = 256;                 // rows per pair tile
 constexpr int PAIR_STAGES = 6;
 constexpr int PAIR_A_BYTES = 128 * GEMM_BK * 2;   // 16 KB per CTA
 constexpr int PAIR_B_BYTES = 128 * GEMM_BK * 2;   // 16 KB per CTA
-constexpr int PAIR_SMEM_BYTES = PAIR_STAGES * (PAIR_A_BYTES + PAIR_B_BYTES) + 1024 + 256;
 // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue: two warps per TMEM lane quarter, each taking half
 // of the accumulator's columns, so that the epilogue of one tile stays shorter than the next
 // tile's MMAs even at the fp8 rate (twice the bf16 K per cycle).
 constexpr int PAIR_EPI_WARPS = 8;
 constexpr int PAIR_THREADS = 64 + 32 * PAIR_EPI_WARPS;
+constexpr int PAIR_STAGE_OUT_BYTES = 2048;        // per epilogue warp: 32 rows x 32 bf16
+constexpr int PAIR_SMEM_BYTES =
+    PAIR_STAGES * (PAIR_A_BYTES + PAIR_B_BYTES) + PAIR_EPI_WARPS * PAIR_STAGE_OUT_BYTES + 1024 + 256;
 
 // Tile walk with 256-row m-tiles (mprefix counts 256-row tiles per group).
 __device__ __forceinline__ int pair_total_tiles(const GemmParams& p, int& routed_tiles) {
@@ -95,7 +97,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + PAIR_STAGES * PAIR_A_BYTES;
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sB + PAIR_STAGES * PAIR_B_BYTES);
+    uint8_t* sOut = sB + PAIR_STAGES * PAIR_B_BYTES;   // epilogue staging, one 2 KB slot per warp
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(sOut + PAIR_EPI_WARPS * PAIR_STAGE_OUT_BYTES);
     uint64_t* empty_bar = full_bar + PAIR_STAGES;
     uint64_t* tfull_bar = empty_bar + PAIR_STAGES;
     uint64_t* tempty_bar = tfull_bar + 2;
@@ -236,6 +239,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
         const int half = (warp - 2) >> 2;         // which half of the columns it converts
         const int row_in_cta = sub * 32 + lane;
         const uint32_t tempty_leader0 = map_to_cta(tempty_bar, 0);
+        uint4* stage = reinterpret_cast<uint4*>(sOut + (warp - 2) * PAIR_STAGE_OUT_BYTES);
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = pair_id; t < total; t += npairs) {
@@ -248,7 +252,9 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
             const int row_in_tile = (int)rank * 128 + row_in_cta;
             const long long orow = c.out_row0 + ti.a_row + row_in_tile;
             const bool row_ok = row_in_tile < ti.rows && orow >= 0 && orow < c.out_rows;
-            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(c.out) + orow * c.ldo;
+            // the warp's 32 rows are consecutive: out0 is its first row, valid has a bit per row
+            __nv_bfloat16* out0 = reinterpret_cast<__nv_bfloat16*>(c.out) + (orow - lane) * c.ldo;
+            const uint32_t valid = __ballot_sync(0xffffffffu, row_ok);
             float sa = 1.f;                        // fp8: activation row scale, weight column scales
             const float *sb = nullptr, *sb2 = nullptr;
             if (F8) {
@@ -266,12 +272,14 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                     tmem_ld_32cols(tbase + 128 + ch * 32, u);
                     tmem_ld_wait();
                     const int col0 = ti.n_idx * 128 + ch * 32;
-                    if (row_ok && col0 < c.n_out) {
+                    if (valid && col0 < c.n_out) {        // warp-uniform
                         if (F8) {
                             scale_cols32(g, sa, sb + col0);
                             scale_cols32(u, sa, sb2 + col0);
                         }
-                        swiglu_store32(g, u, out + col0);
+                        uint32_t packed[16];
+                        swiglu_pack32(g, u, packed);
+                        store_rows_staged(packed, stage, lane, out0 + col0, c.ldo, valid);
                     }
                 }
             } else {
@@ -282,9 +290,11 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                     tmem_ld_32cols(tbase + ch * 32, v);
                     tmem_ld_wait();
                     const int col0 = ti.n_idx * 256 + ch * 32;
-                    if (row_ok && col0 < c.n_out) {
+                    if (valid && col0 < c.n_out) {        // warp-uniform
                         if (F8) scale_cols32(v, sa, sb + col0);
-                        store32(v, out + col0);
+                        uint32_t packed[16];
+                        pack32(v, packed);
+                        store_rows_staged(packed, stage, lane, out0 + col0, c.ldo, valid);
                     }
                 }
             }
