@@ -468,6 +468,14 @@ int moe_workspace_layout(int T, int d, int E, int k, int f, int f_shared, size_t
  */
 int moe_get_error(moe_stream_t stream);
 
+/*
+ * Failure-detection self-test: enqueues one kernel whose single bounded wait on an mbarrier
+ * can never be satisfied.  After the wait limit (2 s) the kernel records MOE_ERR_TIMEOUT in the
+ * device error word and returns; the next moe_get_error() reports it and the device stays
+ * usable.  Returns the host launch status.
+ */
+int moe_selftest_wait_timeout(moe_stream_t stream);
+
 /* Static text for a status code. */
 const char* moe_strerror(int code);
 

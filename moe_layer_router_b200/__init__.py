@@ -120,6 +120,8 @@ for _n in ("moe_pipeline_bytes", "moe_pipeline_create", "moe_pipeline_submit", "
 _lib.moe_update_bias.argtypes = [_vp, _i32, _i64, _vp, _vp]
 _lib.moe_update_bias.restype = _i32
 _lib.moe_get_error.argtypes = [_vp]
+_lib.moe_selftest_wait_timeout.argtypes = [_vp]
+_lib.moe_selftest_wait_timeout.restype = _i32
 _lib.moe_strerror.argtypes = [_i32]
 _lib.moe_strerror.restype = ctypes.c_char_p
 for _n in ("moe_workspace_bytes", "moe_workspace_layout", "moe_route", "moe_permute", "moe_expert_ffn",
@@ -458,6 +460,11 @@ def moe_layer_forward_w8a8(x, Wg, bias, W1q, s1, W3q, s3, W2q, s2, W1sq, s1s, W3
 
 def moe_get_error(stream=None) -> int:
     return int(_lib.moe_get_error(_stream(stream)))
+
+
+def moe_selftest_wait_timeout(stream=None) -> None:
+    """Enqueue the bounded-wait self-test (about 2 s; MOE_ERR_TIMEOUT in the error word)."""
+    _check(_lib.moe_selftest_wait_timeout(_stream(stream)), "moe_selftest_wait_timeout")
 
 
 def workspace_view(ws, layout: dict, name: str, shape, dtype):

@@ -1382,6 +1382,11 @@ int moe_update_bias(const int32_t* counts_raw, int E, int64_t capacity, float* b
     return launch_status();
 }
 
+int moe_selftest_wait_timeout(moe_stream_t stream) {
+    wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+    return launch_status();
+}
+
 int moe_get_error(moe_stream_t stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int v = 0;

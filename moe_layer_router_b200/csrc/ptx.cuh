@@ -82,6 +82,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// Failure-detection self-test: one thread waits on an mbarrier whose phase nothing completes.
+// The bounded wait gives up after kWaitLimitNs, records MOE_ERR_TIMEOUT and the kernel returns,
+// leaving the context usable.
+__global__ void wait_selftest_kernel() {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    mbar_wait(&bar, 0, nullptr);   // no arrival will come
+}
+
 // ---------------------------------------------------------------- TMA
 
 // 2-D tiled bulk tensor load global -> shared, completion counted on `bar` (bytes).
