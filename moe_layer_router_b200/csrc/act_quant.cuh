@@ -3,7 +3,12 @@
 // Every activation row is quantised on its own ([EP-DS3] deployment section, w4afp8: low-bit
 // weights with fp8 activations): s = amax(|x|) / 448 in fp32 (1 for an all-zero row), and each
 // element becomes e4m3(fp32(x) / s), rounded to nearest even and saturating at 448 (the
-// hardware conversion with .satfinite).  One warp per row; 16-byte loads, 8-byte stores.
+// hardware conversion with .satfinite).  Two kernels apply it:
+//   quant_rows_e4m3_kernel      a warp per row in two passes over the row (amax, then codes);
+//                               28 registers, so many warps hide the divisions' latency
+//   quant_rows_e4m3_reg_kernel  the row held in registers (read once), and optionally written
+//                               to several destination rows (a token's k permuted rows)
+// 16-byte loads, 8-byte stores.
 #pragma once
 
 #include <cuda_fp8.h>
