@@ -13,7 +13,8 @@
 //     every epilogue thread of both CTAs (eight warps each) arrives on the leader's
 //     accumulator-empty barrier.
 // Per SM this halves the B operand traffic of a 1-SM M = 128 tile and leaves room for a
-// 6-stage ring (A 16 KB + B 16 KB per stage per CTA).
+// 6-stage ring (A 16 KB + B 16 KB per stage per CTA) and 16 KB of epilogue staging, through
+// which each epilogue warp stores whole 64-byte pieces of 8 output rows at a time.
 #pragma once
 
 #include "grouped_gemm.cuh"
