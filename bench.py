@@ -53,6 +53,7 @@ DESCR = {
     "mixtral2e": "profiling case: Mixtral-like layer cut to T=2048, E=2 (same tile shapes)",
     "dsv3_32e": "profiling case: DeepSeek-V3-like decode cut to T=32, E=32 (same tile shapes)",
     "qwen3_16e": "profiling case: Qwen3-like prefill cut to T=2048, E=16 (same tile shapes)",
+    "qwen3_f128": "profiling case: Qwen3-like batch and routing (T=16384 E=128 top-8) with experts cut to f=128",
 }
 
 
@@ -75,6 +76,9 @@ def parse():
                     help="> 0: expert parallelism with this many ranks emulated on one GPU (the workload's batch "
                          "split over the ranks, experts split contiguously); prints its own line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="at N=1 with bf16 weights the line also carries per_config: every workload of the "
+                         "task timed in the same run (tokens/s, roofline, oracle sample); this skips it")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
 
@@ -196,9 +200,10 @@ def sample_size(oracle, wl, inp, w, seconds):
     return max(1, min(wl.T, S)), dt, s0
 
 
-def cpu_baseline(wl, seconds):
+def cpu_baseline(wl, seconds, inp=None, w=None):
     import oracle
-    inp, w = host_weights(wl)
+    if inp is None:
+        inp, w = host_weights(wl)
     S, _, _ = sample_size(oracle, wl, inp, w, seconds)
     dt = oracle_step(oracle, wl, inp, w, 0, S)
     if dt < 0.6 * seconds and S < wl.T:          # parallel efficiency grows with the sample: rescale once
@@ -273,6 +278,133 @@ def layer_work(wl, N, touched, wbytes=2):
     return flops, b
 
 
+def roofline_and_layer(wl, N, touched, counts, craw, gemm_ms, step_ms, fp8, a8, peaks, peak_src):
+    """The dominant kernel's roofline (GEMM1: tensor-bound for prefill, HBM-bound for decode) and
+    the layer's totals for one timed configuration.  gemm_ms: mean kernel times of the two grouped
+    GEMMs; step_ms: mean layer time."""
+    T, k, E = wl.T, wl.k, wl.E
+    g1_ms = gemm_ms["gate_up"]
+    decode = wl.name.startswith("dsv3")
+    tc_ratio = 2.0 if a8 else 1.0     # fp8 tensor peak = measured bf16 peak x the nominal 4.5 / 2.25
+    if decode:
+        alg = gemm1_bytes(wl, N, touched, 1 if fp8 else 2, 1 if a8 else 2)
+        achieved = alg / (g1_ms / 1000.0) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    else:
+        alg = gemm1_work(wl, N)
+        achieved = alg / (g1_ms / 1000.0) / 1e12
+        roof = {"bound": "latency" if wl.name == "tiny" else "tensor", "achieved": achieved,
+                "peak": peaks["bf16_tflops"] * tc_ratio, "unit": "TFLOP/s",
+                "frac": achieved / (peaks["bf16_tflops"] * tc_ratio)}
+        # the same achieved rate against the power-capped sustained GEMM rate, for context
+        roof["frac_of_sustained"] = achieved / (peaks["bf16_tflops_sustained"] * tc_ratio)
+    roof["traffic"] = recorded_traffic("gate_up" + ("_fp8a8" if a8 else "_fp8" if fp8 else ""), wl.name)
+    pair = T * k >= 256 * E
+    roof["kernel"] = (("grouped_gemm_pair_kernel" if pair else "grouped_gemm_kernel") + "<EPI_SWIGLU, F8> (fp8 x fp8)"
+                      if a8 else
+                      "grouped_gemm_w8_kernel<EPI_SWIGLU>" if fp8 else
+                      "grouped_gemm_pair_kernel<EPI_SWIGLU>" if pair else "grouped_gemm_kernel<EPI_SWIGLU>") + \
+        " (gate_up: W1/W3 + SwiGLU)"
+    roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if decode else 'bf16_tflops'}, burst)" + \
+        ("" if decode or not a8 else " x 2 (nominal fp8 / bf16 dense ratio)")
+    roof["algorithmic_per_launch"] = alg
+    lf, lb = layer_work(wl, N, touched, 1 if fp8 else 2)
+    step_s = step_ms / 1000.0
+    layer = {"tflops": lf / step_s / 1e12, "gbs": lb / step_s / 1e9,
+             # both grouped GEMMs' FLOPs over their kernel times, against the tensor peak
+             # of their operand type (bf16, or fp8 = measured bf16 x 2)
+             "gemms_tensor_frac": gemms_work(wl, N) / ((gemm_ms["gate_up"] + gemm_ms["down"]) / 1e3) / 1e12
+             / (peaks["bf16_tflops"] * tc_ratio),
+             "tensor_frac": lf / step_s / 1e12 / peaks["bf16_tflops"],
+             "hbm_frac": lb / step_s / 1e9 / peaks["hbm_gbs"], "kept_rows": N, "touched_experts": touched,
+             "drop_rate": 1.0 - N / float(T * k), "load_var_raw": float(np.var(craw)),
+             "load_var_kept": float(np.var(counts)), "max_rows": int(counts.max()),
+             "min_rows": int(counts.min())}
+    if wl.zipf_s > 0:
+        p = craw / craw.sum()
+        layer["zipf_l1_error"] = float(np.abs(p - synth.Inputs(wl).zipf_target()).sum())
+    return roof, layer
+
+
+
+PER_CONFIG_STEPS = {"tiny": 50, "mixtral": 20, "qwen3": 20, "dsv3": 20, "skew": 20}
+
+
+def config_entry(wl, value, ms_per_step, steps, roof, layer, stage_ms, gemm_ms, clocks, cpu):
+    """One workload's record in per_config."""
+    r = {k: roof[k] for k in ("bound", "kernel", "achieved", "unit", "peak", "frac", "peak_source")}
+    if "frac_of_sustained" in roof:
+        r["frac_of_sustained"] = roof["frac_of_sustained"]
+    e = {"workload": DESCR[wl.name], "tokens_per_s": value, "ms_per_step": ms_per_step, "steps": steps,
+         "roofline": r, "gemms_tensor_frac": layer["gemms_tensor_frac"], "tensor_frac": layer["tensor_frac"],
+         "hbm_frac": layer["hbm_frac"], "kept_rows": layer["kept_rows"], "drop_rate": layer["drop_rate"],
+         "load_var_raw": layer["load_var_raw"], "load_var_kept": layer["load_var_kept"],
+         "stages_ms": stage_ms, "gemm_ms": gemm_ms, "clocks": clocks, "cpu_baseline": cpu}
+    if "zipf_l1_error" in layer:
+        e["zipf_l1_error"] = layer["zipf_l1_error"]
+    return e
+
+
+def measure_config(name, dev, warmup, peaks, peak_src, cpu_seconds):
+    """Time one workload at N = 1 (bf16 weights; inputs resident in HBM), and the oracle on a sample
+    of it, for per_config.  The host copy of the weights serves both."""
+    import torch
+    import moe_layer_router_b200 as moe
+
+    wl = synth.WORKLOADS[name]
+    T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
+    inp, w = host_weights(wl)
+    dv = lambda a: None if a is None else \
+        torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    W = {n: dv(w[n]) for n in ("wg", "w1", "w3", "w2", "w1s", "w3s", "w2s")}
+    bias = None if w["bias"] is None else torch.from_numpy(w["bias"]).to(dev)
+    x = dv(inp.x())
+    ws = torch.empty(moe.moe_workspace_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device=dev)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+
+    def fwd(events=None):
+        moe.moe_layer_forward_ex(x, W["wg"], bias, W["w1"], W["w3"], W["w2"], W["w1s"], W["w3s"], W["w2s"], fs,
+                                 T, d, E, k, f, wl.capacity_factor, wl.cap_mode, out, ws, events)
+
+    for _ in range(max(3, warmup)):
+        fwd()
+    torch.cuda.synchronize()
+    rc = moe.moe_get_error()
+    if rc != 0:
+        raise RuntimeError(f"{name}: device error after warm-up: {moe.strerror(rc)}")
+    K = PER_CONFIG_STEPS[name]
+    evs = [{n: torch.cuda.Event(enable_timing=True) for n in moe.STAGES} for _ in range(K)]
+    for e in evs:
+        for ev in e.values():
+            ev.record()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        for i in range(K):
+            fwd(evs[i])
+        torch.cuda.synchronize()
+    rc = moe.moe_get_error()
+    if rc != 0:
+        raise RuntimeError(f"{name}: device error: {moe.strerror(rc)}")
+    total_ms = evs[0]["route"].elapsed_time(evs[K - 1]["end"])
+    stage_ms = {a: float(np.mean([e[a].elapsed_time(e[b]) for e in evs]))
+                for a, b in zip(moe.STAGES[:-1], moe.STAGES[1:])}
+    gemm_ms = {"gate_up": stage_ms["gate_up"], "down": stage_ms["down"]}
+    L = moe.moe_workspace_layout(T, d, E, k, f, fs)
+    counts = moe.workspace_view(ws, L, "counts", (E,), torch.int32).cpu().numpy()
+    craw = moe.workspace_view(ws, L, "counts_raw", (E,), torch.int32).cpu().numpy()
+    N = int(counts.sum())
+    touched = int((counts > 0).sum())
+    roof, layer = roofline_and_layer(wl, N, touched, counts, craw, gemm_ms, total_ms / K, False, False, peaks,
+                                     peak_src)
+    del W, bias, x, ws, out
+    torch.cuda.empty_cache()
+    cpu = cpu_baseline(wl, cpu_seconds, inp, w) if cpu_seconds > 0 else None
+    return config_entry(wl, T * K / (total_ms / 1e3), total_ms / K, K, roof, layer, stage_ms, gemm_ms,
+                        clk.summary(), cpu)
+
+
+
 def run_cached(args, base, rank, world, local):
     """Decode with the routed experts in page-locked host memory and an LRU of S HBM slots.
 
@@ -342,7 +474,7 @@ def run_cached(args, base, rank, world, local):
         raise RuntimeError("device error after warm-up")
     c0 = moe.cache_counters(state)
     K = args.steps
-    names = moe.STAGES + ["cache"]
+    names = moe.STAGES + ["cache", "copy_start", "copy_end"]
     evs = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(K)]
     for e in evs:
         for ev in e.values():
@@ -362,7 +494,8 @@ def run_cached(args, base, rank, world, local):
     c1 = moe.cache_counters(state)
     expert_bytes = 3 * f * d + 4 * (2 * f + d) if fp8 else 3 * f * d * 2
     hits, misses = c1["hits"] - c0["hits"], c1["misses"] - c0["misses"]
-    copy_ms = sum(e["cache"].elapsed_time(e["gate_up"]) for e in evs)   # plan + copy kernels, all steps
+    # the copy kernel on the cache's copy stream (it overlaps the resident experts' GEMMs)
+    copy_ms = sum(e["copy_start"].elapsed_time(e["copy_end"]) for e in evs)
     link_gbs = misses * expert_bytes / 1e9 / (copy_ms / 1e3)
     # end to end: every step copies its tokens from page-locked host memory and its output back
     x_pin = xs.cpu().pin_memory()
@@ -414,7 +547,8 @@ def run_cached(args, base, rank, world, local):
                      "peak_source": "measured in this run (cudaMemcpyAsync page-locked -> device, 1 GiB x 5)",
                      "algorithmic_per_launch": misses / K * expert_bytes},
         "cache": {"hits": hits, "misses": misses, "hit_rate": hits / max(1, hits + misses),
-                  "loads_per_step": misses / K, "expert_mb": expert_bytes / 1e6},
+                  "loads_per_step": misses / K, "expert_mb": expert_bytes / 1e6,
+                  "copy_ms_per_step": copy_ms / K, "step_over_copy": total_ms / max(copy_ms, 1e-9)},
         "stages_ms": stage_ms,
         "e2e": {"value": dp.job_throughput(T, world, K, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
                 "d2h_bytes_per_step": T * d * 2},
@@ -612,40 +746,34 @@ def main():
     # neighbouring batches overlap the layer); timed from the first copy in to the last copy out
     x_pin = x_host.pin_memory()
     out_pin = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
-    if fp8:   # the pipeline object takes bf16 weights: copies around each call on one stream
-        x_e2e = torch.empty_like(x)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        e0.record()
-        for _ in range(K):
-            x_e2e.copy_(x_pin, non_blocking=True)
-            fwd(x_e2e, out)
-            out_pin.copy_(out, non_blocking=True)
-        e1.record()
-        torch.cuda.synchronize()
-        return_e2e = dp.max_over_ranks(e0.elapsed_time(e1), device=dev)
-    pmem = torch.empty(0 if fp8 else moe.moe_pipeline_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device=dev)
     if fp8:
-        e2e_ms = return_e2e
+        routed = {n: W[w] for n, w in (("W1q", "w1q"), ("W3q", "w3q"), ("W2q", "w2q"), ("s1", "s1"), ("s3", "s3"),
+                                       ("s2", "s2"))}
+        shared = {n: W[w] for n, w in (("W1q", "w1sq"), ("W3q", "w3sq"), ("W2q", "w2sq"), ("s1", "s1s"),
+                                       ("s3", "s3s"), ("s2", "s2s"))} if fs else None
+        pmem = torch.empty(moe.moe_pipeline_bytes_w8(T, d, E, k, f, fs, a8), dtype=torch.uint8, device=dev)
+        pl = moe.Pipeline(W["wg"], W["bias"], None, None, None, None, None, None, fs, T, d, E, k, f,
+                          wl.capacity_factor, wl.cap_mode, pmem, routed=routed, shared=shared, activations_fp8=a8)
     else:
+        pmem = torch.empty(moe.moe_pipeline_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device=dev)
         pl = moe.Pipeline(W["wg"], W["bias"], W["w1"], W["w3"], W["w2"], W.get("w1s"), W.get("w3s"), W.get("w2s"),
                           fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, pmem)
-        s_h2d, _, s_d2h = pl.streams()
-        for _ in range(3):
-            pl.submit(x_pin, out_pin)
-        pl.sync()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        e0.record(torch.cuda.ExternalStream(s_h2d))
-        for _ in range(K):
-            pl.submit(x_pin, out_pin)
-        e1.record(torch.cuda.ExternalStream(s_d2h))
-        pl.sync()
-        torch.cuda.synchronize()
-        pl.close()
-        e2e_ms = dp.max_over_ranks(e0.elapsed_time(e1), device=dev)
+    s_h2d, _, s_d2h = pl.streams()
+    for _ in range(3):
+        pl.submit(x_pin, out_pin)
+    pl.sync()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(torch.cuda.ExternalStream(s_h2d))
+    for _ in range(K):
+        pl.submit(x_pin, out_pin)
+    e1.record(torch.cuda.ExternalStream(s_d2h))
+    pl.sync()
+    torch.cuda.synchronize()
+    pl.close()
+    e2e_ms = dp.max_over_ranks(e0.elapsed_time(e1), device=dev)
     if world > 1:
         dist.barrier()
     e2e_value = dp.job_throughput(T, world, K, e2e_ms)
@@ -659,33 +787,8 @@ def main():
         return
 
     peaks, peak_src = load_peaks()
-    g1_ms = gemm_ms["gate_up"]
-    decode = wl.name.startswith("dsv3")
-    if decode:
-        alg = gemm1_bytes(wl, N, touched, 1 if fp8 else 2, 1 if a8 else 2)
-        achieved = alg / (g1_ms / 1000.0) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"]}
-    else:
-        tc_ratio = 2.0 if a8 else 1.0     # fp8 tensor peak = measured bf16 peak x the nominal 4.5 / 2.25
-        alg = gemm1_work(wl, N)
-        achieved = alg / (g1_ms / 1000.0) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"] * tc_ratio, "unit": "TFLOP/s",
-                "frac": achieved / (peaks["bf16_tflops"] * tc_ratio)}
-    if not decode:   # the same achieved rate against the power-capped sustained GEMM rate, for context
-        roof["frac_of_sustained"] = achieved / (peaks["bf16_tflops_sustained"] * tc_ratio)
-    roof["traffic"] = recorded_traffic("gate_up" + ("_fp8a8" if a8 else "_fp8" if fp8 else ""), wl.name)
-    pair = T * k >= 256 * E
-    roof["kernel"] = (("grouped_gemm_pair_kernel" if pair else "grouped_gemm_kernel") + "<EPI_SWIGLU, F8> (fp8 x fp8)"
-                      if a8 else
-                      "grouped_gemm_w8_kernel<EPI_SWIGLU>" if fp8 else
-                      "grouped_gemm_pair_kernel<EPI_SWIGLU>" if pair else "grouped_gemm_kernel<EPI_SWIGLU>") + \
-        " (gate_up: W1/W3 + SwiGLU)"
-    roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if decode else 'bf16_tflops'}, burst)" + \
-        ("" if decode or not a8 else " x 2 (nominal fp8 / bf16 dense ratio)")
-    roof["algorithmic_per_launch"] = alg
-    lf, lb = layer_work(wl, N, touched, 1 if fp8 else 2)
-    step_s = total_ms / K / 1000.0
+    roof, layer = roofline_and_layer(wl, N, touched, counts, craw, gemm_ms, total_ms / K, fp8, a8, peaks,
+                                     peak_src)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -696,16 +799,7 @@ def main():
                    "l2": "working set larger than L2 (expert weights %.2f GB per step)" % (
                        touched * 3.0 * f * d * 2 / 1e9)},
         "roofline": roof,
-        "layer": {"tflops": lf / step_s / 1e12, "gbs": lb / step_s / 1e9,
-                  # both grouped GEMMs' FLOPs over their kernel times, against the tensor peak
-                  # of their operand type (bf16, or fp8 = measured bf16 x 2)
-                  "gemms_tensor_frac": gemms_work(wl, N) / ((gemm_ms["gate_up"] + gemm_ms["down"]) / 1e3) / 1e12
-                  / (peaks["bf16_tflops"] * (2.0 if a8 else 1.0)),
-                  "tensor_frac": lf / step_s / 1e12 / peaks["bf16_tflops"],
-                  "hbm_frac": lb / step_s / 1e9 / peaks["hbm_gbs"], "kept_rows": N, "touched_experts": touched,
-                  "drop_rate": 1.0 - N / float(T * k), "load_var_raw": float(np.var(craw)),
-                  "load_var_kept": float(np.var(counts)), "max_rows": int(counts.max()),
-                  "min_rows": int(counts.min())},
+        "layer": layer,
         "stages_ms": stage_ms,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
                 "d2h_bytes_per_step": T * d * 2},
@@ -713,11 +807,21 @@ def main():
         "gpu_launches": launches_per_step(a8, wl.has_shared) * K,
         "clocks": clk.summary(),
     }
-    if wl.zipf_s > 0:
-        p = craw / craw.sum()
-        line["layer"]["zipf_l1_error"] = float(np.abs(p - inp.zipf_target()).sum())
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    if world == 1 and args.weights == "bf16" and not args.no_per_config and wl.name in synth.WORKLOAD_ORDER:
+        # every workload of the task in the same run, one after the other on this GPU
+        del W, tensors, x, ws, out, pmem
+        torch.cuda.empty_cache()
+        per = {}
+        for name in synth.WORKLOAD_ORDER:
+            if name == wl.name:
+                per[name] = config_entry(wl, value, total_ms / K, K, roof, layer, stage_ms, gemm_ms, line["clocks"],
+                                         line.get("cpu_baseline"))
+            else:
+                per[name] = measure_config(name, dev, 3, peaks, peak_src,
+                                           0.0 if args.no_cpu_baseline else min(args.cpu_seconds, 6.0))
+        line["per_config"] = per
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

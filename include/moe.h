@@ -121,7 +121,10 @@ int moe_permute(const moe_bf16* x, const int32_t* idx, int T, int d, int E, int 
  *   - Sizes whose scratch, ceil(T/256)*E*4 + T*k*4 + (E+1)*4 bytes (each part rounded up
  *     to 256), exceeds MOE_NOALLOC_SCRATCH_BYTES return MOE_ERR_WORKSPACE; nothing runs.
  *   - The first call on a device, with that device current, looks up the array's device
- *     address (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     address (cudaGetSymbolAddress) and keeps it for the life of the process; make that
+ *     first call before any stream capture.  A cudaDeviceReset() (or anything else that
+ *     tears down the device's primary context) makes the kept address stale: do not call
+ *     this entry point on that device again in the same process.
  *   - Calls on one device share the array: calls whose kernels overlap on the GPU race.
  *   - Allocates and frees nothing.
  */
@@ -187,6 +190,8 @@ typedef struct moe_stage_events {
     void* cache;     /* before the expert cache plan / copy kernels (moe_layer_forward_cached only) */
     void* gemm1;     /* fp8-activation layers: after quantising GEMM1's rows, before its kernel */
     void* gemm2;     /* fp8-activation layers: after quantising h, before GEMM2's kernel */
+    void* copy_start;  /* cached layers: before the expert copy kernel, on the copy stream */
+    void* copy_end;    /* cached layers: after the expert copy kernel, on the copy stream */
 } moe_stage_events;
 
 /* moe_layer_forward() with optional stage markers (events may be NULL). */
@@ -337,6 +342,14 @@ int moe_layer_permute(const moe_bf16* x, int f_shared, int T, int d, int E, int 
  * moe_ep_expert_ffn: source_major = 0 after moe_ep_dispatch(), 1 after an all-to-all-v.
  */
 int moe_ep_workspace_bytes(int R, int E, size_t* bytes);
+/*
+ * Byte offset inside ep_ws of the split table moe_ep_plan() writes: int32 [2, R], row 0 = rows
+ * this rank sends to each rank q (its kept rows of q's experts), row 1 = rows it receives from
+ * each rank s (s's kept rows of this rank's experts).  These are the split sizes of the two
+ * all-to-all-v exchanges (dispatch: send / receive; return: the same rows swapped), computed on
+ * the device with the rest of the plan.  MOE_ERR_SHAPE as for moe_ep_workspace_bytes().
+ */
+int moe_ep_splits_offset(int R, int E, size_t* offset);
 int moe_ep_plan(const int32_t* all_counts_raw, int R, int rank, int E, int64_t capacity, int max_recv_rows,
                 void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream);
 int moe_ep_dispatch(const moe_bf16* x_perm, int R, int rank, int E, int d, moe_bf16* const* recv_bufs,
@@ -349,6 +362,28 @@ int moe_ep_expert_ffn(const moe_bf16* recv_x, int max_recv_rows, int source_majo
                       size_t ep_ws_bytes, moe_stream_t stream);
 int moe_ep_return(const moe_bf16* y_recv, int R, int rank, int E, int d, moe_bf16* const* y_perm_bufs,
                   const void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream);
+
+/*
+ * Peer buffers for the put exchange with one process per GPU ([EP-KV] section 7: point-to-point
+ * copies into the other ranks' memory).  Each rank exports its receive buffer and its y_perm,
+ * the ranks exchange the handles (any host channel: the caller's collective library), and each
+ * rank imports the others' handles to get device addresses its put kernels can store to
+ * (plain peer stores over NVLink; nothing else reads another GPU's memory).
+ *   moe_ipc_export(ptr, handle)   handle: MOE_IPC_HANDLE_BYTES bytes (host) describing the device
+ *                                 allocation that holds ptr and ptr's offset in it
+ *   moe_ipc_import(handle, &ptr)  maps another process's exported allocation into this process
+ *                                 (cudaIpcOpenMemHandle, peer access enabled lazily) and returns
+ *                                 the address of the exported pointer; a process uses its own
+ *                                 pointers for its own buffers (CUDA IPC maps other processes')
+ *   moe_ipc_close(ptr, handle)    unmaps what moe_ipc_import returned for that handle
+ * The exporter must keep the allocation alive until every importer has closed it.  Errors:
+ * MOE_ERR_INVALID_ARG (null arguments, a pointer that is not device memory, a foreign blob),
+ * MOE_ERR_CUDA (the runtime refused the export, import or close).  Synchronous host calls.
+ */
+#define MOE_IPC_HANDLE_BYTES 96
+int moe_ipc_export(const void* ptr, void* handle);
+int moe_ipc_import(const void* handle, void** ptr);
+int moe_ipc_close(void* ptr, const void* handle);
 
 /*
  * The layer with fp8 e4m3 weights AND fp8 activations: the weights as in moe_layer_forward_w8();
@@ -413,7 +448,12 @@ int moe_cache_reset(void* cache_state, int E, int S, moe_stream_t stream);
  *   S: slots; must be >= min(E, T*k) so that one batch always fits (else MOE_ERR_SHAPE).
  * Per batch, after the counts: the plan kernel updates the state and lists the loads, the copy
  * kernel brings those experts into their slots, the grouped GEMMs read expert e from slot
- * slot_of[e].  The output is the same as moe_layer_forward() with W1/W3/W2 = the sources.
+ * slot_of[e].  The copy overlaps compute ([EP-DS3] section 3.2): it runs on a copy stream of the
+ * library's own (one per device, created on first use), forked from `stream` after the plan;
+ * meanwhile both grouped GEMMs run on `stream` over the experts that were already resident (and
+ * the shared expert), then `stream` waits for the copy and the GEMMs run over the loaded ones.
+ * Cached-layer calls on one device share that copy stream, so their copies run one after
+ * another.  The output is the same as moe_layer_forward() with W1/W3/W2 = the sources.
  * Device-side failure (a batch that needs more than S experts) sets MOE_ERR_CHECK.
  */
 int moe_layer_forward_cached(const moe_bf16* x, const moe_bf16* Wg, const float* bias,
@@ -448,6 +488,21 @@ int moe_layer_forward_cached_w8(const moe_bf16* x, const moe_bf16* Wg, const flo
                                 int f_shared, int T, int d, int E, int k, int f, double capacity_factor, int cap_mode,
                                 moe_bf16* out, void* ws, size_t ws_bytes, moe_stream_t stream,
                                 const moe_stage_events* events);
+
+/*
+ * The host-buffer pipeline (moe_pipeline_*) over the fp8 layers: the same two device slots,
+ * three streams and overlapped copies, with moe_layer_forward_w8() (activations_fp8 = 0) or
+ * moe_layer_forward_w8a8() (activations_fp8 = 1) as the layer.  params gives the router (Wg,
+ * bias), the shapes and the capacity; its W1..W2s are ignored.  routed / shared: the fp8 codes
+ * and row scales (shared may be NULL when f_shared == 0).  moe_pipeline_bytes_w8(): device
+ * memory to pass (2 input + 2 output slots and that layer's workspace).  submit, sync, streams
+ * and destroy are the moe_pipeline_* calls above.  Errors as moe_pipeline_create(), plus
+ * MOE_ERR_INVALID_ARG for missing fp8 arrays; shapes are checked by the layer at submit.
+ */
+int moe_pipeline_bytes_w8(int T, int d, int E, int k, int f, int f_shared, int activations_fp8, size_t* bytes);
+int moe_pipeline_create_w8(const moe_pipeline_params* params, const moe_w8_experts* routed,
+                           const moe_w8_experts* shared, int activations_fp8, void* dev_mem, size_t dev_bytes,
+                           moe_pipeline** out);
 
 /*
  * Byte offsets of the intermediates that moe_layer_forward() leaves in its workspace,

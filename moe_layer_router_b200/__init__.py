@@ -101,6 +101,15 @@ _lib.moe_ep_expert_ffn.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32
 _lib.moe_ep_expert_ffn.restype = _i32
 _lib.moe_ep_return.argtypes = [_vp, _i32, _i32, _i32, _i32, ctypes.POINTER(_vp), _vp, _sz, _vp]
 _lib.moe_ep_return.restype = _i32
+_lib.moe_ep_splits_offset.argtypes = [_i32, _i32, ctypes.POINTER(_sz)]
+_lib.moe_ep_splits_offset.restype = _i32
+_lib.moe_ipc_export.argtypes = [_vp, _vp]
+_lib.moe_ipc_export.restype = _i32
+_lib.moe_ipc_import.argtypes = [_vp, ctypes.POINTER(_vp)]
+_lib.moe_ipc_import.restype = _i32
+_lib.moe_ipc_close.argtypes = [_vp, _vp]
+_lib.moe_ipc_close.restype = _i32
+MOE_IPC_HANDLE_BYTES = 96
 _lib.moe_layer_route_count.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _sz, _vp]
 _lib.moe_layer_route_count.restype = _i32
 _lib.moe_fill_base.argtypes = [_vp, _i32, _i32, _i32, _vp, _vp]
@@ -114,8 +123,11 @@ _lib.moe_pipeline_submit.argtypes = [_vp, _vp, _vp]
 _lib.moe_pipeline_sync.argtypes = [_vp]
 _lib.moe_pipeline_streams.argtypes = [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp)]
 _lib.moe_pipeline_destroy.argtypes = [_vp]
+_lib.moe_pipeline_bytes_w8.argtypes = [_i32, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(_sz)]
+_lib.moe_pipeline_create_w8.argtypes = [_vp, ctypes.POINTER(moe_w8_experts), ctypes.POINTER(moe_w8_experts), _i32,
+                                        _vp, _sz, ctypes.POINTER(_vp)]
 for _n in ("moe_pipeline_bytes", "moe_pipeline_create", "moe_pipeline_submit", "moe_pipeline_sync",
-           "moe_pipeline_streams", "moe_pipeline_destroy"):
+           "moe_pipeline_streams", "moe_pipeline_destroy", "moe_pipeline_bytes_w8", "moe_pipeline_create_w8"):
     getattr(_lib, _n).restype = _i32
 _lib.moe_update_bias.argtypes = [_vp, _i32, _i64, _vp, _vp]
 _lib.moe_update_bias.restype = _i32
@@ -227,7 +239,7 @@ STAGES = ["route", "topk", "permute", "gate_up", "down", "combine", "end"]   # t
 # struct order; "cache" marks the expert cache kernels (between "permute" and "gate_up") in
 # moe_layer_forward_cached; "gemm1" / "gemm2" mark the grouped GEMM kernels themselves in the
 # fp8-activation layer (after the quantisation of their rows, inside "gate_up" / "down")
-_EVENT_FIELDS = STAGES + ["cache", "gemm1", "gemm2"]
+_EVENT_FIELDS = STAGES + ["cache", "gemm1", "gemm2", "copy_start", "copy_end"]
 
 
 class moe_stage_events(ctypes.Structure):
@@ -283,19 +295,35 @@ def moe_pipeline_bytes(T, d, E, k, f, f_shared=0) -> int:
     return int(out.value)
 
 
+def moe_pipeline_bytes_w8(T, d, E, k, f, f_shared=0, activations_fp8=False) -> int:
+    out = _sz(0)
+    _check(_lib.moe_pipeline_bytes_w8(T, d, E, k, f, f_shared, int(bool(activations_fp8)), ctypes.byref(out)),
+           "moe_pipeline_bytes_w8")
+    return int(out.value)
+
+
 class Pipeline:
     """moe_pipeline_* as an object: submit(x_host, out_host) per batch, sync() to wait.
-    dev_mem is a caller-owned device buffer of moe_pipeline_bytes() bytes; weights stay
-    referenced (keep the tensors alive)."""
+    dev_mem is a caller-owned device buffer of moe_pipeline_bytes() bytes (moe_pipeline_bytes_w8()
+    for fp8 experts); weights stay referenced (keep the tensors alive).  fp8: pass W1 = W3 = W2 =
+    None and routed (and, with a shared expert, shared) as dicts of W1q, W3q, W2q, s1, s3, s2
+    tensors; activations_fp8 selects moe_layer_forward_w8a8 over moe_layer_forward_w8."""
 
     def __init__(self, Wg, bias, W1, W3, W2, W1s, W3s, W2s, f_shared, T, d, E, k, f, capacity_factor, cap_mode,
-                 dev_mem):
-        self._keep = (Wg, bias, W1, W3, W2, W1s, W3s, W2s, dev_mem)
+                 dev_mem, routed: Optional[dict] = None, shared: Optional[dict] = None, activations_fp8=False):
+        self._keep = (Wg, bias, W1, W3, W2, W1s, W3s, W2s, dev_mem, routed, shared)
         self.params = moe_pipeline_params(_ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(W1s), _ptr(W3s), _ptr(W2s),
                                           _ptr(bias), T, d, E, k, f, f_shared, float(capacity_factor), cap_mode)
         h = _vp()
-        _check(_lib.moe_pipeline_create(ctypes.byref(self.params), _ptr(dev_mem), _nbytes(dev_mem), ctypes.byref(h)),
-               "moe_pipeline_create")
+        if routed is None:
+            _check(_lib.moe_pipeline_create(ctypes.byref(self.params), _ptr(dev_mem), _nbytes(dev_mem),
+                                            ctypes.byref(h)), "moe_pipeline_create")
+        else:
+            self._q, self._qs = _w8(routed), _w8(shared)
+            _check(_lib.moe_pipeline_create_w8(ctypes.byref(self.params), ctypes.byref(self._q),
+                                               ctypes.byref(self._qs) if self._qs is not None else None,
+                                               int(bool(activations_fp8)), _ptr(dev_mem), _nbytes(dev_mem),
+                                               ctypes.byref(h)), "moe_pipeline_create_w8")
         self.handle = h
 
     def submit(self, x_host, out_host) -> None:
@@ -437,6 +465,36 @@ def moe_ep_return(y_recv, R, rank, E, d, y_perm_bufs, ep_ws, stream=None) -> Non
     """y_perm_bufs: R tensors (or device addresses), rank s's y_perm (in its layer workspace)."""
     _check(_lib.moe_ep_return(_ptr(y_recv), R, rank, E, d, _addr_array(y_perm_bufs), _ptr(ep_ws), _nbytes(ep_ws),
                               _stream(stream)), "moe_ep_return")
+
+
+def moe_ep_splits(ep_ws, R: int, E: int):
+    """The [2, R] int32 split table moe_ep_plan wrote into ep_ws (a view, on the device): row 0 the
+    rows this rank sends to each rank, row 1 the rows it receives from each rank."""
+    import torch
+    off = _sz(0)
+    _check(_lib.moe_ep_splits_offset(R, E, ctypes.byref(off)), "moe_ep_splits_offset")
+    o = int(off.value)
+    return ep_ws[o:o + 8 * R].view(torch.int32).view(2, R)
+
+
+def moe_ipc_export(t) -> bytes:
+    """IPC handle (MOE_IPC_HANDLE_BYTES bytes) of the device allocation holding tensor t."""
+    buf = ctypes.create_string_buffer(MOE_IPC_HANDLE_BYTES)
+    _check(_lib.moe_ipc_export(_ptr(t), buf), "moe_ipc_export")
+    return buf.raw
+
+
+def moe_ipc_import(handle: bytes) -> int:
+    """Device address, in this process, of another process's exported pointer."""
+    if len(handle) != MOE_IPC_HANDLE_BYTES:
+        raise ValueError("IPC handle of the wrong size")
+    out = _vp(0)
+    _check(_lib.moe_ipc_import(handle, ctypes.byref(out)), "moe_ipc_import")
+    return int(out.value)
+
+
+def moe_ipc_close(addr: int, handle: bytes) -> None:
+    _check(_lib.moe_ipc_close(_vp(addr), handle), "moe_ipc_close")
 
 
 def moe_workspace_bytes_a8(T: int, d: int, E: int, k: int, f: int, f_shared: int = 0) -> int:

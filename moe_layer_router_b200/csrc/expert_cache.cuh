@@ -11,7 +11,11 @@
 //   cache_load_kernel   every SM streams the listed experts' weights (W1, W3, W2; or their fp8
 //                       codes and row scales) from page-locked host memory (read directly over
 //                       the host link) into their slots
-// The grouped GEMMs then read weight group slot_of[e] for routed group e.
+// The grouped GEMMs then read weight group slot_of[e] for routed group e.  The plan also splits
+// the GEMM tile prefix in two: tiles of experts that were resident before the batch (hits) and
+// tiles of the experts being loaded (misses), so the hits' GEMMs can run on the layer's stream
+// while the copy runs on a second stream, and only the misses' GEMMs wait for the copy
+// ([EP-DS3] section 3.2: load experts asynchronously on a CUDA stream, overlapped with compute).
 //
 // Pairing the r-th miss with the r-th candidate slot is the same as taking misses one at a time
 // and evicting the oldest candidate each time: a slot that receives a miss is stamped with the
@@ -70,9 +74,40 @@ __global__ void __launch_bounds__(CACHE_MAX) cache_reset_kernel(CacheView v, int
     if (t < 8) reinterpret_cast<long long*>(v.ctr)[t] = 0;
 }
 
+// Exclusive scan over the block (blockDim.x = CACHE_MAX) of one value per thread; the total
+// goes to *total.  s_warp: CACHE_MAX / 32 ints of shared memory.
+__device__ __forceinline__ int cache_block_exscan(int x, int* s_warp, int* total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int v = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+    }
+    __syncthreads();                 // s_warp free from any earlier use
+    if (lane == 31) s_warp[wid] = v;
+    __syncthreads();
+    if (wid == 0) {
+        int w = s_warp[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        s_warp[lane] = w;            // inclusive over warps
+    }
+    __syncthreads();
+    const int pre = (wid ? s_warp[wid - 1] : 0) + v - x;
+    *total = s_warp[CACHE_MAX / 32 - 1];
+    return pre;
+}
+
 // counts[e] = rows routed to expert e and kept (after capacity); an expert is needed iff > 0.
+// tile_rows: rows per m-tile of the expert GEMMs; mp_hit / mp_miss [E+1]: m-tile prefixes over the
+// experts that were resident before this batch / are loaded by it (the other experts count 0).
 __global__ void __launch_bounds__(CACHE_MAX) cache_plan_kernel(const int32_t* __restrict__ counts, int E, int S,
-                                                               CacheView v) {
+                                                               CacheView v, int tile_rows, int32_t* mp_hit,
+                                                               int32_t* mp_miss) {
     __shared__ int s_stamp[CACHE_MAX];
     __shared__ int s_old[CACHE_MAX];      // expert_in before this batch
     __shared__ int s_cand[CACHE_MAX];     // candidate rank -> slot
@@ -129,7 +164,24 @@ __global__ void __launch_bounds__(CACHE_MAX) cache_plan_kernel(const int32_t* __
             v.ctr->loads_last = 0;
             record_error(-7 /* MOE_ERR_CHECK */);
         }
+        if (t <= E) {         // no GEMM tiles in either phase
+            mp_hit[t] = 0;
+            mp_miss[t] = 0;
+        }
         return;
+    }
+    // the tile prefixes of the two GEMM phases
+    const int tiles = need ? (counts[t] + tile_rows - 1) / tile_rows : 0;
+    int hit_total, miss_total;
+    const int hit_pre = cache_block_exscan(miss ? 0 : tiles, s_warp, &hit_total);
+    const int miss_pre = cache_block_exscan(miss ? tiles : 0, s_warp, &miss_total);
+    if (t < E) {
+        mp_hit[t] = hit_pre;
+        mp_miss[t] = miss_pre;
+    }
+    if (t == 0) {
+        mp_hit[E] = hit_total;
+        mp_miss[E] = miss_total;
     }
     if (miss) {
         const int vs = s_cand[miss_rank];

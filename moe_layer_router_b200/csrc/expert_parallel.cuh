@@ -39,11 +39,12 @@ struct EpView {
     int32_t* seg_off;     // [E + 1] source-major segment offsets (all-to-all-v layout)
     int32_t* seg_tiles;   // [E + 1] tile prefix of those segments
     int32_t* group_map;   // [E] segment g -> local expert g % El
+    int32_t* splits;      // [2, R]: rows this rank sends to rank q, rows it receives from rank s
 };
 
 inline size_t ep_pad(size_t b) { return (b + 255) & ~size_t(255); }
 
-inline size_t ep_layout_bytes(int R, int E, size_t off[8]) {
+inline size_t ep_layout_bytes(int R, int E, size_t off[9]) {
     const int El = E / R;
     size_t o = 0;
     off[0] = o; o += ep_pad((size_t)R * E * 4);
@@ -54,15 +55,16 @@ inline size_t ep_layout_bytes(int R, int E, size_t off[8]) {
     off[5] = o; o += ep_pad((size_t)(E + 1) * 4);
     off[6] = o; o += ep_pad((size_t)(E + 1) * 4);
     off[7] = o; o += ep_pad((size_t)E * 4);
+    off[8] = o; o += ep_pad((size_t)2 * R * 4);
     return o;
 }
 
 inline EpView ep_view(void* ws, int R, int E) {
-    size_t off[8];
+    size_t off[9];
     ep_layout_bytes(R, E, off);
     char* b = static_cast<char*>(ws);
     auto at = [&](int i) { return reinterpret_cast<int32_t*>(b + off[i]); };
-    return EpView{at(0), at(1), at(2), at(3), at(4), at(5), at(6), at(7)};
+    return EpView{at(0), at(1), at(2), at(3), at(4), at(5), at(6), at(7), at(8)};
 }
 
 // Block-wide exclusive scan of one value per thread (blockDim.x = 1024); returns the prefix and
@@ -150,10 +152,16 @@ __global__ void __launch_bounds__(1024) ep_plan_kernel(const int32_t* __restrict
     if (e < R) {                     // thread s: where my experts' rows sit in s's x_perm
         int pre = 0;
         for (int x = 0; x < rank * El; ++x) pre += v.kept[(long long)e * E + x];
+        int from = 0, to = 0;
         for (int j = 0; j < El; ++j) {
             v.back[2 * E + e * El + j] = pre;
             pre += v.kept[(long long)e * E + rank * El + j];
+            from += v.kept[(long long)e * E + rank * El + j];     // rank e's rows of my experts
+            to += v.kept[(long long)rank * E + e * El + j];       // my rows of rank e's experts
         }
+        // the split sizes of an all-to-all-v of the rows: what I send to / receive from rank e
+        v.splits[e] = to;
+        v.splits[R + e] = from;
     }
     __syncthreads();
     if (e == 0) {                    // tile prefixes of both layouts, and the source-major offsets

@@ -15,6 +15,18 @@
 // Per SM this halves the B operand traffic of a 1-SM M = 128 tile and leaves room for a
 // 6-stage ring (A 16 KB + B 16 KB per stage per CTA) and 16 KB of epilogue staging, through
 // which each epilogue warp stores whole 64-byte pieces of 8 output rows at a time.
+//
+// Swapped tail tiles.  A group's last m-tile usually holds fewer than 256 rows; as an M = 256
+// tile its MMAs would cost the same as a full one.  A tile of at most PAIR_SWAP_MAX_ROWS rows
+// instead runs with the operands swapped, D^T = W * X^T: the weights are the M = 256 side (each
+// CTA's 128 weight rows in the B slot of the stage) and the tile's tokens the N side (N = rows
+// rounded up to 16, each CTA loading its N / 2 token rows in 32-row boxes into the A slot), so
+// the MMA time follows the real row count.  TMEM then holds one weight row (output feature) per
+// lane and one token per column.  For GEMM1 each CTA loads 64 rows of W1 and the same 64 rows of
+// W3, so that a feature's gate (lanes 0-63) and up (lanes 64-127) values sit in the same CTA: the
+// warps of lanes 64-127 pass their up values through shared memory to the warps of lanes 0-63,
+// which apply SwiGLU.  Stores write one token row's 32 consecutive outputs (64 bytes) per warp
+// instruction.
 #pragma once
 
 #include "grouped_gemm.cuh"
@@ -33,6 +45,20 @@ constexpr int PAIR_THREADS = 64 + 32 * PAIR_EPI_WARPS;
 constexpr int PAIR_STAGE_OUT_BYTES = 2048;        // per epilogue warp: 32 rows x 32 bf16
 constexpr int PAIR_SMEM_BYTES =
     PAIR_STAGES * (PAIR_A_BYTES + PAIR_B_BYTES) + PAIR_EPI_WARPS * PAIR_STAGE_OUT_BYTES + 1024 + 256;
+#ifndef MOE_PAIR_SWAP_MAX_ROWS
+#define MOE_PAIR_SWAP_MAX_ROWS 224
+#endif
+constexpr int PAIR_SWAP_MAX_ROWS = MOE_PAIR_SWAP_MAX_ROWS;   // tail tiles up to this many rows run swapped
+constexpr int PAIR_SWAP_BOX_ROWS = 32;                      // token rows per TMA box of a swapped tile
+constexpr int PAIR_SWAP_BOX_BYTES = PAIR_SWAP_BOX_ROWS * 128;
+
+// Tensor maps only swapped tiles use.
+struct PairSwapMaps {
+    CUtensorMap a0, a1;     // the token rows of class 0 / class 1 in 32-row boxes
+    CUtensorMap w0, w0b;    // GEMM1: W1 / W3 of class 0 in 64-row boxes
+    CUtensorMap w1, w1b;    // GEMM1: W1 / W3 of class 1 in 64-row boxes
+};
+
 
 // Tile walk with 256-row m-tiles (mprefix counts 256-row tiles per group).
 __device__ __forceinline__ int pair_total_tiles(const GemmParams& p, int& routed_tiles) {
@@ -47,6 +73,8 @@ struct PairTile {
     int rows;    // valid rows of the pair tile (<= 256)
     int group;
     int n_idx;
+    bool swap;   // tail tile run with the operands swapped (tokens on the MMA's N side)
+    int n_tok;   // swapped: MMA N = rows rounded up to 16
 };
 
 __device__ __forceinline__ PairTile pair_decode_tile(const GemmParams& p, int t, int routed_tiles) {
@@ -82,6 +110,8 @@ __device__ __forceinline__ PairTile pair_decode_tile(const GemmParams& p, int t,
         ti.n_idx = n;
         (void)c;
     }
+    ti.swap = ti.rows <= PAIR_SWAP_MAX_ROWS;
+    ti.n_tok = (ti.rows + 15) & ~15;
     return ti;
 }
 
@@ -92,7 +122,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                          const __grid_constant__ CUtensorMap tmB0b, const __grid_constant__ CUtensorMap tmA1,
                          const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB1b,
-                         const __grid_constant__ GemmParams p) {
+                         const __grid_constant__ GemmParams p, const __grid_constant__ PairSwapMaps sw) {
     static_assert(EPI == EPI_SWIGLU || EPI == EPI_STORE, "pair tiles serve the expert GEMMs");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -104,7 +134,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
     uint64_t* tfull_bar = empty_bar + PAIR_STAGES;
     uint64_t* tempty_bar = tfull_bar + 2;
     uint64_t* drain_bar = tempty_bar + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+    uint64_t* xch_bar = drain_bar + 1;   // swapped GEMM1 tiles: 2 barriers per gate / up warp pair
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xch_bar + 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -124,6 +155,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
             mbar_init(tempty_bar + a, 2 * 32 * PAIR_EPI_WARPS);  // leader: epilogue threads of 2 CTAs
         }
         mbar_init(drain_bar, 1);
+        for (int i = 0; i < 8; ++i) mbar_init(xch_bar + i, 32);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -175,12 +207,35 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                 const int a_row = ti.a_row + (int)rank * 128;
                 constexpr int KB = F8 ? 2 * GEMM_BK : GEMM_BK;
                 const int nk = c.K / KB;
+                // swapped tile: this CTA's N / 2 token rows in 32-row boxes, and its weight rows
+                // (GEMM1: 64 rows of W1 and the same 64 rows of W3)
+                const int half_tok = ti.n_tok >> 1;
+                const int nld = ti.swap ? (half_tok + PAIR_SWAP_BOX_ROWS - 1) / PAIR_SWAP_BOX_ROWS : 0;
+                const CUtensorMap* mT = ti.cls ? &sw.a1 : &sw.a0;
+                const CUtensorMap* mW = ti.cls ? &sw.w1 : &sw.w0;
+                const CUtensorMap* mWb = ti.cls ? &sw.w1b : &sw.w0b;
+                const int t_row = ti.a_row + (int)rank * half_tok;
+                const int w_row = wg * c.b_group_rows + ti.n_idx * 128 + (int)rank * 64;   // GEMM1 swapped
+                const uint32_t tx = ti.swap ? 2u * (uint32_t)(PAIR_B_BYTES + nld * PAIR_SWAP_BOX_BYTES)
+                                            : 2u * (PAIR_A_BYTES + PAIR_B_BYTES);
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(empty_bar + stage, phase ^ 1u, abort_flag)) { ok = false; break; }
                     const uint32_t fb = full_leader0 + (uint32_t)stage * 8u;
-                    if (leader) mbar_arrive_expect_tx(full_bar + stage, 2u * (PAIR_A_BYTES + PAIR_B_BYTES));
-                    tma_load_2d_pair(sA + stage * PAIR_A_BYTES, mA, fb, kb * KB, a_row, pol_a);
-                    tma_load_2d_pair(sB + stage * PAIR_B_BYTES, mB, fb, kb * KB, b_row, pol_b);
+                    if (leader) mbar_arrive_expect_tx(full_bar + stage, tx);
+                    if (!ti.swap) {
+                        tma_load_2d_pair(sA + stage * PAIR_A_BYTES, mA, fb, kb * KB, a_row, pol_a);
+                        tma_load_2d_pair(sB + stage * PAIR_B_BYTES, mB, fb, kb * KB, b_row, pol_b);
+                    } else {
+                        if (EPI == EPI_SWIGLU) {
+                            tma_load_2d_pair(sB + stage * PAIR_B_BYTES, mW, fb, kb * KB, w_row, pol_b);
+                            tma_load_2d_pair(sB + stage * PAIR_B_BYTES + 64 * 128, mWb, fb, kb * KB, w_row, pol_b);
+                        } else {
+                            tma_load_2d_pair(sB + stage * PAIR_B_BYTES, mB, fb, kb * KB, b_row, pol_b);
+                        }
+                        for (int i = 0; i < nld; ++i)
+                            tma_load_2d_pair(sA + stage * PAIR_A_BYTES + i * PAIR_SWAP_BOX_BYTES, mT, fb, kb * KB,
+                                             t_row + i * PAIR_SWAP_BOX_ROWS, pol_a);
+                    }
                     ++issued;
                     if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -207,18 +262,23 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                 const PairTile ti = pair_decode_tile(p, t, routed_tiles);
                 const GemmClass& c = p.cls[ti.cls];
                 const int nk = c.K / (F8 ? 2 * GEMM_BK : GEMM_BK);
+                // swapped tile: A = the weights (B slot), B = the tokens (A slot), N = n_tok
+                const uint32_t id = !ti.swap ? idesc
+                                    : (F8 ? idesc_e4m3_f32(PAIR_BM, ti.n_tok) : idesc_bf16_f32(PAIR_BM, ti.n_tok));
                 if (!mbar_wait(tempty_bar + acc, acc_phase ^ 1u, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * GEMM_ACC_COLS);
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(full_bar + stage, phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint64_t ad = smem_desc_k_sw128(sA + stage * PAIR_A_BYTES);
-                    const uint64_t bd = smem_desc_k_sw128(sB + stage * PAIR_B_BYTES);
+                    const uint64_t da = smem_desc_k_sw128(sA + stage * PAIR_A_BYTES);
+                    const uint64_t db = smem_desc_k_sw128(sB + stage * PAIR_B_BYTES);
+                    const uint64_t ad = ti.swap ? db : da;
+                    const uint64_t bd = ti.swap ? da : db;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {   // 32 bytes of K per instruction
-                        if (F8) umma_e4m3_pair(d_tmem, ad + 2ull * kk, bd + 2ull * kk, idesc, (kb | kk) != 0);
-                        else umma_bf16_pair(d_tmem, ad + 2ull * kk, bd + 2ull * kk, idesc, (kb | kk) != 0);
+                        if (F8) umma_e4m3_pair(d_tmem, ad + 2ull * kk, bd + 2ull * kk, id, (kb | kk) != 0);
+                        else umma_bf16_pair(d_tmem, ad + 2ull * kk, bd + 2ull * kk, id, (kb | kk) != 0);
                     }
                     umma_commit_pair(empty_bar + stage, 0x3);
                     any = true;
@@ -243,7 +303,9 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
         uint4* stage = reinterpret_cast<uint4*>(sOut + (warp - 2) * PAIR_STAGE_OUT_BYTES);
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = pair_id; t < total; t += npairs) {
+        uint32_t xch_n = 0;         // swapped GEMM1 tiles: 16-token hand-overs so far (per pair)
+        bool swap_ok = true;
+        for (int t = pair_id; t < total && swap_ok; t += npairs) {
             const PairTile ti = pair_decode_tile(p, t, routed_tiles);
             const GemmClass& c = p.cls[ti.cls];
             const bool ready = mbar_wait(tfull_bar + acc, acc_phase, abort_flag);
@@ -264,7 +326,97 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                 sb = c.b_scale + wg * c.b_scale_stride;
                 if (EPI == EPI_SWIGLU) sb2 = c.b_scale2 + wg * c.b_scale_stride;
             }
-            if (EPI == EPI_SWIGLU) {
+            if (ti.swap) {
+                // lane = weight row of this CTA, column j = token a_row + j; warp halves take
+                // alternate 32-token chunks
+                const int nch = (ti.n_tok + 31) >> 5;
+                __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(c.out);
+                if (EPI == EPI_SWIGLU) {
+                    // lanes 0-63: gate of this CTA's 64 features, lanes 64-127: their up values; the
+                    // warp of quarter q + 2 passes its up values to the warp of quarter q (same half)
+                    // through the two warps' staging slots, tokens 0-15 / 16-31 of the chunk
+                    const int q = sub & 1;
+                    const bool up_warp = sub >= 2;
+                    const int feat = ti.n_idx * 128 + (int)rank * 64 + q * 32 + lane;
+                    const bool feat_ok = feat < c.n_out;
+                    // the up warp's own staging slot: 16 tokens x 32 lanes of fp32; the pair's
+                    // two barriers: values staged (up -> gate), values read (gate -> up)
+                    float* st = reinterpret_cast<float*>(sOut + (q + 4 * half) * PAIR_STAGE_OUT_BYTES);
+                    uint64_t* xch_staged = xch_bar + 2 * (q + 2 * half);
+                    uint64_t* xch_read = xch_staged + 1;
+                    float sg = 1.f, su = 1.f;
+                    if (F8 && feat_ok) {
+                        sg = __ldg(sb + feat);
+                        su = __ldg(sb2 + feat);
+                    }
+#pragma unroll 1
+                    for (int ch = half; ch < nch && swap_ok; ch += 2) {
+                        uint32_t v[32];
+                        __syncwarp();
+                        tmem_ld_32cols(tbase + ch * 32, v);
+                        tmem_ld_wait();
+                        if (up_warp) {
+                            // tokens 0-15, then 16-31 of the chunk through this warp's own slot
+#pragma unroll
+                            for (int part = 0; part < 2; ++part) {
+                                if (!mbar_wait(xch_read, (xch_n & 1u) ^ 1u, abort_flag)) { swap_ok = false; break; }
+#pragma unroll
+                                for (int j = 0; j < 16; ++j) st[j * 32 + lane] = __uint_as_float(v[16 * part + j]);
+                                mbar_arrive(xch_staged);
+                                ++xch_n;
+                            }
+                        } else {
+                            float u[32];
+#pragma unroll
+                            for (int part = 0; part < 2; ++part) {
+                                if (!mbar_wait(xch_staged, xch_n & 1u, abort_flag)) { swap_ok = false; break; }
+#pragma unroll
+                                for (int j = 0; j < 16; ++j) u[16 * part + j] = st[j * 32 + lane];
+                                mbar_arrive(xch_read);
+                                ++xch_n;
+                            }
+                            if (!swap_ok) break;
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) {
+                                const int tok = ch * 32 + j;
+                                const long long orow_t = c.out_row0 + ti.a_row + tok;
+                                if (feat_ok && tok < ti.rows && orow_t >= 0 && orow_t < c.out_rows) {
+                                    float g = __uint_as_float(v[j]), uu = u[j];
+                                    if (F8) {
+                                        const float st_a = __ldg(c.a_scale + ti.a_row + tok);
+                                        g = g * st_a * sg;
+                                        uu = uu * st_a * su;
+                                    }
+                                    out[orow_t * c.ldo + feat] = __float2bfloat16_rn(swiglu_f32(g, uu));
+                                }
+                            }
+                        }
+                    }
+                    // the up warp leaves its slot only once the last values were read from it
+                    if (up_warp && swap_ok && !mbar_wait(xch_read, (xch_n & 1u) ^ 1u, abort_flag)) swap_ok = false;
+                } else {
+                    const int col = ti.n_idx * 256 + (int)rank * 128 + sub * 32 + lane;
+                    const bool col_ok = col < c.n_out;
+                    const float sc = (F8 && col_ok) ? __ldg(sb + col) : 1.f;
+#pragma unroll 1
+                    for (int ch = half; ch < nch; ch += 2) {
+                        uint32_t v[32];
+                        __syncwarp();
+                        tmem_ld_32cols(tbase + ch * 32, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int tok = ch * 32 + j;
+                            const long long orow_t = c.out_row0 + ti.a_row + tok;
+                            if (col_ok && tok < ti.rows && orow_t >= 0 && orow_t < c.out_rows) {
+                                float val = __uint_as_float(v[j]);
+                                if (F8) val = val * __ldg(c.a_scale + ti.a_row + tok) * sc;
+                                out[orow_t * c.ldo + col] = __float2bfloat16_rn(val);
+                            }
+                        }
+                    }
+                }
+            } else if (EPI == EPI_SWIGLU) {
 #pragma unroll 1
                 for (int ch = 2 * half; ch < 2 * half + 2; ++ch) {
                     uint32_t g[32], u[32];
@@ -299,6 +451,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                     }
                 }
             }
+            if (!swap_ok) break;      // a hand-over wait gave up: the kernel is being abandoned
             tc_fence_before();
             mbar_arrive_cluster(tempty_leader0 + (uint32_t)acc * 8u);
             acc ^= 1;

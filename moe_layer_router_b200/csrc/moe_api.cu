@@ -27,6 +27,9 @@ struct DeviceInfo {
     int sms = 0;
     bool gemm_attr = false;
     bool permute_attr = false;
+    // expert cache: the stream the expert copies run on, and the fork / join events
+    cudaStream_t copy_stream = nullptr;
+    cudaEvent_t copy_fork = nullptr, copy_join = nullptr;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mutex;
@@ -60,6 +63,17 @@ int device_info(DeviceInfo** out) {
         g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     }
     *out = &di;
+    return MOE_OK;
+}
+
+// The expert cache's copy stream and its fork / join events on this device (created once).
+int copy_stream(DeviceInfo* di) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (di->copy_stream) return MOE_OK;
+    if (cudaStreamCreateWithFlags(&di->copy_stream, cudaStreamNonBlocking) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&di->copy_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&di->copy_join, cudaEventDisableTiming) != cudaSuccess)
+        return MOE_ERR_CUDA;
     return MOE_OK;
 }
 
@@ -146,9 +160,17 @@ int launch_gemm(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b0, co
 // double while the tile count stays under one CTA per SM of a B200 (148), each slice keeps
 // >= 256 of K and the partial sums stay under 16 MB.  A pure function of the shapes, so the
 // workspace size does not depend on the device.
+// K slices of the router GEMM.  Precision first: one fp32 tensor-memory accumulation runs over at
+// most ROUTER_MAX_K of the hidden dimension (measured on B200: over K = 4096 the logits drift up to
+// 3.5e-5 from the exactly rounded sums, over K <= 1024 at most 5e-6); the slices are summed in fp32
+// by the top-k kernel.  Then parallelism: small batches split further while the tiles do not fill
+// the GPU.  Slices must be whole 64-element k-blocks of equal length.
+constexpr int ROUTER_MAX_K = 512;
 int router_ksplit(int T, int d, int E) {
     const long long tiles = (long long)((T + GEMM_BM - 1) / GEMM_BM) * ((E + 255) / 256);
     int ks = 1;
+    while (d / ks > ROUTER_MAX_K && d % (GEMM_BK * ks * 2) == 0 && (long long)ks * 2 * T * E * 4 <= (512ll << 20))
+        ks *= 2;
     while (tiles * ks * 2 <= 148 && d % (GEMM_BK * ks * 2) == 0 && d / (ks * 2) >= 256 &&
            (long long)ks * 2 * T * E * 4 <= (16ll << 20))
         ks *= 2;
@@ -162,7 +184,7 @@ size_t router_partial_bytes(int T, int d, int E) {
 template <int EPI, bool F8 = false>
 int launch_gemm_pair(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b0, const CUtensorMap& b0b,
                      const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& b1b, const GemmParams& p,
-                     long long tiles_upper, cudaStream_t s) {
+                     const PairSwapMaps& sw, long long tiles_upper, cudaStream_t s) {
     {
         std::lock_guard<std::mutex> lock(g_mutex);
         static bool attr_set[kMaxDevices][3] = {};
@@ -178,18 +200,41 @@ int launch_gemm_pair(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b
     if (tiles_upper <= 0) return MOE_OK;
     const long long pairs = di->sms / 2;
     const int grid = 2 * (int)(tiles_upper < pairs ? tiles_upper : pairs);
-    grouped_gemm_pair_kernel<EPI, F8><<<grid, PAIR_THREADS, PAIR_SMEM_BYTES, s>>>(a0, b0, b0b, a1, b1, b1b, p);
+    grouped_gemm_pair_kernel<EPI, F8><<<grid, PAIR_THREADS, PAIR_SMEM_BYTES, s>>>(a0, b0, b0b, a1, b1, b1b, p, sw);
     return launch_status();
 }
 
 // Pair (2-SM) tiles pay off when experts average at least one full 256-row tile.
 bool use_pair_tiles(long long rows, int E) { return rows >= 256ll * E; }
 
+// Tensor maps of the pair kernel's swapped tail tiles: the token rows of each class in 32-row
+// boxes and (GEMM1) W1 / W3 of each class in 64-row boxes.  A null base leaves that map unused
+// (its class has no rows, or the GEMM has no gate / up pair); it then copies another map.
+// f8: e4m3 operands (128-byte K rows) instead of bf16.
+int make_swap_maps(PairSwapMaps* m, bool f8, const void* t0, uint64_t k0, uint64_t rows0, const void* t1, uint64_t k1,
+                   uint64_t rows1, const void* w1_0, const void* w3_0, uint64_t wrows0, const void* w1_1,
+                   const void* w3_1, uint64_t wrows1) {
+    memset(m, 0, sizeof(*m));
+    auto mk = [&](CUtensorMap* d, const void* base, uint64_t inner, uint64_t rows, uint32_t box) {
+        return f8 ? make_map_e4m3(d, base, inner, rows, box) : make_map(d, base, inner, rows, box);
+    };
+    int rc;
+    if (t0 && (rc = mk(&m->a0, t0, k0, rows0, PAIR_SWAP_BOX_ROWS)) != MOE_OK) return rc;
+    if (t1 && (rc = mk(&m->a1, t1, k1, rows1, PAIR_SWAP_BOX_ROWS)) != MOE_OK) return rc;
+    if (w1_0 && (rc = mk(&m->w0, w1_0, k0, wrows0, 64)) != MOE_OK) return rc;
+    if (w3_0 && (rc = mk(&m->w0b, w3_0, k0, wrows0, 64)) != MOE_OK) return rc;
+    if (w1_1 && (rc = mk(&m->w1, w1_1, k1, wrows1, 64)) != MOE_OK) return rc;
+    if (w3_1 && (rc = mk(&m->w1b, w3_1, k1, wrows1, 64)) != MOE_OK) return rc;
+    if (!t0) { m->a0 = m->a1; m->w0 = m->w1; m->w0b = m->w1b; }
+    if (!t1) { m->a1 = m->a0; m->w1 = m->w0; m->w1b = m->w0b; }
+    return MOE_OK;
+}
+
 // ------------------------------------------------------------------ workspace layouts
 
 struct LayerLayout {
     size_t off[12];
-    size_t blk_cnt, rank_local, mprefix, h_shared, router_part;
+    size_t blk_cnt, rank_local, mprefix, h_shared, router_part, mp_hit, mp_miss;
     size_t total;
 };
 
@@ -221,6 +266,8 @@ LayerLayout layer_layout(int T, int d, int E, int k, int f, int f_shared) {
     L.rank_local = take(Tk * 4);
     L.mprefix = take((size_t)(E + 1) * 4);
     L.router_part = take(router_partial_bytes(T, d, E));
+    L.mp_hit = take((size_t)(E + 1) * 4);      // expert cache: tile prefixes of resident / loaded experts
+    L.mp_miss = take((size_t)(E + 1) * 4);
     L.total = cur;
     return L;
 }
@@ -410,7 +457,13 @@ int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t
         const int bm = a.pair ? PAIR_BM : GEMM_BM;
         if (routed) tiles += ((long long)(a.max_rows + bm - 1) / bm + a.E) * c0.ntiles;
         if (shared) tiles += (long long)((a.T + bm - 1) / bm) * c1.ntiles;
-        rc = a.pair ? launch_gemm_pair<EPI_SWIGLU>(di, A0, B0, B0b, A1, B1, B1b, p, tiles, s)
+        PairSwapMaps sw;
+        if (a.pair && (rc = make_swap_maps(&sw, false, routed ? a.x_perm : nullptr, a.d, a.max_rows,
+                                           shared ? a.x : nullptr, a.d, a.T, routed ? a.W1 : nullptr,
+                                           routed ? a.W3 : nullptr, weight_groups(a) * a.f, shared ? a.W1s : nullptr,
+                                           shared ? a.W3s : nullptr, a.f_shared)) != MOE_OK)
+            return rc;
+        rc = a.pair ? launch_gemm_pair<EPI_SWIGLU>(di, A0, B0, B0b, A1, B1, B1b, p, sw, tiles, s)
                     : launch_gemm<EPI_SWIGLU>(di, A0, B0, B0b, A1, B1, B1b, p, tiles, s);
         if (rc != MOE_OK) return rc;
     }
@@ -448,7 +501,12 @@ int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t
         const int bm = a.pair ? PAIR_BM : GEMM_BM;
         if (routed) tiles += ((long long)(a.max_rows + bm - 1) / bm + a.E) * c0.ntiles;
         if (shared) tiles += (long long)((a.T + bm - 1) / bm) * c1.ntiles;
-        rc = a.pair ? launch_gemm_pair<EPI_STORE>(di, A0, B0, B0, A1, B1, B1, p, tiles, s)
+        PairSwapMaps sw;
+        if (a.pair && (rc = make_swap_maps(&sw, false, routed ? a.h : nullptr, a.f, a.max_rows,
+                                           shared ? a.h_shared : nullptr, a.f_shared, a.T, nullptr, nullptr, 0,
+                                           nullptr, nullptr, 0)) != MOE_OK)
+            return rc;
+        rc = a.pair ? launch_gemm_pair<EPI_STORE>(di, A0, B0, B0, A1, B1, B1, p, sw, tiles, s)
                     : launch_gemm<EPI_STORE>(di, A0, B0, B0, A1, B1, B1, p, tiles, s);
         if (rc != MOE_OK) return rc;
     }
@@ -683,7 +741,14 @@ int run_expert_ffn_a8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, cons
         const int bm = a.pair ? PAIR_BM : GEMM_BM;
         if (routed) tiles += ((long long)(a.max_rows + bm - 1) / bm + a.E) * c0.ntiles;
         if (shared) tiles += (long long)((a.T + bm - 1) / bm) * c1.ntiles;
-        rc = a.pair ? launch_gemm_pair<EPI_SWIGLU, true>(di, A0, B0, B0b, A1, B1, B1b, p, tiles, s)
+        PairSwapMaps sw;
+        if (a.pair && (rc = make_swap_maps(&sw, true, routed ? b.xq : nullptr, a.d, a.max_rows,
+                                           shared ? b.xqs : nullptr, a.d, a.T, routed ? q.W1q : nullptr,
+                                           routed ? q.W3q : nullptr, weight_groups(a) * a.f,
+                                           shared ? q.W1sq : nullptr, shared ? q.W3sq : nullptr, a.f_shared)) !=
+                          MOE_OK)
+            return rc;
+        rc = a.pair ? launch_gemm_pair<EPI_SWIGLU, true>(di, A0, B0, B0b, A1, B1, B1b, p, sw, tiles, s)
                     : launch_gemm<EPI_SWIGLU, true>(di, A0, B0, B0b, A1, B1, B1b, p, tiles, s);
         if (rc != MOE_OK) return rc;
     }
@@ -726,7 +791,12 @@ int run_expert_ffn_a8(DeviceInfo* di, const FfnArgs& a, const W8Weights& q, cons
         const int bm = a.pair ? PAIR_BM : GEMM_BM;
         if (routed) tiles += ((long long)(a.max_rows + bm - 1) / bm + a.E) * c0.ntiles;
         if (shared) tiles += (long long)((a.T + bm - 1) / bm) * c1.ntiles;
-        rc = a.pair ? launch_gemm_pair<EPI_STORE, true>(di, A0, B0, B0, A1, B1, B1, p, tiles, s)
+        PairSwapMaps sw;
+        if (a.pair && (rc = make_swap_maps(&sw, true, routed ? b.hq : nullptr, a.f, a.max_rows,
+                                           shared ? b.hqs : nullptr, a.f_shared, a.T, nullptr, nullptr, 0, nullptr,
+                                           nullptr, 0)) != MOE_OK)
+            return rc;
+        rc = a.pair ? launch_gemm_pair<EPI_STORE, true>(di, A0, B0, B0, A1, B1, B1, p, sw, tiles, s)
                     : launch_gemm<EPI_STORE, true>(di, A0, B0, B0, A1, B1, B1, p, tiles, s);
         if (rc != MOE_OK) return rc;
     }
@@ -990,22 +1060,37 @@ int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float*
                           rank_local, mprefix, s, pair ? PAIR_BM : GEMM_BM, fill_base, false, !(w8 && act8))) != MOE_OK)
         return rc;
     CacheView cv{};
+    int32_t* mp_hit = reinterpret_cast<int32_t*>(base + L.mp_hit);
+    int32_t* mp_miss = reinterpret_cast<int32_t*>(base + L.mp_miss);
     if (cache) {
+        // plan on the layer's stream; the copy of the missed experts on the copy stream, which
+        // forks after the plan and joins before the misses' GEMMs
+        if ((rc = copy_stream(di)) != MOE_OK) return rc;
         if (!mark(ev.cache)) return MOE_ERR_CUDA;
         cv = cache_view(cache->state, E, cache->S);
-        cache_plan_kernel<<<1, CACHE_MAX, 0, s>>>(counts, E, cache->S, cv);
+        cache_plan_kernel<<<1, CACHE_MAX, 0, s>>>(counts, E, cache->S, cv, pair ? PAIR_BM : GEMM_BM, mp_hit, mp_miss);
         if ((rc = launch_status()) != MOE_OK) return rc;
-        cache_load_kernel<<<2 * di->sms, CACHE_LOAD_THREADS, 0, s>>>(cv.ctr, cv.load_expert, cv.load_slot, cache->cp);
+        if (cudaEventRecord(di->copy_fork, s) != cudaSuccess ||
+            cudaStreamWaitEvent(di->copy_stream, di->copy_fork, 0) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        if (ev.copy_start && cudaEventRecord(static_cast<cudaEvent_t>(ev.copy_start), di->copy_stream) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        cache_load_kernel<<<2 * di->sms, CACHE_LOAD_THREADS, 0, di->copy_stream>>>(cv.ctr, cv.load_expert,
+                                                                                   cv.load_slot, cache->cp);
         if ((rc = launch_status()) != MOE_OK) return rc;
+        if (ev.copy_end && cudaEventRecord(static_cast<cudaEvent_t>(ev.copy_end), di->copy_stream) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        if (cudaEventRecord(di->copy_join, di->copy_stream) != cudaSuccess) return MOE_ERR_CUDA;
     }
     if (!mark(ev.gate_up)) return MOE_ERR_CUDA;
     FfnArgs a;
     memset(&a, 0, sizeof(a));
     a.x_perm = x_perm; a.offsets = offsets; a.mprefix = mprefix; a.max_rows = T * k; a.E = E; a.d = d; a.f = f;
     a.W1 = W1; a.W3 = W3; a.W2 = W2; a.h = h; a.y_perm = y_perm;
-    if (cache) {     // W1/W3/W2 (or w8) already point at the slots
+    if (cache) {     // W1/W3/W2 (or w8) already point at the slots; first the resident experts
         a.group_map = cv.slot_of;
         a.w_groups = cache->S;
+        a.mprefix = mp_hit;
     }
     a.x = x; a.T = T; a.f_shared = f_shared; a.W1s = W1s; a.W3s = W3s; a.W2s = W2s;
     a.h_shared = h_shared; a.y_shared = y_shared;
@@ -1028,6 +1113,22 @@ int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float*
     } else {
         rc = w8 ? run_expert_ffn_w8(di, a, *w8, s, static_cast<cudaEvent_t>(ev.down))
                 : run_expert_ffn(di, a, s, static_cast<cudaEvent_t>(ev.down));
+        if (rc == MOE_OK && cache) {
+            // then the experts this batch loaded, once their copy is done (routed groups only)
+            if (cudaStreamWaitEvent(s, di->copy_join, 0) != cudaSuccess) return MOE_ERR_CUDA;
+            FfnArgs m = a;
+            m.mprefix = mp_miss;
+            m.f_shared = 0;
+            m.h_shared = m.y_shared = nullptr;
+            m.W1s = m.W3s = m.W2s = nullptr;
+            W8Weights qm;
+            if (w8) {
+                qm = *w8;
+                qm.W1sq = qm.W3sq = qm.W2sq = nullptr;
+                qm.s1s = qm.s3s = qm.s2s = nullptr;
+            }
+            rc = w8 ? run_expert_ffn_w8(di, m, qm, s, nullptr) : run_expert_ffn(di, m, s);
+        }
     }
     if (rc != MOE_OK) return rc;
     if (!mark(ev.combine)) return MOE_ERR_CUDA;
@@ -1248,7 +1349,7 @@ int ep_check(int R, int rank, int E, int d) {
 }
 
 size_t ep_bytes(int R, int E) {
-    size_t off[8];
+    size_t off[9];
     return moe::ep_layout_bytes(R, E, off);
 }
 
@@ -1276,6 +1377,91 @@ int moe_ep_workspace_bytes(int R, int E, size_t* bytes) {
     int rc = ep_check(R, 0, E, 64);
     if (rc != MOE_OK) return rc;
     *bytes = ep_bytes(R, E);
+    return MOE_OK;
+}
+
+int moe_ep_splits_offset(int R, int E, size_t* offset) {
+    MOE_REQUIRE(offset, MOE_ERR_INVALID_ARG);
+    int rc = ep_check(R, 0, E, 64);
+    if (rc != MOE_OK) return rc;
+    size_t off[9];
+    moe::ep_layout_bytes(R, E, off);
+    *offset = off[8];
+    return MOE_OK;
+}
+
+// ---- peer buffers: CUDA IPC handles of device allocations
+
+namespace {
+
+using cuMemGetAddressRange_t = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
+
+cuMemGetAddressRange_t address_range_fn() {
+    static cuMemGetAddressRange_t fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<cuMemGetAddressRange_t>(p);
+    });
+    return fn;
+}
+
+struct IpcBlob {                 // layout of the MOE_IPC_HANDLE_BYTES a handle occupies
+    cudaIpcMemHandle_t mem;      // handle of the allocation that holds the pointer
+    uint64_t offset;             // the pointer's offset from the allocation's base
+    uint64_t magic;
+};
+static_assert(sizeof(IpcBlob) <= MOE_IPC_HANDLE_BYTES, "IPC handle blob");
+constexpr uint64_t kIpcMagic = 0x6d6f652d69706331ull;
+
+}  // namespace
+
+int moe_ipc_export(const void* ptr, void* handle) {
+    MOE_REQUIRE(ptr && handle, MOE_ERR_INVALID_ARG);
+    cuMemGetAddressRange_t range = address_range_fn();
+    if (!range) return MOE_ERR_CUDA;
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (range(&base, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS) return MOE_ERR_INVALID_ARG;
+    IpcBlob b;
+    memset(&b, 0, sizeof(b));
+    if (cudaIpcGetMemHandle(&b.mem, reinterpret_cast<void*>(base)) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    b.offset = reinterpret_cast<uint64_t>(ptr) - static_cast<uint64_t>(base);
+    b.magic = kIpcMagic;
+    memset(handle, 0, MOE_IPC_HANDLE_BYTES);
+    memcpy(handle, &b, sizeof(b));
+    return MOE_OK;
+}
+
+int moe_ipc_import(const void* handle, void** ptr) {
+    MOE_REQUIRE(handle && ptr, MOE_ERR_INVALID_ARG);
+    IpcBlob b;
+    memcpy(&b, handle, sizeof(b));
+    MOE_REQUIRE(b.magic == kIpcMagic, MOE_ERR_INVALID_ARG);
+    void* base = nullptr;
+    if (cudaIpcOpenMemHandle(&base, b.mem, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    *ptr = static_cast<char*>(base) + b.offset;
+    return MOE_OK;
+}
+
+int moe_ipc_close(void* ptr, const void* handle) {
+    MOE_REQUIRE(ptr && handle, MOE_ERR_INVALID_ARG);
+    IpcBlob b;
+    memcpy(&b, handle, sizeof(b));
+    MOE_REQUIRE(b.magic == kIpcMagic, MOE_ERR_INVALID_ARG);
+    if (cudaIpcCloseMemHandle(static_cast<char*>(ptr) - b.offset) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
     return MOE_OK;
 }
 

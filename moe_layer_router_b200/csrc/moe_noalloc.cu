@@ -15,7 +15,9 @@
 // process exits.  Host code cannot use the array's name as a device address (on the host
 // the name is only a stand-in), so the first call on each device, with that device
 // current, asks the runtime for the real address with cudaGetSymbolAddress() and caches
-// it; that first call should therefore come before any stream capture.
+// it; that first call should therefore come before any stream capture.  The cached address
+// belongs to the device's primary context: after a cudaDeviceReset() it is stale, and the
+// entry point must not be called on that device again in the same process.
 //
 // Sharing.  All calls on a device share the one array and the array keeps the previous
 // call's contents.  Nothing in it needs to start at zero: the count kernel writes every

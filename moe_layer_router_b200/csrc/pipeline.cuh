@@ -16,8 +16,14 @@
 
 namespace moe {
 
+// weights: 0 = bf16 (moe_layer_forward), 1 = fp8 weights (moe_layer_forward_w8),
+// 2 = fp8 weights and activations (moe_layer_forward_w8a8)
+enum { PIPE_BF16 = 0, PIPE_W8 = 1, PIPE_W8A8 = 2 };
+
 struct Pipeline {
     moe_pipeline_params prm;
+    int weights;
+    moe_w8_experts q, qs;       // fp8 routed and shared experts (weights != PIPE_BF16)
     char* x_dev[2];
     char* out_dev[2];
     void* ws;
@@ -42,21 +48,47 @@ int moe_pipeline_bytes(int T, int d, int E, int k, int f, int f_shared, size_t* 
     return MOE_OK;
 }
 
-int moe_pipeline_create(const moe_pipeline_params* prm, void* dev_mem, size_t dev_bytes, moe_pipeline** out) {
+int moe_pipeline_bytes_w8(int T, int d, int E, int k, int f, int f_shared, int activations_fp8, size_t* bytes) {
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    size_t ws = 0;
+    int rc = activations_fp8 ? moe_workspace_bytes_a8(T, d, E, k, f, f_shared, &ws)
+                             : moe_workspace_bytes(T, d, E, k, f, f_shared, &ws);
+    if (rc != MOE_OK) return rc;
+    *bytes = 4 * moe::pipeline_io_bytes(T, d) + moe::align256(ws);
+    return MOE_OK;
+}
+
+namespace {
+
+int pipeline_create(const moe_pipeline_params* prm, int weights, const moe_w8_experts* q, const moe_w8_experts* qs,
+                    void* dev_mem, size_t dev_bytes, moe_pipeline** out) {
     using namespace moe;
     if (!prm || !dev_mem || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(dev_mem)) return MOE_ERR_ALIGN;
     size_t need = 0;
-    int rc = moe_pipeline_bytes(prm->T, prm->d, prm->E, prm->k, prm->f, prm->f_shared, &need);
+    int rc = weights == PIPE_BF16
+                 ? moe_pipeline_bytes(prm->T, prm->d, prm->E, prm->k, prm->f, prm->f_shared, &need)
+                 : moe_pipeline_bytes_w8(prm->T, prm->d, prm->E, prm->k, prm->f, prm->f_shared,
+                                         weights == PIPE_W8A8, &need);
     if (rc != MOE_OK) return rc;
     if (dev_bytes < need) return MOE_ERR_WORKSPACE;
-    if (!prm->Wg || !prm->W1 || !prm->W3 || !prm->W2) return MOE_ERR_INVALID_ARG;
+    if (!prm->Wg) return MOE_ERR_INVALID_ARG;
+    if (weights == PIPE_BF16 && !(prm->W1 && prm->W3 && prm->W2)) return MOE_ERR_INVALID_ARG;
+    if (weights != PIPE_BF16 && !(q && q->W1q && q->W3q && q->W2q && q->s1 && q->s3 && q->s2)) return MOE_ERR_INVALID_ARG;
+    if (weights != PIPE_BF16 && prm->f_shared > 0 &&
+        !(qs && qs->W1q && qs->W3q && qs->W2q && qs->s1 && qs->s3 && qs->s2))
+        return MOE_ERR_INVALID_ARG;
     DeviceInfo* di;
     if ((rc = device_info(&di)) != MOE_OK) return rc;
     Pipeline* pl = new (std::nothrow) Pipeline;
     if (!pl) return MOE_ERR_INVALID_ARG;
     memset(pl, 0, sizeof(Pipeline));
     pl->prm = *prm;
+    pl->weights = weights;
+    if (weights != PIPE_BF16) {
+        pl->q = *q;
+        if (prm->f_shared > 0) pl->qs = *qs;
+    }
     char* base = static_cast<char*>(dev_mem);
     const size_t io = pipeline_io_bytes(prm->T, prm->d);
     pl->x_dev[0] = base;
@@ -80,6 +112,18 @@ int moe_pipeline_create(const moe_pipeline_params* prm, void* dev_mem, size_t de
     return MOE_OK;
 }
 
+}  // namespace
+
+int moe_pipeline_create(const moe_pipeline_params* prm, void* dev_mem, size_t dev_bytes, moe_pipeline** out) {
+    return pipeline_create(prm, moe::PIPE_BF16, nullptr, nullptr, dev_mem, dev_bytes, out);
+}
+
+int moe_pipeline_create_w8(const moe_pipeline_params* prm, const moe_w8_experts* routed, const moe_w8_experts* shared,
+                           int activations_fp8, void* dev_mem, size_t dev_bytes, moe_pipeline** out) {
+    return pipeline_create(prm, activations_fp8 ? moe::PIPE_W8A8 : moe::PIPE_W8, routed, shared, dev_mem, dev_bytes,
+                           out);
+}
+
 int moe_pipeline_submit(moe_pipeline* handle, const moe_bf16* x_host, moe_bf16* out_host) {
     using namespace moe;
     Pipeline* pl = reinterpret_cast<Pipeline*>(handle);
@@ -95,9 +139,20 @@ int moe_pipeline_submit(moe_pipeline* handle, const moe_bf16* x_host, moe_bf16* 
     // compute: after the copy in, and after the slot's previous output went back to the host
     if (cudaStreamWaitEvent(pl->compute, pl->h2d_done[s], 0) != cudaSuccess) return MOE_ERR_CUDA;
     if (pl->submitted >= 2 && cudaStreamWaitEvent(pl->compute, pl->d2h_done[s], 0) != cudaSuccess) return MOE_ERR_CUDA;
-    int rc = moe_layer_forward(reinterpret_cast<const moe_bf16*>(pl->x_dev[s]), p.Wg, p.bias, p.W1, p.W3, p.W2, p.W1s,
-                               p.W3s, p.W2s, p.f_shared, p.T, p.d, p.E, p.k, p.f, p.capacity_factor, p.cap_mode,
-                               reinterpret_cast<moe_bf16*>(pl->out_dev[s]), pl->ws, pl->ws_bytes, pl->compute);
+    const moe_bf16* xd = reinterpret_cast<const moe_bf16*>(pl->x_dev[s]);
+    moe_bf16* od = reinterpret_cast<moe_bf16*>(pl->out_dev[s]);
+    int rc;
+    if (pl->weights == PIPE_BF16) {
+        rc = moe_layer_forward(xd, p.Wg, p.bias, p.W1, p.W3, p.W2, p.W1s, p.W3s, p.W2s, p.f_shared, p.T, p.d, p.E, p.k,
+                               p.f, p.capacity_factor, p.cap_mode, od, pl->ws, pl->ws_bytes, pl->compute);
+    } else {
+        const moe_w8_experts& q = pl->q;
+        const moe_w8_experts& qs = pl->qs;
+        auto call = pl->weights == PIPE_W8A8 ? moe_layer_forward_w8a8 : moe_layer_forward_w8;
+        rc = call(xd, p.Wg, p.bias, q.W1q, q.s1, q.W3q, q.s3, q.W2q, q.s2, qs.W1q, qs.s1, qs.W3q, qs.s3, qs.W2q,
+                  qs.s2, p.f_shared, p.T, p.d, p.E, p.k, p.f, p.capacity_factor, p.cap_mode, od, pl->ws,
+                  pl->ws_bytes, pl->compute, nullptr);
+    }
     if (rc != MOE_OK) return rc;
     if (cudaEventRecord(pl->layer_done[s], pl->compute) != cudaSuccess) return MOE_ERR_CUDA;
     // d2h: after the layer

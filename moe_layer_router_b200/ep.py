@@ -8,42 +8,22 @@ send the results back and combine ([EP-KV] sections 6-7).  Every step of the pat
 library's kernels; this module only moves pointers, sizes and (for the NCCL path) the two
 all-to-all-v exchanges.
 
-Two drivers:
+Three drivers:
   * ``EmulatedEP``: R ranks on one device in one process.  The row exchanges are the library's
     put kernels writing into the other ranks' buffers (expert-major receive order, one GEMM group
     per local expert); the all-gather is a device copy.
   * ``ep_layer_forward_dist``: one process per GPU over ``torch.distributed``; counts are
-    all-gathered and rows moved with ``all_to_all_single`` (NCCL), whose split sizes
-    ``ep_row_splits`` computes on the host from the gathered counts; rows arrive source-major and
-    the local GEMM runs one segment per (source rank, local expert).
+    all-gathered and rows moved with ``all_to_all_single`` (NCCL), whose split sizes the
+    device-side plan writes (``moe_ep_splits``; the host only reads them back, as the collective
+    wants them on the host); rows arrive source-major and the local GEMM runs one segment per
+    (source rank, local expert).
+  * ``ep_layer_forward_put_dist``: one process per GPU, rows moved by the library's put kernels
+    straight into the other ranks' buffers (``PeerBuffers``: CUDA IPC handles exchanged over
+    ``torch.distributed``), with a barrier between the puts and the reads of each exchange.
 """
 from __future__ import annotations
 
 from typing import List, Optional, Sequence
-
-import numpy as np
-
-
-def kept_counts(all_counts_raw: np.ndarray, capacity: int) -> np.ndarray:
-    """[R, E] rows each rank keeps per expert: the rows of rank r for expert e come after the
-    rows of ranks < r in token order, so r keeps min(c[r][e], max(0, C - sum_{s<r} c[s][e]))."""
-    c = np.asarray(all_counts_raw, dtype=np.int64)
-    if capacity < 0:
-        return c.copy()
-    before = np.cumsum(c, axis=0) - c
-    return np.clip(np.minimum(c, capacity - before), 0, None)
-
-
-def ep_row_splits(all_counts_raw: np.ndarray, capacity: int, rank: int):
-    """-> (send_rows [R], recv_rows [R]): rows `rank` sends to each rank (its kept rows of that
-    rank's experts, in rank order = x_perm order) and rows it receives from each rank."""
-    R, E = all_counts_raw.shape
-    if E % R:
-        raise ValueError("E must be a multiple of the number of ranks")
-    El = E // R
-    kept = kept_counts(all_counts_raw, capacity)
-    per_rank = kept.reshape(R, R, El).sum(axis=2)       # [src, dst]
-    return per_rank[rank].tolist(), per_rank[:, rank].tolist()
 
 
 def exchange_rows(src, send_rows: Sequence[int], recv_rows: Sequence[int], out, group=None) -> None:
@@ -121,9 +101,9 @@ class EmulatedEP:
         x_perm = [b.view(moe, "x_perm", (T * k, d), xs[r].dtype) for r, b in enumerate(self.ranks)]
         y_perm = [b.view(moe, "y_perm", (T * k, d), xs[r].dtype) for r, b in enumerate(self.ranks)]
         a2a = self.exchange == "a2a"
-        if a2a:     # split sizes on the host, as an all-to-all-v caller has them
-            counts = self.all_counts.cpu().numpy()
-            splits = [ep_row_splits(counts, C, r) for r in range(R)]
+        if a2a:     # the plans' split sizes, on the host, as an all-to-all-v caller has them
+            tabs = [moe.moe_ep_splits(b.ep_ws, R, E).cpu().tolist() for b in self.ranks]
+            splits = [(t[0], t[1]) for t in tabs]
         mark("dispatch")
         if a2a:
             self._a2a([x_perm[r] for r in range(R)], recv, [sp[0] for sp in splits], [sp[1] for sp in splits])
@@ -187,7 +167,7 @@ def ep_layer_forward_dist(x, Wg, bias, W1_local, W3_local, W2_local, W1s, W3s, W
     moe.moe_fill_base(all_counts, R, rank, E, bufs.fill_base)
     moe.moe_layer_permute(x, f_shared, T, d, E, k, f, C, bufs.fill_base, bufs.ws)
     moe.moe_ep_plan(all_counts, R, rank, E, C, R * T * k, bufs.ep_ws)
-    send_rows, recv_rows = ep_row_splits(all_counts.cpu().numpy(), C, rank)
+    send_rows, recv_rows = moe.moe_ep_splits(bufs.ep_ws, R, E).cpu().tolist()   # host split sizes
     x_perm = bufs.view(moe, "x_perm", (T * k, d), x.dtype)
     y_perm = bufs.view(moe, "y_perm", (T * k, d), x.dtype)
     exchange_rows(x_perm, send_rows, recv_rows, bufs.recv, group)
@@ -197,3 +177,70 @@ def ep_layer_forward_dist(x, Wg, bias, W1_local, W3_local, W2_local, W1s, W3s, W
     moe.moe_combine(y_perm, bufs.view(moe, "dest", (T, k), torch.int32), bufs.view(moe, "w", (T, k), torch.float32),
                     bufs.y_shared, T, d, k, out)
     return bufs
+
+
+class PeerBuffers:
+    """Device addresses, in this process, of every rank's receive buffer and y_perm: the put
+    kernels' destinations on several GPUs.  Each rank exports its two buffers (CUDA IPC handles),
+    the handles are all-gathered over torch.distributed, and each rank imports the other ranks'
+    (its own entry is its own pointer).  export / import_ / close default to the library's
+    moe_ipc_* calls; tests pass stand-ins to check the exchange on CPU ranks."""
+
+    def __init__(self, recv, y_perm, group=None, export=None, import_=None, close=None):
+        import torch.distributed as dist
+        import moe_layer_router_b200 as moe
+        self._import = import_ or moe.moe_ipc_import
+        self._close = close or moe.moe_ipc_close
+        export = export or moe.moe_ipc_export
+        self.R, self.rank = dist.get_world_size(group), dist.get_rank(group)
+        mine = (export(recv), export(y_perm))
+        handles = [None] * self.R
+        dist.all_gather_object(handles, mine, group=group)
+        self.recv, self.y_perm, self._opened = [], [], []
+        for s, (h_recv, h_y) in enumerate(handles):
+            if s == self.rank:
+                self.recv.append(recv)
+                self.y_perm.append(y_perm)
+                continue
+            for h, dst in ((h_recv, self.recv), (h_y, self.y_perm)):
+                a = self._import(h)
+                self._opened.append((a, h))
+                dst.append(a)
+
+    def close(self) -> None:
+        while self._opened:
+            a, h = self._opened.pop()
+            self._close(a, h)
+
+
+def ep_layer_forward_put_dist(x, Wg, bias, W1_local, W3_local, W2_local, W1s, W3s, W2s, f_shared, T, d, E, k, f,
+                              capacity_factor, cap_mode, out, bufs: _RankBuffers, peers: PeerBuffers, group=None):
+    """One rank of an expert-parallel layer whose row exchanges are the library's put kernels
+    storing into the other ranks' buffers (peers: PeerBuffers over bufs.recv and bufs' y_perm).
+    Rows arrive expert-major, so each local expert is one GEMM group.  The collectives: an
+    all-gather of the raw counts and two barriers, each after this rank's stream has finished its
+    puts, so that no rank reads a buffer before every rank has written it."""
+    import torch
+    import torch.distributed as dist
+    import moe_layer_router_b200 as moe
+
+    R, rank = dist.get_world_size(group), dist.get_rank(group)
+    max_recv = bufs.recv.shape[0]
+    C = moe.moe_capacity(R * T, E, k, capacity_factor, cap_mode)
+    moe.moe_layer_route_count(x, Wg, bias, f_shared, T, d, E, k, f, bufs.ws)
+    all_counts = torch.empty((R, E), dtype=torch.int32, device=x.device)
+    dist.all_gather_into_tensor(all_counts, bufs.view(moe, "counts_raw", (E,), torch.int32), group=group)
+    moe.moe_fill_base(all_counts, R, rank, E, bufs.fill_base)
+    moe.moe_layer_permute(x, f_shared, T, d, E, k, f, C, bufs.fill_base, bufs.ws)
+    moe.moe_ep_plan(all_counts, R, rank, E, C, max_recv, bufs.ep_ws)
+    x_perm = bufs.view(moe, "x_perm", (T * k, d), x.dtype)
+    moe.moe_ep_dispatch(x_perm, R, rank, E, d, peers.recv, bufs.ep_ws)
+    torch.cuda.current_stream(x.device).synchronize()
+    dist.barrier(group=group)              # every rank's rows are in every receive buffer
+    moe.moe_ep_expert_ffn(bufs.recv, max_recv, R, rank, E, d, f, W1_local, W3_local, W2_local, bufs.h, bufs.y_recv,
+                          x, T, W1s, W3s, W2s, f_shared, bufs.h_shared, bufs.y_shared, bufs.ep_ws, source_major=False)
+    moe.moe_ep_return(bufs.y_recv, R, rank, E, d, peers.y_perm, bufs.ep_ws)
+    torch.cuda.current_stream(x.device).synchronize()
+    dist.barrier(group=group)              # every result is back in its token's y_perm
+    moe.moe_combine(bufs.view(moe, "y_perm", (T * k, d), x.dtype), bufs.view(moe, "dest", (T, k), torch.int32),
+                    bufs.view(moe, "w", (T, k), torch.float32), bufs.y_shared, T, d, k, out)

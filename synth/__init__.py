@@ -163,6 +163,9 @@ PROFILE_WORKLOADS = {
     "mixtral2e": Workload("mixtral2e", 2048, 4096, 2, 2, 14336),
     "dsv3_32e": Workload("dsv3_32e", 32, 7168, 32, 8, 2048, f_shared=2048, bias_range=0.1),
     "qwen3_16e": Workload("qwen3_16e", 2048, 4096, 16, 8, 1536),
+    # the Qwen3-like batch (same x, router and routing) with experts cut to f = 128: the router
+    # GEMM, top-k, permutation, gather and combine at their full size, ~2.5 GB on the device
+    "qwen3_f128": Workload("qwen3_f128", 16384, 4096, 128, 8, 128),
 }
 WORKLOADS.update(PROFILE_WORKLOADS)
 

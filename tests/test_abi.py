@@ -205,3 +205,28 @@ def test_binding_stage_events_match_the_header():
 def test_binding_structs_match_the_header(name):
     import moe_layer_router_b200 as moe
     assert [n for n, _ in getattr(moe, name)._fields_] == header_struct_fields(name)
+
+
+def test_ep_split_table_offset_and_ipc_validation(lib):
+    sz = ctypes.c_size_t(0)
+    lib.moe_ep_splits_offset.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
+    lib.moe_ep_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
+    for R, E in [(1, 8), (4, 32), (8, 256), (64, 1024)]:
+        assert lib.moe_ep_splits_offset(R, E, ctypes.byref(sz)) == 0
+        off = sz.value
+        assert lib.moe_ep_workspace_bytes(R, E, ctypes.byref(sz)) == 0
+        assert off % 256 == 0 and off + 8 * R <= sz.value          # the [2, R] table fits, aligned
+    assert lib.moe_ep_splits_offset(3, 8, ctypes.byref(sz)) == -2     # E not a multiple of R
+    assert lib.moe_ep_splits_offset(4, 32, None) == -1
+    vp = ctypes.c_void_p
+    lib.moe_ipc_export.argtypes = [vp, vp]
+    lib.moe_ipc_import.argtypes = [vp, ctypes.POINTER(vp)]
+    lib.moe_ipc_close.argtypes = [vp, vp]
+    blob = ctypes.create_string_buffer(96)
+    out = vp(0)
+    assert lib.moe_ipc_export(None, blob) == -1
+    assert lib.moe_ipc_export(4096, None) == -1
+    assert lib.moe_ipc_import(blob, ctypes.byref(out)) == -1          # not a handle this library wrote
+    assert lib.moe_ipc_import(None, ctypes.byref(out)) == -1
+    assert lib.moe_ipc_close(None, blob) == -1
+    assert lib.moe_ipc_close(4096, blob) == -1

@@ -11,7 +11,8 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 import oracle
-from moe_layer_router_b200.ep import ep_row_splits, exchange_rows, kept_counts
+from _ep_reference import ep_row_splits, kept_counts
+from moe_layer_router_b200.ep import exchange_rows
 
 
 def _batch(R, T, E, k, seed):
@@ -138,3 +139,54 @@ def test_all_to_all_v_exchange_between_gloo_ranks(R, C):
         assert ok_recv, f"rank {rank}: received rows out of (source, expert) order"
         assert ok_back, f"rank {rank}: results did not come back to their rows"
     assert sum(n for *_, n in res) > 0
+
+
+def _peer_worker(rank, R, port, q):
+    """PeerBuffers on gloo ranks with stand-in export / import / close: every rank ends up with its
+    own buffers at its own index and the other ranks' imported addresses, in rank order, and
+    closes exactly what it imported."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=R)
+    try:
+        from moe_layer_router_b200.ep import PeerBuffers
+        opened, closed = [], []
+
+        def export(buf):
+            return f"{rank}:{buf}".encode()
+
+        def import_(h):
+            s, name = h.decode().split(":")
+            a = 1000 * int(s) + (1 if name == "recv" else 2)
+            opened.append(a)
+            return a
+
+        def close(a, h):
+            assert import_(h) == a
+            closed.append(a)
+
+        pb = PeerBuffers("recv", "y_perm", export=export, import_=import_, close=close)
+        ok = pb.recv[rank] == "recv" and pb.y_perm[rank] == "y_perm"
+        ok &= all(pb.recv[s] == 1000 * s + 1 and pb.y_perm[s] == 1000 * s + 2 for s in range(R) if s != rank)
+        ok &= len(opened) == 2 * (R - 1)
+        n_open = len(opened)
+        pb.close()
+        ok &= sorted(closed) == sorted(opened[:n_open]) and not pb._opened
+        q.put((rank, bool(ok)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("R", [2, 3])
+def test_peer_buffer_handle_exchange_between_gloo_ranks(R):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_peer_worker, args=(r, R, port, q)) for r in range(R)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(R)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(ok for _, ok in res), res

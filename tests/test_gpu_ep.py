@@ -120,3 +120,112 @@ def test_nccl_driver_single_rank_matches_layer(moe):
         assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
     finally:
         dist.destroy_process_group()
+
+
+def test_plan_split_table_matches_host_reference(moe):
+    """moe_ep_plan's [2, R] split table (the all-to-all-v split sizes) against the host restatement
+    of the whole-batch capacity over ranks, for every rank of a skewed batch with capacity."""
+    from _ep_reference import ep_row_splits
+    R, E = 4, 32
+    rng = np.random.default_rng(5)
+    counts = rng.integers(0, 60, size=(R, E)).astype(np.int32)
+    counts[:, :3] += 100                                   # hot experts, so the capacity bites
+    for C in (-1, 0, 70, 150):
+        dev_counts = torch.from_numpy(counts).cuda()
+        for r in range(R):
+            ep_ws = torch.empty(moe.moe_ep_workspace_bytes(R, E), dtype=torch.uint8, device="cuda")
+            moe.moe_ep_plan(dev_counts, R, r, E, C, R * 512, ep_ws)
+            got = moe.moe_ep_splits(ep_ws, R, E).cpu().tolist()
+            send, recv = ep_row_splits(counts, C, r)
+            assert got == [send, recv], (C, r)
+    assert moe.moe_get_error() == 0
+
+
+def test_put_driver_single_rank_matches_layer(moe):
+    """ep_layer_forward_put_dist on one NCCL rank (its own buffers, no IPC import; the barriers and
+    the expert-major put path run): bit-identical to the single-GPU layer."""
+    import os
+    import socket
+    import torch.distributed as dist
+    from moe_layer_router_b200.ep import PeerBuffers, _RankBuffers, ep_layer_forward_put_dist
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        wl = synth.Workload("ep_put", 96, 256, 8, 2, 128, f_shared=128, cap_mode=synth.CAP_PER_TOKEN,
+                            capacity_factor=1.0, seed=6)
+        inp = synth.Inputs(wl)
+        T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
+        dv = to_dev_bf16
+        x, wg = dv(inp.x()), dv(inp.wg())
+        W1, W3, W2 = dv(inp.w1()), dv(inp.w3()), dv(inp.w2())
+        sh = [dv(inp.shared(n)) for n in ("w1s", "w3s", "w2s")]
+        bufs = _RankBuffers(moe, 1, T, d, E, k, f, fs, T * k, x.device)
+        peers = PeerBuffers(bufs.recv, bufs.view(moe, "y_perm", (T * k, d), torch.bfloat16))
+        out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+        for _ in range(2):                       # a second call reuses the buffers
+            ep_layer_forward_put_dist(x, wg, None, W1, W3, W2, *sh, fs, T, d, E, k, f, wl.capacity_factor,
+                                      wl.cap_mode, out, bufs, peers)
+        peers.close()
+        ref = torch.empty_like(out)
+        ws = torch.empty(moe.moe_workspace_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device="cuda")
+        moe.moe_layer_forward(x, wg, None, W1, W3, W2, *sh, fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode,
+                              ref, ws)
+        torch.cuda.synchronize()
+        assert moe.moe_get_error() == 0
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    finally:
+        dist.destroy_process_group()
+
+
+def _ipc_child(handle, rows, d, E, q):
+    """Imports the parent's receive buffer and puts its rows there with the dispatch kernel (R = 1:
+    the whole x_perm goes to rank 0's buffer, expert-major = x_perm order)."""
+    try:
+        import torch
+        import moe_layer_router_b200 as moe
+        torch.cuda.set_device(0)
+        x_perm = to_dev_bf16(synth.normal_bf16(9, 1, 0, rows * d, 1.0).reshape(rows, d))
+        counts = np.full((1, E), rows // E, np.int32)
+        ep_ws = torch.empty(moe.moe_ep_workspace_bytes(1, E), dtype=torch.uint8, device="cuda")
+        moe.moe_ep_plan(torch.from_numpy(counts).cuda(), 1, 0, E, -1, rows, ep_ws)
+        addr = moe.moe_ipc_import(handle)
+        moe.moe_ep_dispatch(x_perm, 1, 0, E, d, [addr], ep_ws)
+        torch.cuda.synchronize()
+        rc = moe.moe_get_error()
+        moe.moe_ipc_close(addr, handle)
+        q.put(("ok", rc))
+    except Exception as e:      # reported to the parent, which fails the test
+        q.put(("error", repr(e)))
+
+
+def test_ipc_peer_put_from_another_process(moe):
+    """A second process on the same GPU imports this process's receive buffer (moe_ipc_export /
+    moe_ipc_import) and the library's put kernel stores rows into it: the rows arrive intact, at the
+    exported pointer's offset inside its allocation."""
+    import subprocess
+    import torch.multiprocessing as mp
+    mode = subprocess.run(["nvidia-smi", "--query-gpu=compute_mode", "--format=csv,noheader", "-i", "0"],
+                          capture_output=True, text=True).stdout.strip()
+    if "Exclusive" in mode:
+        pytest.skip(f"compute mode {mode}: a second process cannot use the GPU")
+    rows, d, E = 512, 256, 4
+    pad = torch.zeros(4096, dtype=torch.uint8, device="cuda")        # an allocation with an offset inside
+    recv = torch.zeros((rows + 8, d), dtype=torch.bfloat16, device="cuda")
+    handle = moe.moe_ipc_export(recv[8:])
+    assert len(handle) == moe.MOE_IPC_HANDLE_BYTES
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_ipc_child, args=(handle, rows, d, E, q))
+    p.start()
+    status, info = q.get(timeout=300)
+    p.join(timeout=120)
+    assert status == "ok" and info == 0, info
+    assert p.exitcode == 0
+    want = synth.normal_bf16(9, 1, 0, rows * d, 1.0).reshape(rows, d)
+    assert np.array_equal(bf16_bits(recv[8:]), want)
+    assert not bf16_bits(recv[:8]).any()                  # nothing before the exported pointer
+    del pad

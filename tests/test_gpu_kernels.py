@@ -383,6 +383,41 @@ def test_pipeline_matches_layer_forward_batch_by_batch(moe):
     assert moe.moe_get_error() == 0
 
 
+@pytest.mark.parametrize("a8", [False, True], ids=["fp8-weights", "fp8-weights-and-activations"])
+def test_fp8_pipeline_matches_layer_forward_batch_by_batch(moe, a8):
+    """moe_pipeline_create_w8: the fp8 layers through the host-buffer pipeline, bit for bit the
+    same as the layer called on each batch."""
+    wl = synth.Workload("pipe8", 384, 256, 8, 2, 256, f_shared=128, bias_range=0.1,
+                        cap_mode=synth.CAP_PER_TOKEN, capacity_factor=1.5)
+    T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
+    inp = synth.Inputs(wl)
+    Wg = to_dev_bf16(inp.wg())
+    bias = torch.from_numpy(inp.bias()).cuda()
+    Q = synth.device_tensors_q8(wl, "cuda")
+    routed = {"W1q": Q["w1q"], "W3q": Q["w3q"], "W2q": Q["w2q"], "s1": Q["s1"], "s3": Q["s3"], "s2": Q["s2"]}
+    shared = {"W1q": Q["w1sq"], "W3q": Q["w3sq"], "W2q": Q["w2sq"], "s1": Q["s1s"], "s3": Q["s3s"], "s2": Q["s2s"]}
+    nb = 4
+    xs = [torch.from_numpy(inp.x_rows(b * T, T).view(np.int16)).view(torch.bfloat16).reshape(T, d).pin_memory()
+          for b in range(nb)]
+    outs = [torch.zeros((T, d), dtype=torch.bfloat16).pin_memory() for _ in range(nb)]
+    mem = torch.empty(moe.moe_pipeline_bytes_w8(T, d, E, k, f, fs, a8), dtype=torch.uint8, device="cuda")
+    pl = moe.Pipeline(Wg, bias, None, None, None, None, None, None, fs, T, d, E, k, f, wl.capacity_factor,
+                      wl.cap_mode, mem, routed=routed, shared=shared, activations_fp8=a8)
+    for b in range(nb):
+        pl.submit(xs[b], outs[b])
+    pl.sync()
+    pl.close()
+    call = moe.moe_layer_forward_w8a8 if a8 else moe.moe_layer_forward_w8
+    ws_bytes = moe.moe_workspace_bytes_a8(T, d, E, k, f, fs) if a8 else moe.moe_workspace_bytes(T, d, E, k, f, fs)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    ref = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    for b in range(nb):
+        call(xs[b].cuda(), Wg, bias, Q["w1q"], Q["s1"], Q["w3q"], Q["s3"], Q["w2q"], Q["s2"], Q["w1sq"], Q["s1s"],
+             Q["w3sq"], Q["s3s"], Q["w2sq"], Q["s2s"], fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, ref, ws)
+        assert torch.equal(outs[b].view(torch.int16), ref.cpu().view(torch.int16)), f"batch {b}"
+    assert moe.moe_get_error() == 0
+
+
 # ----------------------------------------------------------------------------- fp8 expert weights
 
 def _q8_reference(wl, x, logits, inp, k, C):
