@@ -75,6 +75,9 @@ def parse():
     ap.add_argument("--ep-ranks", type=int, default=0,
                     help="> 0: expert parallelism with this many ranks emulated on one GPU (the workload's batch "
                          "split over the ranks, experts split contiguously); prints its own line")
+    ap.add_argument("--ep-exchange", default="fused", choices=["put", "fused", "a2a"],
+                    help="with --ep-ranks: put kernels both ways; put dispatch + return from GEMM2's own stores "
+                         "(fused); or all-to-all-v style copies")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
                     help="at N=1 with bf16 weights the line also carries per_config: every workload of the "
@@ -580,7 +583,7 @@ def run_ep(args, wl, local):
     W = synth.device_tensors(wl, dev, names=["x", "wg", "w1", "w3", "w2", "w1s", "w3s", "w2s", "bias"])
     xs = [W["x"][r * Tr:(r + 1) * Tr] for r in range(R)]
     outs = [torch.empty((Tr, d), dtype=torch.bfloat16, device=dev) for _ in range(R)]
-    ep = EmulatedEP(R, Tr, d, E, k, f, fs, device=dev)
+    ep = EmulatedEP(R, Tr, d, E, k, f, fs, device=dev, exchange=args.ep_exchange)
 
     def step(events=None):
         ep.forward(xs, W["wg"], W["bias"], W["w1"], W["w3"], W["w2"], W.get("w1s"), W.get("w3s"), W.get("w2s"),
@@ -622,9 +625,13 @@ def run_ep(args, wl, local):
     if moe.moe_get_error() != 0:
         raise RuntimeError("device error")
     N = sum(int(moe.workspace_view(b.ws, b.layout, "counts", (E,), torch.int32).sum()) for b in ep.ranks)
-    moved = 2 * N * d * 2                       # rows out and back, bf16
-    put_ms = stage_ms["dispatch"] + stage_ms["return"]
+    fused = args.ep_exchange == "fused"
+    moved = (1 if fused else 2) * N * d * 2     # rows out (and back, unless GEMM2 returns them), bf16
+    put_ms = stage_ms["dispatch"] + (0.0 if fused else stage_ms["return"])
     achieved = 2 * moved / 1e9 / (put_ms / 1e3)  # read + write
+    put_kernel = ("ep_put_rows_kernel (dispatch row ranges; GEMM2's epilogue stores the results into the "
+                  "tokens' ranks' y_perm)" if fused else
+                  "ep_put_rows_kernel (dispatch + return row ranges between the ranks' buffers)")
     peaks, peak_src = load_peaks()
     line = {
         "metric": "MoE-layer tokens/s on 1 B200, experts split over R expert-parallel ranks emulated on the GPU",
@@ -637,8 +644,10 @@ def run_ep(args, wl, local):
                    "l2": "working set larger than L2 (expert weights streamed every step)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                     "kernel": "ep_put_rows_kernel (dispatch + return row ranges between the ranks' buffers)",
-                     "peak_source": f"{peak_src} (hbm_gbs, burst)", "algorithmic_per_launch": 2 * moved / (2 * R)},
+                     "kernel": put_kernel,
+                     "peak_source": f"{peak_src} (hbm_gbs, burst)",
+                     "algorithmic_per_launch": 2 * moved / ((1 if fused else 2) * R)},
+        "exchange": args.ep_exchange,
         "single_gpu_layer_ms": single_ms / K,
         "stages_ms": stage_ms,
         "e2e": None,

@@ -362,6 +362,23 @@ int moe_ep_expert_ffn(const moe_bf16* recv_x, int max_recv_rows, int source_majo
                       size_t ep_ws_bytes, moe_stream_t stream);
 int moe_ep_return(const moe_bf16* y_recv, int R, int rank, int E, int d, moe_bf16* const* y_perm_bufs,
                   const void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream);
+/*
+ * Steps 6 and 7 in one: moe_ep_expert_ffn() (expert-major receive buffer, after
+ * moe_ep_dispatch()) whose second grouped GEMM stores every result row straight into the y_perm of
+ * the rank the row came from, at the row it had there ([EP-KV] section 7: the combine-side
+ * exchange fused into the expert computation), so the rows cross to the other GPUs while later
+ * tiles are still being computed and no y_recv buffer or return copy is needed.  A small kernel
+ * first writes the byte address of every received row's destination into row_dest
+ * [max_recv_rows] int64 (device, 16-byte aligned, caller-owned scratch).  y_perm_bufs: as for
+ * moe_ep_return().  The shared expert's output goes to y_shared as in moe_ep_expert_ffn().  The
+ * results are the same bits as moe_ep_expert_ffn() + moe_ep_return().
+ */
+int moe_ep_expert_ffn_return(const moe_bf16* recv_x, int max_recv_rows, int R, int rank, int E, int d, int f,
+                             const moe_bf16* W1_local, const moe_bf16* W3_local, const moe_bf16* W2_local,
+                             moe_bf16* h, const moe_bf16* x, int T, const moe_bf16* W1s, const moe_bf16* W3s,
+                             const moe_bf16* W2s, int f_shared, moe_bf16* h_shared, moe_bf16* y_shared,
+                             moe_bf16* const* y_perm_bufs, int64_t* row_dest, const void* ep_ws, size_t ep_ws_bytes,
+                             moe_stream_t stream);
 
 /*
  * Peer buffers for the put exchange with one process per GPU ([EP-KV] section 7: point-to-point

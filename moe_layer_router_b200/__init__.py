@@ -101,6 +101,9 @@ _lib.moe_ep_expert_ffn.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32
 _lib.moe_ep_expert_ffn.restype = _i32
 _lib.moe_ep_return.argtypes = [_vp, _i32, _i32, _i32, _i32, ctypes.POINTER(_vp), _vp, _sz, _vp]
 _lib.moe_ep_return.restype = _i32
+_lib.moe_ep_expert_ffn_return.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp,
+                                          _vp, _vp, _i32, _vp, _vp, ctypes.POINTER(_vp), _vp, _vp, _sz, _vp]
+_lib.moe_ep_expert_ffn_return.restype = _i32
 _lib.moe_ep_splits_offset.argtypes = [_i32, _i32, ctypes.POINTER(_sz)]
 _lib.moe_ep_splits_offset.restype = _i32
 _lib.moe_ipc_export.argtypes = [_vp, _vp]
@@ -465,6 +468,19 @@ def moe_ep_return(y_recv, R, rank, E, d, y_perm_bufs, ep_ws, stream=None) -> Non
     """y_perm_bufs: R tensors (or device addresses), rank s's y_perm (in its layer workspace)."""
     _check(_lib.moe_ep_return(_ptr(y_recv), R, rank, E, d, _addr_array(y_perm_bufs), _ptr(ep_ws), _nbytes(ep_ws),
                               _stream(stream)), "moe_ep_return")
+
+
+def moe_ep_expert_ffn_return(recv_x, max_recv_rows, R, rank, E, d, f, W1_local, W3_local, W2_local, h, x, T, W1s,
+                             W3s, W2s, f_shared, h_shared, y_shared, y_perm_bufs, row_dest, ep_ws,
+                             stream=None) -> None:
+    """The local experts with the return exchange fused into GEMM2's stores: result rows go straight
+    to y_perm_bufs[source rank] (R tensors or device addresses); row_dest: int64 scratch
+    [max_recv_rows]."""
+    _check(_lib.moe_ep_expert_ffn_return(_ptr(recv_x), max_recv_rows, R, rank, E, d, f, _ptr(W1_local),
+                                         _ptr(W3_local), _ptr(W2_local), _ptr(h), _ptr(x), T, _ptr(W1s), _ptr(W3s),
+                                         _ptr(W2s), f_shared, _ptr(h_shared), _ptr(y_shared),
+                                         _addr_array(y_perm_bufs), _ptr(row_dest), _ptr(ep_ws), _nbytes(ep_ws),
+                                         _stream(stream)), "moe_ep_expert_ffn_return")
 
 
 def moe_ep_splits(ep_ws, R: int, E: int):

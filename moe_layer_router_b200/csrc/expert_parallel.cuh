@@ -204,4 +204,19 @@ __global__ void __launch_bounds__(256) ep_put_rows_kernel(const int32_t* __restr
         d[i] = s[i];
 }
 
+// The fused return: the byte address, in its source rank's y_perm, of every received row's
+// result, from the return table ([3, E]: row in the receive buffer, rows, row in the source
+// rank's y_perm; range g = s El + j goes to rank s = g / El).  GEMM2's epilogue then stores each
+// result row straight there (peer stores on several GPUs), instead of a separate put kernel.
+// blockIdx.y = range, grid-stride over its rows.
+__global__ void __launch_bounds__(256) ep_row_dest_kernel(const int32_t* __restrict__ table, int E, int El,
+                                                          EpDests dest, long long row_bytes,
+                                                          long long* __restrict__ row_addr) {
+    const int g = blockIdx.y;
+    const int row0 = table[g], rows = table[E + g], dst0 = table[2 * E + g];
+    const long long base = reinterpret_cast<long long>(dest.base[g / El]);
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < rows; i += gridDim.x * blockDim.x)
+        row_addr[row0 + i] = base + (long long)(dst0 + i) * row_bytes;
+}
+
 }  // namespace moe

@@ -70,6 +70,9 @@ struct GemmClass {
     const float* b_scale;
     const float* b_scale2;
     long long b_scale_stride;
+    // nullable: output row r (A-row index) goes to the byte address row_addr[r] instead of
+    // out + (out_row0 + r) * ldo (rows of another rank's buffer, for the fused return exchange)
+    const long long* row_addr;
 };
 
 struct GemmParams {
@@ -199,6 +202,25 @@ __device__ __forceinline__ void store_rows_staged(const uint32_t (&packed)[16], 
         const int r = 8 * j + (lane >> 2), q = lane & 3;
         const uint4 w = stage[r * 4 + (q ^ ((r >> 1) & 3))];
         if ((valid >> r) & 1u) reinterpret_cast<uint4*>(out0 + r * ldo)[q] = w;
+    }
+}
+
+// store_rows_staged with one base pointer per row: lane l holds row l's (column 0) address in
+// `row_ptr` (any value for rows whose bit in `valid` is clear); the 32 columns go to col0 onwards.
+__device__ __forceinline__ void store_rows_staged_ptr(const uint32_t (&packed)[16], uint4* stage, int lane,
+                                                      unsigned long long row_ptr, int col0, uint32_t valid) {
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        stage[lane * 4 + (q ^ ((lane >> 1) & 3))] =
+            make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int r = 8 * j + (lane >> 2), q = lane & 3;
+        const uint4 w = stage[r * 4 + (q ^ ((r >> 1) & 3))];
+        const unsigned long long p = __shfl_sync(0xffffffffu, row_ptr, r);
+        if ((valid >> r) & 1u) reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p) + col0)[q] = w;
     }
 }
 
@@ -412,6 +434,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
                 }
             } else if (EPI == EPI_STORE) {
                 __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(c.out) + orow * c.ldo;
+                if (c.row_addr && row_ok)
+                    out = reinterpret_cast<__nv_bfloat16*>(__ldg(c.row_addr + ti.a_row + row_in_tile));
 #pragma unroll 1
                 for (int ch = 0; ch < c.mma_n / 32; ++ch) {
                     uint32_t v[32];

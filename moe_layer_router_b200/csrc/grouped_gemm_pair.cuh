@@ -316,8 +316,11 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
             const long long orow = c.out_row0 + ti.a_row + row_in_tile;
             const bool row_ok = row_in_tile < ti.rows && orow >= 0 && orow < c.out_rows;
             // the warp's 32 rows are consecutive: out0 is its first row, valid has a bit per row
+            // (with a row table: each lane's own row address instead)
             __nv_bfloat16* out0 = reinterpret_cast<__nv_bfloat16*>(c.out) + (orow - lane) * c.ldo;
             const uint32_t valid = __ballot_sync(0xffffffffu, row_ok);
+            const unsigned long long row_ptr =
+                (c.row_addr && row_ok) ? (unsigned long long)__ldg(c.row_addr + ti.a_row + row_in_tile) : 0ull;
             float sa = 1.f;                        // fp8: activation row scale, weight column scales
             const float *sb = nullptr, *sb2 = nullptr;
             if (F8) {
@@ -411,7 +414,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                             if (col_ok && tok < ti.rows && orow_t >= 0 && orow_t < c.out_rows) {
                                 float val = __uint_as_float(v[j]);
                                 if (F8) val = val * __ldg(c.a_scale + ti.a_row + tok) * sc;
-                                out[orow_t * c.ldo + col] = __float2bfloat16_rn(val);
+                                __nv_bfloat16* o = c.row_addr ? reinterpret_cast<__nv_bfloat16*>(
+                                                                    __ldg(c.row_addr + ti.a_row + tok))
+                                                              : out + orow_t * c.ldo;
+                                o[col] = __float2bfloat16_rn(val);
                             }
                         }
                     }
@@ -447,7 +453,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                         if (F8) scale_cols32(v, sa, sb + col0);
                         uint32_t packed[16];
                         pack32(v, packed);
-                        store_rows_staged(packed, stage, lane, out0 + col0, c.ldo, valid);
+                        if (c.row_addr) store_rows_staged_ptr(packed, stage, lane, row_ptr, col0, valid);
+                        else store_rows_staged(packed, stage, lane, out0 + col0, c.ldo, valid);
                     }
                 }
             }

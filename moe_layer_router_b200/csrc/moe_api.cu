@@ -413,6 +413,7 @@ struct FfnArgs {
     bool pair;   // 2-SM tiles (mprefix counts 256-row tiles) instead of 1-SM tiles (128 rows)
     const int32_t* group_map;   // routed group -> weight group (expert cache slots), nullptr = identity
     int w_groups;               // weight groups in W1/W3/W2 (0 = E)
+    const long long* y_row_addr;  // nullable: GEMM2 stores routed row r at this byte address (fused return)
 };
 
 inline uint64_t weight_groups(const FfnArgs& a) { return (uint64_t)(a.w_groups ? a.w_groups : a.E); }
@@ -486,6 +487,7 @@ int run_expert_ffn(DeviceInfo* di, const FfnArgs& a, cudaStream_t s, cudaEvent_t
         GemmClass& c0 = p.cls[0];
         c0.K = a.f; c0.n_out = a.d; c0.ntiles = (a.d + 255) / 256; c0.b_group_rows = a.d; c0.b_tile_rows = 256;
         c0.mma_n = 256; c0.out = a.y_perm; c0.ldo = a.d; c0.out_row0 = 0; c0.out_rows = a.max_rows;
+        c0.row_addr = a.y_row_addr;
         GemmClass& c1 = p.cls[1];
         c1.K = a.f_shared; c1.n_out = a.d; c1.ntiles = (a.d + 255) / 256; c1.b_group_rows = 0; c1.b_tile_rows = 256;
         c1.mma_n = 256; c1.out = a.y_shared; c1.ldo = a.d; c1.out_row0 = 0; c1.out_rows = a.T;
@@ -1554,6 +1556,63 @@ int moe_ep_return(const moe_bf16* y_recv, int R, int rank, int E, int d, moe_bf1
     MOE_REQUIRE(ep_ws_bytes >= ep_bytes(R, E), MOE_ERR_WORKSPACE);
     const EpView v = ep_view(const_cast<void*>(ep_ws), R, E);
     return ep_put(y_recv, v.back, y_perm_bufs, R, E, d, static_cast<cudaStream_t>(stream));
+}
+
+int moe_ep_expert_ffn_return(const moe_bf16* recv_x, int max_recv_rows, int R, int rank, int E, int d, int f,
+                             const moe_bf16* W1_local, const moe_bf16* W3_local, const moe_bf16* W2_local,
+                             moe_bf16* h, const moe_bf16* x, int T, const moe_bf16* W1s, const moe_bf16* W3s,
+                             const moe_bf16* W2s, int f_shared, moe_bf16* h_shared, moe_bf16* y_shared,
+                             moe_bf16* const* y_perm_bufs, int64_t* row_dest, const void* ep_ws, size_t ep_ws_bytes,
+                             moe_stream_t stream) {
+    using namespace moe;
+    int rc = ep_check(R, rank, E, d);
+    if (rc != MOE_OK) return rc;
+    MOE_REQUIRE(max_recv_rows >= 0 && f >= 64 && f % 64 == 0 && f_shared >= 0 && f_shared % 64 == 0, MOE_ERR_SHAPE);
+    const bool shared = f_shared > 0;
+    MOE_REQUIRE(ep_ws && y_perm_bufs && (max_recv_rows == 0 || (recv_x && W1_local && W3_local && W2_local && h &&
+                                                                 row_dest)),
+                MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(!shared || (x && T >= 1 && W1s && W3s && W2s && h_shared && y_shared), MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(recv_x) && aligned16(W1_local) && aligned16(W3_local) && aligned16(W2_local) &&
+                    aligned16(h) && aligned16(x) && aligned16(W1s) && aligned16(W3s) && aligned16(W2s) &&
+                    aligned16(h_shared) && aligned16(y_shared) && aligned16(ep_ws) && aligned16(row_dest),
+                MOE_ERR_ALIGN);
+    MOE_REQUIRE(ep_ws_bytes >= ep_bytes(R, E), MOE_ERR_WORKSPACE);
+    EpDests dst;
+    memset(&dst, 0, sizeof(dst));
+    for (int q = 0; q < R; ++q) {
+        MOE_REQUIRE(y_perm_bufs[q] && aligned16(y_perm_bufs[q]), MOE_ERR_INVALID_ARG);
+        dst.base[q] = reinterpret_cast<char*>(y_perm_bufs[q]);
+    }
+    DeviceInfo* di;
+    if ((rc = device_info(&di)) != MOE_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const EpView v = ep_view(const_cast<void*>(ep_ws), R, E);
+    const int El = E / R;
+    if (max_recv_rows > 0) {
+        const int bx = std::max(1, std::min(8, (2 * di->sms + E - 1) / E));
+        ep_row_dest_kernel<<<dim3(bx, E), 256, 0, s>>>(v.back, E, El, dst, (long long)d * 2,
+                                                      reinterpret_cast<long long*>(row_dest));
+        if ((rc = launch_status()) != MOE_OK) return rc;
+    }
+    FfnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x_perm = recv_x;
+    a.max_rows = max_recv_rows;
+    a.offsets = max_recv_rows ? v.exp_off : nullptr;
+    a.mprefix = v.exp_tiles;
+    a.E = El;
+    a.d = d;
+    a.f = f;
+    a.W1 = W1_local; a.W3 = W3_local; a.W2 = W2_local;
+    a.h = h;
+    a.y_perm = reinterpret_cast<moe_bf16*>(dst.base[rank]);   // only for the tensor-map checks: rows go by row_dest
+    a.y_row_addr = reinterpret_cast<const long long*>(row_dest);
+    a.x = x; a.T = T; a.f_shared = f_shared; a.W1s = W1s; a.W3s = W3s; a.W2s = W2s;
+    a.h_shared = h_shared; a.y_shared = y_shared;
+    a.pair = use_pair_tiles(max_recv_rows, El);
+    if (max_recv_rows == 0 && !shared) return MOE_OK;
+    return run_expert_ffn(di, a, s);
 }
 
 int moe_update_bias(const int32_t* counts_raw, int E, int64_t capacity, float* bias, moe_stream_t stream) {

@@ -48,6 +48,7 @@ class _RankBuffers:
         self.y_recv = torch.empty((rows, d), dtype=torch.bfloat16, device=device)
         self.h_shared = torch.empty((T, fs), dtype=torch.bfloat16, device=device) if fs else None
         self.y_shared = torch.empty((T, d), dtype=torch.bfloat16, device=device) if fs else None
+        self.row_dest = torch.empty(rows, dtype=torch.int64, device=device)   # fused return: row addresses
 
     def view(self, moe, name, shape, dtype):
         return moe.workspace_view(self.ws, self.layout, name, shape, dtype)
@@ -58,13 +59,14 @@ class EmulatedEP:
 
     def __init__(self, R, T, d, E, k, f, f_shared=0, device="cuda", exchange="put"):
         """exchange: "put" moves rows with the library's put kernels (expert-major receive order);
-        "a2a" moves them like an all-to-all-v would (source-major, device copies sized on the
-        host from the gathered counts) and runs the source-major GEMM segments."""
+        "fused" dispatches the same way and returns the results from GEMM2's own stores
+        (moe_ep_expert_ffn_return); "a2a" moves them like an all-to-all-v would (source-major,
+        device copies sized by the plans' split tables) and runs the source-major GEMM segments."""
         import moe_layer_router_b200 as moe
         if E % R:
             raise ValueError("E must be a multiple of R")
-        if exchange not in ("put", "a2a"):
-            raise ValueError("exchange must be 'put' or 'a2a'")
+        if exchange not in ("put", "fused", "a2a"):
+            raise ValueError("exchange must be 'put', 'fused' or 'a2a'")
         self.exchange = exchange
         self.moe, self.R, self.T, self.d, self.E, self.k, self.f, self.fs = moe, R, T, d, E, k, f, f_shared
         self.max_recv = R * T * k
@@ -111,12 +113,20 @@ class EmulatedEP:
             for r, b in enumerate(self.ranks):
                 moe.moe_ep_dispatch(x_perm[r], R, r, E, d, recv, b.ep_ws)
         mark("experts")
+        fused = self.exchange == "fused"
         for r, b in enumerate(self.ranks):
             sl = slice(r * El, (r + 1) * El)
-            moe.moe_ep_expert_ffn(b.recv, self.max_recv, R, r, E, d, f, W1[sl], W3[sl], W2[sl], b.h, b.y_recv, xs[r],
-                                  T, W1s, W3s, W2s, fs, b.h_shared, b.y_shared, b.ep_ws, source_major=a2a)
+            if fused:     # the results go straight to the tokens' ranks from GEMM2's stores
+                moe.moe_ep_expert_ffn_return(b.recv, self.max_recv, R, r, E, d, f, W1[sl], W3[sl], W2[sl], b.h,
+                                             xs[r], T, W1s, W3s, W2s, fs, b.h_shared, b.y_shared, y_perm, b.row_dest,
+                                             b.ep_ws)
+            else:
+                moe.moe_ep_expert_ffn(b.recv, self.max_recv, R, r, E, d, f, W1[sl], W3[sl], W2[sl], b.h, b.y_recv,
+                                      xs[r], T, W1s, W3s, W2s, fs, b.h_shared, b.y_shared, b.ep_ws, source_major=a2a)
         mark("return")
-        if a2a:
+        if fused:
+            pass
+        elif a2a:
             self._a2a([b.y_recv for b in self.ranks], y_perm, [sp[1] for sp in splits], [sp[0] for sp in splits])
         else:
             for r, b in enumerate(self.ranks):
@@ -215,9 +225,10 @@ class PeerBuffers:
 
 def ep_layer_forward_put_dist(x, Wg, bias, W1_local, W3_local, W2_local, W1s, W3s, W2s, f_shared, T, d, E, k, f,
                               capacity_factor, cap_mode, out, bufs: _RankBuffers, peers: PeerBuffers, group=None):
-    """One rank of an expert-parallel layer whose row exchanges are the library's put kernels
-    storing into the other ranks' buffers (peers: PeerBuffers over bufs.recv and bufs' y_perm).
-    Rows arrive expert-major, so each local expert is one GEMM group.  The collectives: an
+    """One rank of an expert-parallel layer whose row exchanges are peer stores into the other ranks'
+    buffers (peers: PeerBuffers over bufs.recv and bufs' y_perm): the put kernel for the dispatch,
+    GEMM2's own epilogue for the return (moe_ep_expert_ffn_return).  Rows arrive expert-major, so
+    each local expert is one GEMM group.  The collectives: an
     all-gather of the raw counts and two barriers, each after this rank's stream has finished its
     puts, so that no rank reads a buffer before every rank has written it."""
     import torch
@@ -237,9 +248,10 @@ def ep_layer_forward_put_dist(x, Wg, bias, W1_local, W3_local, W2_local, W1s, W3
     moe.moe_ep_dispatch(x_perm, R, rank, E, d, peers.recv, bufs.ep_ws)
     torch.cuda.current_stream(x.device).synchronize()
     dist.barrier(group=group)              # every rank's rows are in every receive buffer
-    moe.moe_ep_expert_ffn(bufs.recv, max_recv, R, rank, E, d, f, W1_local, W3_local, W2_local, bufs.h, bufs.y_recv,
-                          x, T, W1s, W3s, W2s, f_shared, bufs.h_shared, bufs.y_shared, bufs.ep_ws, source_major=False)
-    moe.moe_ep_return(bufs.y_recv, R, rank, E, d, peers.y_perm, bufs.ep_ws)
+    # the local experts; GEMM2 stores each result row straight into its token's rank's y_perm
+    moe.moe_ep_expert_ffn_return(bufs.recv, max_recv, R, rank, E, d, f, W1_local, W3_local, W2_local, bufs.h, x, T,
+                                 W1s, W3s, W2s, f_shared, bufs.h_shared, bufs.y_shared, peers.y_perm, bufs.row_dest,
+                                 bufs.ep_ws)
     torch.cuda.current_stream(x.device).synchronize()
     dist.barrier(group=group)              # every result is back in its token's y_perm
     moe.moe_combine(bufs.view(moe, "y_perm", (T * k, d), x.dtype), bufs.view(moe, "dest", (T, k), torch.int32),

@@ -30,7 +30,7 @@ CASES = {
 }
 
 
-@pytest.mark.parametrize("exchange", ["put", "a2a"])
+@pytest.mark.parametrize("exchange", ["put", "fused", "a2a"])
 @pytest.mark.parametrize("case", list(CASES))
 def test_emulated_expert_parallel_layer(moe, case, exchange):
     from moe_layer_router_b200.ep import EmulatedEP

@@ -106,11 +106,13 @@ def check_x_perm(moe, ws, L, wl, x, r):
     assert np.array_equal(bf16_bits(xp), oracle.gather(x, r["dest"], r["N"]))
 
 
-def check_experts_and_out(moe, ws, L, wl, x, toks, g_idx, dest, w_o, out, expert, shared, label, h_from_gpu=False):
+def check_experts_and_out(moe, ws, L, wl, x, toks, g_idx, dest, w_o, out, expert, shared, label, own=None):
     """h, y_perm (and y_shared) of every assignment of the tokens `toks`, and their outputs.
 
     expert(e, xe, g_h) -> (h_ref, y_ref) of expert e on rows xe; g_h is the GPU's h of those rows
-    (used by the fp8-activation oracle for its second GEMM).  shared(xs, g_h) likewise."""
+    (used by the fp8-activation oracle for its second GEMM).  shared(xs, g_h) likewise.
+    own: optional (expert_own(e, xe) -> y, shared_own(xs) -> y), an oracle that does not take the
+    GPU's h; the outputs it gives are reported against the bar (printed, not asserted)."""
     T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
     toks = np.asarray(sorted(toks), dtype=np.int64)
     S = len(toks)
@@ -123,6 +125,7 @@ def check_experts_and_out(moe, ws, L, wl, x, toks, g_idx, dest, w_o, out, expert
     h_dev = moe.workspace_view(ws, L, "h", (T * k, f), torch.bfloat16)
     y_dev = moe.workspace_view(ws, L, "y_perm", (T * k, d), torch.bfloat16)
     y_ref = np.zeros((len(tt), d), np.uint16)
+    y_own = np.zeros((len(tt), d), np.uint16) if own else None
     worst_h = worst_y = 0.0
     for e in np.unique(ee):
         sel = np.nonzero(ee == e)[0]
@@ -131,6 +134,8 @@ def check_experts_and_out(moe, ws, L, wl, x, toks, g_idx, dest, w_o, out, expert
         worst_h = max(worst_h, _max_rel_excess(g_h, h_ref, H_BAR))
         worst_y = max(worst_y, _max_rel_excess(_rows(y_dev, dd[sel]), ye, OUT_BAR))
         y_ref[sel] = ye
+        if own:
+            y_own[sel] = own[0](int(e), x[tt[sel]])
     assert worst_h <= 1.0, f"{label}: h outside its bar (worst |d| / bar = {worst_h:.3f})"
     assert worst_y <= 1.0, f"{label}: y_perm outside its bar (worst |d| / bar = {worst_y:.3f})"
     ysh = None
@@ -152,6 +157,12 @@ def check_experts_and_out(moe, ws, L, wl, x, toks, g_idx, dest, w_o, out, expert
           f"worst |d|/bar: out {_max_rel_excess(got, ref_out, OUT_BAR):.3f}, y_perm {worst_y:.3f}, h {worst_h:.3f}; "
           f"relative rms {rel_rms:.2e}")
     assert rel_rms < 5e-3                                                  # no systematic drift
+    if own:      # the oracle with its own h throughout: how many outputs leave the bar
+        ref_own = oracle.combine(y_own, mini_dest, w_o[toks], own[1](x[toks]) if fs else None)
+        o64 = bits_to_f64(ref_own)
+        bad = np.abs(g64 - o64) > OUT_BAR[0] + OUT_BAR[1] * np.abs(o64)
+        print(f"{label}: against the oracle with its own h: {int(bad.sum())} of {bad.size} outputs outside the "
+              f"bar, max |d| = {np.abs(g64 - o64).max():.3e}")
 
 
 def token_set(wl, r, mode, seed):
@@ -285,6 +296,13 @@ def test_full_size_fp8_weights_and_activations(moe, name):
         h = oracle.expert_gate_up_w8a8(xs, qs[0][0], qs[0][1], qs[1][0], qs[1][1])
         return h, oracle.expert_down_w8a8(g_h, qs[2][0], qs[2][1])
 
+    def expert_own(e, xe):
+        (q1, s1), (q3, s3), (q2, s2) = q8_weights(inp, wl, e)
+        return oracle.expert_ffn_w8a8(xe, q1, s1, q3, s3, q2, s2)[1]
+
+    def shared_own(xs):
+        return oracle.expert_ffn_w8a8(xs, qs[0][0], qs[0][1], qs[1][0], qs[1][1], qs[2][0], qs[2][1])[1]
+
     toks = token_set(wl, r, "all" if name == "dsv3" else "cover", seed=13)
     check_experts_and_out(moe, ws, L, wl, x, toks, g_idx, r["dest"], w_o, out, expert, shared,
-                          f"{name} fp8 x fp8")
+                          f"{name} fp8 x fp8", own=(expert_own, shared_own))
