@@ -301,6 +301,10 @@ int moe_pipeline_destroy(moe_pipeline* pipeline);
  */
 int moe_layer_permute(const moe_bf16* x, int f_shared, int T, int d, int E, int k, int f, int64_t capacity,
                       const int32_t* fill_base, void* ws, size_t ws_bytes, moe_stream_t stream);
+/* moe_layer_permute() without the row gather: counts, offsets, dest and src_token only; x_perm is
+ * left unwritten (for moe_ep_dispatch_gather(), which moves x's rows itself). */
+int moe_layer_permute_indices(const moe_bf16* x, int f_shared, int T, int d, int E, int k, int f, int64_t capacity,
+                              const int32_t* fill_base, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
  * Expert parallelism: the E routed experts are split over R ranks, rank r holding experts
@@ -354,6 +358,15 @@ int moe_ep_plan(const int32_t* all_counts_raw, int R, int rank, int E, int64_t c
                 void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream);
 int moe_ep_dispatch(const moe_bf16* x_perm, int R, int rank, int E, int d, moe_bf16* const* recv_bufs,
                     const void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream);
+/*
+ * moe_ep_dispatch() fused with the permutation's gather: after moe_layer_permute_indices() and
+ * moe_ep_plan(), each kept row is copied from x (token src_token[r] for x_perm row r; src_token
+ * is the layer workspace's) straight into the receive buffer of its expert's rank, at the row
+ * moe_ep_dispatch() would have put it, so x_perm is never written or read.  Same receive layout
+ * and errors as moe_ep_dispatch().
+ */
+int moe_ep_dispatch_gather(const moe_bf16* x, const int32_t* src_token, int R, int rank, int E, int d,
+                           moe_bf16* const* recv_bufs, const void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream);
 int moe_ep_expert_ffn(const moe_bf16* recv_x, int max_recv_rows, int source_major, int R, int rank, int E, int d,
                       int f,
                       const moe_bf16* W1_local, const moe_bf16* W3_local, const moe_bf16* W2_local, moe_bf16* h,

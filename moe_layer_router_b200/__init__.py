@@ -104,6 +104,10 @@ _lib.moe_ep_return.restype = _i32
 _lib.moe_ep_expert_ffn_return.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _i32, _vp,
                                           _vp, _vp, _i32, _vp, _vp, ctypes.POINTER(_vp), _vp, _vp, _sz, _vp]
 _lib.moe_ep_expert_ffn_return.restype = _i32
+_lib.moe_ep_dispatch_gather.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, ctypes.POINTER(_vp), _vp, _sz, _vp]
+_lib.moe_ep_dispatch_gather.restype = _i32
+_lib.moe_layer_permute_indices.argtypes = _lib.moe_layer_permute.argtypes
+_lib.moe_layer_permute_indices.restype = _i32
 _lib.moe_ep_splits_offset.argtypes = [_i32, _i32, ctypes.POINTER(_sz)]
 _lib.moe_ep_splits_offset.restype = _i32
 _lib.moe_ipc_export.argtypes = [_vp, _vp]
@@ -468,6 +472,18 @@ def moe_ep_return(y_recv, R, rank, E, d, y_perm_bufs, ep_ws, stream=None) -> Non
     """y_perm_bufs: R tensors (or device addresses), rank s's y_perm (in its layer workspace)."""
     _check(_lib.moe_ep_return(_ptr(y_recv), R, rank, E, d, _addr_array(y_perm_bufs), _ptr(ep_ws), _nbytes(ep_ws),
                               _stream(stream)), "moe_ep_return")
+
+
+def moe_layer_permute_indices(x, f_shared, T, d, E, k, f, capacity, fill_base, ws, stream=None) -> None:
+    """moe_layer_permute without the gather: dest and src_token only (x_perm unwritten)."""
+    _check(_lib.moe_layer_permute_indices(_ptr(x), f_shared, T, d, E, k, f, int(capacity), _ptr(fill_base), _ptr(ws),
+                                          _nbytes(ws), _stream(stream)), "moe_layer_permute_indices")
+
+
+def moe_ep_dispatch_gather(x, src_token, R, rank, E, d, recv_bufs, ep_ws, stream=None) -> None:
+    """The dispatch fused with the gather: x's kept rows straight into the receive buffers."""
+    _check(_lib.moe_ep_dispatch_gather(_ptr(x), _ptr(src_token), R, rank, E, d, _addr_array(recv_bufs), _ptr(ep_ws),
+                                       _nbytes(ep_ws), _stream(stream)), "moe_ep_dispatch_gather")
 
 
 def moe_ep_expert_ffn_return(recv_x, max_recv_rows, R, rank, E, d, f, W1_local, W3_local, W2_local, h, x, T, W1s,

@@ -204,6 +204,25 @@ __global__ void __launch_bounds__(256) ep_put_rows_kernel(const int32_t* __restr
         d[i] = s[i];
 }
 
+// The fused dispatch: this rank's kept rows go from x (row src_token[r] for x_perm row r) straight
+// into the receive buffer of each expert's rank, so x_perm is never written or read.  Same ranges
+// as the dispatch put ([3, E] send table); blockIdx.y = range, a warp per row, 16-byte chunks.
+__global__ void __launch_bounds__(256) ep_gather_put_kernel(const int32_t* __restrict__ table, int E, int El,
+                                                            const uint4* __restrict__ x,
+                                                            const int32_t* __restrict__ src_token, EpDests dest,
+                                                            int row_chunks) {
+    const int r = blockIdx.y;
+    const int row0 = table[r], rows = table[E + r], dst0 = table[2 * E + r];
+    uint4* d = reinterpret_cast<uint4*>(dest.base[r / El]) + (long long)dst0 * row_chunks;
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); i < rows; i += warps) {
+        const uint4* src = x + (long long)__ldg(src_token + row0 + i) * row_chunks;
+        uint4* dst = d + (long long)i * row_chunks;
+        for (int c = lane; c < row_chunks; c += 32) dst[c] = __ldg(src + c);
+    }
+}
+
 // The fused return: the byte address, in its source rank's y_perm, of every received row's
 // result, from the return table ([3, E]: row in the receive buffer, rows, row in the source
 // rank's y_perm; range g = s El + j goes to rank s = g / El).  GEMM2's epilogue then stores each

@@ -962,7 +962,7 @@ int moe_layer_forward(const moe_bf16* x, const moe_bf16* Wg, const float* bias, 
 namespace moe {
 namespace {
 
-enum { LAYER_ROUTE = 1, LAYER_COUNT = 2, LAYER_FINISH = 4, LAYER_PERMUTE = 8 };
+enum { LAYER_ROUTE = 1, LAYER_COUNT = 2, LAYER_FINISH = 4, LAYER_PERMUTE = 8, LAYER_INDICES = 16 };
 
 // The layer in phases over one workspace:
 //   LAYER_ROUTE   router GEMM + top-k                 (needs x, Wg, bias)
@@ -1052,9 +1052,9 @@ int layer_phases(int phases, const moe_bf16* x, const moe_bf16* Wg, const float*
                               rank_local, mprefix, s, GEMM_BM, nullptr, true)) != MOE_OK)
             return rc;
     }
-    if (phases & LAYER_PERMUTE)
+    if (phases & (LAYER_PERMUTE | LAYER_INDICES))   // LAYER_INDICES: dest / src_token only, no x_perm
         return run_permute(di, x, idx, T, d, E, k, C, counts_raw, counts, offsets, dest, src, x_perm, blk_cnt,
-                           rank_local, mprefix, s, GEMM_BM, fill_base);
+                           rank_local, mprefix, s, GEMM_BM, fill_base, false, !(phases & LAYER_INDICES));
     if (!(phases & LAYER_FINISH)) return MOE_OK;
     if (!mark(ev.permute)) return MOE_ERR_CUDA;
     // fp8 activations: each x row is quantised once and written to its rows by dest: no x_perm
@@ -1339,6 +1339,13 @@ int moe_layer_permute(const moe_bf16* x, int f_shared, int T, int d, int E, int 
                         ws_bytes, static_cast<cudaStream_t>(stream), nullptr);
 }
 
+int moe_layer_permute_indices(const moe_bf16* x, int f_shared, int T, int d, int E, int k, int f, int64_t capacity,
+                              const int32_t* fill_base, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    return layer_phases(LAYER_INDICES, x, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                        f_shared, T, d, E, k, f, capacity < 0 ? -1 : (long long)capacity, fill_base, nullptr, ws,
+                        ws_bytes, static_cast<cudaStream_t>(stream), nullptr);
+}
+
 // ------------------------------------------------------------------ expert parallelism
 
 namespace {
@@ -1556,6 +1563,29 @@ int moe_ep_return(const moe_bf16* y_recv, int R, int rank, int E, int d, moe_bf1
     MOE_REQUIRE(ep_ws_bytes >= ep_bytes(R, E), MOE_ERR_WORKSPACE);
     const EpView v = ep_view(const_cast<void*>(ep_ws), R, E);
     return ep_put(y_recv, v.back, y_perm_bufs, R, E, d, static_cast<cudaStream_t>(stream));
+}
+
+int moe_ep_dispatch_gather(const moe_bf16* x, const int32_t* src_token, int R, int rank, int E, int d,
+                           moe_bf16* const* recv_bufs, const void* ep_ws, size_t ep_ws_bytes, moe_stream_t stream) {
+    using namespace moe;
+    int rc = ep_check(R, rank, E, d);
+    if (rc != MOE_OK) return rc;
+    MOE_REQUIRE(x && src_token && recv_bufs && ep_ws, MOE_ERR_INVALID_ARG);
+    MOE_REQUIRE(aligned16(x) && aligned16(ep_ws), MOE_ERR_ALIGN);
+    MOE_REQUIRE(ep_ws_bytes >= ep_bytes(R, E), MOE_ERR_WORKSPACE);
+    EpDests dst;
+    memset(&dst, 0, sizeof(dst));
+    for (int q = 0; q < R; ++q) {
+        MOE_REQUIRE(recv_bufs[q] && aligned16(recv_bufs[q]), MOE_ERR_INVALID_ARG);
+        dst.base[q] = reinterpret_cast<char*>(recv_bufs[q]);
+    }
+    DeviceInfo* di;
+    if ((rc = device_info(&di)) != MOE_OK) return rc;
+    const EpView v = ep_view(const_cast<void*>(ep_ws), R, E);
+    const int bx = std::max(1, std::min(16, (4 * di->sms + E - 1) / E));
+    ep_gather_put_kernel<<<dim3(bx, E), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        v.send, E, E / R, reinterpret_cast<const uint4*>(x), src_token, dst, d / 8);
+    return launch_status();
 }
 
 int moe_ep_expert_ffn_return(const moe_bf16* recv_x, int max_recv_rows, int R, int rank, int E, int d, int f,

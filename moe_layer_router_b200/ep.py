@@ -59,9 +59,10 @@ class EmulatedEP:
 
     def __init__(self, R, T, d, E, k, f, f_shared=0, device="cuda", exchange="put"):
         """exchange: "put" moves rows with the library's put kernels (expert-major receive order);
-        "fused" dispatches the same way and returns the results from GEMM2's own stores
-        (moe_ep_expert_ffn_return); "a2a" moves them like an all-to-all-v would (source-major,
-        device copies sized by the plans' split tables) and runs the source-major GEMM segments."""
+        "fused" gathers x's rows straight into the receive buffers (moe_ep_dispatch_gather, no
+        x_perm) and returns the results from GEMM2's own stores (moe_ep_expert_ffn_return); "a2a"
+        moves them like an all-to-all-v would (source-major, device copies sized by the plans' split
+        tables) and runs the source-major GEMM segments."""
         import moe_layer_router_b200 as moe
         if E % R:
             raise ValueError("E must be a multiple of R")
@@ -95,9 +96,13 @@ class EmulatedEP:
         mark("permute")
         for r, b in enumerate(self.ranks):          # the all-gather of raw counts
             self.all_counts[r].copy_(b.view(moe, "counts_raw", (E,), self.all_counts.dtype))
+        fused = self.exchange == "fused"
         for r, b in enumerate(self.ranks):
             moe.moe_fill_base(self.all_counts, R, r, E, b.fill_base)
-            moe.moe_layer_permute(xs[r], fs, T, d, E, k, f, C, b.fill_base, b.ws)
+            if fused:       # no x_perm: the dispatch gathers x's rows itself
+                moe.moe_layer_permute_indices(xs[r], fs, T, d, E, k, f, C, b.fill_base, b.ws)
+            else:
+                moe.moe_layer_permute(xs[r], fs, T, d, E, k, f, C, b.fill_base, b.ws)
             moe.moe_ep_plan(self.all_counts, R, r, E, C, self.max_recv, b.ep_ws)
         recv = [b.recv for b in self.ranks]
         x_perm = [b.view(moe, "x_perm", (T * k, d), xs[r].dtype) for r, b in enumerate(self.ranks)]
@@ -109,11 +114,14 @@ class EmulatedEP:
         mark("dispatch")
         if a2a:
             self._a2a([x_perm[r] for r in range(R)], recv, [sp[0] for sp in splits], [sp[1] for sp in splits])
+        elif fused:
+            for r, b in enumerate(self.ranks):
+                moe.moe_ep_dispatch_gather(xs[r], b.view(moe, "src_token", (T * k,), self.all_counts.dtype), R, r, E,
+                                           d, recv, b.ep_ws)
         else:
             for r, b in enumerate(self.ranks):
                 moe.moe_ep_dispatch(x_perm[r], R, r, E, d, recv, b.ep_ws)
         mark("experts")
-        fused = self.exchange == "fused"
         for r, b in enumerate(self.ranks):
             sl = slice(r * El, (r + 1) * El)
             if fused:     # the results go straight to the tokens' ranks from GEMM2's stores
@@ -226,8 +234,9 @@ class PeerBuffers:
 def ep_layer_forward_put_dist(x, Wg, bias, W1_local, W3_local, W2_local, W1s, W3s, W2s, f_shared, T, d, E, k, f,
                               capacity_factor, cap_mode, out, bufs: _RankBuffers, peers: PeerBuffers, group=None):
     """One rank of an expert-parallel layer whose row exchanges are peer stores into the other ranks'
-    buffers (peers: PeerBuffers over bufs.recv and bufs' y_perm): the put kernel for the dispatch,
-    GEMM2's own epilogue for the return (moe_ep_expert_ffn_return).  Rows arrive expert-major, so
+    buffers (peers: PeerBuffers over bufs.recv and bufs' y_perm): a gather kernel that copies x's
+    kept rows straight to their experts' ranks for the dispatch (moe_ep_dispatch_gather), GEMM2's
+    own epilogue for the return (moe_ep_expert_ffn_return).  Rows arrive expert-major, so
     each local expert is one GEMM group.  The collectives: an
     all-gather of the raw counts and two barriers, each after this rank's stream has finished its
     puts, so that no rank reads a buffer before every rank has written it."""
@@ -242,10 +251,11 @@ def ep_layer_forward_put_dist(x, Wg, bias, W1_local, W3_local, W2_local, W1s, W3
     all_counts = torch.empty((R, E), dtype=torch.int32, device=x.device)
     dist.all_gather_into_tensor(all_counts, bufs.view(moe, "counts_raw", (E,), torch.int32), group=group)
     moe.moe_fill_base(all_counts, R, rank, E, bufs.fill_base)
-    moe.moe_layer_permute(x, f_shared, T, d, E, k, f, C, bufs.fill_base, bufs.ws)
+    moe.moe_layer_permute_indices(x, f_shared, T, d, E, k, f, C, bufs.fill_base, bufs.ws)
     moe.moe_ep_plan(all_counts, R, rank, E, C, max_recv, bufs.ep_ws)
-    x_perm = bufs.view(moe, "x_perm", (T * k, d), x.dtype)
-    moe.moe_ep_dispatch(x_perm, R, rank, E, d, peers.recv, bufs.ep_ws)
+    # x's kept rows straight into the experts' ranks' receive buffers (no x_perm)
+    moe.moe_ep_dispatch_gather(x, bufs.view(moe, "src_token", (T * k,), torch.int32), R, rank, E, d, peers.recv,
+                               bufs.ep_ws)
     torch.cuda.current_stream(x.device).synchronize()
     dist.barrier(group=group)              # every rank's rows are in every receive buffer
     # the local experts; GEMM2 stores each result row straight into its token's rank's y_perm
