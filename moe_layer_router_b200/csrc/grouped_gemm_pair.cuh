@@ -60,6 +60,27 @@ struct PairSwapMaps {
 };
 
 
+// Swapped tiles: a warp's 32 consecutive output columns (lane = column) x 32 tokens (vals[j] =
+// token j, fp32 bits) as bf16, written through the warp's 2 KB staging slot so that each lane stores 16-byte
+// pieces of token rows (a warp store covers 8 token rows x 64 bytes).  Token j goes to
+// rowptr(j) + col0 (elements); tokens with j >= ntok are skipped.  Warp-collective.
+template <typename RowPtr>
+__device__ __forceinline__ void store_cols_transposed(const uint32_t (&vals)[32], __nv_bfloat16* stage, int lane,
+                                                      int col0, int ntok, RowPtr rowptr) {
+    __syncwarp();                                   // the slot's previous reads are done
+#pragma unroll
+    for (int j = 0; j < 32; ++j) stage[j * 32 + lane] = __float2bfloat16_rn(__uint_as_float(vals[j]));
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int piece = lane + 32 * i, j = piece >> 2, q = piece & 3;
+        if (j < ntok) {
+            const uint4 w = reinterpret_cast<const uint4*>(stage + j * 32)[q];
+            reinterpret_cast<uint4*>(rowptr(j) + col0)[q] = w;
+        }
+    }
+}
+
 // Tile walk with 256-row m-tiles (mprefix counts 256-row tiles per group).
 __device__ __forceinline__ int pair_total_tiles(const GemmParams& p, int& routed_tiles) {
     routed_tiles = p.offsets ? __ldg(p.mprefix + p.E) * p.cls[0].ntiles : 0;
@@ -340,8 +361,11 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                     // through the two warps' staging slots, tokens 0-15 / 16-31 of the chunk
                     const int q = sub & 1;
                     const bool up_warp = sub >= 2;
-                    const int feat = ti.n_idx * 128 + (int)rank * 64 + q * 32 + lane;
+                    const int feat0 = ti.n_idx * 128 + (int)rank * 64 + q * 32;   // this warp's first feature
+                    const int feat = feat0 + lane;
                     const bool feat_ok = feat < c.n_out;
+                    __nv_bfloat16* own_stage =
+                        reinterpret_cast<__nv_bfloat16*>(sOut + (warp - 2) * PAIR_STAGE_OUT_BYTES);
                     // the up warp's own staging slot: 16 tokens x 32 lanes of fp32; the pair's
                     // two barriers: values staged (up -> gate), values read (gate -> up)
                     float* st = reinterpret_cast<float*>(sOut + (q + 4 * half) * PAIR_STAGE_OUT_BYTES);
@@ -380,45 +404,57 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                             }
                             if (!swap_ok) break;
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) {
-                                const int tok = ch * 32 + j;
-                                const long long orow_t = c.out_row0 + ti.a_row + tok;
-                                if (feat_ok && tok < ti.rows && orow_t >= 0 && orow_t < c.out_rows) {
-                                    float g = __uint_as_float(v[j]), uu = u[j];
-                                    if (F8) {
-                                        const float st_a = __ldg(c.a_scale + ti.a_row + tok);
-                                        g = g * st_a * sg;
-                                        uu = uu * st_a * su;
-                                    }
-                                    out[orow_t * c.ldo + feat] = __float2bfloat16_rn(swiglu_f32(g, uu));
+                            for (int j = 0; j < 32; ++j) {     // h replaces the gate values in v
+                                float g = __uint_as_float(v[j]), uu = u[j];
+                                if (F8) {
+                                    const int tok = min(ch * 32 + j, ti.rows - 1);
+                                    const float st_a = __ldg(c.a_scale + ti.a_row + tok);
+                                    g = g * st_a * sg;
+                                    uu = uu * st_a * su;
                                 }
+                                v[j] = __float_as_uint(swiglu_f32(g, uu));
                             }
+                            // this warp's 32 features are whole 64-byte pieces of h rows; the tile's
+                            // features are all inside n_out (n_out is a multiple of 64)
+                            const int ntok = min(32, ti.rows - ch * 32);
+                            const long long row0 = c.out_row0 + ti.a_row + ch * 32;
+                            if (feat0 < c.n_out)
+                                store_cols_transposed(v, own_stage, lane, feat0, ntok, [&](int j) {
+                                    return out + (row0 + j) * c.ldo;
+                                });
                         }
                     }
                     // the up warp leaves its slot only once the last values were read from it
                     if (up_warp && swap_ok && !mbar_wait(xch_read, (xch_n & 1u) ^ 1u, abort_flag)) swap_ok = false;
                 } else {
-                    const int col = ti.n_idx * 256 + (int)rank * 128 + sub * 32 + lane;
-                    const bool col_ok = col < c.n_out;
-                    const float sc = (F8 && col_ok) ? __ldg(sb + col) : 1.f;
+                    const int col0 = ti.n_idx * 256 + (int)rank * 128 + sub * 32;   // this warp's 32 columns
+                    const float sc = (F8 && col0 + lane < c.n_out) ? __ldg(sb + col0 + lane) : 1.f;
+                    __nv_bfloat16* own_stage =
+                        reinterpret_cast<__nv_bfloat16*>(sOut + (warp - 2) * PAIR_STAGE_OUT_BYTES);
 #pragma unroll 1
                     for (int ch = half; ch < nch; ch += 2) {
                         uint32_t v[32];
                         __syncwarp();
                         tmem_ld_32cols(tbase + ch * 32, v);
                         tmem_ld_wait();
+                        if (F8) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int tok = ch * 32 + j;
-                            const long long orow_t = c.out_row0 + ti.a_row + tok;
-                            if (col_ok && tok < ti.rows && orow_t >= 0 && orow_t < c.out_rows) {
-                                float val = __uint_as_float(v[j]);
-                                if (F8) val = val * __ldg(c.a_scale + ti.a_row + tok) * sc;
-                                __nv_bfloat16* o = c.row_addr ? reinterpret_cast<__nv_bfloat16*>(
-                                                                    __ldg(c.row_addr + ti.a_row + tok))
-                                                              : out + orow_t * c.ldo;
-                                o[col] = __float2bfloat16_rn(val);
-                            }
+                            for (int j = 0; j < 32; ++j)
+                                v[j] = __float_as_uint(__uint_as_float(v[j]) *
+                                                       __ldg(c.a_scale + ti.a_row + min(ch * 32 + j, ti.rows - 1)) *
+                                                       sc);
+                        }
+                        const int ntok = min(32, ti.rows - ch * 32);
+                        const int r0 = ti.a_row + ch * 32;
+                        if (col0 < c.n_out) {
+                            if (c.row_addr)
+                                store_cols_transposed(v, own_stage, lane, col0, ntok, [&](int j) {
+                                    return reinterpret_cast<__nv_bfloat16*>(__ldg(c.row_addr + r0 + j));
+                                });
+                            else
+                                store_cols_transposed(v, own_stage, lane, col0, ntok, [&](int j) {
+                                    return out + (c.out_row0 + r0 + j) * c.ldo;
+                                });
                         }
                     }
                 }

@@ -306,11 +306,12 @@ def device_tensors(wl: Workload, device, names=None, chunk_elems: int = 1 << 27)
     return out
 
 
-def device_tensors_q8(wl: Workload, device, chunk_rows: int = 1 << 16) -> dict:
+def device_tensors_q8(wl: Workload, device, chunk_rows: int = 1 << 16, host: Optional[dict] = None) -> dict:
     """fp8 e4m3 expert weights with fp32 row scales, quantised from the workload's bf16 weights
     (quantize_e4m3_rows) chunk by chunk on the host and copied to `device`.
     Keys: w1q, w3q [E,f,d] uint8, s1, s3 [E,f]; w2q [E,d,f], s2 [E,d]; w1sq, w3sq, w2sq, s1s,
-    s3s, s2s for the shared expert."""
+    s3s, s2s for the shared expert.  host: a dict that receives the same arrays as numpy
+    (host copies, e.g. for a checker that needs every expert's codes)."""
     import torch
 
     inp = Inputs(wl)
@@ -320,12 +321,18 @@ def device_tensors_q8(wl: Workload, device, chunk_rows: int = 1 << 16) -> dict:
         q_dev = torch.empty((wl.E * rows_per_e, K), dtype=torch.uint8, device=device)
         s_dev = torch.empty(wl.E * rows_per_e, dtype=torch.float32, device=device)
         ne = max(1, min(wl.E, chunk_rows // rows_per_e))
+        if host is not None:
+            host[name + "q"] = np.empty((wl.E, rows_per_e, K), np.uint8)
+            host["s" + name[1]] = np.empty((wl.E, rows_per_e), np.float32)
         for e0 in range(0, wl.E, ne):
             n = min(ne, wl.E - e0)
             w = inp.expert_rows(name, e0, n)
             q, sc = quantize_e4m3_rows(w, K)
             q_dev[e0 * rows_per_e:(e0 + n) * rows_per_e].copy_(torch.from_numpy(q))
             s_dev[e0 * rows_per_e:(e0 + n) * rows_per_e].copy_(torch.from_numpy(sc))
+            if host is not None:
+                host[name + "q"][e0:e0 + n] = q.reshape(n, rows_per_e, K)
+                host["s" + name[1]][e0:e0 + n] = sc.reshape(n, rows_per_e)
         out[name + "q"] = q_dev.view(wl.E, rows_per_e, K)
         out["s" + name[1]] = s_dev.view(wl.E, rows_per_e)
     if wl.has_shared:
@@ -334,5 +341,8 @@ def device_tensors_q8(wl: Workload, device, chunk_rows: int = 1 << 16) -> dict:
             q, sc = quantize_e4m3_rows(a, a.shape[1])
             out[name[:2] + "sq"] = torch.from_numpy(q).to(device)
             out["s" + name[1] + "s"] = torch.from_numpy(sc).to(device)
+            if host is not None:
+                host[name[:2] + "sq"] = q
+                host["s" + name[1] + "s"] = sc
     return out
 

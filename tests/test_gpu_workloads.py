@@ -12,6 +12,10 @@ weights are regenerated from the seeded generator (never read back from the GPU)
   - for the Qwen3-like layer (131 072 kept rows) the tokens of a covering set of rows: the
     first, the last and one seeded row of every 128-row block of every expert's rows, which
     reaches both halves of every 256-row pair tile, every 128-row tile and every ragged tail.
+The fp8 layers (bench.py --weights fp8 / fp8a8) route exactly like the bf16 layer (checked on
+every token again); their expert GEMMs are checked on 64 seeded tokens of the decode layer and,
+for the prefill layer, on the tokens of the first, last and one seeded row of every 256-row tile
+of every expert (the fp8 oracle is the slowest part of the suite).
 Each test prints the largest logit error and the largest output difference (pytest -rA).
 """
 import gc
@@ -165,14 +169,20 @@ def check_experts_and_out(moe, ws, L, wl, x, toks, g_idx, dest, w_o, out, expert
               f"bar, max |d| = {np.abs(g64 - o64).max():.3e}")
 
 
-def token_set(wl, r, mode, seed):
+def token_set(wl, r, mode, seed, block=128, min_tokens=512):
+    """"all": every token; "cover": the tokens of covering_rows (first, last and one seeded row of
+    every `block`-row block of every expert), padded with seeded tokens to min_tokens;
+    "sample:N": N seeded tokens including the first and the last."""
     if mode == "all":
         return np.arange(wl.T)
-    rows = covering_rows(r["offsets"], seed)
+    rng = np.random.default_rng(seed + 1)
+    if mode.startswith("sample:"):
+        n = int(mode.split(":")[1])
+        return np.union1d([0, wl.T - 1], rng.choice(wl.T, n - 2, replace=False))
+    rows = covering_rows(r["offsets"], seed, block)
     toks = np.unique(r["src_token"][rows])
-    if len(toks) < 512:                      # at least 512 tokens: seeded extra ones
-        rng = np.random.default_rng(seed + 1)
-        extra = rng.choice(np.setdiff1d(np.arange(wl.T), toks), 512 - len(toks), replace=False)
+    if len(toks) < min_tokens:                      # seeded extra tokens
+        extra = rng.choice(np.setdiff1d(np.arange(wl.T), toks), min_tokens - len(toks), replace=False)
         toks = np.union1d(toks, extra)
     return toks
 
@@ -188,14 +198,27 @@ def bf16_expert(inp, wl):
     return expert, shared
 
 
-def q8_weights(inp, wl, e):
-    return (synth.quantize_e4m3_rows(inp.expert_rows("w1", e, 1), wl.d),
-            synth.quantize_e4m3_rows(inp.expert_rows("w3", e, 1), wl.d),
-            synth.quantize_e4m3_rows(inp.expert_rows("w2", e, 1), wl.f))
+def q8_weights(host, e):
+    """Expert e's fp8 codes and row scales (the same arrays the GPU was given)."""
+    return ((host["w1q"][e], host["s1"][e]), (host["w3q"][e], host["s3"][e]), (host["w2q"][e], host["s2"][e]))
 
 
-def q8_shared(inp):
-    return [synth.quantize_e4m3_rows(inp.shared(n), inp.shared(n).shape[1]) for n in ("w1s", "w3s", "w2s")]
+def q8_shared(host):
+    return [(host["w1sq"], host["s1s"]), (host["w3sq"], host["s3s"]), (host["w2sq"], host["s2s"])]
+
+
+@pytest.fixture(scope="module")
+def dsv3_q8():
+    """The DeepSeek-V3-like layer's fp8 weights, quantised once for both fp8 decode tests: device
+    tensors for the layer and the same codes on the host for the oracle."""
+    wl = synth.WORKLOADS["dsv3"]
+    host = {}
+    W = synth.device_tensors(wl, "cuda", names=["x", "wg", "bias"])
+    Q = synth.device_tensors_q8(wl, "cuda", host=host)
+    yield wl, W, Q, host
+    del W, Q
+    gc.collect()
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("name", ["mixtral", "qwen3", "dsv3", "skew"])
@@ -232,77 +255,87 @@ def test_full_size_layer(moe, name):
     torch.cuda.empty_cache()
 
 
-def test_full_size_decode_fp8_weights(moe):
+def test_full_size_decode_fp8_weights(moe, dsv3_q8):
     """The DeepSeek-V3-like decode layer with fp8 e4m3 expert weights (bench.py --weights fp8):
-    routing bit-exact for every token, every token's outputs against the oracle's fp8 experts on
-    weights regenerated and quantised on the host."""
-    wl = synth.WORKLOADS["dsv3"]
+    routing bit-exact for every token; h, y_perm, the shared expert and the outputs of 64 seeded
+    tokens against the oracle's fp8 experts on the same codes."""
+    wl, W, Q, host = dsv3_q8
     T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
-    W = synth.device_tensors(wl, "cuda", names=["x", "wg", "bias"])
-    Q = synth.device_tensors_q8(wl, "cuda")
     ws = torch.empty(moe.moe_workspace_bytes(T, d, E, k, f, fs), dtype=torch.uint8, device="cuda")
     out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
     moe.moe_layer_forward_w8(W["x"], W["wg"], W["bias"], Q["w1q"], Q["s1"], Q["w3q"], Q["s3"], Q["w2q"], Q["s2"],
                              Q["w1sq"], Q["s1s"], Q["w3sq"], Q["s3s"], Q["w2sq"], Q["s2s"], fs, T, d, E, k, f,
                              wl.capacity_factor, wl.cap_mode, out, ws)
     assert moe.moe_get_error() == 0
-    del Q, W
     L = moe.moe_workspace_layout(T, d, E, k, f, fs)
     inp = synth.Inputs(wl)
     x, g_idx, r, w_o = check_routing(moe, ws, L, wl, inp, "dsv3 fp8 weights")
 
     def expert(e, xe, g_h):
-        (q1, s1), (q3, s3), (q2, s2) = q8_weights(inp, wl, e)
+        (q1, s1), (q3, s3), (q2, s2) = q8_weights(host, e)
         return oracle.expert_ffn_q8(xe, q1, s1, q3, s3, q2, s2)
 
-    qs = q8_shared(inp)
+    qs = q8_shared(host)
 
     def shared(xs, g_h):
         return oracle.expert_ffn_q8(xs, qs[0][0], qs[0][1], qs[1][0], qs[1][1], qs[2][0], qs[2][1])
 
-    check_experts_and_out(moe, ws, L, wl, x, np.arange(T), g_idx, r["dest"], w_o, out, expert, shared,
-                          "dsv3 fp8 weights")
+    check_experts_and_out(moe, ws, L, wl, x, token_set(wl, r, "sample:64", seed=11), g_idx, r["dest"], w_o, out,
+                          expert, shared, "dsv3 fp8 weights")
 
 
-@pytest.mark.parametrize("name", ["dsv3", "mixtral"])
-def test_full_size_fp8_weights_and_activations(moe, name):
-    """bench.py --weights fp8a8 at full size (decode on 1-SM tiles, prefill on 2-SM tiles): routing
-    bit-exact for every token; h against the oracle's fp8 x fp8 first GEMM; the oracle's second GEMM
-    is given the kernel's h, so both sides quantise the same h rows (the quantised codes are a
-    decision taken on h, like the routing on the logits).  Every token of the decode layer, the
-    covering set of rows of the prefill layer."""
-    wl = synth.WORKLOADS[name]
+def _run_w8a8(moe, wl, W, Q, host, mode, own):
     T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
-    W = synth.device_tensors(wl, "cuda", names=["x", "wg", "bias"])
-    Q = synth.device_tensors_q8(wl, "cuda")
     ws = torch.empty(moe.moe_workspace_bytes_a8(T, d, E, k, f, fs), dtype=torch.uint8, device="cuda")
     out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
     moe.moe_layer_forward_w8a8(W["x"], W["wg"], W.get("bias"), Q["w1q"], Q["s1"], Q["w3q"], Q["s3"], Q["w2q"],
                                Q["s2"], Q.get("w1sq"), Q.get("s1s"), Q.get("w3sq"), Q.get("s3s"), Q.get("w2sq"),
                                Q.get("s2s"), fs, T, d, E, k, f, wl.capacity_factor, wl.cap_mode, out, ws)
     assert moe.moe_get_error() == 0
-    del Q, W
     L = moe.moe_workspace_layout(T, d, E, k, f, fs)
     inp = synth.Inputs(wl)
-    x, g_idx, r, w_o = check_routing(moe, ws, L, wl, inp, f"{name} fp8 x fp8")
+    label = f"{wl.name} fp8 x fp8"
+    x, g_idx, r, w_o = check_routing(moe, ws, L, wl, inp, label)
 
     def expert(e, xe, g_h):
-        (q1, s1), (q3, s3), (q2, s2) = q8_weights(inp, wl, e)
+        (q1, s1), (q3, s3), (q2, s2) = q8_weights(host, e)
         return oracle.expert_gate_up_w8a8(xe, q1, s1, q3, s3), oracle.expert_down_w8a8(g_h, q2, s2)
 
-    qs = q8_shared(inp) if fs else None
+    qs = q8_shared(host) if fs else None
 
     def shared(xs, g_h):
         h = oracle.expert_gate_up_w8a8(xs, qs[0][0], qs[0][1], qs[1][0], qs[1][1])
         return h, oracle.expert_down_w8a8(g_h, qs[2][0], qs[2][1])
 
     def expert_own(e, xe):
-        (q1, s1), (q3, s3), (q2, s2) = q8_weights(inp, wl, e)
+        (q1, s1), (q3, s3), (q2, s2) = q8_weights(host, e)
         return oracle.expert_ffn_w8a8(xe, q1, s1, q3, s3, q2, s2)[1]
 
     def shared_own(xs):
         return oracle.expert_ffn_w8a8(xs, qs[0][0], qs[0][1], qs[1][0], qs[1][1], qs[2][0], qs[2][1])[1]
 
-    toks = token_set(wl, r, "all" if name == "dsv3" else "cover", seed=13)
-    check_experts_and_out(moe, ws, L, wl, x, toks, g_idx, r["dest"], w_o, out, expert, shared,
-                          f"{name} fp8 x fp8", own=(expert_own, shared_own))
+    check_experts_and_out(moe, ws, L, wl, x, mode(r), g_idx, r["dest"], w_o, out, expert, shared, label,
+                          own=(expert_own, shared_own) if own else None)
+
+
+def test_full_size_fp8_weights_and_activations_decode(moe, dsv3_q8):
+    """bench.py --weights fp8a8 on the DeepSeek-V3-like decode layer (1-SM tiles): routing bit-exact
+    for every token; h against the oracle's fp8 x fp8 first GEMM; the oracle's second GEMM is given
+    the kernel's h, so both sides quantise the same h rows (the quantised codes are a decision
+    taken on h, like the routing on the logits); 64 seeded tokens.  Also reported: the outputs
+    against the oracle that quantises its own h."""
+    wl, W, Q, host = dsv3_q8
+    _run_w8a8(moe, wl, W, Q, host, lambda r: token_set(wl, r, "sample:64", seed=13), own=True)
+
+
+def test_full_size_fp8_weights_and_activations_prefill(moe):
+    """The same on the Mixtral-like prefill layer (2-SM tiles, swapped tail tiles): the tokens of
+    the first, last and one seeded row of every 256-row tile of every expert."""
+    wl = synth.WORKLOADS["mixtral"]
+    host = {}
+    W = synth.device_tensors(wl, "cuda", names=["x", "wg", "bias"])
+    Q = synth.device_tensors_q8(wl, "cuda", host=host)
+    _run_w8a8(moe, wl, W, Q, host, lambda r: token_set(wl, r, "cover", seed=13, block=256, min_tokens=0), own=False)
+    del W, Q
+    gc.collect()
+    torch.cuda.empty_cache()
