@@ -84,6 +84,7 @@ struct GemmParams {
     int stages;              // ring slots (<= GEMM_MAX_STAGES)
     int b_slot;              // bytes of one B slot (multiple of 1024)
     const int32_t* group_map;  // [E] routed group -> weight group (expert cache slots); nullptr = identity
+    int swap_max;              // pair kernel: tail tiles of at most this many rows run swapped (0 = none)
 };
 
 // Weight group that routed group g reads its B rows from.
