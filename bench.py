@@ -555,7 +555,7 @@ def run_cached(args, base, rank, world, local):
         "stages_ms": stage_ms,
         "e2e": {"value": dp.job_throughput(T, world, K, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
                 "d2h_bytes_per_step": T * d * 2},
-        "gpu_launches": (KERNELS_PER_STEP + 2) * K,
+        "gpu_launches": (KERNELS_PER_STEP + 4) * K,   # + cache plan, copy, the loaded experts' two GEMMs
         "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)

@@ -22,10 +22,11 @@
 // CTA's 128 weight rows in the B slot of the stage) and the tile's tokens the N side (N = rows
 // rounded up to 16, each CTA loading its N / 2 token rows in 32-row boxes into the A slot), so
 // the MMA time follows the real row count.  TMEM then holds one weight row (output feature) per
-// lane and one token per column.  For GEMM1 each CTA loads 64 features as four groups of 16 W1
-// rows each followed by the same 16 rows of W3, so that a feature's gate and up values sit in
-// lanes l and l + 16 of one warp and one shuffle pairs them.  Outputs go through the warp's
-// staging slot and leave as 16-byte pieces of token rows.
+// lane and one token per column.  For GEMM1 each CTA loads 64 rows of W1 and the same 64 rows of
+// W3, so that a feature's gate (lanes 0-63) and up (lanes 64-127) values sit in the same CTA: the
+// warps of lanes 64-127 pass their up values through shared memory to the warps of lanes 0-63,
+// which apply SwiGLU.  Stores write one token row's 32 consecutive outputs (64 bytes) per warp
+// instruction.
 #pragma once
 
 #include "grouped_gemm.cuh"
@@ -50,8 +51,8 @@ constexpr int PAIR_SWAP_BOX_BYTES = PAIR_SWAP_BOX_ROWS * 128;
 // Tensor maps only swapped tiles use.
 struct PairSwapMaps {
     CUtensorMap a0, a1;     // the token rows of class 0 / class 1 in 32-row boxes
-    CUtensorMap w0, w0b;    // GEMM1: W1 / W3 of class 0 in 16-row boxes
-    CUtensorMap w1, w1b;    // GEMM1: W1 / W3 of class 1 in 16-row boxes
+    CUtensorMap w0, w0b;    // GEMM1: W1 / W3 of class 0 in 64-row boxes
+    CUtensorMap w1, w1b;    // GEMM1: W1 / W3 of class 1 in 64-row boxes
 };
 
 
@@ -151,7 +152,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
     uint64_t* tfull_bar = empty_bar + PAIR_STAGES;
     uint64_t* tempty_bar = tfull_bar + 2;
     uint64_t* drain_bar = tempty_bar + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+    uint64_t* xch_bar = drain_bar + 1;   // swapped GEMM1 tiles: 2 barriers per gate / up warp pair
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xch_bar + 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -171,6 +173,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
             mbar_init(tempty_bar + a, 2 * 32 * PAIR_EPI_WARPS);  // leader: epilogue threads of 2 CTAs
         }
         mbar_init(drain_bar, 1);
+        for (int i = 0; i < 8; ++i) mbar_init(xch_bar + i, 32);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -223,7 +226,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                 constexpr int KB = F8 ? 2 * GEMM_BK : GEMM_BK;
                 const int nk = c.K / KB;
                 // swapped tile: this CTA's N / 2 token rows in 32-row boxes, and its weight rows
-                // (GEMM1: 64 features, each 16 W1 rows followed by the same 16 rows of W3)
+                // (GEMM1: 64 rows of W1 and the same 64 rows of W3)
                 const int half_tok = ti.n_tok >> 1;
                 const int nld = ti.swap ? (half_tok + PAIR_SWAP_BOX_ROWS - 1) / PAIR_SWAP_BOX_ROWS : 0;
                 const CUtensorMap* mT = ti.cls ? &sw.a1 : &sw.a0;
@@ -241,13 +244,9 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                         tma_load_2d_pair(sA + stage * PAIR_A_BYTES, mA, fb, kb * KB, a_row, pol_a);
                         tma_load_2d_pair(sB + stage * PAIR_B_BYTES, mB, fb, kb * KB, b_row, pol_b);
                     } else {
-                        if (EPI == EPI_SWIGLU) {      // rows 32 q .. +15: W1, 32 q + 16 .. +15: W3
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                uint8_t* dst = sB + stage * PAIR_B_BYTES + q * 32 * 128;
-                                tma_load_2d_pair(dst, mW, fb, kb * KB, w_row + 16 * q, pol_b);
-                                tma_load_2d_pair(dst + 16 * 128, mWb, fb, kb * KB, w_row + 16 * q, pol_b);
-                            }
+                        if (EPI == EPI_SWIGLU) {
+                            tma_load_2d_pair(sB + stage * PAIR_B_BYTES, mW, fb, kb * KB, w_row, pol_b);
+                            tma_load_2d_pair(sB + stage * PAIR_B_BYTES + 64 * 128, mWb, fb, kb * KB, w_row, pol_b);
                         } else {
                             tma_load_2d_pair(sB + stage * PAIR_B_BYTES, mB, fb, kb * KB, b_row, pol_b);
                         }
@@ -322,7 +321,9 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
         uint4* stage = reinterpret_cast<uint4*>(sOut + (warp - 2) * PAIR_STAGE_OUT_BYTES);
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = pair_id; t < total; t += npairs) {
+        uint32_t xch_n = 0;         // swapped GEMM1 tiles: 16-token hand-overs so far (per pair)
+        bool swap_ok = true;
+        for (int t = pair_id; t < total && swap_ok; t += npairs) {
             const PairTile ti = pair_decode_tile(p, t, routed_tiles, swap_max);
             const GemmClass& c = p.cls[ti.cls];
             const bool ready = mbar_wait(tfull_bar + acc, acc_phase, abort_flag);
@@ -352,58 +353,76 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                 const int nch = (ti.n_tok + 31) >> 5;
                 __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(c.out);
                 if (EPI == EPI_SWIGLU) {
-                    // this CTA's 64 features in four 16-feature groups, one per lane quarter: lanes
-                    // 0-15 of the quarter hold the gate (W1) rows, lanes 16-31 the up (W3) rows of the
-                    // same features.  A lane pair (l, l + 16) swaps half its tokens with one shuffle:
-                    // lane l then has gate and up of tokens 0-15, lane l + 16 of tokens 16-31.
-                    const int fbase = ti.n_idx * 128 + (int)rank * 64 + sub * 16;   // this warp's features
-                    const bool upper = lane >= 16;
-                    const int feat = fbase + (lane & 15);
+                    // lanes 0-63: gate of this CTA's 64 features, lanes 64-127: their up values; the
+                    // warp of quarter q + 2 passes its up values to the warp of quarter q (same half)
+                    // through the two warps' staging slots, tokens 0-15 / 16-31 of the chunk
+                    const int q = sub & 1;
+                    const bool up_warp = sub >= 2;
+                    const int feat0 = ti.n_idx * 128 + (int)rank * 64 + q * 32;   // this warp's first feature
+                    const int feat = feat0 + lane;
+                    const bool feat_ok = feat < c.n_out;
+                    __nv_bfloat16* own_stage =
+                        reinterpret_cast<__nv_bfloat16*>(sOut + (warp - 2) * PAIR_STAGE_OUT_BYTES);
+                    // the up warp's own staging slot: 16 tokens x 32 lanes of fp32; the pair's
+                    // two barriers: values staged (up -> gate), values read (gate -> up)
+                    float* st = reinterpret_cast<float*>(sOut + (q + 4 * half) * PAIR_STAGE_OUT_BYTES);
+                    uint64_t* xch_staged = xch_bar + 2 * (q + 2 * half);
+                    uint64_t* xch_read = xch_staged + 1;
                     float sg = 1.f, su = 1.f;
-                    if (F8 && feat < c.n_out) {
+                    if (F8 && feat_ok) {
                         sg = __ldg(sb + feat);
                         su = __ldg(sb2 + feat);
                     }
-                    __nv_bfloat16* stage16 =
-                        reinterpret_cast<__nv_bfloat16*>(sOut + (warp - 2) * PAIR_STAGE_OUT_BYTES);
-                    // token t's 16 features at stage16 + srow(t) (the upper tokens shifted by 32 bytes
-                    // so that both lane halves write different banks)
-                    auto srow = [](int t) { return t * 16 + (t >> 4) * 16; };
 #pragma unroll 1
-                    for (int ch = half; ch < nch; ch += 2) {
+                    for (int ch = half; ch < nch && swap_ok; ch += 2) {
                         uint32_t v[32];
                         __syncwarp();
                         tmem_ld_32cols(tbase + ch * 32, v);
                         tmem_ld_wait();
-                        __syncwarp();                       // the previous chunk's staging reads are done
+                        if (up_warp) {
+                            // tokens 0-15, then 16-31 of the chunk through this warp's own slot
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const uint32_t sent = upper ? v[j] : v[16 + j];
-                            const uint32_t got = __shfl_xor_sync(0xffffffffu, sent, 16);
-                            float g = __uint_as_float(upper ? got : v[j]);
-                            float u = __uint_as_float(upper ? v[16 + j] : got);
-                            const int t = upper ? 16 + j : j;   // token within the chunk
-                            if (F8) {
-                                const float sa_t = __ldg(c.a_scale + ti.a_row + min(ch * 32 + t, ti.rows - 1));
-                                g = g * sa_t * sg;
-                                u = u * sa_t * su;
-                            }
-                            stage16[srow(t) + (lane & 15)] = __float2bfloat16_rn(swiglu_f32(g, u));
-                        }
-                        __syncwarp();
-                        // 32 token rows x 16 features (32 bytes, a whole sector) as 16-byte pieces
-                        const int ntok = min(32, ti.rows - ch * 32);
-                        const long long row0 = c.out_row0 + ti.a_row + ch * 32;
-                        if (fbase < c.n_out) {
+                            for (int part = 0; part < 2; ++part) {
+                                if (!mbar_wait(xch_read, (xch_n & 1u) ^ 1u, abort_flag)) { swap_ok = false; break; }
 #pragma unroll
-                            for (int i = 0; i < 2; ++i) {
-                                const int piece = lane + 32 * i, t = piece >> 1, q8 = piece & 1;
-                                if (t < ntok)
-                                    reinterpret_cast<uint4*>(out + (row0 + t) * c.ldo + fbase)[q8] =
-                                        reinterpret_cast<const uint4*>(stage16 + srow(t))[q8];
+                                for (int j = 0; j < 16; ++j) st[j * 32 + lane] = __uint_as_float(v[16 * part + j]);
+                                mbar_arrive(xch_staged);
+                                ++xch_n;
                             }
+                        } else {
+                            float u[32];
+#pragma unroll
+                            for (int part = 0; part < 2; ++part) {
+                                if (!mbar_wait(xch_staged, xch_n & 1u, abort_flag)) { swap_ok = false; break; }
+#pragma unroll
+                                for (int j = 0; j < 16; ++j) u[16 * part + j] = st[j * 32 + lane];
+                                mbar_arrive(xch_read);
+                                ++xch_n;
+                            }
+                            if (!swap_ok) break;
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) {     // h replaces the gate values in v
+                                float g = __uint_as_float(v[j]), uu = u[j];
+                                if (F8) {
+                                    const int tok = min(ch * 32 + j, ti.rows - 1);
+                                    const float st_a = __ldg(c.a_scale + ti.a_row + tok);
+                                    g = g * st_a * sg;
+                                    uu = uu * st_a * su;
+                                }
+                                v[j] = __float_as_uint(swiglu_f32(g, uu));
+                            }
+                            // this warp's 32 features are whole 64-byte pieces of h rows; the tile's
+                            // features are all inside n_out (n_out is a multiple of 64)
+                            const int ntok = min(32, ti.rows - ch * 32);
+                            const long long row0 = c.out_row0 + ti.a_row + ch * 32;
+                            if (feat0 < c.n_out)
+                                store_cols_transposed(v, own_stage, lane, feat0, ntok, [&](int j) {
+                                    return out + (row0 + j) * c.ldo;
+                                });
                         }
                     }
+                    // the up warp leaves its slot only once the last values were read from it
+                    if (up_warp && swap_ok && !mbar_wait(xch_read, (xch_n & 1u) ^ 1u, abort_flag)) swap_ok = false;
                 } else {
                     const int col0 = ti.n_idx * 256 + (int)rank * 128 + sub * 32;   // this warp's 32 columns
                     const float sc = (F8 && col0 + lane < c.n_out) ? __ldg(sb + col0 + lane) : 1.f;
@@ -472,6 +491,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                     }
                 }
             }
+            if (!swap_ok) break;      // a hand-over wait gave up: the kernel is being abandoned
             tc_fence_before();
             mbar_arrive_cluster(tempty_leader0 + (uint32_t)acc * 8u);
             acc ^= 1;

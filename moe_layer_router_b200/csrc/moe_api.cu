@@ -182,8 +182,9 @@ size_t router_partial_bytes(int T, int d, int E) {
 }
 
 // Tail tiles of at most this many rows run with the operands swapped in the pair kernel (GEMM1,
-// GEMM2); measured on the prefill workloads.
-constexpr int kPairSwapMaxGemm1 = 128;
+// GEMM2); measured on the prefill workloads (same-box A/B): swapped SwiGLU tiles pay for their
+// gate / up hand-over between warps, so GEMM1 swaps only short tails.
+constexpr int kPairSwapMaxGemm1 = 64;
 constexpr int kPairSwapMaxGemm2 = 128;
 
 template <int EPI, bool F8 = false>
@@ -215,7 +216,7 @@ int launch_gemm_pair(DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b
 bool use_pair_tiles(long long rows, int E) { return rows >= 256ll * E; }
 
 // Tensor maps of the pair kernel's swapped tail tiles: the token rows of each class in 32-row
-// boxes and (GEMM1) W1 / W3 of each class in 16-row boxes.  A null base leaves that map unused
+// boxes and (GEMM1) W1 / W3 of each class in 64-row boxes.  A null base leaves that map unused
 // (its class has no rows, or the GEMM has no gate / up pair); it then copies another map.
 // f8: e4m3 operands (128-byte K rows) instead of bf16.
 int make_swap_maps(PairSwapMaps* m, bool f8, const void* t0, uint64_t k0, uint64_t rows0, const void* t1, uint64_t k1,
@@ -228,10 +229,10 @@ int make_swap_maps(PairSwapMaps* m, bool f8, const void* t0, uint64_t k0, uint64
     int rc;
     if (t0 && (rc = mk(&m->a0, t0, k0, rows0, PAIR_SWAP_BOX_ROWS)) != MOE_OK) return rc;
     if (t1 && (rc = mk(&m->a1, t1, k1, rows1, PAIR_SWAP_BOX_ROWS)) != MOE_OK) return rc;
-    if (w1_0 && (rc = mk(&m->w0, w1_0, k0, wrows0, 16)) != MOE_OK) return rc;
-    if (w3_0 && (rc = mk(&m->w0b, w3_0, k0, wrows0, 16)) != MOE_OK) return rc;
-    if (w1_1 && (rc = mk(&m->w1, w1_1, k1, wrows1, 16)) != MOE_OK) return rc;
-    if (w3_1 && (rc = mk(&m->w1b, w3_1, k1, wrows1, 16)) != MOE_OK) return rc;
+    if (w1_0 && (rc = mk(&m->w0, w1_0, k0, wrows0, 64)) != MOE_OK) return rc;
+    if (w3_0 && (rc = mk(&m->w0b, w3_0, k0, wrows0, 64)) != MOE_OK) return rc;
+    if (w1_1 && (rc = mk(&m->w1, w1_1, k1, wrows1, 64)) != MOE_OK) return rc;
+    if (w3_1 && (rc = mk(&m->w1b, w3_1, k1, wrows1, 64)) != MOE_OK) return rc;
     if (!t0) { m->a0 = m->a1; m->w0 = m->w1; m->w0b = m->w1b; }
     if (!t1) { m->a1 = m->a0; m->w1 = m->w0; m->w1b = m->w0b; }
     return MOE_OK;
