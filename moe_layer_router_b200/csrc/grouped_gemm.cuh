@@ -278,7 +278,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull_bar + a, 1);
-            mbar_init(tempty_bar + a, 128);
+            mbar_init(tempty_bar + a, 4);      // one arrival per epilogue warp
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -474,9 +474,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
                     }
                 }
             }
-            __syncwarp();
             tc_fence_before();
-            mbar_arrive(tempty_bar + acc);
+            __syncwarp();                     // every lane's tensor-memory reads are done
+            if (lane == 0) mbar_arrive(tempty_bar + acc);
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }

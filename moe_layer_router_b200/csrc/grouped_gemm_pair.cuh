@@ -10,8 +10,8 @@
 //     issues tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16), which reads both CTAs'
 //     halves and accumulates rows [128 r, 128 r + 128) into CTA r's tensor memory.
 //   - the leader's commits arrive on both CTAs' barriers (empty stage, accumulator full);
-//     every epilogue thread of both CTAs (eight warps each) arrives on the leader's
-//     accumulator-empty barrier.
+//     every epilogue warp of both CTAs (eight each) arrives once on the leader's
+//     accumulator-empty barrier, after all its lanes' tensor-memory reads.
 // Per SM this halves the B operand traffic of a 1-SM M = 128 tile and leaves room for a
 // 6-stage ring (A 16 KB + B 16 KB per stage per CTA) and 16 KB of epilogue staging, through
 // which each epilogue warp stores whole 64-byte pieces of 8 output rows at a time.
@@ -170,7 +170,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull_bar + a, 1);     // one multicast commit
-            mbar_init(tempty_bar + a, 2 * 32 * PAIR_EPI_WARPS);  // leader: epilogue threads of 2 CTAs
+            mbar_init(tempty_bar + a, 2 * PAIR_EPI_WARPS);  // leader: one arrival per epilogue warp of 2 CTAs
         }
         mbar_init(drain_bar, 1);
         for (int i = 0; i < 8; ++i) mbar_init(xch_bar + i, 32);
@@ -400,12 +400,14 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                                 ++xch_n;
                             }
                             if (!swap_ok) break;
+                            // fp8: lane j holds token j's activation scale, broadcast per column
+                            const float my_sa =
+                                F8 ? __ldg(c.a_scale + ti.a_row + min(ch * 32 + lane, ti.rows - 1)) : 1.f;
 #pragma unroll
                             for (int j = 0; j < 32; ++j) {     // h replaces the gate values in v
                                 float g = __uint_as_float(v[j]), uu = u[j];
                                 if (F8) {
-                                    const int tok = min(ch * 32 + j, ti.rows - 1);
-                                    const float st_a = __ldg(c.a_scale + ti.a_row + tok);
+                                    const float st_a = __shfl_sync(0xffffffffu, my_sa, j);
                                     g = g * st_a * sg;
                                     uu = uu * st_a * su;
                                 }
@@ -435,11 +437,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                         tmem_ld_32cols(tbase + ch * 32, v);
                         tmem_ld_wait();
                         if (F8) {
+                            const float my_sa = __ldg(c.a_scale + ti.a_row + min(ch * 32 + lane, ti.rows - 1));
 #pragma unroll
                             for (int j = 0; j < 32; ++j)
-                                v[j] = __float_as_uint(__uint_as_float(v[j]) *
-                                                       __ldg(c.a_scale + ti.a_row + min(ch * 32 + j, ti.rows - 1)) *
-                                                       sc);
+                                v[j] = __float_as_uint(__uint_as_float(v[j]) * __shfl_sync(0xffffffffu, my_sa, j) * sc);
                         }
                         const int ntok = min(32, ti.rows - ch * 32);
                         const int r0 = ti.a_row + ch * 32;
@@ -493,7 +494,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
             }
             if (!swap_ok) break;      // a hand-over wait gave up: the kernel is being abandoned
             tc_fence_before();
-            mbar_arrive_cluster(tempty_leader0 + (uint32_t)acc * 8u);
+            __syncwarp();             // every lane's tensor-memory reads are done: one arrival per warp
+            if (lane == 0) mbar_arrive_cluster(tempty_leader0 + (uint32_t)acc * 8u);
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
