@@ -476,7 +476,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_const
             }
             tc_fence_before();
             __syncwarp();                     // every lane's tensor-memory reads are done
-            if (lane == 0) mbar_arrive(tempty_bar + acc);
+            if (lane == 0) mbar_arrive_relaxed(tempty_bar + acc);
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }

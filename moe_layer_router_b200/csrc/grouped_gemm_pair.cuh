@@ -495,7 +495,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
             if (!swap_ok) break;      // a hand-over wait gave up: the kernel is being abandoned
             tc_fence_before();
             __syncwarp();             // every lane's tensor-memory reads are done: one arrival per warp
-            if (lane == 0) mbar_arrive_cluster(tempty_leader0 + (uint32_t)acc * 8u);
+            if (lane == 0) mbar_arrive_cluster_relaxed(tempty_leader0 + (uint32_t)acc * 8u);
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }

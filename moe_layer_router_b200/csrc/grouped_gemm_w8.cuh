@@ -149,7 +149,7 @@ grouped_gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(acc_full + a, 1);
-            mbar_init(acc_empty + a, 128);
+            mbar_init(acc_empty + a, 4);       // one arrival per epilogue warp
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -417,15 +417,17 @@ grouped_gemm_w8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
                     }
                 }
             }
-            __syncwarp();
             tc_fence_before();
+            __syncwarp();                     // every lane's tensor-memory reads are done
             if (wide) {
-                mbar_arrive(acc_empty + 0);
-                mbar_arrive(acc_empty + 1);
+                if (lane == 0) {
+                    mbar_arrive_relaxed(acc_empty + 0);
+                    mbar_arrive_relaxed(acc_empty + 1);
+                }
                 aph[0] ^= 1u;
                 aph[1] ^= 1u;
             } else {
-                mbar_arrive(acc_empty + slot);
+                if (lane == 0) mbar_arrive_relaxed(acc_empty + slot);
                 aph[slot] ^= 1u;
                 slot ^= 1;
             }

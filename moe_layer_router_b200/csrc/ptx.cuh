@@ -51,6 +51,14 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Arrival without release semantics, for the accumulator-empty barriers: the arriving warp has
+// completed its tensor-memory reads (tcgen05.wait::ld, then tcgen05.fence::before_thread_sync),
+// which is all the waiting MMA issuer needs; a release would first wait for the warp's outstanding
+// global stores of the tile, which need no ordering with the next MMAs.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -218,6 +226,11 @@ __device__ __forceinline__ void cluster_sync_all() {
 // arrive on an mbarrier given by its shared::cluster address (possibly in the peer CTA)
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+}
+
+// the same without release semantics (see mbar_arrive_relaxed)
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t bar_cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
 }
 
 // 2-D TMA load into this CTA's shared memory whose completion is counted on an mbarrier of
