@@ -281,6 +281,55 @@ def layer_work(wl, N, touched, wbytes=2):
     return flops, b
 
 
+L2_BYTES = 126 * 10**6          # B200 L2
+
+
+def working_set_bytes(wl, wbytes: int = 2) -> float:
+    """Upper bound of the bytes one layer step touches: every expert's weights, the shared expert,
+    the router, x and out, and the permuted rows / h / y_perm of all T k assignments."""
+    T, d, E, k, f, fs = wl.T, wl.d, wl.E, wl.k, wl.f, wl.f_shared
+    return (3.0 * E * f * d * wbytes + 3.0 * fs * d * wbytes + E * d * 2 + 2.0 * T * d * 2 +
+            T * k * (2.0 * d + f) * 2 + (T * (d + fs) * 2 if fs else 0))
+
+
+class L2Flush:
+    """Writes a buffer twice the size of L2 between timed steps whose working set fits in L2, so
+    that every step starts with cold caches."""
+
+    def __init__(self, dev):
+        import torch
+        self.buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.buf.zero_()
+
+
+def timed_steps(fwd, evs, flush, sync=None):
+    """Run len(evs) timed layer steps; with `flush`, L2 is flushed before each step and the step
+    time is the sum of the per-step (route -> end) intervals, so the flushes stay outside it;
+    without, it is the span from the first step's start to the last step's end."""
+    K = len(evs)
+    for i in range(K):
+        if flush is not None:
+            flush()
+        fwd(evs[i])
+    if sync is None:
+        import torch
+        sync = torch.cuda.synchronize
+    sync()
+    if flush is not None:
+        return float(sum(e["route"].elapsed_time(e["end"]) for e in evs))
+    return evs[0]["route"].elapsed_time(evs[K - 1]["end"])
+
+
+def l2_note(wl, flush, wbytes: int = 2) -> str:
+    ws = working_set_bytes(wl, wbytes)
+    if flush is not None:
+        return "L2 flushed before every timed step (a %d MB write; working set %.1f MB < L2)" % (
+            2 * L2_BYTES // 10**6, ws / 1e6)
+    return "working set larger than L2 (%.2f GB per step)" % (ws / 1e9)
+
+
 def roofline_and_layer(wl, N, touched, counts, craw, gemm_ms, step_ms, fp8, a8, peaks, peak_src):
     """The dominant kernel's roofline (GEMM1: tensor-bound for prefill, HBM-bound for decode) and
     the layer's totals for one timed configuration.  gemm_ms: mean kernel times of the two grouped
@@ -334,7 +383,7 @@ def roofline_and_layer(wl, N, touched, counts, craw, gemm_ms, step_ms, fp8, a8, 
 PER_CONFIG_STEPS = {"tiny": 50, "mixtral": 20, "qwen3": 20, "dsv3": 20, "skew": 20}
 
 
-def config_entry(wl, value, ms_per_step, steps, roof, layer, stage_ms, gemm_ms, clocks, cpu):
+def config_entry(wl, value, ms_per_step, steps, roof, layer, stage_ms, gemm_ms, clocks, cpu, l2=None):
     """One workload's record in per_config."""
     r = {k: roof[k] for k in ("bound", "kernel", "achieved", "unit", "peak", "frac", "peak_source")}
     if "frac_of_sustained" in roof:
@@ -344,6 +393,8 @@ def config_entry(wl, value, ms_per_step, steps, roof, layer, stage_ms, gemm_ms, 
          "hbm_frac": layer["hbm_frac"], "kept_rows": layer["kept_rows"], "drop_rate": layer["drop_rate"],
          "load_var_raw": layer["load_var_raw"], "load_var_kept": layer["load_var_kept"],
          "stages_ms": stage_ms, "gemm_ms": gemm_ms, "clocks": clocks, "cpu_baseline": cpu}
+    if l2 is not None:
+        e["l2"] = l2
     if "zipf_l1_error" in layer:
         e["zipf_l1_error"] = layer["zipf_l1_error"]
     return e
@@ -381,15 +432,15 @@ def measure_config(name, dev, warmup, peaks, peak_src, cpu_seconds):
     for e in evs:
         for ev in e.values():
             ev.record()
+    flush = L2Flush(dev) if working_set_bytes(wl) < L2_BYTES else None
     torch.cuda.synchronize()
     with ClockSampler(dev.index) as clk:
-        for i in range(K):
-            fwd(evs[i])
-        torch.cuda.synchronize()
+        total_ms = timed_steps(fwd, evs, flush)
     rc = moe.moe_get_error()
     if rc != 0:
         raise RuntimeError(f"{name}: device error: {moe.strerror(rc)}")
-    total_ms = evs[0]["route"].elapsed_time(evs[K - 1]["end"])
+    l2 = l2_note(wl, flush)
+    del flush
     stage_ms = {a: float(np.mean([e[a].elapsed_time(e[b]) for e in evs]))
                 for a, b in zip(moe.STAGES[:-1], moe.STAGES[1:])}
     gemm_ms = {"gate_up": stage_ms["gate_up"], "down": stage_ms["down"]}
@@ -404,7 +455,7 @@ def measure_config(name, dev, warmup, peaks, peak_src, cpu_seconds):
     torch.cuda.empty_cache()
     cpu = cpu_baseline(wl, cpu_seconds, inp, w) if cpu_seconds > 0 else None
     return config_entry(wl, T * K / (total_ms / 1e3), total_ms / K, K, roof, layer, stage_ms, gemm_ms,
-                        clk.summary(), cpu)
+                        clk.summary(), cpu, l2)
 
 
 
@@ -720,16 +771,16 @@ def main():
     for e in evs:               # torch creates the CUDA event on its first record
         for ev in e.values():
             ev.record()
+    flush = L2Flush(dev) if working_set_bytes(wl, 1 if fp8 else 2) < L2_BYTES else None
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        for i in range(K):
-            fwd(x, out, evs[i])
-        torch.cuda.synchronize()
+        total_ms = timed_steps(lambda e: fwd(x, out, e), evs, flush)
     if world > 1:
         dist.barrier()
-    total_ms = evs[0]["route"].elapsed_time(evs[K - 1]["end"])
+    l2 = l2_note(wl, flush, 1 if fp8 else 2)
+    del flush
     stage_ms = {}
     for a, b in zip(moe.STAGES[:-1], moe.STAGES[1:]):
         stage_ms[a] = float(np.mean([e[a].elapsed_time(e[b]) for e in evs]))
@@ -805,8 +856,7 @@ def main():
                   "bf16 activations, fp8 e4m3 expert weights" if fp8 else "bf16"),
         "data": "synthetic (seeded Philox4x32-10 + Box-Muller; random-init weights)",
         "config": {"workload": DESCR[wl.name], "global_batch": world * T, "seq_len": T, "parallelism": f"dp{world}",
-                   "l2": "working set larger than L2 (expert weights %.2f GB per step)" % (
-                       touched * 3.0 * f * d * 2 / 1e9)},
+                   "l2": l2},
         "roofline": roof,
         "layer": layer,
         "stages_ms": stage_ms,

@@ -44,3 +44,34 @@ def test_launches_per_step():
     # fp8 activations: no gather; x quantiser (routed + shared rows in one), h quantiser, shared h
     assert bench.launches_per_step(True, False) == 10      # 70 launches over 7 layer steps in the ncu list
     assert bench.launches_per_step(True, True) == 11
+
+
+class _Ev:
+    """Stand-in for a timed CUDA event: a timestamp in ms."""
+
+    def __init__(self, t):
+        self.t = t
+
+    def elapsed_time(self, other):
+        return other.t - self.t
+
+
+def test_timed_steps_keeps_l2_flushes_outside_the_timed_steps():
+    # step i runs from 10 i to 10 i + 3 (ms); a flush, when asked for, sits in the gaps
+    evs = [{"route": _Ev(10.0 * i), "end": _Ev(10.0 * i + 3.0)} for i in range(4)]
+    calls = []
+    ran = []
+    t = bench.timed_steps(lambda e: ran.append(e), evs, lambda: calls.append(1), sync=lambda: None)
+    assert t == 4 * 3.0 and len(calls) == 4 and ran == evs
+    # without a flush: the span from the first start to the last end
+    assert bench.timed_steps(lambda e: None, evs, None, sync=lambda: None) == 33.0
+
+
+def test_only_workloads_smaller_than_l2_are_flushed():
+    import synth
+    small = [n for n in ("tiny", "mixtral", "qwen3", "dsv3", "skew")
+             if bench.working_set_bytes(synth.WORKLOADS[n]) < bench.L2_BYTES]
+    assert small == ["tiny"]
+    # the weights alone bound the estimate from below
+    wl = synth.WORKLOADS["mixtral"]
+    assert bench.working_set_bytes(wl) >= 3.0 * wl.E * wl.f * wl.d * 2
