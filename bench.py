@@ -876,7 +876,7 @@ def main():
         for name in synth.WORKLOAD_ORDER:
             if name == wl.name:
                 per[name] = config_entry(wl, value, total_ms / K, K, roof, layer, stage_ms, gemm_ms, line["clocks"],
-                                         line.get("cpu_baseline"))
+                                         line.get("cpu_baseline"), l2)
             else:
                 per[name] = measure_config(name, dev, 3, peaks, peak_src,
                                            0.0 if args.no_cpu_baseline else min(args.cpu_seconds, 6.0))
